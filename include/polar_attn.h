@@ -1,0 +1,191 @@
+/*
+ * polar_attn.h -- C ABI of the B200 (sm_100a) Polar Attention library.
+ *
+ * The library computes the Polar Attention mixing step of "ATMA: Length-
+ * Invariant Language Modeling via Polar Attention and Gated-Delta Compression
+ * Memory" (H. Akbar; gist.science technical summary, section 2.1 "Polar
+ * Attention: A Three-Channel Decomposition") without its recurrent-memory
+ * stream:
+ *
+ *     out = content + count
+ *
+ * For query row i of head h with visible keys j < n (n = i + 1 in causal
+ * prefill, n = seqlen in decode) and kv head g = h / (Hq / Hkv):
+ *
+ *   tau     = 1 + alpha * ln(n / L_train)  if n > L_train, else 1
+ *   z_j     = logit_scale * tau * <q_i, k_j>
+ *   p_j     = softmax_j(z)
+ *   content = (sum_j p_j v_j) / |sum_j p_j v_j|          direction channel
+ *   n_eff   = 1 / sum_j p_j^2  (= l^2 / l2)              participation ratio
+ *   z0      = mean(z) + std(z) * sqrt(2 ln n)            null-floor logit
+ *   gate    = 1 / (1 + exp(-beta * (max_j z_j - z0)))    detection confidence
+ *   count   = gate * tanh(ln(n_eff) / ln(L_train)) * u_h magnitude channel
+ *
+ * std is the population standard deviation of the n visible logits, and the
+ * null logit (whose value vector is zero) enters only the gate, not n_eff.
+ *
+ * Conventions for every entry point:
+ *  - Pointers named *_h are host memory; every other tensor pointer is device
+ *    memory on the current CUDA device.  The caller owns all memory; the
+ *    library allocates nothing, neither device nor pinned memory.
+ *  - Calls are asynchronous and ordered on `stream` (a cudaStream_t; NULL is
+ *    the legacy default stream), except the *_host calls, which synchronise
+ *    `stream` before they return.
+ *  - Argument, shape and alignment errors are detected on the host and
+ *    returned at once, and nothing is launched.  Errors found on the device
+ *    (a page id out of range, a sequence length out of range, a wait that
+ *    timed out) are recorded in a per-device status word that
+ *    polar_attn_get_status() reads.  The kernel involved skips the offending
+ *    work; it never traps.
+ *  - Inputs q and k must be L2-normalised rows (the method normalises queries
+ *    and keys, section 2.1 "Stability Mechanism"); the library does not check
+ *    this.  head_dim must be 64.
+ *  - All tensors are contiguous, with 16-byte aligned base pointers.
+ */
+#ifndef POLAR_ATTN_H
+#define POLAR_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    POLAR_OK = 0,
+    POLAR_ERR_INVALID_ARG = 1, /* bad pointer, shape, stride or parameter */
+    POLAR_ERR_UNSUPPORTED = 2, /* valid but not built (e.g. head_dim != 64) */
+    POLAR_ERR_WORKSPACE = 3,   /* workspace or staging buffer too small */
+    POLAR_ERR_BAD_PAGE = 4,    /* device: page id outside [0, num_pages) */
+    POLAR_ERR_TIMEOUT = 5,     /* device: a bounded wait ran out */
+    POLAR_ERR_CUDA = 6,        /* a CUDA runtime call failed */
+    POLAR_ERR_BAD_SEQLEN = 7   /* device: seqlen outside [1, max_pages*64] */
+} polar_status_t;
+
+typedef enum { POLAR_BF16 = 0, POLAR_FP32 = 1 } polar_dtype_t;
+
+/* Implementation choice for polar_attn_fwd. */
+typedef enum {
+    POLAR_IMPL_AUTO = 0,  /* tensor-core kernel for bf16, SIMT kernel for fp32 */
+    POLAR_IMPL_SIMT = 1,  /* CUDA-core kernel: fp32 FFMA on the exact inputs */
+    POLAR_IMPL_TC = 2     /* tcgen05/TMEM tensor-core kernel (bf16 only) */
+} polar_impl_t;
+
+typedef struct {
+    int B;            /* batch (prefill); ignored by decode */
+    int T;            /* sequence length (prefill); ignored by decode */
+    int Hq, Hkv;      /* query heads, key/value heads; Hq % Hkv == 0, Hq/Hkv <= 8 */
+    int head_dim;     /* must be 64 */
+    int dtype;        /* polar_dtype_t of q, k, v, kv pages and out */
+    float logit_scale;/* s: logits are s * tau * <q, k>; typical 8 */
+    float alpha;      /* length-temperature slope; typical 0.3 */
+    int L_train;      /* training length L_train >= 2; typical 2048 */
+    float beta;       /* gate slope; typical 1.0 */
+    int causal;       /* prefill: must be 1 (row i sees keys 0..i) */
+    int impl;         /* polar_impl_t, prefill only */
+} polar_params_t;
+
+/* Fills *p with the typical constants above for the given shape. */
+void polar_attn_default_params(polar_params_t *p, int B, int T, int Hq, int Hkv, int dtype);
+
+/*
+ * Causal prefill: the fused Polar Attention step over a whole sequence
+ * ("Fused Polar Attention Kernel", section 2.2: participation ratios computed
+ * online with O(block) memory from streaming accumulators with squared
+ * correction factors; no T x T score matrix is stored).
+ *
+ *  q        [B, T, Hq,  64] dtype, device
+ *  k, v     [B, T, Hkv, 64] dtype, device
+ *  u        [Hq, 64] float32, device: the per-head count vectors u_h
+ *  out      [B, T, Hq, 64] dtype, device: content + count
+ *  neff_out [B, Hq, T] float32, device: n_eff per row (may be NULL)
+ *
+ * Returns POLAR_OK once the work is enqueued.  B = 0 or T = 0 is a no-op.
+ */
+polar_status_t polar_attn_fwd(const void *q, const void *k, const void *v, const float *u,
+                              const polar_params_t *params, void *out, float *neff_out,
+                              void *stream);
+
+/* Bytes of device staging that polar_attn_fwd_host needs for this shape. */
+size_t polar_attn_fwd_staging_size(const polar_params_t *params);
+
+/*
+ * polar_attn_fwd on host buffers: copies q, k, v, u from host memory (pinned
+ * memory gives full copy bandwidth) into `staging` (device memory owned by the
+ * caller, at least polar_attn_fwd_staging_size bytes), runs the prefill, copies
+ * out and n_eff back to host memory, and synchronises `stream`.
+ */
+polar_status_t polar_attn_fwd_host(const void *q_h, const void *k_h, const void *v_h,
+                                   const float *u_h, const polar_params_t *params, void *out_h,
+                                   float *neff_h, void *staging, size_t staging_bytes,
+                                   void *stream);
+
+/*
+ * Paged GQA decode: one query token per sequence against a paged KV cache
+ * ("GQA-Grouped Paged Decode Kernel", section 2.2: decode reads the paged KV
+ * cache blocks directly, and each key/value page is read once for all the
+ * query heads of its group).
+ *
+ *  q          [num_seqs, Hq, 64] dtype, device
+ *  kv_pages   [num_pages, 2, Hkv, 64, 64] dtype, device: page p holds 64
+ *             tokens; [p][0] are keys and [p][1] values, head-major, so each
+ *             (page, K|V, head) is one contiguous 64 x 64 block
+ *  page_table [num_seqs, max_pages] int32, device: logical page -> physical
+ *             page; entries at or past ceil(seqlen/64) are never read
+ *  seqlens    [num_seqs] int32, device: tokens in the cache of each sequence,
+ *             1 <= seqlen <= 64 * max_pages; the query sees all of them (its
+ *             own key and value must already be in the cache)
+ *  u          [Hq, 64] float32, device
+ *  out        [num_seqs, Hq, 64] dtype, device
+ *  neff_out   [num_seqs, Hq] float32, device (may be NULL)
+ *  workspace  device scratch of at least polar_attn_decode_workspace_size()
+ *             bytes for the per-split partial states; contents on entry are
+ *             ignored.  Calls that share a workspace must not overlap.
+ *
+ * A page id outside [0, num_pages) sets POLAR_ERR_BAD_PAGE and that page is
+ * skipped; a seqlen out of range sets POLAR_ERR_BAD_SEQLEN and that sequence
+ * is skipped (its outputs are left unwritten).
+ */
+size_t polar_attn_decode_workspace_size(int num_seqs, int max_pages, const polar_params_t *params);
+
+polar_status_t polar_attn_decode_paged(const void *q, const void *kv_pages, int num_pages,
+                                       const int32_t *page_table, int max_pages,
+                                       const int32_t *seqlens, int num_seqs, const float *u,
+                                       const polar_params_t *params, void *out, float *neff_out,
+                                       void *workspace, size_t ws_bytes, void *stream);
+
+/* Bytes of device staging that polar_attn_decode_paged_host needs. */
+size_t polar_attn_decode_staging_size(int num_seqs, int max_pages, const polar_params_t *params);
+
+/*
+ * polar_attn_decode_paged with the per-step inputs (q, page_table, seqlens,
+ * u) in host memory and the outputs returned to host memory; the KV pool stays
+ * resident on the device.  Uses `staging` (device, caller-owned, at least
+ * polar_attn_decode_staging_size bytes, which includes the workspace) and
+ * synchronises `stream` before returning.
+ */
+polar_status_t polar_attn_decode_paged_host(const void *q_h, const void *kv_pages, int num_pages,
+                                            const int32_t *page_table_h, int max_pages,
+                                            const int32_t *seqlens_h, int num_seqs,
+                                            const float *u_h, const polar_params_t *params,
+                                            void *out_h, float *neff_h, void *staging,
+                                            size_t staging_bytes, void *stream);
+
+/*
+ * Synchronises `stream`, returns the first device-side error recorded on the
+ * current device since the last call (POLAR_OK if none) and clears it.
+ */
+polar_status_t polar_attn_get_status(void *stream);
+
+/* Static English description of a status code. */
+const char *polar_attn_status_string(polar_status_t status);
+
+/* Number of kernel launches the library has enqueued on this process so far. */
+uint64_t polar_attn_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* POLAR_ATTN_H */

@@ -1,0 +1,324 @@
+// api.cu -- the C ABI declared in include/polar_attn.h: argument validation,
+// the per-device status word, tensor-map encoding and dispatch to the kernels.
+#include <atomic>
+#include <cmath>
+#include <cstring>
+#include <mutex>
+
+#include <cudaTypedefs.h>
+
+#include "polar_common.cuh"
+#include "polar_internal.h"
+
+namespace polar {
+
+__device__ int g_status = 0;  // first device-side error since the last polar_attn_get_status
+
+namespace {
+
+std::atomic<uint64_t> g_launches{0};
+std::mutex g_mu;
+constexpr int kMaxDevices = 64;
+int *g_status_addr[kMaxDevices] = {nullptr};
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+// Device address of g_status on the current device (looked up once per device).
+int *status_ptr() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!g_status_addr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_status) != cudaSuccess) return nullptr;
+        g_status_addr[dev] = static_cast<int *>(p);
+    }
+    return g_status_addr[dev];
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+size_t dtype_bytes(int dtype) { return dtype == POLAR_FP32 ? 4 : 2; }
+
+polar_status_t check_common(const polar_params_t *p) {
+    if (!p) return POLAR_ERR_INVALID_ARG;
+    if (p->head_dim != kHeadDim) return POLAR_ERR_UNSUPPORTED;
+    if (p->Hq <= 0 || p->Hkv <= 0 || p->Hq % p->Hkv != 0) return POLAR_ERR_INVALID_ARG;
+    if (p->dtype != POLAR_BF16 && p->dtype != POLAR_FP32) return POLAR_ERR_INVALID_ARG;
+    if (!(p->logit_scale > 0.0f) || !std::isfinite(p->logit_scale)) return POLAR_ERR_INVALID_ARG;
+    if (!(p->alpha >= 0.0f) || !std::isfinite(p->alpha)) return POLAR_ERR_INVALID_ARG;
+    if (!std::isfinite(p->beta)) return POLAR_ERR_INVALID_ARG;
+    if (p->L_train < 2) return POLAR_ERR_INVALID_ARG;
+    return POLAR_OK;
+}
+
+polar_status_t check_fwd(const polar_params_t *p) {
+    polar_status_t st = check_common(p);
+    if (st != POLAR_OK) return st;
+    if (p->B < 0 || p->T < 0) return POLAR_ERR_INVALID_ARG;
+    if (p->causal != 1) return POLAR_ERR_UNSUPPORTED;
+    if (p->impl < POLAR_IMPL_AUTO || p->impl > POLAR_IMPL_TC) return POLAR_ERR_INVALID_ARG;
+    if (p->T > (1 << 30) / 64 || p->B > 65535 || p->Hq > 65535) return POLAR_ERR_UNSUPPORTED;
+    return POLAR_OK;
+}
+
+polar_status_t check_decode(const polar_params_t *p, int num_seqs, int max_pages) {
+    polar_status_t st = check_common(p);
+    if (st != POLAR_OK) return st;
+    if (p->dtype != POLAR_BF16) return POLAR_ERR_UNSUPPORTED;
+    const int G = p->Hq / p->Hkv;
+    if (G != 1 && G != 2 && G != 4 && G != 8) return POLAR_ERR_UNSUPPORTED;
+    if (num_seqs < 0 || num_seqs > 65535 || max_pages < 1) return POLAR_ERR_INVALID_ARG;
+    if (static_cast<long long>(max_pages) * kPage > (1ll << 31) - 1) return POLAR_ERR_INVALID_ARG;
+    return POLAR_OK;
+}
+
+polar_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? POLAR_OK : POLAR_ERR_CUDA; }
+
+FwdLaunch make_fwd(const void *q, const void *k, const void *v, const float *u,
+                   const polar_params_t *p, void *out, float *neff, int *status,
+                   cudaStream_t stream) {
+    FwdLaunch a;
+    a.q = q; a.k = k; a.v = v; a.u = u; a.out = out; a.neff = neff;
+    a.B = p->B; a.T = p->T; a.Hq = p->Hq; a.Hkv = p->Hkv; a.dtype = p->dtype;
+    a.s = p->logit_scale; a.alpha = p->alpha; a.beta = p->beta; a.L = p->L_train;
+    a.status = status; a.stream = stream;
+    return a;
+}
+
+}  // namespace
+
+void count_launches(int n) { g_launches.fetch_add(static_cast<uint64_t>(n)); }
+
+CUresult encode_tiled(CUtensorMap *map, CUtensorMapDataType dtype, uint32_t rank, void *base,
+                      const uint64_t *dims, const uint64_t *strides_bytes, const uint32_t *box,
+                      CUtensorMapSwizzle swizzle) {
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        if (!g_encode) {
+            void *fn = nullptr;
+            cudaDriverEntryPointQueryResult q;
+            if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) !=
+                    cudaSuccess ||
+                q != cudaDriverEntryPointSuccess || !fn)
+                return CUDA_ERROR_NOT_FOUND;
+            g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+        }
+    }
+    uint32_t estr[5] = {1, 1, 1, 1, 1};
+    return g_encode(map, dtype, rank, base, dims, strides_bytes, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+}
+
+}  // namespace polar
+
+using namespace polar;
+
+extern "C" {
+
+void polar_attn_default_params(polar_params_t *p, int B, int T, int Hq, int Hkv, int dtype) {
+    if (!p) return;
+    std::memset(p, 0, sizeof *p);
+    p->B = B; p->T = T; p->Hq = Hq; p->Hkv = Hkv; p->head_dim = kHeadDim; p->dtype = dtype;
+    p->logit_scale = 8.0f; p->alpha = 0.3f; p->L_train = 2048; p->beta = 1.0f;
+    p->causal = 1; p->impl = POLAR_IMPL_AUTO;
+}
+
+polar_status_t polar_attn_fwd(const void *q, const void *k, const void *v, const float *u,
+                              const polar_params_t *params, void *out, float *neff_out,
+                              void *stream) {
+    polar_status_t st = check_fwd(params);
+    if (st != POLAR_OK) return st;
+    if (params->B == 0 || params->T == 0) return POLAR_OK;
+    if (!q || !k || !v || !u || !out) return POLAR_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(u) || !aligned16(out) ||
+        (neff_out && (reinterpret_cast<uintptr_t>(neff_out) & 3u)))
+        return POLAR_ERR_INVALID_ARG;
+    int *status = status_ptr();
+    if (!status) return POLAR_ERR_CUDA;
+    FwdLaunch a = make_fwd(q, k, v, u, params, out, neff_out, status,
+                           static_cast<cudaStream_t>(stream));
+    const bool tc = params->impl == POLAR_IMPL_TC ||
+                    (params->impl == POLAR_IMPL_AUTO && params->dtype == POLAR_BF16);
+    if (tc) {
+        if (params->dtype != POLAR_BF16) return POLAR_ERR_UNSUPPORTED;
+        return from_cuda(launch_fwd_tc(a));
+    }
+    return from_cuda(launch_fwd_simt(a));
+}
+
+size_t polar_attn_fwd_staging_size(const polar_params_t *p) {
+    if (check_fwd(p) != POLAR_OK) return 0;
+    const size_t e = dtype_bytes(p->dtype);
+    const size_t rows = static_cast<size_t>(p->B) * p->T;
+    size_t n = 0;
+    n += round_up(rows * p->Hq * kHeadDim * e, 256);       // q
+    n += 2 * round_up(rows * p->Hkv * kHeadDim * e, 256);  // k, v
+    n += round_up(static_cast<size_t>(p->Hq) * kHeadDim * 4, 256);  // u
+    n += round_up(rows * p->Hq * kHeadDim * e, 256);       // out
+    n += round_up(rows * p->Hq * 4, 256);                  // neff
+    return n;
+}
+
+polar_status_t polar_attn_fwd_host(const void *q_h, const void *k_h, const void *v_h,
+                                   const float *u_h, const polar_params_t *p, void *out_h,
+                                   float *neff_h, void *staging, size_t staging_bytes,
+                                   void *stream) {
+    polar_status_t st = check_fwd(p);
+    if (st != POLAR_OK) return st;
+    if (p->B == 0 || p->T == 0) return POLAR_OK;
+    if (!q_h || !k_h || !v_h || !u_h || !out_h || !staging) return POLAR_ERR_INVALID_ARG;
+    if (staging_bytes < polar_attn_fwd_staging_size(p)) return POLAR_ERR_WORKSPACE;
+    if (!aligned16(staging)) return POLAR_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const size_t e = dtype_bytes(p->dtype);
+    const size_t rows = static_cast<size_t>(p->B) * p->T;
+    const size_t qb = rows * p->Hq * kHeadDim * e, kb = rows * p->Hkv * kHeadDim * e;
+    const size_t ub = static_cast<size_t>(p->Hq) * kHeadDim * 4, nb = rows * p->Hq * 4;
+    char *base = static_cast<char *>(staging);
+    char *dq = base;
+    char *dk = dq + round_up(qb, 256);
+    char *dv = dk + round_up(kb, 256);
+    char *du = dv + round_up(kb, 256);
+    char *dout = du + round_up(ub, 256);
+    char *dne = dout + round_up(qb, 256);
+    if (cudaMemcpyAsync(dq, q_h, qb, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+        cudaMemcpyAsync(dk, k_h, kb, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+        cudaMemcpyAsync(dv, v_h, kb, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+        cudaMemcpyAsync(du, u_h, ub, cudaMemcpyHostToDevice, s) != cudaSuccess)
+        return POLAR_ERR_CUDA;
+    st = polar_attn_fwd(dq, dk, dv, reinterpret_cast<float *>(du), p, dout,
+                        neff_h ? reinterpret_cast<float *>(dne) : nullptr, stream);
+    if (st != POLAR_OK) return st;
+    if (cudaMemcpyAsync(out_h, dout, qb, cudaMemcpyDeviceToHost, s) != cudaSuccess) return POLAR_ERR_CUDA;
+    if (neff_h && cudaMemcpyAsync(neff_h, dne, nb, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+        return POLAR_ERR_CUDA;
+    return from_cuda(cudaStreamSynchronize(s));
+}
+
+size_t polar_attn_decode_workspace_size(int num_seqs, int max_pages, const polar_params_t *p) {
+    if (check_decode(p, num_seqs, max_pages) != POLAR_OK) return 0;
+    return decode_partials_bytes(num_seqs, max_pages, p->Hq, p->Hkv);
+}
+
+polar_status_t polar_attn_decode_paged(const void *q, const void *kv_pages, int num_pages,
+                                       const int32_t *page_table, int max_pages,
+                                       const int32_t *seqlens, int num_seqs, const float *u,
+                                       const polar_params_t *p, void *out, float *neff_out,
+                                       void *workspace, size_t ws_bytes, void *stream) {
+    polar_status_t st = check_decode(p, num_seqs, max_pages);
+    if (st != POLAR_OK) return st;
+    if (num_seqs == 0) return POLAR_OK;
+    if (num_pages < 1 || static_cast<long long>(num_pages) * 2 * p->Hkv * kPage > (1ll << 31) - 1)
+        return POLAR_ERR_INVALID_ARG;
+    if (!q || !kv_pages || !page_table || !seqlens || !u || !out || !workspace)
+        return POLAR_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(kv_pages) || !aligned16(u) || !aligned16(out) ||
+        !aligned16(workspace) || (reinterpret_cast<uintptr_t>(page_table) & 3u) ||
+        (reinterpret_cast<uintptr_t>(seqlens) & 3u) ||
+        (neff_out && (reinterpret_cast<uintptr_t>(neff_out) & 3u)))
+        return POLAR_ERR_INVALID_ARG;
+    if (ws_bytes < decode_partials_bytes(num_seqs, max_pages, p->Hq, p->Hkv))
+        return POLAR_ERR_WORKSPACE;
+    int *status = status_ptr();
+    if (!status) return POLAR_ERR_CUDA;
+    DecodeLaunch a;
+    a.q = q; a.kv_pages = kv_pages; a.num_pages = num_pages; a.page_table = page_table;
+    a.max_pages = max_pages; a.seqlens = seqlens; a.num_seqs = num_seqs; a.u = u; a.out = out;
+    a.neff = neff_out; a.Hq = p->Hq; a.Hkv = p->Hkv; a.s = p->logit_scale; a.alpha = p->alpha;
+    a.beta = p->beta; a.L = p->L_train; a.workspace = workspace; a.status = status;
+    a.stream = static_cast<cudaStream_t>(stream);
+    return from_cuda(launch_decode(a));
+}
+
+size_t polar_attn_decode_staging_size(int num_seqs, int max_pages, const polar_params_t *p) {
+    if (check_decode(p, num_seqs, max_pages) != POLAR_OK) return 0;
+    const size_t e = dtype_bytes(p->dtype);
+    size_t n = 0;
+    n += round_up(static_cast<size_t>(num_seqs) * p->Hq * kHeadDim * e, 256);  // q
+    n += round_up(static_cast<size_t>(num_seqs) * max_pages * 4, 256);         // page table
+    n += round_up(static_cast<size_t>(num_seqs) * 4, 256);                     // seqlens
+    n += round_up(static_cast<size_t>(p->Hq) * kHeadDim * 4, 256);             // u
+    n += round_up(static_cast<size_t>(num_seqs) * p->Hq * kHeadDim * e, 256);  // out
+    n += round_up(static_cast<size_t>(num_seqs) * p->Hq * 4, 256);             // neff
+    n += round_up(decode_partials_bytes(num_seqs, max_pages, p->Hq, p->Hkv), 256);
+    return n;
+}
+
+polar_status_t polar_attn_decode_paged_host(const void *q_h, const void *kv_pages, int num_pages,
+                                            const int32_t *page_table_h, int max_pages,
+                                            const int32_t *seqlens_h, int num_seqs,
+                                            const float *u_h, const polar_params_t *p,
+                                            void *out_h, float *neff_h, void *staging,
+                                            size_t staging_bytes, void *stream) {
+    polar_status_t st = check_decode(p, num_seqs, max_pages);
+    if (st != POLAR_OK) return st;
+    if (num_seqs == 0) return POLAR_OK;
+    if (!q_h || !page_table_h || !seqlens_h || !u_h || !out_h || !staging)
+        return POLAR_ERR_INVALID_ARG;
+    if (staging_bytes < polar_attn_decode_staging_size(num_seqs, max_pages, p))
+        return POLAR_ERR_WORKSPACE;
+    if (!aligned16(staging)) return POLAR_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const size_t e = dtype_bytes(p->dtype);
+    const size_t qb = static_cast<size_t>(num_seqs) * p->Hq * kHeadDim * e;
+    const size_t ptb = static_cast<size_t>(num_seqs) * max_pages * 4;
+    const size_t slb = static_cast<size_t>(num_seqs) * 4;
+    const size_t ub = static_cast<size_t>(p->Hq) * kHeadDim * 4;
+    const size_t nb = static_cast<size_t>(num_seqs) * p->Hq * 4;
+    const size_t wsb = decode_partials_bytes(num_seqs, max_pages, p->Hq, p->Hkv);
+    char *dq = static_cast<char *>(staging);
+    char *dpt = dq + round_up(qb, 256);
+    char *dsl = dpt + round_up(ptb, 256);
+    char *du = dsl + round_up(slb, 256);
+    char *dout = du + round_up(ub, 256);
+    char *dne = dout + round_up(qb, 256);
+    char *dws = dne + round_up(nb, 256);
+    if (cudaMemcpyAsync(dq, q_h, qb, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+        cudaMemcpyAsync(dpt, page_table_h, ptb, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+        cudaMemcpyAsync(dsl, seqlens_h, slb, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+        cudaMemcpyAsync(du, u_h, ub, cudaMemcpyHostToDevice, s) != cudaSuccess)
+        return POLAR_ERR_CUDA;
+    st = polar_attn_decode_paged(dq, kv_pages, num_pages, reinterpret_cast<int32_t *>(dpt),
+                                 max_pages, reinterpret_cast<int32_t *>(dsl), num_seqs,
+                                 reinterpret_cast<float *>(du), p, dout,
+                                 neff_h ? reinterpret_cast<float *>(dne) : nullptr, dws, wsb,
+                                 stream);
+    if (st != POLAR_OK) return st;
+    if (cudaMemcpyAsync(out_h, dout, qb, cudaMemcpyDeviceToHost, s) != cudaSuccess) return POLAR_ERR_CUDA;
+    if (neff_h && cudaMemcpyAsync(neff_h, dne, nb, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+        return POLAR_ERR_CUDA;
+    return from_cuda(cudaStreamSynchronize(s));
+}
+
+polar_status_t polar_attn_get_status(void *stream) {
+    int *status = status_ptr();
+    if (!status) return POLAR_ERR_CUDA;
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return POLAR_ERR_CUDA;
+    int v = 0;
+    if (cudaMemcpy(&v, status, sizeof v, cudaMemcpyDeviceToHost) != cudaSuccess) return POLAR_ERR_CUDA;
+    const int zero = 0;
+    if (cudaMemcpy(status, &zero, sizeof zero, cudaMemcpyHostToDevice) != cudaSuccess)
+        return POLAR_ERR_CUDA;
+    return static_cast<polar_status_t>(v);
+}
+
+const char *polar_attn_status_string(polar_status_t s) {
+    switch (s) {
+        case POLAR_OK: return "ok";
+        case POLAR_ERR_INVALID_ARG: return "invalid argument, shape, stride or alignment";
+        case POLAR_ERR_UNSUPPORTED: return "unsupported configuration";
+        case POLAR_ERR_WORKSPACE: return "workspace or staging buffer too small";
+        case POLAR_ERR_BAD_PAGE: return "page id outside the page pool";
+        case POLAR_ERR_TIMEOUT: return "a bounded device wait timed out";
+        case POLAR_ERR_CUDA: return "CUDA runtime error";
+        case POLAR_ERR_BAD_SEQLEN: return "sequence length outside [1, 64*max_pages]";
+    }
+    return "unknown status";
+}
+
+uint64_t polar_attn_launch_count(void) { return g_launches.load(); }
+
+}  // extern "C"

@@ -1,0 +1,58 @@
+// polar_internal.h -- host-side interface between the C ABI (api.cu) and the
+// kernel launchers.  Not installed; not part of the public ABI.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace polar {
+
+struct FwdLaunch {
+    const void *q, *k, *v;
+    const float *u;
+    void *out;
+    float *neff;  // may be null
+    int B, T, Hq, Hkv;
+    int dtype;    // POLAR_BF16 / POLAR_FP32
+    float s, alpha, beta;
+    int L;
+    int *status;  // device status word
+    cudaStream_t stream;
+};
+
+struct DecodeLaunch {
+    const void *q, *kv_pages;
+    int num_pages;
+    const int32_t *page_table;
+    int max_pages;
+    const int32_t *seqlens;
+    int num_seqs;
+    const float *u;
+    void *out;
+    float *neff;
+    int Hq, Hkv;
+    float s, alpha, beta;
+    int L;
+    void *workspace;
+    int *status;
+    cudaStream_t stream;
+};
+
+// Launchers return cudaSuccess or the launch error.
+cudaError_t launch_fwd_simt(const FwdLaunch &a);
+cudaError_t launch_fwd_tc(const FwdLaunch &a);
+cudaError_t launch_decode(const DecodeLaunch &a);
+
+// Decode work split: pages per split and the partial-state bytes it needs.
+int decode_pages_per_split(int num_seqs, int max_pages, int Hkv);
+size_t decode_partials_bytes(int num_seqs, int max_pages, int Hq, int Hkv);
+
+// Bookkeeping shared by the launchers.
+void count_launches(int n);
+CUresult encode_tiled(CUtensorMap *map, CUtensorMapDataType dtype, uint32_t rank, void *base,
+                      const uint64_t *dims, const uint64_t *strides_bytes, const uint32_t *box,
+                      CUtensorMapSwizzle swizzle);
+
+}  // namespace polar

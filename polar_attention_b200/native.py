@@ -1,0 +1,220 @@
+"""ctypes binding of libpolar_attn.so, the C ABI of include/polar_attn.h.
+
+Argument marshalling only: torch tensors supply device memory and streams, and
+every step of the computation runs in the library's CUDA kernels.  There is no
+CPU or PyTorch fallback; a missing or unloadable library raises at once.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libpolar_attn.so")
+
+POLAR_BF16, POLAR_FP32 = 0, 1
+IMPLS = {"auto": 0, "simt": 1, "tc": 2}
+STATUS = {0: "POLAR_OK", 1: "POLAR_ERR_INVALID_ARG", 2: "POLAR_ERR_UNSUPPORTED",
+          3: "POLAR_ERR_WORKSPACE", 4: "POLAR_ERR_BAD_PAGE", 5: "POLAR_ERR_TIMEOUT",
+          6: "POLAR_ERR_CUDA", 7: "POLAR_ERR_BAD_SEQLEN"}
+
+# Every entry point include/polar_attn.h declares.
+EXPORTS = ["polar_attn_default_params", "polar_attn_fwd", "polar_attn_fwd_staging_size",
+           "polar_attn_fwd_host", "polar_attn_decode_workspace_size", "polar_attn_decode_paged",
+           "polar_attn_decode_staging_size", "polar_attn_decode_paged_host",
+           "polar_attn_get_status", "polar_attn_status_string", "polar_attn_launch_count"]
+
+
+class PolarError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: {STATUS.get(code, code)} ({status_string(code)})")
+
+
+class Params(ctypes.Structure):
+    """polar_params_t."""
+    _fields_ = [("B", ctypes.c_int), ("T", ctypes.c_int), ("Hq", ctypes.c_int),
+                ("Hkv", ctypes.c_int), ("head_dim", ctypes.c_int), ("dtype", ctypes.c_int),
+                ("logit_scale", ctypes.c_float), ("alpha", ctypes.c_float),
+                ("L_train", ctypes.c_int), ("beta", ctypes.c_float), ("causal", ctypes.c_int),
+                ("impl", ctypes.c_int)]
+
+
+_lib = None
+_lock = threading.Lock()
+
+
+def lib() -> ctypes.CDLL:
+    """Loads libpolar_attn.so (build it with ``python -m polar_attention_b200.build``)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise RuntimeError(f"{LIB_PATH} is missing: build the CUDA library with "
+                                   "`python -m polar_attention_b200.build` (no fallback exists)")
+            L = ctypes.CDLL(LIB_PATH)
+            P, I, Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+            PP = ctypes.POINTER(Params)
+            L.polar_attn_default_params.argtypes = [PP, I, I, I, I, I]
+            L.polar_attn_default_params.restype = None
+            L.polar_attn_fwd.argtypes = [P, P, P, P, PP, P, P, P]
+            L.polar_attn_fwd_staging_size.argtypes = [PP]
+            L.polar_attn_fwd_staging_size.restype = Z
+            L.polar_attn_fwd_host.argtypes = [P, P, P, P, PP, P, P, P, Z, P]
+            L.polar_attn_decode_workspace_size.argtypes = [I, I, PP]
+            L.polar_attn_decode_workspace_size.restype = Z
+            L.polar_attn_decode_paged.argtypes = [P, P, I, P, I, P, I, P, PP, P, P, P, Z, P]
+            L.polar_attn_decode_staging_size.argtypes = [I, I, PP]
+            L.polar_attn_decode_staging_size.restype = Z
+            L.polar_attn_decode_paged_host.argtypes = [P, P, I, P, I, P, I, P, PP, P, P, P, Z, P]
+            L.polar_attn_get_status.argtypes = [P]
+            L.polar_attn_status_string.argtypes = [I]
+            L.polar_attn_status_string.restype = ctypes.c_char_p
+            L.polar_attn_launch_count.restype = ctypes.c_uint64
+            for name in ("polar_attn_fwd", "polar_attn_fwd_host", "polar_attn_decode_paged",
+                         "polar_attn_decode_paged_host", "polar_attn_get_status"):
+                getattr(L, name).restype = I
+            _lib = L
+    return _lib
+
+
+def status_string(code: int) -> str:
+    try:
+        return lib().polar_attn_status_string(int(code)).decode()
+    except Exception:  # the library may be what failed
+        return "?"
+
+
+def make_params(B=0, T=0, Hq=16, Hkv=4, dtype=POLAR_BF16, s=8.0, alpha=0.3, L=2048, beta=1.0,
+                impl="auto") -> Params:
+    p = Params()
+    lib().polar_attn_default_params(ctypes.byref(p), B, T, Hq, Hkv, dtype)
+    p.logit_scale, p.alpha, p.L_train, p.beta = s, alpha, L, beta
+    p.impl = IMPLS[impl] if isinstance(impl, str) else int(impl)
+    return p
+
+
+def _dt(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return POLAR_BF16
+    if t.dtype == torch.float32:
+        return POLAR_FP32
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _check(code: int, where: str):
+    if code != 0:
+        raise PolarError(code, where)
+
+
+def fwd(q, k, v, u, out=None, neff=None, *, s=8.0, alpha=0.3, L=2048, beta=1.0, impl="auto",
+        stream=None, want_neff=True):
+    """Causal prefill.  q [B,T,Hq,64], k/v [B,T,Hkv,64] (bf16 or fp32, CUDA,
+    contiguous), u [Hq,64] fp32.  Returns (out [B,T,Hq,64], neff [B,Hq,T])."""
+    B, T, Hq, D = q.shape
+    Hkv = k.shape[2]
+    for t in (q, k, v, u):
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError("inputs must be contiguous CUDA tensors")
+    if u.dtype != torch.float32:
+        raise TypeError("u must be float32")
+    if out is None:
+        out = torch.empty_like(q)
+    if neff is None and want_neff:
+        neff = torch.empty((B, Hq, T), device=q.device, dtype=torch.float32)
+    p = make_params(B, T, Hq, Hkv, _dt(q), s, alpha, L, beta, impl)
+    p.head_dim = D
+    _check(lib().polar_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(u), ctypes.byref(p), _ptr(out),
+                                _ptr(neff), _stream(stream)), "polar_attn_fwd")
+    return out, neff
+
+
+def decode_workspace_size(num_seqs: int, max_pages: int, Hq: int, Hkv: int) -> int:
+    p = make_params(0, 0, Hq, Hkv, POLAR_BF16)
+    return int(lib().polar_attn_decode_workspace_size(num_seqs, max_pages, ctypes.byref(p)))
+
+
+def decode_paged(q, kv_pages, page_table, seqlens, u, out=None, neff=None, workspace=None, *,
+                 s=8.0, alpha=0.3, L=2048, beta=1.0, stream=None, want_neff=True):
+    """Paged GQA decode.  q [N,Hq,64] bf16; kv_pages [P,2,Hkv,64,64] bf16;
+    page_table [N,max_pages] int32; seqlens [N] int32; u [Hq,64] fp32.
+    Returns (out [N,Hq,64], neff [N,Hq])."""
+    N, Hq, D = q.shape
+    P_, _, Hkv, _, _ = kv_pages.shape
+    max_pages = page_table.shape[1]
+    if page_table.dtype != torch.int32 or seqlens.dtype != torch.int32:
+        raise TypeError("page_table and seqlens must be int32")
+    p = make_params(0, 0, Hq, Hkv, _dt(q), s, alpha, L, beta)
+    p.head_dim = D
+    ws_need = int(lib().polar_attn_decode_workspace_size(N, max_pages, ctypes.byref(p)))
+    if workspace is None:
+        workspace = torch.empty(max(ws_need, 16), device=q.device, dtype=torch.uint8)
+    if out is None:
+        out = torch.empty_like(q)
+    if neff is None and want_neff:
+        neff = torch.empty((N, Hq), device=q.device, dtype=torch.float32)
+    _check(lib().polar_attn_decode_paged(
+        _ptr(q), _ptr(kv_pages), P_, _ptr(page_table), max_pages, _ptr(seqlens), N, _ptr(u),
+        ctypes.byref(p), _ptr(out), _ptr(neff), _ptr(workspace), workspace.numel(),
+        _stream(stream)), "polar_attn_decode_paged")
+    return out, neff
+
+
+def fwd_staging_size(B, T, Hq, Hkv, dtype=POLAR_BF16) -> int:
+    p = make_params(B, T, Hq, Hkv, dtype)
+    return int(lib().polar_attn_fwd_staging_size(ctypes.byref(p)))
+
+
+def fwd_host(q_h, k_h, v_h, u_h, out_h, neff_h, staging, *, s=8.0, alpha=0.3, L=2048, beta=1.0,
+             impl="auto", stream=None):
+    """polar_attn_fwd_host on (pinned) host tensors; staging is a CUDA uint8
+    tensor of at least fwd_staging_size bytes.  Synchronises the stream."""
+    B, T, Hq, D = q_h.shape
+    p = make_params(B, T, Hq, k_h.shape[2], _dt(q_h), s, alpha, L, beta, impl)
+    p.head_dim = D
+    _check(lib().polar_attn_fwd_host(_ptr(q_h), _ptr(k_h), _ptr(v_h), _ptr(u_h), ctypes.byref(p),
+                                     _ptr(out_h), _ptr(neff_h), _ptr(staging), staging.numel(),
+                                     _stream(stream)), "polar_attn_fwd_host")
+
+
+def decode_staging_size(num_seqs, max_pages, Hq, Hkv) -> int:
+    p = make_params(0, 0, Hq, Hkv, POLAR_BF16)
+    return int(lib().polar_attn_decode_staging_size(num_seqs, max_pages, ctypes.byref(p)))
+
+
+def decode_paged_host(q_h, kv_pages, page_table_h, seqlens_h, u_h, out_h, neff_h, staging, *,
+                      s=8.0, alpha=0.3, L=2048, beta=1.0, stream=None):
+    """polar_attn_decode_paged_host: per-step inputs and outputs in (pinned)
+    host memory, the KV pool resident on the device.  Synchronises the stream."""
+    N, Hq, D = q_h.shape
+    P_, _, Hkv, _, _ = kv_pages.shape
+    p = make_params(0, 0, Hq, Hkv, _dt(q_h), s, alpha, L, beta)
+    p.head_dim = D
+    _check(lib().polar_attn_decode_paged_host(
+        _ptr(q_h), _ptr(kv_pages), P_, _ptr(page_table_h), page_table_h.shape[1], _ptr(seqlens_h),
+        N, _ptr(u_h), ctypes.byref(p), _ptr(out_h), _ptr(neff_h), _ptr(staging), staging.numel(),
+        _stream(stream)), "polar_attn_decode_paged_host")
+
+
+def get_status(stream=None) -> int:
+    """Synchronises the stream; returns and clears the device status word."""
+    return int(lib().polar_attn_get_status(_stream(stream)))
+
+
+def launch_count() -> int:
+    return int(lib().polar_attn_launch_count())
