@@ -140,10 +140,12 @@ polar_status_t polar_attn_fwd(const void *q, const void *k, const void *v, const
     if (!status) return POLAR_ERR_CUDA;
     FwdLaunch a = make_fwd(q, k, v, u, params, out, neff_out, status,
                            static_cast<cudaStream_t>(stream));
-    const bool tc = params->impl == POLAR_IMPL_TC ||
-                    (params->impl == POLAR_IMPL_AUTO && params->dtype == POLAR_BF16);
+    // The tensor-core kernel pairs two query heads of one key/value group per
+    // CTA, so it needs an even group size; fp32 inputs use the CUDA-core kernel.
+    const bool tc_ok = params->dtype == POLAR_BF16 && (params->Hq / params->Hkv) % 2 == 0;
+    const bool tc = params->impl == POLAR_IMPL_TC || (params->impl == POLAR_IMPL_AUTO && tc_ok);
     if (tc) {
-        if (params->dtype != POLAR_BF16) return POLAR_ERR_UNSUPPORTED;
+        if (!tc_ok) return POLAR_ERR_UNSUPPORTED;
         return from_cuda(launch_fwd_tc(a));
     }
     return from_cuda(launch_fwd_simt(a));
