@@ -1,0 +1,477 @@
+"""Benchmark of the Polar Attention hot path on B200.
+
+One step = one pass of the whole path on one GPU's batch of synthetic input:
+  * causal prefill, B=2, Hq=16, Hkv=4, T=16384, d=64, bf16, length temperature
+    active (the extrapolation workload), through polar_attn_fwd; then
+  * paged GQA decode, 32 sequences with 128K-256K tokens of context in 64-token
+    pages behind a shuffled page table, Hq=16, Hkv=4, bf16, through
+    polar_attn_decode_paged.
+value: prefill TFLOP/s (algorithmic flops of the visible causal triangle,
+4*d per visible query-key pair) over all ranks / max-over-ranks prefill time;
+decode.value: HBM GB/s (algorithmic KV bytes, 1024 per cached token per
+sequence: K and V, 4 heads, 64 dims, bf16) likewise.  Times come from CUDA
+events on the launching stream.  Multi-GPU (torchrun) runs independent
+replicas, one batch per rank with its own seed ("scaling": "weak"); the only
+collectives are the barrier and the max of the timings.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl {ours,reference}]
+"""
+from __future__ import annotations
+
+import argparse
+import csv
+import hashlib
+import io
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from polar_attention_b200 import workloads as W  # noqa: E402
+
+METRIC = "Polar-attn fwd TFLOP/s & % BF16 peak at T=16K; decode HBM GB/s at 256K ctx"
+PREFILL = W.EXTRAP
+DECODE = W.DECODE
+KV_BYTES_PER_TOKEN = DECODE.Hkv * DECODE.D * 2 * 2  # K and V, 4 heads, 64 dims, bf16: 1024
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ----------------------------------------------------------------- plumbing --
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0,
+                    help="CPU work budget of the oracle baseline sample")
+    ap.add_argument("--only", choices=["both", "prefill", "decode"], default="both",
+                    help="time one half of the step (profiling runs)")
+    ap.add_argument("--prefill", choices=sorted(W.PREFILL_WORKLOADS), default=W.EXTRAP.name,
+                    help="prefill workload (profiling runs use a smaller one)")
+    ap.add_argument("--decode-seqs", type=int, default=W.DECODE.num_seqs,
+                    help="decode sequences (profiling runs use fewer)")
+    return ap.parse_args(argv)
+
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def rank_seed(base: int, rank: int) -> int:
+    """Each rank draws its own batch: weak scaling over independent problems."""
+    return base + 1000 * rank
+
+
+def max_over_ranks(x: float, world: int, device) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int, device=None):
+    if world > 1:
+        import torch.distributed as dist
+        if device is not None and device.type == "cuda":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+def aggregate_throughput(work_per_rank: float, world: int, max_seconds: float) -> float:
+    """Whole-job throughput: every rank's work over the slowest rank's time."""
+    return work_per_rank * world / max_seconds
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def source_sha(*names) -> str:
+    h = hashlib.sha256()
+    for n in names:
+        with open(os.path.join(ROOT, "polar_attention_b200", "csrc", n), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(kernel: str, sha: str):
+    """dram bytes per launch from the committed ncu summary, if it was taken on
+    the kernel as it is now (same source hash); else None."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    e = d.get(kernel)
+    if not e or e.get("source_sha") != sha:
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling during the timed region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,utilization.gpu,"
+              "clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_indices):
+        self.idx = [str(i) for i in gpu_indices]
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100", "-i", ",".join(self.idx)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, ValueError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                self.out = ""
+        return False
+
+    def summary(self):
+        if self.proc is None or not getattr(self, "out", ""):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        rows = [r for r in csv.reader(io.StringIO(self.out)) if len(r) >= 10]
+        sm, mx, reasons, load = [], [], set(), []
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            try:
+                s, m, util = float(r[1]), float(r[2]), float(r[4])
+            except ValueError:
+                continue
+            mx.append(m)
+            if util >= 50:
+                load.append(s)
+                for n, v in zip(names, r[6:10]):
+                    if v.strip().lower() == "active":
+                        reasons.add(n)
+            sm.append(s)
+        use = load if load else sm
+        return {"sm_mhz": statistics.median(use) if use else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": sorted(reasons),
+                "samples": len(rows), "samples_under_load": len(load)}
+
+
+# -------------------------------------------------------------- CPU oracle --
+
+def _oracle_prefill_rows(x_host, rows, w):
+    import oracle
+    return oracle.polar_fwd(x_host["q"], x_host["k"], x_host["v"], x_host["u"],
+                            oracle.Params(s=w.s, alpha=w.alpha, L=w.L, beta=w.beta), rows=rows)
+
+
+def prefill_rows_flops(rows, w) -> float:
+    i = np.asarray(rows) % w.T
+    return float(4.0 * w.D * np.sum(i + 1))
+
+
+def cpu_prefill_inputs(seed=0):
+    x = W.prefill_inputs(PREFILL, "cpu", seed=seed)
+    return {"q": W.to_host_bits(x["q"]), "k": W.to_host_bits(x["k"]), "v": W.to_host_bits(x["v"]),
+            "u": x["u"].numpy()}
+
+
+def oracle_threads() -> int:
+    return int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+
+
+def calibrated_rows(x_host, budget_s: float, rng, probe_rows=32):
+    """Seeded sample of prefill rows sized to about budget_s of oracle time."""
+    total = PREFILL.B * PREFILL.Hq * PREFILL.T
+    probe = rng.integers(0, total, size=probe_rows)
+    t0 = time.perf_counter()
+    _oracle_prefill_rows(x_host, probe, PREFILL)
+    dt = max(time.perf_counter() - t0, 1e-3)
+    n = int(max(probe_rows, min(200000, probe_rows * budget_s / dt)))
+    return rng.integers(0, total, size=n)
+
+
+def cpu_baseline(budget_s: float, seed=0) -> dict:
+    x_host = cpu_prefill_inputs(seed)
+    rng = np.random.default_rng(seed + 7)
+    rows = calibrated_rows(x_host, budget_s, rng)
+    t0 = time.perf_counter()
+    _oracle_prefill_rows(x_host, rows, PREFILL)
+    dt = time.perf_counter() - t0
+    return {"value": prefill_rows_flops(rows, PREFILL) / dt / 1e12, "unit": "TFLOP/s",
+            "cores": oracle_threads(), "kind": "oracle",
+            "sample": f"{rows.size} seeded random rows of the T=16384 prefill workload "
+                      f"(fp64 two-pass oracle, {dt:.1f} s)"}
+
+
+# ------------------------------------------------------------------ GPU arm --
+
+def run_ours(args):
+    import dataclasses
+
+    import polar_attention_b200 as pa
+
+    global PREFILL, DECODE
+    PREFILL = W.PREFILL_WORKLOADS[args.prefill]
+    DECODE = dataclasses.replace(W.DECODE, num_seqs=args.decode_seqs)
+    do_pre = args.only in ("both", "prefill")
+    do_dec = args.only in ("both", "decode")
+
+    rank, world, local = dist_env()
+    if world > 1:
+        import torch.distributed as dist
+        from datetime import timedelta
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300))
+    dev = torch.device("cuda", local if world > 1 else 0)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+
+    seed = rank_seed(0, rank)
+    if do_pre:
+        xp = W.prefill_inputs(PREFILL, dev, seed=seed)
+        out_p = torch.empty_like(xp["q"])
+        neff_p = torch.empty((PREFILL.B, PREFILL.Hq, PREFILL.T), device=dev)
+    kv_bytes, tokens = 0.0, 0
+    if do_dec:
+        xd = W.decode_inputs(DECODE, dev, seed=seed)
+        out_d = torch.empty_like(xd["q"])
+        neff_d = torch.empty((DECODE.num_seqs, DECODE.Hq), device=dev)
+        ws = torch.empty(pa.decode_workspace_size(DECODE.num_seqs, xd["max_pages"], DECODE.Hq,
+                                                  DECODE.Hkv), device=dev, dtype=torch.uint8)
+        tokens = int(xd["seqlens"].to(torch.int64).sum().item())
+        kv_bytes = float(tokens) * KV_BYTES_PER_TOKEN
+    p = dict(s=PREFILL.s, alpha=PREFILL.alpha, L=PREFILL.L, beta=PREFILL.beta)
+
+    def prefill():
+        if not do_pre:
+            return
+        pa.fwd(xp["q"], xp["k"], xp["v"], xp["u"], out_p, neff_p, stream=stream, **p)
+
+    def decode():
+        if not do_dec:
+            return
+        pa.decode_paged(xd["q"], xd["kv_pages"], xd["page_table"], xd["seqlens"], xd["u"], out_d,
+                        neff_d, ws, stream=stream, **p)
+
+    K, Wm = args.steps, args.warmup
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    outer = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    for _ in range(Wm):
+        prefill()
+        decode()
+    torch.cuda.synchronize(dev)
+    st = pa.get_status()
+    if st != 0:
+        raise RuntimeError(f"device status {st} after warm-up")
+
+    with ClockSampler([dev.index]) as clk:
+        time.sleep(0.3)  # let the sampler start before the timed region
+        barrier(world, dev)
+        torch.cuda.synchronize(dev)
+        n0 = pa.launch_count()
+        outer[0].record(stream)
+        for i in range(K):
+            ev[i][0].record(stream)
+            prefill()
+            ev[i][1].record(stream)
+            decode()
+            ev[i][2].record(stream)
+        outer[1].record(stream)
+        torch.cuda.synchronize(dev)
+        launches = pa.launch_count() - n0
+        barrier(world, dev)
+    st = pa.get_status()
+    if st != 0:
+        raise RuntimeError(f"device status {st} after timing")
+
+    t_pre = sum(ev[i][0].elapsed_time(ev[i][1]) for i in range(K)) / 1e3
+    t_dec = sum(ev[i][1].elapsed_time(ev[i][2]) for i in range(K)) / 1e3
+    t_all = outer[0].elapsed_time(outer[1]) / 1e3
+    t_pre_max = max_over_ranks(t_pre, world, dev)
+    t_dec_max = max_over_ranks(t_dec, world, dev)
+    t_all_max = max_over_ranks(t_all, world, dev)
+
+    # ---- end to end through the host-buffer C ABI (pinned host memory) ----
+    e2e = None
+    if args.e2e_steps > 0 and do_pre and do_dec:
+        pin = lambda t: t.detach().cpu().pin_memory()  # noqa: E731
+        hq, hk, hv, hu = pin(xp["q"]), pin(xp["k"]), pin(xp["v"]), pin(xp["u"])
+        ho = torch.empty_like(hq).pin_memory()
+        hn = torch.empty((PREFILL.B, PREFILL.Hq, PREFILL.T)).pin_memory()
+        stg = torch.empty(pa.fwd_staging_size(PREFILL.B, PREFILL.T, PREFILL.Hq, PREFILL.Hkv),
+                          device=dev, dtype=torch.uint8)
+        dq, dpt, dsl, du = pin(xd["q"]), pin(xd["page_table"]), pin(xd["seqlens"]), pin(xd["u"])
+        do = torch.empty_like(dq).pin_memory()
+        dn = torch.empty((DECODE.num_seqs, DECODE.Hq)).pin_memory()
+        dstg = torch.empty(pa.decode_staging_size(DECODE.num_seqs, xd["max_pages"], DECODE.Hq,
+                                                  DECODE.Hkv), device=dev, dtype=torch.uint8)
+        h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hu, dq, dpt, dsl, du))
+        d2h = sum(t.numel() * t.element_size() for t in (ho, hn, do, dn))
+        e_pre = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+        tp = td = 0.0
+        for i in range(args.e2e_steps + 1):
+            barrier(world, dev)
+            e_pre[0].record(stream)
+            pa.fwd_host(hq, hk, hv, hu, ho, hn, stg, stream=stream, **p)
+            e_pre[1].record(stream)
+            torch.cuda.synchronize(dev)
+            a = e_pre[0].elapsed_time(e_pre[1]) / 1e3
+            e_pre[0].record(stream)
+            pa.decode_paged_host(dq, xd["kv_pages"], dpt, dsl, du, do, dn, dstg, stream=stream, **p)
+            e_pre[1].record(stream)
+            torch.cuda.synchronize(dev)
+            b = e_pre[0].elapsed_time(e_pre[1]) / 1e3
+            if i > 0:  # the first is a warm-up
+                tp += a
+                td += b
+        tp = max_over_ranks(tp, world, dev)
+        td = max_over_ranks(td, world, dev)
+        ns = args.e2e_steps
+        e2e = {"value": aggregate_throughput(PREFILL.flops * ns, world, tp) / 1e12,
+               "unit": "TFLOP/s", "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+               "decode_value": aggregate_throughput(kv_bytes * ns, world, td) / 1e9,
+               "decode_unit": "GB/s", "steps": ns,
+               "note": "host-buffer C ABI calls (pinned), copies inside the timed region"}
+
+    result = None
+    if rank == 0:
+        peaks, peak_src = measured_peaks()
+        pre_launch_s = t_pre / K
+        dec_launch_s = t_dec / K
+        tf = PREFILL.flops / pre_launch_s / 1e12 if do_pre else 0.0
+        gbs = kv_bytes / dec_launch_s / 1e9 if do_dec else 0.0
+        sha_p = source_sha("fwd_tc.cu", "polar_common.cuh")
+        sha_d = source_sha("decode.cu", "polar_common.cuh")
+        value = aggregate_throughput(PREFILL.flops * K, world, t_pre_max) / 1e12 if do_pre else 0.0
+        dec_value = aggregate_throughput(kv_bytes * K, world, t_dec_max) / 1e9 if do_dec else 0.0
+        result = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K,
+            "warmup": Wm, "ms_per_step": t_all_max / K * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {
+                "workload": f"{PREFILL.describe()} + {DECODE.describe()}",
+                "prefill": {"B": PREFILL.B, "T": PREFILL.T, "Hq": PREFILL.Hq, "Hkv": PREFILL.Hkv,
+                            "head_dim": PREFILL.D, "alpha": PREFILL.alpha, "L_train": PREFILL.L,
+                            "logit_scale": PREFILL.s, "flops_per_launch": PREFILL.flops},
+                "decode": {"num_seqs": DECODE.num_seqs, "ctx": [DECODE.min_len, DECODE.max_len],
+                           "Hq": DECODE.Hq, "Hkv": DECODE.Hkv, "page": W.PAGE,
+                           "kv_bytes_per_launch": kv_bytes, "tokens": tokens},
+                "l2": "inputs larger than L2: each step streams the 6.5 GB KV pool, which "
+                      "evicts the prefill operands between prefill launches",
+                "parallelism": f"replicas x{world} (one batch per rank)"},
+            "prefill": {"value": value, "unit": "TFLOP/s", "ms_per_launch": pre_launch_s * 1e3,
+                        "pct_bf16_peak": 100 * tf / peaks["bf16_tflops"],
+                        "tokens_per_s": aggregate_throughput(PREFILL.B * PREFILL.T * K, world,
+                                                             t_pre_max) if do_pre else 0.0},
+            "decode": {"value": dec_value, "unit": "GB/s", "ms_per_launch": dec_launch_s * 1e3,
+                       "pct_hbm_peak": 100 * gbs / peaks["hbm_gbs"],
+                       "tokens_per_s": aggregate_throughput(DECODE.num_seqs * K, world,
+                                                            t_dec_max) if do_dec else 0.0},
+            "roofline": {"bound": "tensor", "kernel": "fwd_tc_kernel", "achieved": tf,
+                         "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                         "frac": tf / peaks["bf16_tflops"],
+                         "frac_of_sustained": tf / peaks.get("bf16_tflops_sustained",
+                                                              peaks["bf16_tflops"]),
+                         "traffic": profiled_traffic("fwd_tc_kernel", sha_p),
+                         "peak_source": f"{peak_src} (burst cuBLAS bf16)"},
+            "roofline_decode": {"bound": "hbm", "kernel": "decode_split_kernel+decode_merge_kernel",
+                                "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                                "frac": gbs / peaks["hbm_gbs"],
+                                "traffic": profiled_traffic("decode", sha_d),
+                                "peak_source": f"{peak_src} (copy bandwidth)"},
+            "gpu_launches": int(launches),
+            "clocks": clk.summary(),
+            "e2e": e2e,
+        }
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier(device_ids=[dev.index])
+        dist.destroy_process_group()
+    return result
+
+
+# ---------------------------------------------------------- reference arm --
+
+def run_reference(args):
+    """The fp64 CPU oracle as it stands, on the host cores, on the same metric
+    and unit: each step is a bounded seeded sample of prefill rows."""
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return None
+    x_host = cpu_prefill_inputs(0)
+    rng = np.random.default_rng(11)
+    rows_per_step = 8
+    total = PREFILL.B * PREFILL.Hq * PREFILL.T
+    for _ in range(args.warmup):
+        _oracle_prefill_rows(x_host, rng.integers(0, total, size=rows_per_step), PREFILL)
+    flops = 0.0
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        rows = rng.integers(0, total, size=rows_per_step)
+        _oracle_prefill_rows(x_host, rows, PREFILL)
+        flops += prefill_rows_flops(rows, PREFILL)
+    dt = time.perf_counter() - t0
+    v = flops / dt / 1e12
+    return {"impl": "reference", "metric": METRIC, "value": v, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic",
+            "config": {"workload": PREFILL.describe(),
+                       "sample": f"{rows_per_step} seeded random rows per step"},
+            "cpu_baseline": {"value": v, "unit": "TFLOP/s", "cores": oracle_threads(),
+                             "kind": "oracle",
+                             "sample": f"{rows_per_step} random rows of the T=16384 prefill "
+                                       "per step"},
+            "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    if args.impl == "reference":
+        res = run_reference(args)
+    else:
+        res = run_ours(args)
+        rank, world, _ = dist_env()
+        if res is not None and args.only != "both":
+            res["partial_step"] = f"only the {args.only} half was timed (profiling run)"
+        if res is not None and world == 1 and not args.no_cpu_baseline and args.only == "both":
+            res["cpu_baseline"] = cpu_baseline(args.cpu_seconds)
+        elif res is not None:
+            res["cpu_baseline"] = None
+    if res is not None:
+        print(json.dumps(res), flush=True)
+
+
+if __name__ == "__main__":
+    main()
