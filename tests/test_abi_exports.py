@@ -1,0 +1,46 @@
+"""The C-ABI library loads on a machine without a GPU and exports every
+function that include/*.h declares (no compute call is made)."""
+import ctypes
+import glob
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    names = set()
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        src = open(h).read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        for m in re.finditer(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\s*\*?\s*(polar_attn_[A-Za-z0-9_]+)\s*\(",
+                             src, flags=re.M):
+            names.add(m.group(1))
+    return sorted(names)
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for must in ("polar_attn_fwd", "polar_attn_decode_paged", "polar_attn_get_status"):
+        assert must in names
+
+
+def test_library_exports_every_declared_symbol():
+    from polar_attention_b200 import native
+    if not os.path.exists(native.LIB_PATH):
+        from polar_attention_b200 import build
+        build.build()
+    lib = ctypes.CDLL(native.LIB_PATH)
+    missing = [n for n in declared_functions() if not hasattr(lib, n)]
+    assert not missing, f"not exported: {missing}"
+    assert set(native.EXPORTS) == set(declared_functions())
+
+
+def test_binding_fails_loudly_without_the_library(monkeypatch, tmp_path):
+    from polar_attention_b200 import native
+    monkeypatch.setattr(native, "_lib", None)
+    monkeypatch.setattr(native, "LIB_PATH", str(tmp_path / "missing.so"))
+    with pytest.raises(RuntimeError, match="no fallback"):
+        native.lib()
