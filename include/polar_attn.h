@@ -173,6 +173,39 @@ polar_status_t polar_attn_decode_paged_host(const void *q_h, const void *kv_page
                                             size_t staging_bytes, void *stream);
 
 /*
+ * Paged GQA decode for callers that cannot allocate device memory -- for
+ * example a serving process that handed all free device memory to its KV-cache
+ * pool at start-up, or a plug-in whose host framework gives it no device
+ * allocator -- and so have no workspace to pass.  The paper has no counterpart;
+ * this is a property of the library, not of the method.
+ *
+ * Same arguments, layouts, results and error reporting as
+ * polar_attn_decode_paged, without the workspace: the per-split scratch lives
+ * in a fixed array of POLAR_NOALLOC_SCRATCH_BYTES bytes of device memory that
+ * the library holds on every device that loads it, until the process exits.
+ * The call itself allocates nothing and calls no allocating routine.
+ *  - A shape whose scratch (polar_attn_decode_workspace_size) exceeds
+ *    POLAR_NOALLOC_SCRATCH_BYTES is rejected with POLAR_ERR_WORKSPACE and
+ *    nothing is launched.
+ *  - The first call on a device looks up the array's device address with that
+ *    device current (a synchronous runtime query); make that first call before
+ *    any stream capture.
+ *  - Every call on a device shares the one array and leaves its contents
+ *    behind.  Nothing in it has to start at zero: each split writes its whole
+ *    partial state before the merge reads it.  Calls whose work overlaps on the
+ *    GPU (concurrent streams, or other host threads) race on the array; order
+ *    them on one stream or serialise them.
+ */
+#define POLAR_NOALLOC_SCRATCH_BYTES (16u << 20)
+
+polar_status_t polar_attn_decode_paged_noalloc(const void *q, const void *kv_pages,
+                                               int num_pages, const int32_t *page_table,
+                                               int max_pages, const int32_t *seqlens,
+                                               int num_seqs, const float *u,
+                                               const polar_params_t *params, void *out,
+                                               float *neff_out, void *stream);
+
+/*
  * Synchronises `stream`, returns the first device-side error recorded on the
  * current device since the last call (POLAR_OK if none) and clears it.
  */

@@ -25,7 +25,8 @@ STATUS = {0: "POLAR_OK", 1: "POLAR_ERR_INVALID_ARG", 2: "POLAR_ERR_UNSUPPORTED",
 EXPORTS = ["polar_attn_default_params", "polar_attn_fwd", "polar_attn_fwd_staging_size",
            "polar_attn_fwd_host", "polar_attn_decode_workspace_size", "polar_attn_decode_paged",
            "polar_attn_decode_staging_size", "polar_attn_decode_paged_host",
-           "polar_attn_get_status", "polar_attn_status_string", "polar_attn_launch_count"]
+           "polar_attn_get_status", "polar_attn_status_string", "polar_attn_launch_count",
+           "polar_attn_decode_paged_noalloc"]
 
 
 class PolarError(RuntimeError):
@@ -72,12 +73,14 @@ def lib() -> ctypes.CDLL:
             L.polar_attn_decode_staging_size.argtypes = [I, I, PP]
             L.polar_attn_decode_staging_size.restype = Z
             L.polar_attn_decode_paged_host.argtypes = [P, P, I, P, I, P, I, P, PP, P, P, P, Z, P]
+            L.polar_attn_decode_paged_noalloc.argtypes = [P, P, I, P, I, P, I, P, PP, P, P, P]
             L.polar_attn_get_status.argtypes = [P]
             L.polar_attn_status_string.argtypes = [I]
             L.polar_attn_status_string.restype = ctypes.c_char_p
             L.polar_attn_launch_count.restype = ctypes.c_uint64
             for name in ("polar_attn_fwd", "polar_attn_fwd_host", "polar_attn_decode_paged",
-                         "polar_attn_decode_paged_host", "polar_attn_get_status"):
+                         "polar_attn_decode_paged_host", "polar_attn_get_status",
+                         "polar_attn_decode_paged_noalloc"):
                 getattr(L, name).restype = I
             _lib = L
     return _lib
@@ -172,6 +175,26 @@ def decode_paged(q, kv_pages, page_table, seqlens, u, out=None, neff=None, works
         _ptr(q), _ptr(kv_pages), P_, _ptr(page_table), max_pages, _ptr(seqlens), N, _ptr(u),
         ctypes.byref(p), _ptr(out), _ptr(neff), _ptr(workspace), workspace.numel(),
         _stream(stream)), "polar_attn_decode_paged")
+    return out, neff
+
+
+# Bytes of the fixed device scratch behind decode_paged_noalloc (POLAR_NOALLOC_SCRATCH_BYTES).
+NOALLOC_SCRATCH_BYTES = 16 << 20
+
+
+def decode_paged_noalloc(q, kv_pages, page_table, seqlens, u, out, neff=None, *, s=8.0,
+                         alpha=0.3, L=2048, beta=1.0, stream=None):
+    """polar_attn_decode_paged_noalloc: the paged decode with no workspace, for
+    callers that cannot allocate device memory.  out (and neff, if given) must
+    be preallocated by the caller; this wrapper allocates nothing."""
+    N, Hq, D = q.shape
+    P_, _, Hkv, _, _ = kv_pages.shape
+    p = make_params(0, 0, Hq, Hkv, _dt(q), s, alpha, L, beta)
+    p.head_dim = D
+    _check(lib().polar_attn_decode_paged_noalloc(
+        _ptr(q), _ptr(kv_pages), P_, _ptr(page_table), page_table.shape[1], _ptr(seqlens), N,
+        _ptr(u), ctypes.byref(p), _ptr(out), _ptr(neff), _stream(stream)),
+        "polar_attn_decode_paged_noalloc")
     return out, neff
 
 
