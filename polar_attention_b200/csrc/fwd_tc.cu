@@ -26,6 +26,7 @@
 // lets softmax i rescale O_i in place before it releases P_i(j+1).
 #include <atomic>
 
+#include "polar_attn_selftest.h"
 #include "polar_common.cuh"
 #include "polar_internal.h"
 
@@ -54,6 +55,19 @@ __device__ __forceinline__ void tmem_alloc_512(uint32_t *dst_smem) {
 
 __device__ __forceinline__ void tmem_dealloc_512(uint32_t taddr) {
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" ::"r"(taddr) : "memory");
+}
+
+// Register rebalancing between warpgroups (must be executed by all four warps
+// of a warpgroup).  Budget: launched at 168 per thread x 384 threads = 64512;
+// the producer/MMA warpgroup drops to 64 and the two softmax warpgroups rise to
+// 216: 64*128 + 216*256 = 63488, within the launch total.
+template <int N>
+__device__ __forceinline__ void reg_dealloc() {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void reg_alloc() {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
 }
 
 __device__ __forceinline__ void tc_fence_before() {
@@ -164,6 +178,140 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     return r;
 }
 
+// ----------------------------------------------- packed fp32 (f32x2) math --
+
+__device__ __forceinline__ float2 f2_add(float2 a, float2 b) {
+    float2 d;
+    asm("add.rn.f32x2 %0, %1, %2;"
+        : "=l"(reinterpret_cast<uint64_t &>(d))
+        : "l"(reinterpret_cast<const uint64_t &>(a)), "l"(reinterpret_cast<const uint64_t &>(b)));
+    return d;
+}
+
+__device__ __forceinline__ float2 f2_fma(float2 a, float2 b, float2 c) {
+    float2 d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;"
+        : "=l"(reinterpret_cast<uint64_t &>(d))
+        : "l"(reinterpret_cast<const uint64_t &>(a)), "l"(reinterpret_cast<const uint64_t &>(b)),
+          "l"(reinterpret_cast<const uint64_t &>(c)));
+    return d;
+}
+
+__device__ __forceinline__ float max3(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
+// 2^x on the FMA pipe for two values at once (Cody-Waite range reduction and a
+// degree-4 minimax polynomial; the FlashAttention-4 write-up publishes the
+// idea of sharing the exponentials between this and the MUFU unit).  x = n + f
+// with n = round(x), f in [-1/2, 1/2]; p(f) ~ 2^f with relative error below
+// 4e-6 in fp32 (coefficients from exp2_poly_coeffs.py, which derives them by
+// a Remez exchange); 2^n enters as an integer add to the exponent field.
+// Valid for -126 < x < 128; callers guarantee the range.
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+    constexpr float kShift = 12582912.0f;  // 1.5 * 2^23: x + kShift rounds x to an integer
+    const float2 j = f2_add(x, make_float2(kShift, kShift));
+    const float2 r = f2_add(j, make_float2(-kShift, -kShift));
+    const float2 f = f2_fma(r, make_float2(-1.f, -1.f), x);
+    float2 p = make_float2(9.570102207e-03f, 9.570102207e-03f);
+    p = f2_fma(p, f, make_float2(5.591785908e-02f, 5.591785908e-02f));
+    p = f2_fma(p, f, make_float2(2.402474433e-01f, 2.402474433e-01f));
+    p = f2_fma(p, f, make_float2(6.931217909e-01f, 6.931217909e-01f));
+    p = f2_fma(p, f, make_float2(1.0f, 1.0f));
+    const uint32_t px = __float_as_uint(p.x) + (__float_as_uint(j.x) << 23);
+    const uint32_t py = __float_as_uint(p.y) + (__float_as_uint(j.y) << 23);
+    return make_float2(__uint_as_float(px), __uint_as_float(py));
+}
+
+#ifndef POLAR_TC_POLY_MASK
+// Which of every 16 exponential pairs of a full tile go to the polynomial
+// (bit e set: pair e); the rest use MUFU ex2.  0x2222 = 4 of 16 (one quarter).
+#define POLAR_TC_POLY_MASK 0x2222
+#endif
+
+// Row statistics of one 128-key tile of S (raw dots, one row per thread):
+// max, sum and sum of squares over the visible keys.  Independent partial
+// accumulators keep the dependency chains short.  kDiag: the tile holds the
+// row's own position t; keys after it are invisible and are set to -inf in sr.
+template <bool kDiag>
+__device__ __forceinline__ void row_stats(uint32_t (&sr)[4][32], int t, float &tmax, float &ts1,
+                                          float &ts2) {
+    if (!kDiag) {
+        float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+        float2 a1[4], a2[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) a1[q] = a2[q] = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int e = 0; e < 64; ++e) {
+            const float x0 = __uint_as_float(sr[e >> 4][2 * (e & 15)]);
+            const float x1 = __uint_as_float(sr[e >> 4][2 * (e & 15) + 1]);
+            mx[e & 3] = max3(mx[e & 3], x0, x1);
+            const float2 v = make_float2(x0, x1);
+            a1[e & 3] = f2_add(a1[e & 3], v);
+            a2[e & 3] = f2_fma(v, v, a2[e & 3]);
+        }
+        tmax = fmaxf(max3(mx[0], mx[1], mx[2]), mx[3]);
+        const float2 b1 = f2_add(f2_add(a1[0], a1[1]), f2_add(a1[2], a1[3]));
+        const float2 b2 = f2_add(f2_add(a2[0], a2[1]), f2_add(a2[2], a2[3]));
+        ts1 = b1.x + b1.y;
+        ts2 = b2.x + b2.y;
+    } else {
+        float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+        float a1[4] = {0.f, 0.f, 0.f, 0.f}, a2[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int e = 0; e < 128; ++e) {
+            const bool vis = e <= t;
+            const float x = __uint_as_float(sr[e >> 5][e & 31]);
+            const float xv = vis ? x : 0.f;
+            sr[e >> 5][e & 31] = __float_as_uint(vis ? x : -INFINITY);
+            mx[e & 3] = fmaxf(mx[e & 3], vis ? x : -INFINITY);
+            a1[e & 3] += xv;
+            a2[e & 3] = fmaf(xv, xv, a2[e & 3]);
+        }
+        tmax = fmaxf(max3(mx[0], mx[1], mx[2]), mx[3]);
+        ts1 = (a1[0] + a1[1]) + (a1[2] + a1[3]);
+        ts2 = (a2[0] + a2[1]) + (a2[2] + a2[3]);
+    }
+}
+
+// Weights p = 2^(c*log2e*S - m_ref) of one tile: their sum and sum of squares
+// (for l and l2), and the bf16 P tile written to tensor memory for the PV MMA.
+// kPoly: the pairs selected by POLAR_TC_POLY_MASK use the FMA-pipe polynomial
+// (full tiles only; the diagonal tile's -inf entries use ex2, which gives 0).
+template <bool kPoly>
+__device__ __forceinline__ void row_weights(const uint32_t (&sr)[4][32], float2 sc2, float neg_m,
+                                            uint32_t tP, float &tl, float &tl2) {
+    const float2 nm = make_float2(neg_m, neg_m);
+    float2 la[2], l2a[2];
+    la[0] = la[1] = l2a[0] = l2a[1] = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int cc = 0; cc < 4; ++cc) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+            const float2 sv = make_float2(__uint_as_float(sr[cc][2 * e]),
+                                          __uint_as_float(sr[cc][2 * e + 1]));
+            const float2 x = f2_fma(sv, sc2, nm);
+            float2 p;
+            if (kPoly && ((POLAR_TC_POLY_MASK >> e) & 1)) {
+                p = exp2_poly2(make_float2(fmaxf(x.x, -126.f), fmaxf(x.y, -126.f)));
+            } else {
+                p.x = ex2(x.x);
+                p.y = ex2(x.y);
+            }
+            la[e & 1] = f2_add(la[e & 1], p);
+            l2a[e & 1] = f2_fma(p, p, l2a[e & 1]);
+            pk[e] = pack_bf16(p.x, p.y);
+        }
+        tmem_st16(tP + 16 * cc, pk);
+    }
+    const float2 sl = f2_add(la[0], la[1]), sl2 = f2_add(l2a[0], l2a[1]);
+    tl = sl.x + sl.y;
+    tl2 = sl2.x + sl2.y;
+}
+
 struct TcArgs {
     const float *u;
     __nv_bfloat16 *out;
@@ -219,7 +367,9 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CU
     tc_fence_after();
     const uint32_t tmem = tmem_base_sh;
 
-    if (warp == 0) {
+    if (warp < 4) {
+      reg_dealloc<64>();
+      if (warp == 0) {
         // ------------------------------------------------------ TMA producer
         if (lane == 0) {
             tma_prefetch_desc(&tq);
@@ -300,7 +450,9 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CU
             tc_commit(&mma_done);
             mbar_wait(&mma_done, 0, a.status);
         }
-    } else if (warp >= 4) {
+      }
+    } else {
+        reg_alloc<216>();
         // ------------------------------------------------ softmax warpgroups
         const int slot = (warp - 4) >> 2;          // head slot 0 or 1
         const int t = threadIdx.x - 128 * (1 + slot);  // row within the tile = TMEM lane
@@ -316,6 +468,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CU
         const float cl2 = c * kLog2e;
 
         float m_ref = -INFINITY, m_raw = -INFINITY, l = 0.f, l2 = 0.f, s1 = 0.f, s2 = 0.f;
+        const float2 sc2 = make_float2(cl2, cl2);
         bool ok = true;
         for (int j = 0; j < nkv; ++j) {
             ok = mbar_wait(&s_full[slot], j & 1, a.status);
@@ -326,21 +479,11 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CU
             for (int cc = 0; cc < 4; ++cc) tmem_ld32(tS + 32 * cc, sr[cc]);
             tmem_wait_ld();
             const bool diag = (j == nkv - 1);
-            float tmax = -INFINITY, ts1 = 0.f, ts2 = 0.f;
-#pragma unroll
-            for (int cc = 0; cc < 4; ++cc) {
-#pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    const int col = 32 * cc + e;
-                    float x = __uint_as_float(sr[cc][e]);
-                    if (diag && col > t) x = -INFINITY;  // key after the row: invisible
-                    sr[cc][e] = __float_as_uint(x);
-                    tmax = fmaxf(tmax, x);
-                    const float xv = (diag && col > t) ? 0.f : x;
-                    ts1 += xv;
-                    ts2 = fmaf(xv, xv, ts2);
-                }
-            }
+            float tmax, ts1, ts2;
+            if (diag)
+                row_stats<true>(sr, t, tmax, ts1, ts2);
+            else
+                row_stats<false>(sr, t, tmax, ts1, ts2);
             s1 += ts1;
             s2 += ts2;
             m_raw = fmaxf(m_raw, tmax);
@@ -353,20 +496,11 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CU
                 l2 *= r * r;
                 m_ref = zmax;
             }
-            float tl = 0.f, tl2 = 0.f;
-#pragma unroll
-            for (int cc = 0; cc < 4; ++cc) {
-                uint32_t pk[16];
-#pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    const float p0 = ex2(fmaf(__uint_as_float(sr[cc][2 * e]), cl2, -m_ref));
-                    const float p1 = ex2(fmaf(__uint_as_float(sr[cc][2 * e + 1]), cl2, -m_ref));
-                    tl += p0 + p1;
-                    tl2 = fmaf(p0, p0, fmaf(p1, p1, tl2));
-                    pk[e] = pack_bf16(p0, p1);
-                }
-                tmem_st16(tP + 16 * cc, pk);
-            }
+            float tl, tl2;
+            if (diag)
+                row_weights<false>(sr, sc2, -m_ref, tP, tl, tl2);
+            else
+                row_weights<true>(sr, sc2, -m_ref, tP, tl, tl2);
             l += tl;
             l2 += tl2;
             // Rescale the output accumulator when this row's reference max moved.
@@ -438,6 +572,14 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CU
     }
 }
 
+__global__ void selftest_exp2_kernel(const float2 *x, float2 *poly, float2 *mufu, int npairs) {
+    const int i = blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= npairs) return;
+    const float2 v = x[i];
+    poly[i] = exp2_poly2(v);
+    mufu[i] = make_float2(ex2(v.x), ex2(v.y));
+}
+
 }  // namespace
 
 cudaError_t launch_fwd_tc(const FwdLaunch &a) {
@@ -494,3 +636,18 @@ cudaError_t launch_fwd_tc(const FwdLaunch &a) {
 }
 
 }  // namespace polar
+
+extern "C" polar_status_t polar_attn_selftest_exp2(const float *x, float *poly, float *mufu, int n,
+                                                   void *stream) {
+    if (!x || !poly || !mufu || n < 0 || (n & 1)) return POLAR_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(poly) |
+         reinterpret_cast<uintptr_t>(mufu)) & 7u)
+        return POLAR_ERR_INVALID_ARG;
+    if (n == 0) return POLAR_OK;
+    const int np = n / 2;
+    polar::selftest_exp2_kernel<<<(np + 255) / 256, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+        reinterpret_cast<const float2 *>(x), reinterpret_cast<float2 *>(poly),
+        reinterpret_cast<float2 *>(mufu), np);
+    polar::count_launches(1);
+    return cudaGetLastError() == cudaSuccess ? POLAR_OK : POLAR_ERR_CUDA;
+}

@@ -26,7 +26,7 @@ EXPORTS = ["polar_attn_default_params", "polar_attn_fwd", "polar_attn_fwd_stagin
            "polar_attn_fwd_host", "polar_attn_decode_workspace_size", "polar_attn_decode_paged",
            "polar_attn_decode_staging_size", "polar_attn_decode_paged_host",
            "polar_attn_get_status", "polar_attn_status_string", "polar_attn_launch_count",
-           "polar_attn_decode_paged_noalloc"]
+           "polar_attn_decode_paged_noalloc", "polar_attn_selftest_exp2"]
 
 
 class PolarError(RuntimeError):
@@ -74,13 +74,14 @@ def lib() -> ctypes.CDLL:
             L.polar_attn_decode_staging_size.restype = Z
             L.polar_attn_decode_paged_host.argtypes = [P, P, I, P, I, P, I, P, PP, P, P, P, Z, P]
             L.polar_attn_decode_paged_noalloc.argtypes = [P, P, I, P, I, P, I, P, PP, P, P, P]
+            L.polar_attn_selftest_exp2.argtypes = [P, P, P, I, P]
             L.polar_attn_get_status.argtypes = [P]
             L.polar_attn_status_string.argtypes = [I]
             L.polar_attn_status_string.restype = ctypes.c_char_p
             L.polar_attn_launch_count.restype = ctypes.c_uint64
             for name in ("polar_attn_fwd", "polar_attn_fwd_host", "polar_attn_decode_paged",
                          "polar_attn_decode_paged_host", "polar_attn_get_status",
-                         "polar_attn_decode_paged_noalloc"):
+                         "polar_attn_decode_paged_noalloc", "polar_attn_selftest_exp2"):
                 getattr(L, name).restype = I
             _lib = L
     return _lib
@@ -232,6 +233,15 @@ def decode_paged_host(q_h, kv_pages, page_table_h, seqlens_h, u_h, out_h, neff_h
         _ptr(q_h), _ptr(kv_pages), P_, _ptr(page_table_h), page_table_h.shape[1], _ptr(seqlens_h),
         N, _ptr(u_h), ctypes.byref(p), _ptr(out_h), _ptr(neff_h), _ptr(staging), staging.numel(),
         _stream(stream)), "polar_attn_decode_paged_host")
+
+
+def selftest_exp2(x, stream=None):
+    """The prefill kernel's FMA-pipe 2^x and MUFU ex2.approx on a CUDA fp32
+    tensor x (even length).  Returns (poly, mufu)."""
+    poly, mufu = torch.empty_like(x), torch.empty_like(x)
+    _check(lib().polar_attn_selftest_exp2(_ptr(x), _ptr(poly), _ptr(mufu), x.numel(),
+                                          _stream(stream)), "polar_attn_selftest_exp2")
+    return poly, mufu
 
 
 def get_status(stream=None) -> int:

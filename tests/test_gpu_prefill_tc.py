@@ -62,3 +62,30 @@ def test_train_length_sampled(cuda_ok):
     ref = PT.oracle_prefill(w, x, rows)
     o, n, grp = PT.gpu_rows_prefill(out, neff, rows, w.B, w.T, w.Hq)
     PT.compare(o, n, ref, grp, PT.OUT_TOL_BF16, what="train_len")
+
+
+def test_extrapolation_T16384_sampled(cuda_ok):
+    """Full-size T=16384 workload (temperature active up to tau=1.62), in the
+    launch configuration the bench times; sampled rows against the oracle."""
+    w = W.EXTRAP
+    x, out, neff = _run(w)
+    rows = PT.sample_rows(w.B, w.Hq, w.T, 600, seed=2)
+    ref = PT.oracle_prefill(w, x, rows)
+    o, n, grp = PT.gpu_rows_prefill(out, neff, rows, w.B, w.T, w.Hq)
+    PT.compare(o, n, ref, grp, PT.OUT_TOL_BF16, what="extrapolation_T16384")
+
+
+def test_long_T65536_sampled(cuda_ok):
+    """T=65536 with a 16-key needle per kv head matched by the last 64 queries:
+    the needle rows and random rows against the oracle, and the needle rows
+    concentrate (n_eff well below the unplanted rows')."""
+    w = W.LONG
+    x, out, neff = _run(w)
+    T, Hq = w.T, w.Hq
+    needle = [h * T + i for h in (0, 5, 10, 15) for i in range(T - 64, T, 8)]
+    rows = PT.sample_rows(w.B, Hq, T, 200, seed=3, include=needle)
+    ref = PT.oracle_prefill(w, x, rows)
+    o, n, grp = PT.gpu_rows_prefill(out, neff, rows, w.B, T, Hq)
+    PT.compare(o, n, ref, grp, PT.OUT_TOL_BF16, what="long_T65536")
+    nn = neff[0, :, T - 64:].float()
+    assert nn.median() < 0.01 * neff[0, :, T // 2:T - 64].float().median()
