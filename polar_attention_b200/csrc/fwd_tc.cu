@@ -19,11 +19,12 @@
 //   warps 8-11  softmax warpgroup for head slot 1
 // Tensor memory (512 columns): S0 S1 (128 fp32 columns each), P0 P1 (128 bf16
 // packed in 64 columns each), O0 O1 (64 fp32 columns each).
-// Issue order of the MMA thread, per key tile j:
-//   PV0(j), S0(j+1), PV1(j), S1(j+1)
-// so the tensor core computes one head's next scores while the other head's
-// softmax runs.  A tcgen05.commit after S_i(j+1) also covers PV_i(j), which
-// lets softmax i rescale O_i in place before it releases P_i(j+1).
+// Per key tile j the MMA thread issues S0(j+1) and S1(j+1) as soon as each
+// softmax warpgroup has copied S_i(j) into registers (barrier s_free), then
+// PV0(j) and PV1(j) once P_i(j) is in tensor memory (p_full).  The next scores
+// are thus computed while the softmax of tile j runs.  A commit after PV_i(j)
+// (pv_done) tells softmax i that P_i may be overwritten and that O_i is
+// current, so it can rescale O_i in place before it releases P_i(j+1).
 #include <atomic>
 
 #include "polar_attn_selftest.h"
@@ -37,7 +38,6 @@ constexpr int kBM = 128;               // query rows per head slot
 constexpr int kBN = 128;               // keys per tile
 constexpr int kStagesKV = 4;           // K/V ring depth
 constexpr int kTileBytes = 128 * 128;  // 128 rows x 64 bf16
-constexpr int kThreads = 384;
 constexpr int kSmemBytes = (2 + 2 * kStagesKV) * kTileBytes + 1024;
 
 // Tensor-memory column map.
@@ -83,25 +83,35 @@ __device__ __forceinline__ void tc_commit(uint64_t *bar) {
                  : "memory");
 }
 
-// D[tmem] (+)= A[smem] * B[smem]^T, kind::f16 (bf16 in, fp32 accumulate).
-__device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
-                                       uint32_t idesc, uint32_t accumulate) {
+// tcgen05.mma kind::f16 (bf16 in, fp32 accumulate in TMEM), each shared-memory
+// descriptor given as its two 32-bit halves (low: start address >> 4 and
+// leading byte offset; high: stride byte offset, version, layout), packed
+// inside the asm.  The issuing thread then
+// steps through a tile by adding a constant to the low half: about four
+// instructions per MMA, which matters because this thread shares its
+// scheduler with busy softmax warps.
+template <uint32_t kAcc>
+__device__ __forceinline__ void mma_ss2(uint32_t d_tmem, uint32_t a_lo, uint32_t a_hi, uint32_t b_lo,
+                                        uint32_t b_hi, uint32_t idesc) {
     asm volatile(
-        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        "{\n\t.reg .b64 da, db;\n\t.reg .pred p;\n\t"
+        "mov.b64 da, {%1, %2};\n\tmov.b64 db, {%3, %4};\n\tsetp.ne.b32 p, %6, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %5, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_lo), "r"(a_hi), "r"(b_lo), "r"(b_hi), "r"(idesc), "n"(kAcc)
         : "memory");
 }
 
-// D[tmem] (+)= A[tmem] * B[smem].
-__device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
-                                       uint32_t idesc, uint32_t accumulate) {
+__device__ __forceinline__ void mma_ts2(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_lo,
+                                        uint32_t b_hi, uint32_t idesc, uint32_t accumulate) {
     asm volatile(
-        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        "{\n\t.reg .b64 db;\n\t.reg .pred p;\n\t"
+        "mov.b64 db, {%2, %3};\n\tsetp.ne.b32 p, %5, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], db, %4, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "r"(b_lo), "r"(b_hi), "r"(idesc), "r"(accumulate)
         : "memory");
 }
+
+
 
 #define POLAR_R32(r)                                                                      \
     "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),   \
@@ -151,14 +161,6 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
         : "memory");
 }
 
-// Shared-memory matrix descriptor for a 128B-swizzled tile (rows of 128
-// bytes, 8-row groups 1024 bytes apart): start address, leading and stride
-// byte offsets, descriptor version 1, layout SWIZZLE_128B.
-__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
-    return static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4) |
-           (static_cast<uint64_t>(lbo >> 4) << 16) | (static_cast<uint64_t>(sbo >> 4) << 32) |
-           (1ull << 46) | (2ull << 61);
-}
 
 // Instruction descriptor, kind::f16: bf16 A and B, fp32 D, dense.
 __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool b_mn_major) {
@@ -225,10 +227,22 @@ __device__ __forceinline__ float2 exp2_poly2(float2 x) {
     return make_float2(__uint_as_float(px), __uint_as_float(py));
 }
 
+#ifndef POLAR_TC_GROUP_PV
+// 1: the MMA thread waits for both P tiles and issues the 16 PV MMAs of the two
+// heads back to back (one queue refill per tile instead of two).
+#define POLAR_TC_GROUP_PV 1
+#endif
+
+#ifndef POLAR_TC_SPLIT_POLY_MASK
+// The same for the half-row pass of the split softmax (16 pairs per chunk):
+// 0x0101 = 2 of 16, the best of the measured shares on B200.
+#define POLAR_TC_SPLIT_POLY_MASK 0x0101
+#endif
+
 #ifndef POLAR_TC_POLY_MASK
 // Which of every 16 exponential pairs of a full tile go to the polynomial
-// (bit e set: pair e); the rest use MUFU ex2.  0x2222 = 4 of 16 (one quarter).
-#define POLAR_TC_POLY_MASK 0x2222
+// (bit e set: pair e); the rest use MUFU ex2.  0x0202 = 2 of 16.
+#define POLAR_TC_POLY_MASK 0x0202
 #endif
 
 // Row statistics of one 128-key tile of S (raw dots, one row per thread):
@@ -277,18 +291,17 @@ __device__ __forceinline__ void row_stats(uint32_t (&sr)[4][32], int t, float &t
 }
 
 // Weights p = 2^(c*log2e*S - m_ref) of one tile: their sum and sum of squares
-// (for l and l2), and the bf16 P tile written to tensor memory for the PV MMA.
+// (for l and l2), and the bf16 pairs of the P tile in pk.
 // kPoly: the pairs selected by POLAR_TC_POLY_MASK use the FMA-pipe polynomial
 // (full tiles only; the diagonal tile's -inf entries use ex2, which gives 0).
 template <bool kPoly>
 __device__ __forceinline__ void row_weights(const uint32_t (&sr)[4][32], float2 sc2, float neg_m,
-                                            uint32_t tP, float &tl, float &tl2) {
+                                            uint32_t (&pk)[4][16], float &tl, float &tl2) {
     const float2 nm = make_float2(neg_m, neg_m);
     float2 la[2], l2a[2];
     la[0] = la[1] = l2a[0] = l2a[1] = make_float2(0.f, 0.f);
 #pragma unroll
     for (int cc = 0; cc < 4; ++cc) {
-        uint32_t pk[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
             const float2 sv = make_float2(__uint_as_float(sr[cc][2 * e]),
@@ -303,13 +316,119 @@ __device__ __forceinline__ void row_weights(const uint32_t (&sr)[4][32], float2 
             }
             la[e & 1] = f2_add(la[e & 1], p);
             l2a[e & 1] = f2_fma(p, p, l2a[e & 1]);
-            pk[e] = pack_bf16(p.x, p.y);
+            pk[cc][e] = pack_bf16(p.x, p.y);
         }
-        tmem_st16(tP + 16 * cc, pk);
     }
     const float2 sl = f2_add(la[0], la[1]), sl2 = f2_add(l2a[0], l2a[1]);
     tl = sl.x + sl.y;
     tl2 = sl2.x + sl2.y;
+}
+
+// One pass over a tile with a fixed exponential reference (see the kernel's
+// kFixedRef): the weights p = 2^(c*log2e*S + neg_m) are computed at once, with
+// no wait for the tile max, and returned packed as bf16 pairs in pk; the max,
+// sum and sum of squares of the raw dots (for the gate and the null floor) and
+// the sums of p and p^2 (l, l2) accumulate alongside.  kDiag masks the keys
+// after the row's own position t (p = 0, excluded from every sum).
+template <bool kDiag, bool kPoly>
+__device__ __forceinline__ void fused_tile(const uint32_t (&sr)[4][32], int t, float2 sc2,
+                                           float neg_m, uint32_t (&pk)[4][16], float &tmax,
+                                           float &ts1, float &ts2, float &tl, float &tl2) {
+    const float2 nm = make_float2(neg_m, neg_m);
+    float mx[2] = {-INFINITY, -INFINITY};
+    float2 a1 = make_float2(0.f, 0.f), a2 = a1, la = a1, l2a = a1;
+#pragma unroll
+    for (int cc = 0; cc < 4; ++cc) {
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+            float2 sv = make_float2(__uint_as_float(sr[cc][2 * e]), __uint_as_float(sr[cc][2 * e + 1]));
+            float2 x;
+            if (kDiag) {
+                const int col = 32 * cc + 2 * e;
+                const bool v0 = col <= t, v1 = col + 1 <= t;
+                mx[e & 1] = max3(mx[e & 1], v0 ? sv.x : -INFINITY, v1 ? sv.y : -INFINITY);
+                x = f2_fma(sv, sc2, nm);
+                x.x = v0 ? x.x : -INFINITY;
+                x.y = v1 ? x.y : -INFINITY;
+                sv.x = v0 ? sv.x : 0.f;
+                sv.y = v1 ? sv.y : 0.f;
+            } else {
+                mx[e & 1] = max3(mx[e & 1], sv.x, sv.y);
+                x = f2_fma(sv, sc2, nm);
+            }
+            a1 = f2_add(a1, sv);
+            a2 = f2_fma(sv, sv, a2);
+            float2 p;
+            if (!kDiag && kPoly && ((POLAR_TC_POLY_MASK >> e) & 1)) {
+                p = exp2_poly2(make_float2(fmaxf(x.x, -126.f), fmaxf(x.y, -126.f)));
+            } else {
+                p.x = ex2(x.x);
+                p.y = ex2(x.y);
+            }
+            la = f2_add(la, p);
+            l2a = f2_fma(p, p, l2a);
+            pk[cc][e] = pack_bf16(p.x, p.y);
+        }
+    }
+    tmax = fmaxf(mx[0], mx[1]);
+    ts1 = a1.x + a1.y;
+    ts2 = a2.x + a2.y;
+    tl = la.x + la.y;
+    tl2 = l2a.x + l2a.y;
+}
+
+// fused_tile for a half row: 64 keys (keys 64*half .. 64*half + 63 of the
+// tile, in sr[0..1][0..31]) of one row, used when two softmax threads share a
+// row.  tlim = t - 64*half: key c of this half is visible iff c <= tlim.
+template <bool kDiag>
+__device__ __forceinline__ void fused_half(const uint32_t (&sr)[2][32], int tlim, float2 sc2,
+                                           float neg_m, uint32_t (&pk)[2][16], float &tmax,
+                                           float &ts1, float &ts2, float &tl, float &tl2) {
+    const float2 nm = make_float2(neg_m, neg_m);
+    float mx[2] = {-INFINITY, -INFINITY};
+    float2 a1 = make_float2(0.f, 0.f), a2 = a1, la = a1, l2a = a1;
+#pragma unroll
+    for (int cc = 0; cc < 2; ++cc) {
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+            float2 sv = make_float2(__uint_as_float(sr[cc][2 * e]), __uint_as_float(sr[cc][2 * e + 1]));
+            float2 x;
+            if (kDiag) {
+                const int col = 32 * cc + 2 * e;
+                const bool v0 = col <= tlim, v1 = col + 1 <= tlim;
+                mx[e & 1] = max3(mx[e & 1], v0 ? sv.x : -INFINITY, v1 ? sv.y : -INFINITY);
+                x = f2_fma(sv, sc2, nm);
+                x.x = v0 ? x.x : -INFINITY;
+                x.y = v1 ? x.y : -INFINITY;
+                sv.x = v0 ? sv.x : 0.f;
+                sv.y = v1 ? sv.y : 0.f;
+            } else {
+                mx[e & 1] = max3(mx[e & 1], sv.x, sv.y);
+                x = f2_fma(sv, sc2, nm);
+            }
+            a1 = f2_add(a1, sv);
+            a2 = f2_fma(sv, sv, a2);
+            float2 p;
+            if (!kDiag && ((POLAR_TC_SPLIT_POLY_MASK >> e) & 1)) {
+                p = exp2_poly2(make_float2(fmaxf(x.x, -126.f), fmaxf(x.y, -126.f)));
+            } else {
+                p.x = ex2(x.x);
+                p.y = ex2(x.y);
+            }
+            la = f2_add(la, p);
+            l2a = f2_fma(p, p, l2a);
+            pk[cc][e] = pack_bf16(p.x, p.y);
+        }
+    }
+    tmax = fmaxf(mx[0], mx[1]);
+    ts1 = a1.x + a1.y;
+    ts2 = a2.x + a2.y;
+    tl = la.x + la.y;
+    tl2 = l2a.x + l2a.y;
+}
+
+__device__ __forceinline__ void named_barrier(int id, int nthreads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
 struct TcArgs {
@@ -321,7 +440,55 @@ struct TcArgs {
     float s, alpha, L, beta, inv_ln_L;
 };
 
-__global__ void __launch_bounds__(kThreads, 1)
+// Epilogue of one row: content = O/|O|, the magnitude channel from the row's
+// streaming state, out = content + count (bf16, 128-bit stores) and n_eff.
+__device__ __forceinline__ void store_row(const uint32_t (&o)[2][32], float l, float l2,
+                                          float m_raw, float s1, float s2, float c, float n,
+                                          const TcArgs &a, int b, int row, int h) {
+    float ne;
+    const float mag = polar_magnitude(l, l2, m_raw, s1, s2, c, n, a.beta, a.inv_ln_L, &ne);
+    float nrm = 0.f;
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh)
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+            const float x = __uint_as_float(o[hh][e]);
+            nrm = fmaf(x, x, nrm);
+        }
+    const float inv = 1.0f / fmaxf(sqrtf(nrm), 1e-30f);
+    const float4 *u4 = reinterpret_cast<const float4 *>(a.u + static_cast<size_t>(h) * kHeadDim);
+    uint4 *dst = reinterpret_cast<uint4 *>(a.out + ((static_cast<size_t>(b) * a.T + row) * a.Hq + h) *
+                                                       kHeadDim);
+#pragma unroll
+    for (int ch = 0; ch < 8; ++ch) {
+        const float4 ua = __ldg(u4 + 2 * ch), ub = __ldg(u4 + 2 * ch + 1);
+        const float uu[8] = {ua.x, ua.y, ua.z, ua.w, ub.x, ub.y, ub.z, ub.w};
+        uint32_t w4[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const int d0 = 8 * ch + 2 * e;
+            const float x0 = __uint_as_float(o[d0 >> 5][d0 & 31]) * inv;
+            const float x1 = __uint_as_float(o[(d0 + 1) >> 5][(d0 + 1) & 31]) * inv;
+            w4[e] = pack_bf16(fmaf(mag, uu[2 * e], x0), fmaf(mag, uu[2 * e + 1], x1));
+        }
+        dst[ch] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+    }
+    if (a.neff) a.neff[(static_cast<size_t>(b) * a.Hq + h) * a.T + row] = ne;
+}
+
+// kFixedRef: the exponentials use the fixed per-row reference m_ref = c*log2e,
+// the largest logit L2-normalised q and k allow (|<q,k>| <= 1); weights then
+// stay <= ~1 and no rescale is needed, so a tile's weights do not wait for
+// its max.  A logit above the reference by more than the rescale threshold can
+// only come from inputs that break the normalisation precondition; it is
+// reported as POLAR_ERR_INVALID_ARG through the status word.
+// The host picks kFixedRef only when the smallest weight squared, 2^(-4c*log2e),
+// stays a normal fp32; otherwise the reference follows the running max.
+// kSplit: softmax warpgroups per head slot.  1: one thread per row (128
+// columns; any reference).  2: two threads per row, each with 64 of the keys
+// (fixed reference only: the halves need no exchange until the epilogue).
+template <bool kFixedRef, int kSplit>
+__global__ void __launch_bounds__(128 + 256 * kSplit, 1)
 fwd_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
               const __grid_constant__ CUtensorMap tv, const TcArgs a) {
     extern __shared__ uint8_t smem_raw[];
@@ -332,8 +499,12 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CU
     uint8_t *sV = sK + kStagesKV * kTileBytes;    // kStagesKV tiles
 
     __shared__ __align__(8) uint64_t q_full, kv_full[kStagesKV], kv_empty[kStagesKV];
-    __shared__ __align__(8) uint64_t s_full[2], p_full[2], o_done[2], mma_done;
+    __shared__ __align__(8) uint64_t s_full[2], s_free[2], p_full[2], pv_done[2], mma_done;
     __shared__ uint32_t tmem_base_sh;
+    // kSplit == 2: per-row partial statistics of the upper key half
+    // (m_raw, S1, S2, l, l2), handed to the lower half for the epilogue.
+    __shared__ float part[kSplit == 2 ? 2 : 1][kSplit == 2 ? kBM : 1][5];
+    static_assert(kSplit == 1 || kFixedRef, "split rows need the fixed reference");
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -355,8 +526,9 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CU
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&s_full[i], 1);
-            mbar_init(&p_full[i], kBM);
-            mbar_init(&o_done[i], 1);
+            mbar_init(&s_free[i], kBM * kSplit);
+            mbar_init(&p_full[i], kBM * kSplit);
+            mbar_init(&pv_done[i], 1);
         }
         mbar_init(&mma_done, 1);
         fence_barrier_init();
@@ -402,20 +574,31 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CU
             const uint32_t sQa = smem_u32(sQ), sKa = smem_u32(sK), sVa = smem_u32(sV);
             const uint32_t colS[2] = {kColS0, kColS1}, colP[2] = {kColP0, kColP1},
                            colO[2] = {kColO0, kColO1};
+            // Descriptor halves: low = (address >> 4) | (LBO >> 4) << 16, high =
+            // (SBO >> 4) | version 1 << 14 | SWIZZLE_128B << 29.  Q and K are
+            // K-major (LBO 16, SBO 1024); V is MN-major (LBO 8192, SBO 1024).
+            const uint32_t hi = (1024u >> 4) | (1u << 14) | (2u << 29);
+            const uint32_t q_lo0 = ((sQa & 0x3FFFFu) >> 4) | (1u << 16);
+            const uint32_t k_lo0 = ((sKa & 0x3FFFFu) >> 4) | (1u << 16);
+            const uint32_t v_lo0 = ((sVa & 0x3FFFFu) >> 4) | ((8192u >> 4) << 16);
+            constexpr uint32_t kStage = kTileBytes >> 4;
             auto issue_s = [&](int i, int j) {
-                const uint32_t qa = sQa + i * kTileBytes, ka = sKa + (j % kStagesKV) * kTileBytes;
-#pragma unroll
-                for (int kk = 0; kk < kHeadDim / 16; ++kk)
-                    mma_ss(tmem + colS[i], sw128_desc(qa + 32 * kk, 16, 1024),
-                           sw128_desc(ka + 32 * kk, 16, 1024), idesc_qk, kk > 0);
+                const uint32_t qa = q_lo0 + i * kStage, ka = k_lo0 + (j % kStagesKV) * kStage;
+                const uint32_t d = tmem + colS[i];
+                mma_ss2<0>(d, qa, hi, ka, hi, idesc_qk);
+                mma_ss2<1>(d, qa + 2, hi, ka + 2, hi, idesc_qk);
+                mma_ss2<1>(d, qa + 4, hi, ka + 4, hi, idesc_qk);
+                mma_ss2<1>(d, qa + 6, hi, ka + 6, hi, idesc_qk);
                 tc_commit(&s_full[i]);
             };
             auto issue_pv = [&](int i, int j) {
-                const uint32_t va = sVa + (j % kStagesKV) * kTileBytes;
+                const uint32_t va = v_lo0 + (j % kStagesKV) * kStage;
+                const uint32_t d = tmem + colO[i], pa = tmem + colP[i];
+                const uint32_t acc0 = j > 0;
+                mma_ts2(d, pa, va, hi, idesc_pv, acc0);
 #pragma unroll
-                for (int kk = 0; kk < kBN / 16; ++kk)
-                    mma_ts(tmem + colO[i], tmem + colP[i] + 8 * kk,
-                           sw128_desc(va + 2048 * kk, 8192, 1024), idesc_pv, (j > 0 || kk > 0));
+                for (int kk = 1; kk < kBN / 16; ++kk)
+                    mma_ts2(d, pa + 8 * kk, va + 128 * kk, hi, idesc_pv, 1u);
             };
             bool ok = mbar_wait(&q_full, 0, a.status) && mbar_wait(&kv_full[0], 0, a.status);
             if (ok) {
@@ -424,33 +607,123 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CU
                 issue_s(1, 0);
             }
             for (int j = 0; j < nkv && ok; ++j) {
-                ok = mbar_wait(&p_full[0], j & 1, a.status);
+                // Next scores first: S_i(j+1) goes as soon as softmax i has read
+                // S_i(j) into registers, so it overlaps the softmax of tile j.
+                if (j + 1 < nkv) {
+                    ok = mbar_wait(&kv_full[(j + 1) % kStagesKV], ((j + 1) / kStagesKV) & 1, a.status);
+                    for (int i = 0; i < 2 && ok; ++i) {
+                        ok = mbar_wait(&s_free[i], j & 1, a.status);
+                        if (!ok) break;
+                        tc_fence_after();
+                        issue_s(i, j + 1);
+                    }
+                    if (!ok) break;
+                }
+#if POLAR_TC_GROUP_PV
+                // Both P tiles first, then one back-to-back run of 16 PV MMAs.
+                ok = mbar_wait(&p_full[0], j & 1, a.status) && mbar_wait(&p_full[1], j & 1, a.status);
                 if (!ok) break;
                 tc_fence_after();
                 issue_pv(0, j);
-                if (j + 1 < nkv) {
-                    ok = mbar_wait(&kv_full[(j + 1) % kStagesKV], ((j + 1) / kStagesKV) & 1, a.status);
+                tc_commit(&pv_done[0]);
+                issue_pv(1, j);
+                tc_commit(&pv_done[1]);
+#else
+                for (int i = 0; i < 2 && ok; ++i) {
+                    ok = mbar_wait(&p_full[i], j & 1, a.status);
                     if (!ok) break;
                     tc_fence_after();
-                    issue_s(0, j + 1);
-                } else {
-                    tc_commit(&o_done[0]);
+                    issue_pv(i, j);
+                    tc_commit(&pv_done[i]);
                 }
-                ok = mbar_wait(&p_full[1], j & 1, a.status);
+#endif
                 if (!ok) break;
-                tc_fence_after();
-                issue_pv(1, j);
                 tc_commit(&kv_empty[j % kStagesKV]);
-                if (j + 1 < nkv)
-                    issue_s(1, j + 1);
-                else
-                    tc_commit(&o_done[1]);
             }
             // All MMAs this thread issued complete before tensor memory is freed.
             tc_commit(&mma_done);
             mbar_wait(&mma_done, 0, a.status);
         }
       }
+    } else if constexpr (kSplit == 2) {
+        reg_alloc<104>();
+        // --------------------------------- softmax: two warpgroups per head
+        const int sw = warp - 4;                 // 0..15
+        const int slot = sw >> 3;                // head slot
+        const int half = (sw >> 2) & 1;          // keys 64*half .. 64*half + 63 of a tile
+        const int wq = warp & 3;                 // TMEM lane quarter
+        const int t = 32 * wq + lane;            // row within the tile = TMEM lane
+        const int h = h0 + slot;
+        const uint32_t lane_base = tmem + (static_cast<uint32_t>(32 * wq) << 16);
+        const uint32_t tS = lane_base + (slot ? kColS1 : kColS0) + 64 * half;
+        const uint32_t tP = lane_base + (slot ? kColP1 : kColP0) + 32 * half;
+        const uint32_t tO = lane_base + (slot ? kColO1 : kColO0);
+        const int row = q0 + t;
+        const float n = static_cast<float>(row + 1);
+        const float c = a.s * length_temperature(n, a.alpha, a.L);
+        const float cl2 = c * kLog2e;
+        const float m_ref = cl2;
+        const float2 sc2 = make_float2(cl2, cl2);
+        float m_raw = -INFINITY, l = 0.f, l2 = 0.f, s1 = 0.f, s2 = 0.f;
+        bool ok = true;
+        for (int j = 0; j < nkv; ++j) {
+            ok = mbar_wait(&s_full[slot], j & 1, a.status);
+            if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+            tc_fence_after();
+            uint32_t sr[2][32];
+            tmem_ld32(tS, sr[0]);
+            tmem_ld32(tS + 32, sr[1]);
+            tmem_wait_ld();
+            tc_fence_before();
+            mbar_arrive(&s_free[slot]);
+            uint32_t pk[2][16];
+            float tmax, ts1, ts2, tl, tl2;
+            if (j == nkv - 1)
+                fused_half<true>(sr, t - 64 * half, sc2, -m_ref, pk, tmax, ts1, ts2, tl, tl2);
+            else
+                fused_half<false>(sr, t - 64 * half, sc2, -m_ref, pk, tmax, ts1, ts2, tl, tl2);
+            s1 += ts1;
+            s2 += ts2;
+            l += tl;
+            l2 += tl2;
+            m_raw = fmaxf(m_raw, tmax);
+            if (tmax * cl2 > m_ref + kRescaleThreshold) record_error(a.status, POLAR_ERR_INVALID_ARG);
+            if (j > 0) {
+                ok = mbar_wait(&pv_done[slot], (j - 1) & 1, a.status);
+                if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+                tc_fence_after();
+            }
+            tmem_st16(tP, pk[0]);
+            tmem_st16(tP + 16, pk[1]);
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(&p_full[slot]);
+        }
+        // Combine the two halves of every row; the lower half runs the epilogue.
+        if (half == 1) {
+            part[slot][t][0] = m_raw;
+            part[slot][t][1] = s1;
+            part[slot][t][2] = s2;
+            part[slot][t][3] = l;
+            part[slot][t][4] = l2;
+        }
+        named_barrier(1 + slot, 256);
+        if (half == 0) {
+            m_raw = fmaxf(m_raw, part[slot][t][0]);
+            s1 += part[slot][t][1];
+            s2 += part[slot][t][2];
+            l += part[slot][t][3];
+            l2 += part[slot][t][4];
+            if (ok) ok = mbar_wait(&pv_done[slot], (nkv - 1) & 1, a.status);
+            if (__all_sync(0xffffffffu, ok)) {
+                tc_fence_after();
+                uint32_t o[2][32];
+                tmem_ld32(tO, o[0]);
+                tmem_ld32(tO + 32, o[1]);
+                tmem_wait_ld();
+                if (row < a.T) store_row(o, l, l2, m_raw, s1, s2, c, n, a, b, row, h);
+            }
+        }
     } else {
         reg_alloc<216>();
         // ------------------------------------------------ softmax warpgroups
@@ -467,8 +740,23 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CU
         const float c = a.s * length_temperature(n, a.alpha, a.L);
         const float cl2 = c * kLog2e;
 
-        float m_ref = -INFINITY, m_raw = -INFINITY, l = 0.f, l2 = 0.f, s1 = 0.f, s2 = 0.f;
+        float m_ref = kFixedRef ? cl2 : -INFINITY;
+        float m_raw = -INFINITY, l = 0.f, l2 = 0.f, s1 = 0.f, s2 = 0.f;
         const float2 sc2 = make_float2(cl2, cl2);
+        // O_i *= r for this thread's row (a warp-collective TMEM round trip).
+        auto rescale_o = [&](float r) {
+            uint32_t o[2][32];
+            tmem_ld32(tO, o[0]);
+            tmem_ld32(tO + 32, o[1]);
+            tmem_wait_ld();
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh)
+#pragma unroll
+                for (int e = 0; e < 32; ++e)
+                    o[hh][e] = __float_as_uint(__uint_as_float(o[hh][e]) * r);
+            tmem_st32(tO, o[0]);
+            tmem_st32(tO + 32, o[1]);
+        };
         bool ok = true;
         for (int j = 0; j < nkv; ++j) {
             ok = mbar_wait(&s_full[slot], j & 1, a.status);
@@ -478,88 +766,75 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CU
 #pragma unroll
             for (int cc = 0; cc < 4; ++cc) tmem_ld32(tS + 32 * cc, sr[cc]);
             tmem_wait_ld();
+            // S_i(j) is in registers: the MMA thread may overwrite it with S_i(j+1).
+            tc_fence_before();
+            mbar_arrive(&s_free[slot]);
             const bool diag = (j == nkv - 1);
-            float tmax, ts1, ts2;
-            if (diag)
-                row_stats<true>(sr, t, tmax, ts1, ts2);
-            else
-                row_stats<false>(sr, t, tmax, ts1, ts2);
-            s1 += ts1;
-            s2 += ts2;
-            m_raw = fmaxf(m_raw, tmax);
-            const float zmax = tmax * cl2;
-            const bool need = zmax > m_ref + kRescaleThreshold;
+            uint32_t pk[4][16];
             float r = 1.f;
-            if (need) {
-                r = ex2(m_ref - zmax);  // 0 on the first tile
-                l *= r;
-                l2 *= r * r;
-                m_ref = zmax;
+            bool need = false;
+            if (kFixedRef) {
+                float tmax, ts1, ts2, tl, tl2;
+                if (diag)
+                    fused_tile<true, false>(sr, t, sc2, -m_ref, pk, tmax, ts1, ts2, tl, tl2);
+                else
+                    fused_tile<false, true>(sr, t, sc2, -m_ref, pk, tmax, ts1, ts2, tl, tl2);
+                s1 += ts1;
+                s2 += ts2;
+                l += tl;
+                l2 += tl2;
+                m_raw = fmaxf(m_raw, tmax);
+                // A logit this far above the unit-vector bound means q or k was not
+                // L2-normalised: the precondition is broken and is reported.
+                if (tmax * cl2 > m_ref + kRescaleThreshold) record_error(a.status, POLAR_ERR_INVALID_ARG);
+            } else {
+                float tmax, ts1, ts2;
+                if (diag)
+                    row_stats<true>(sr, t, tmax, ts1, ts2);
+                else
+                    row_stats<false>(sr, t, tmax, ts1, ts2);
+                s1 += ts1;
+                s2 += ts2;
+                m_raw = fmaxf(m_raw, tmax);
+                const float zmax = tmax * cl2;
+                need = zmax > m_ref + kRescaleThreshold;
+                if (need) {
+                    r = ex2(m_ref - zmax);  // 0 on the first tile
+                    l *= r;
+                    l2 *= r * r;
+                    m_ref = zmax;
+                }
+                float tl, tl2;
+                if (diag)
+                    row_weights<false>(sr, sc2, -m_ref, pk, tl, tl2);
+                else
+                    row_weights<true>(sr, sc2, -m_ref, pk, tl, tl2);
+                l += tl;
+                l2 += tl2;
             }
-            float tl, tl2;
-            if (diag)
-                row_weights<false>(sr, sc2, -m_ref, tP, tl, tl2);
-            else
-                row_weights<true>(sr, sc2, -m_ref, tP, tl, tl2);
-            l += tl;
-            l2 += tl2;
+            // PV_i(j-1) done: P_i may be overwritten and O_i is current.  Waiting only
+            // now lets this tile's weights overlap PV_i(j-1).
+            if (j > 0) {
+                ok = mbar_wait(&pv_done[slot], (j - 1) & 1, a.status);
+                if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+                tc_fence_after();
+            }
+#pragma unroll
+            for (int cc = 0; cc < 4; ++cc) tmem_st16(tP + 16 * cc, pk[cc]);
             // Rescale the output accumulator when this row's reference max moved.
-            // Safe: S(j) landing implies PV(j-1) has completed (one commit covers both).
-            if (j > 0 && __any_sync(0xffffffffu, need)) {
-                uint32_t o[2][32];
-                tmem_ld32(tO, o[0]);
-                tmem_ld32(tO + 32, o[1]);
-                tmem_wait_ld();
-#pragma unroll
-                for (int hh = 0; hh < 2; ++hh)
-#pragma unroll
-                    for (int e = 0; e < 32; ++e)
-                        o[hh][e] = __float_as_uint(__uint_as_float(o[hh][e]) * r);
-                tmem_st32(tO, o[0]);
-                tmem_st32(tO + 32, o[1]);
-            }
+            if (!kFixedRef && j > 0 && __any_sync(0xffffffffu, need)) rescale_o(r);
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(&p_full[slot]);
         }
-        if (ok) ok = mbar_wait(&o_done[slot], 0, a.status);
+        if (ok) ok = mbar_wait(&pv_done[slot], (nkv - 1) & 1, a.status);
         if (__all_sync(0xffffffffu, ok)) {
             tc_fence_after();
             uint32_t o[2][32];
             tmem_ld32(tO, o[0]);
             tmem_ld32(tO + 32, o[1]);
             tmem_wait_ld();
-            if (row < a.T) {
-                float ne;
-                const float mag = polar_magnitude(l, l2, m_raw, s1, s2, c, n, a.beta, a.inv_ln_L, &ne);
-                float nrm = 0.f;
-#pragma unroll
-                for (int hh = 0; hh < 2; ++hh)
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) {
-                        const float x = __uint_as_float(o[hh][e]);
-                        nrm = fmaf(x, x, nrm);
-                    }
-                const float inv = 1.0f / fmaxf(sqrtf(nrm), 1e-30f);
-                const float4 *u4 = reinterpret_cast<const float4 *>(a.u + static_cast<size_t>(h) * kHeadDim);
-                uint4 *dst = reinterpret_cast<uint4 *>(
-                    a.out + ((static_cast<size_t>(b) * a.T + row) * a.Hq + h) * kHeadDim);
-#pragma unroll
-                for (int ch = 0; ch < 8; ++ch) {
-                    const float4 ua = __ldg(u4 + 2 * ch), ub = __ldg(u4 + 2 * ch + 1);
-                    const float uu[8] = {ua.x, ua.y, ua.z, ua.w, ub.x, ub.y, ub.z, ub.w};
-                    uint32_t w4[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int d0 = 8 * ch + 2 * e;
-                        const float x0 = __uint_as_float(o[d0 >> 5][d0 & 31]) * inv;
-                        const float x1 = __uint_as_float(o[(d0 + 1) >> 5][(d0 + 1) & 31]) * inv;
-                        w4[e] = pack_bf16(fmaf(mag, uu[2 * e], x0), fmaf(mag, uu[2 * e + 1], x1));
-                    }
-                    dst[ch] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
-                }
-                if (a.neff) a.neff[(static_cast<size_t>(b) * a.Hq + h) * a.T + row] = ne;
-            }
+            if (row < a.T) store_row(o, l, l2, m_raw, s1, s2, c, n, a, b, row, h);
         }
     }
 
@@ -586,14 +861,25 @@ cudaError_t launch_fwd_tc(const FwdLaunch &a) {
     const int G = a.Hq / a.Hkv;
     if (a.dtype != POLAR_BF16 || G % 2 != 0) return cudaErrorNotSupported;
     static std::atomic<uint64_t> configured{0};
+    static std::atomic<uint64_t> split_ok{0};  // per device: the split kernel's register plan holds
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     const uint64_t bit = 1ull << (dev & 63);
     if (!(configured.load() & bit)) {
-        e = cudaFuncSetAttribute(fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        e = cudaFuncSetAttribute(fwd_tc_kernel<true, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  kSmemBytes);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(fwd_tc_kernel<false, 1>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
         if (e != cudaSuccess) return e;
+        // setmaxnreg can only hand out the registers the block was launched with:
+        // 64 for the producer/MMA warpgroup plus 104 for each of the four softmax
+        // warpgroups must fit in (registers per thread at launch) x 640.
+        cudaFuncAttributes fa;
+        e = cudaFuncGetAttributes(&fa, fwd_tc_kernel<true, 2>);
+        if (e != cudaSuccess) return e;
+        if (static_cast<long long>(fa.numRegs) * 640 >= 64ll * 128 + 104ll * 512) split_ok.fetch_or(bit);
         configured.fetch_or(bit);
     }
     // [B, T, H, 64] bf16 as a 4-D tensor (d, head, t, b); tiles of 128 rows x 64.
@@ -630,7 +916,15 @@ cudaError_t launch_fwd_tc(const FwdLaunch &a) {
     const long long ctas = static_cast<long long>(ta.nqt) * ta.npairs * a.B;
     if (ctas <= 0) return cudaSuccess;
     if (ctas > 0x7fffffffll) return cudaErrorInvalidValue;
-    fwd_tc_kernel<<<static_cast<unsigned>(ctas), kThreads, kSmemBytes, a.stream>>>(tq, tk, tv, ta);
+    // Fixed exponential reference while the smallest weight squared, 2^(-4 c_max log2e)
+    // with c_max the largest logit scale of any row, stays well inside fp32.
+    const float cl2_max = a.s *
+                          (a.T > a.L ? 1.0f + a.alpha * logf(static_cast<float>(a.T) / a.L) : 1.0f) *
+                          1.4426950408889634f;
+    if (cl2_max <= 28.0f && (split_ok.load() & bit))
+        fwd_tc_kernel<true, 2><<<static_cast<unsigned>(ctas), 640, kSmemBytes, a.stream>>>(tq, tk, tv, ta);
+    else
+        fwd_tc_kernel<false, 1><<<static_cast<unsigned>(ctas), 384, kSmemBytes, a.stream>>>(tq, tk, tv, ta);
     count_launches(1);
     return cudaGetLastError();
 }

@@ -89,3 +89,30 @@ def test_long_T65536_sampled(cuda_ok):
     PT.compare(o, n, ref, grp, PT.OUT_TOL_BF16, what="long_T65536")
     nn = neff[0, :, T - 64:].float()
     assert nn.median() < 0.01 * neff[0, :, T // 2:T - 64].float().median()
+
+
+@pytest.mark.parametrize("T", [300, 1000])
+def test_large_logit_scale_uses_running_max(cuda_ok, T):
+    """A logit scale whose weights could underflow against the fixed reference
+    (s * log2e > 28) takes the running-max kernel; it must match too."""
+    w = W.small_prefill(B=1, T=T, Hq=8, Hkv=2, dtype="bf16", seed=T, plant="frac",
+                        plant_frac=0.02, s=24.0, L=256)
+    x, out, neff = _run(w)
+    ref = PT.oracle_prefill(w, x)
+    rows = np.arange(w.B * w.Hq * w.T)
+    o, n, grp = PT.gpu_rows_prefill(out, neff, rows, w.B, w.T, w.Hq)
+    PT.compare(o, n, ref, grp, PT.OUT_TOL_BF16, what=f"running max T={T}")
+
+
+def test_unnormalised_inputs_are_reported(cuda_ok):
+    """q scaled by 3 breaks the L2-normalisation precondition: the fixed-
+    reference kernel sees logits past the unit-vector bound and reports
+    POLAR_ERR_INVALID_ARG through the status word (no fault, finite output)."""
+    w = W.small_prefill(B=1, T=256, Hq=4, Hkv=2, dtype="bf16", seed=2, plant="frac",
+                        plant_frac=0.05)
+    x = PT.to_device(W.prefill_inputs(w, "cpu"))
+    assert pa.get_status() == 0
+    out, neff = pa.fwd((x["q"].float() * 3).bfloat16(), x["k"], x["v"], x["u"], impl="tc")
+    torch.cuda.synchronize()
+    assert pa.get_status() == 1  # POLAR_ERR_INVALID_ARG
+    assert pa.get_status() == 0
