@@ -46,20 +46,66 @@ struct SplitArgs {
 };
 
 // Byte offset of logical 16-byte chunk c of row t inside a 128B-swizzled tile.
-__device__ __forceinline__ int swz(int t, int c) { return t * 128 + ((c ^ (t & 7)) << 4); }
+__device__ __forceinline__ uint32_t swz(int t, int c) {
+    return static_cast<uint32_t>(t * 128 + ((c ^ (t & 7)) << 4));
+}
 
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr));
+}
+
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t (&r)[4]) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr));
+}
+
+// d += A(16x16, rows g and g+8 of the lane) * B(16x8), bf16 in, fp32 accumulate.
+// Rows g+8 (a1, a3) are the zero padding of the query-head dimension.
+__device__ __forceinline__ void mma_bf16(float (&d)[4], uint32_t a0, uint32_t a2, uint32_t b0,
+                                         uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    uint32_t r;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+// Keep the low / high bf16 half of x only if the corresponding token is valid.
+__device__ __forceinline__ uint32_t mask_pair(uint32_t x, bool lo_ok, bool hi_ok) {
+    return (lo_ok ? (x & 0xFFFFu) : 0u) | (hi_ok ? (x & 0xFFFF0000u) : 0u);
+}
+
+// Split kernel: CTA (split, kv head g, sequence), 4 warps.  Warp w owns tokens
+// 16w .. 16w+15 of every page and keeps, for each query head of the group
+// (mma rows; rows >= G are zero padding), the streaming state of the method:
+// reference max m_ref (log2 units), l, l2 (rescaled by r, r^2 when m_ref
+// moves past the lazy threshold), the raw-dot sums S1, S2 and max, and the
+// value accumulator O (mma accumulator fragments).  The scores S = Q K^T and
+// O += P V run on mma.sync (bf16 in, fp32 accumulate); the S fragments are
+// reused as the P operand in registers.  At the end the four warps' states are
+// merged exactly in shared memory into one partial per (split, query head).
 template <int G>
-__global__ void __launch_bounds__(32 * G)
+__global__ void __launch_bounds__(128)
 decode_split_kernel(const __grid_constant__ CUtensorMap kv_map, const SplitArgs a) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     __shared__ __align__(8) uint64_t full_bar[kStages];
-    __shared__ __align__(16) float ps[G][kPage];
+    __shared__ float mst[4][G][6];          // per warp, head: m_ref, m_raw, l, l2, S1, S2
+    __shared__ float macc[4][G][kHeadDim];  // per warp, head: O row
 
     const int split = blockIdx.x, g = blockIdx.y, seq = blockIdx.z;
     const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int h = g * G + w;
+    const int gq = lane >> 2, tq = lane & 3;  // mma row (query head) and column pair
 
     const int seqlen = a.seqlens[seq];
     if (seqlen < 1 || seqlen > a.max_pages * kPage) {
@@ -99,30 +145,28 @@ decode_split_kernel(const __grid_constant__ CUtensorMap kv_map, const SplitArgs 
     if (threadIdx.x == 0)
         for (int kk = 0; kk < min(kStages, np); ++kk) issue(kk);
 
-    // The query row of head h, fp32, in every lane.
-    float qr[kHeadDim];
+    // Query fragments (A operand of S = Q K^T): row gq = query head g*G + gq.
+    const bool real = gq < G;
+    uint32_t qa[4][2];
     {
-        const uint4 *qp = reinterpret_cast<const uint4 *>(
-            a.q + (static_cast<size_t>(seq) * a.Hq + h) * kHeadDim);
+        const uint32_t *qrow = reinterpret_cast<const uint32_t *>(
+            a.q + (static_cast<size_t>(seq) * a.Hq + g * G + (real ? gq : 0)) * kHeadDim);
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-            const uint4 raw = __ldg(qp + c);
-            const __nv_bfloat162 *pr = reinterpret_cast<const __nv_bfloat162 *>(&raw);
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const float2 f = __bfloat1622float2(pr[e]);
-                qr[c * 8 + 2 * e] = f.x;
-                qr[c * 8 + 2 * e + 1] = f.y;
-            }
+        for (int kk = 0; kk < 4; ++kk) {
+            qa[kk][0] = real ? __ldg(qrow + 8 * kk + tq) : 0u;
+            qa[kk][1] = real ? __ldg(qrow + 8 * kk + 4 + tq) : 0u;
         }
     }
     const float n = static_cast<float>(seqlen);
     const float cl2 = a.s * length_temperature(n, a.alpha, a.L) * kLog2e;
 
     float m_ref = -INFINITY, m_raw = -INFINITY, l = 0.f, l2 = 0.f, s1 = 0.f, s2 = 0.f;
-    float acc0 = 0.f, acc1 = 0.f;  // d = 2*lane, 2*lane + 1
+    float acc[8][4];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
     int issued = min(kStages, np), consumed = 0;
     bool ok = true;
+    const uint32_t sbase = smem_u32(smem);
 
     for (int kk = 0; kk < np; ++kk) {
         const int st = kk % kStages;
@@ -134,59 +178,81 @@ decode_split_kernel(const __grid_constant__ CUtensorMap kv_map, const SplitArgs 
         if (phys >= 0 && phys < a.num_pages) {
             const int page = p0 + kk;
             const int ntok = page == npg - 1 ? seqlen - page * kPage : kPage;
-            const uint8_t *kb = smem + st * kStageBytes;
-            const uint8_t *vb = kb + kChunkBytes;
-            // logits of tokens lane and lane + 32 for head h
-            float sd[2];
+            const uint32_t kb = sbase + st * kStageBytes, vb = kb + kChunkBytes;
+            // S = Q K^T for this warp's 16 tokens (two n-tiles of 8).
+            float sc[2][4];
 #pragma unroll
-            for (int r = 0; r < 2; ++r) {
-                const int t = lane + 32 * r;
-                float acc = 0.f;
+            for (int nt = 0; nt < 2; ++nt) {
+                sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
+                const int tok = 16 * w + 8 * nt + (lane & 7);
+                uint32_t b[2][4];
+                ldsm_x4(kb + swz(tok, lane >> 3), b[0]);
+                ldsm_x4(kb + swz(tok, 4 + (lane >> 3)), b[1]);
 #pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    const uint4 raw = *reinterpret_cast<const uint4 *>(kb + swz(t, c));
-                    const __nv_bfloat162 *pr = reinterpret_cast<const __nv_bfloat162 *>(&raw);
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float2 f = __bfloat1622float2(pr[e]);
-                        acc = fmaf(qr[c * 8 + 2 * e], f.x, acc);
-                        acc = fmaf(qr[c * 8 + 2 * e + 1], f.y, acc);
-                    }
-                }
-                sd[r] = acc;
+                for (int ks = 0; ks < 4; ++ks)
+                    mma_bf16(sc[nt], qa[ks][0], qa[ks][1], b[ks >> 1][2 * (ks & 1)],
+                             b[ks >> 1][2 * (ks & 1) + 1]);
             }
-            const bool v0 = lane < ntok, v1 = lane + 32 < ntok;
-            const float z0 = v0 ? sd[0] * cl2 : -INFINITY;
-            const float z1 = v1 ? sd[1] * cl2 : -INFINITY;
-            s1 += (v0 ? sd[0] : 0.f) + (v1 ? sd[1] : 0.f);
-            s2 += (v0 ? sd[0] * sd[0] : 0.f) + (v1 ? sd[1] * sd[1] : 0.f);
-            m_raw = fmaxf(m_raw, fmaxf(v0 ? sd[0] : -INFINITY, v1 ? sd[1] : -INFINITY));
-            const float tmax = warp_max(fmaxf(z0, z1));
-            if (tmax > m_ref + kRescaleThreshold) {  // warp-uniform
-                const float r = exp2f(m_ref - tmax);
+            // Streaming statistics of the valid tokens (rows gq; c0/c1 of each n-tile).
+            bool vld[2][2];
+            float tmax = -INFINITY, ts1 = 0.f, ts2 = 0.f;
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    vld[nt][e] = 16 * w + 8 * nt + 2 * tq + e < ntok;
+                    const float x = sc[nt][e];
+                    tmax = fmaxf(tmax, vld[nt][e] ? x : -INFINITY);
+                    ts1 += vld[nt][e] ? x : 0.f;
+                    ts2 += vld[nt][e] ? x * x : 0.f;
+                }
+            tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 1));
+            tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 2));
+            s1 += ts1;
+            s2 += ts2;
+            m_raw = fmaxf(m_raw, tmax);
+            const float zmax = tmax * cl2;
+            if (zmax > m_ref + kRescaleThreshold) {  // uniform over the quad of row gq
+                const float r = exp2f(m_ref - zmax);
                 l *= r;
                 l2 *= r * r;
-                acc0 *= r;
-                acc1 *= r;
-                m_ref = tmax;
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    acc[i][0] *= r;
+                    acc[i][1] *= r;
+                }
+                m_ref = zmax;
             }
-            const float pa = exp2f(z0 - m_ref), pb = exp2f(z1 - m_ref);
-            l += pa + pb;
-            l2 += pa * pa + pb * pb;
-            ps[w][lane] = pa;
-            ps[w][lane + 32] = pb;
-            __syncwarp();
-            // acc[d] += sum_t p_t v_t[d] for this lane's two columns
-            const int cw = lane >> 2, sub = (lane & 3) * 4;
-            for (int t = 0; t < ntok; ++t) {
-                const float p = ps[w][t];
-                const __nv_bfloat162 vv = *reinterpret_cast<const __nv_bfloat162 *>(
-                    vb + t * 128 + ((cw ^ (t & 7)) << 4) + sub);
-                const float2 f = __bfloat1622float2(vv);
-                acc0 = fmaf(p, f.x, acc0);
-                acc1 = fmaf(p, f.y, acc1);
+            float pv[2][2];
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const float pp = vld[nt][e] ? exp2f(fmaf(sc[nt][e], cl2, -m_ref)) : 0.f;
+                    pv[nt][e] = pp;
+                    l += pp;
+                    l2 = fmaf(pp, pp, l2);
+                }
+            const uint32_t pa0 = pack_bf16x2(pv[0][0], pv[0][1]);
+            const uint32_t pa2 = pack_bf16x2(pv[1][0], pv[1][1]);
+            // O += P V: V^T fragments by transposed ldmatrix; tokens past the end
+            // of the sequence are zeroed so no stale value can enter the sum.
+            const bool last = ntok < kPage;
+            const int trow = 16 * w + 8 * ((lane >> 3) & 1) + (lane & 7);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                uint32_t v[4];
+                ldsm_x4_t(vb + swz(trow, 2 * i + (lane >> 4)), v);
+                if (last) {
+                    const int t0 = 16 * w + 2 * tq;
+                    v[0] = mask_pair(v[0], t0 < ntok, t0 + 1 < ntok);
+                    v[1] = mask_pair(v[1], t0 + 8 < ntok, t0 + 9 < ntok);
+                    v[2] = mask_pair(v[2], t0 < ntok, t0 + 1 < ntok);
+                    v[3] = mask_pair(v[3], t0 + 8 < ntok, t0 + 9 < ntok);
+                }
+                mma_bf16(acc[2 * i], pa0, pa2, v[0], v[1]);
+                mma_bf16(acc[2 * i + 1], pa0, pa2, v[2], v[3]);
             }
-            __syncwarp();
         }
         __syncthreads();  // every warp is done with stage st
         if (threadIdx.x == 0 && issued < np) issue(issued++);
@@ -201,17 +267,58 @@ decode_split_kernel(const __grid_constant__ CUtensorMap kv_map, const SplitArgs 
         return;
     }
 
-    l = warp_sum(l);
-    l2 = warp_sum(l2);
-    s1 = warp_sum(s1);
-    s2 = warp_sum(s2);
-    m_raw = warp_max(m_raw);
-    float *dst = a.partials +
-                 ((static_cast<size_t>(seq) * a.Hq + h) * a.max_splits + split) * kPartialFloats;
-    reinterpret_cast<float2 *>(dst)[lane] = make_float2(acc0, acc1);
-    if (lane == 0) {
-        reinterpret_cast<float4 *>(dst + 64)[0] = make_float4(m_ref, m_raw, l, l2);
-        reinterpret_cast<float2 *>(dst + 68)[0] = make_float2(s1, s2);
+    // Reduce the quad of each row, then merge the four warps exactly.
+#pragma unroll
+    for (int o = 1; o <= 2; o <<= 1) {
+        l += __shfl_xor_sync(0xffffffffu, l, o);
+        l2 += __shfl_xor_sync(0xffffffffu, l2, o);
+        s1 += __shfl_xor_sync(0xffffffffu, s1, o);
+        s2 += __shfl_xor_sync(0xffffffffu, s2, o);
+        m_raw = fmaxf(m_raw, __shfl_xor_sync(0xffffffffu, m_raw, o));
+    }
+    if (real) {
+        if (tq == 0) {
+            mst[w][gq][0] = m_ref;
+            mst[w][gq][1] = m_raw;
+            mst[w][gq][2] = l;
+            mst[w][gq][3] = l2;
+            mst[w][gq][4] = s1;
+            mst[w][gq][5] = s2;
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            macc[w][gq][8 * i + 2 * tq] = acc[i][0];
+            macc[w][gq][8 * i + 2 * tq + 1] = acc[i][1];
+        }
+    }
+    __syncthreads();
+    for (int hh = w; hh < G; hh += 4) {
+        float M = -INFINITY;
+#pragma unroll
+        for (int ww = 0; ww < 4; ++ww) M = fmaxf(M, mst[ww][hh][0]);
+        float r[4];
+#pragma unroll
+        for (int ww = 0; ww < 4; ++ww) r[ww] = M == -INFINITY ? 0.f : exp2f(mst[ww][hh][0] - M);
+        float2 o = make_float2(0.f, 0.f);
+        float ml = 0.f, ml2 = 0.f, ms1 = 0.f, ms2 = 0.f, mraw = -INFINITY;
+#pragma unroll
+        for (int ww = 0; ww < 4; ++ww) {
+            o.x = fmaf(macc[ww][hh][2 * lane], r[ww], o.x);
+            o.y = fmaf(macc[ww][hh][2 * lane + 1], r[ww], o.y);
+            ml = fmaf(mst[ww][hh][2], r[ww], ml);
+            ml2 = fmaf(mst[ww][hh][3], r[ww] * r[ww], ml2);
+            ms1 += mst[ww][hh][4];
+            ms2 += mst[ww][hh][5];
+            mraw = fmaxf(mraw, mst[ww][hh][1]);
+        }
+        const int h = g * G + hh;
+        float *dst = a.partials +
+                     ((static_cast<size_t>(seq) * a.Hq + h) * a.max_splits + split) * kPartialFloats;
+        reinterpret_cast<float2 *>(dst)[lane] = o;
+        if (lane == 0) {
+            reinterpret_cast<float4 *>(dst + 64)[0] = make_float4(M, mraw, ml, ml2);
+            reinterpret_cast<float2 *>(dst + 68)[0] = make_float2(ms1, ms2);
+        }
     }
 }
 
@@ -275,7 +382,7 @@ cudaError_t launch_split(const CUtensorMap &map, const SplitArgs &sa, int num_se
         configured.fetch_or(bit);
     }
     dim3 grid(sa.max_splits, sa.Hkv, num_seqs);
-    decode_split_kernel<G><<<grid, 32 * G, kSplitSmem, stream>>>(map, sa);
+    decode_split_kernel<G><<<grid, 128, kSplitSmem, stream>>>(map, sa);
     return cudaGetLastError();
 }
 
