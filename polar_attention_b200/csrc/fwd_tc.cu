@@ -19,12 +19,12 @@
 //   warps 8-11  softmax warpgroup for head slot 1
 // Tensor memory (512 columns): S0 S1 (128 fp32 columns each), P0 P1 (128 bf16
 // packed in 64 columns each), O0 O1 (64 fp32 columns each).
-// Per key tile j the MMA thread issues S0(j+1) and S1(j+1) as soon as each
-// softmax warpgroup has copied S_i(j) into registers (barrier s_free), then
-// PV0(j) and PV1(j) once P_i(j) is in tensor memory (p_full).  The next scores
-// are thus computed while the softmax of tile j runs.  A commit after PV_i(j)
-// (pv_done) tells softmax i that P_i may be overwritten and that O_i is
-// current, so it can rescale O_i in place before it releases P_i(j+1).
+// The MMA thread keeps the scores one tile ahead of the softmax: when P_0(j)
+// and P_1(j) are in tensor memory (barrier p_full) it issues S0(j+2) and
+// S1(j+2) (each once softmax i has copied S_i(j+1) into registers, barrier
+// s_free), then PV0(j) and PV1(j).  A commit after PV_i(j) (pv_done) tells
+// softmax i that P_i may be overwritten and that O_i is current, so it can
+// rescale O_i in place before it releases P_i(j+1).
 #include <atomic>
 
 #include "polar_attn_selftest.h"
@@ -227,11 +227,6 @@ __device__ __forceinline__ float2 exp2_poly2(float2 x) {
     return make_float2(__uint_as_float(px), __uint_as_float(py));
 }
 
-#ifndef POLAR_TC_GROUP_PV
-// 1: the MMA thread waits for both P tiles and issues the 16 PV MMAs of the two
-// heads back to back (one queue refill per tile instead of two).
-#define POLAR_TC_GROUP_PV 1
-#endif
 
 #ifndef POLAR_TC_SPLIT_POLY_MASK
 // The same for the half-row pass of the split softmax (16 pairs per chunk):
@@ -431,6 +426,7 @@ __device__ __forceinline__ void named_barrier(int id, int nthreads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
+
 struct TcArgs {
     const float *u;
     __nv_bfloat16 *out;
@@ -600,44 +596,32 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CU
                 for (int kk = 1; kk < kBN / 16; ++kk)
                     mma_ts2(d, pa + 8 * kk, va + 128 * kk, hi, idesc_pv, 1u);
             };
-            bool ok = mbar_wait(&q_full, 0, a.status) && mbar_wait(&kv_full[0], 0, a.status);
-            if (ok) {
-                tc_fence_after();
-                issue_s(0, 0);
-                issue_s(1, 0);
-            }
-            for (int j = 0; j < nkv && ok; ++j) {
-                // Next scores first: S_i(j+1) goes as soon as softmax i has read
-                // S_i(j) into registers, so it overlaps the softmax of tile j.
-                if (j + 1 < nkv) {
-                    ok = mbar_wait(&kv_full[(j + 1) % kStagesKV], ((j + 1) / kStagesKV) & 1, a.status);
-                    for (int i = 0; i < 2 && ok; ++i) {
-                        ok = mbar_wait(&s_free[i], j & 1, a.status);
-                        if (!ok) break;
-                        tc_fence_after();
-                        issue_s(i, j + 1);
-                    }
-                    if (!ok) break;
+            // Waits for S_i(jn)'s K tile and for softmax i to have copied S_i(jn-1)
+            // out of tensor memory, then issues S_i(jn) for both heads.
+            auto next_scores = [&](int jn) -> bool {
+                if (!mbar_wait(&kv_full[jn % kStagesKV], (jn / kStagesKV) & 1, a.status)) return false;
+                for (int i = 0; i < 2; ++i) {
+                    if (jn > 0 && !mbar_wait(&s_free[i], (jn - 1) & 1, a.status)) return false;
+                    tc_fence_after();
+                    issue_s(i, jn);
                 }
-#if POLAR_TC_GROUP_PV
-                // Both P tiles first, then one back-to-back run of 16 PV MMAs.
+                return true;
+            };
+            bool ok = mbar_wait(&q_full, 0, a.status) && next_scores(0);
+            if (ok && nkv > 1) ok = next_scores(1);
+            for (int j = 0; j < nkv && ok; ++j) {
+                // P_0(j) and P_1(j) are in tensor memory.  The scores two tiles ahead
+                // go first: S_i(j+2) may overwrite S_i once softmax i has loaded
+                // S_i(j+1), which it does right after releasing P_i(j).  PV(j) is
+                // needed only at the end of softmax tile j+1, so it can wait behind.
                 ok = mbar_wait(&p_full[0], j & 1, a.status) && mbar_wait(&p_full[1], j & 1, a.status);
                 if (!ok) break;
+                if (j + 2 < nkv && !(ok = next_scores(j + 2))) break;
                 tc_fence_after();
                 issue_pv(0, j);
                 tc_commit(&pv_done[0]);
                 issue_pv(1, j);
                 tc_commit(&pv_done[1]);
-#else
-                for (int i = 0; i < 2 && ok; ++i) {
-                    ok = mbar_wait(&p_full[i], j & 1, a.status);
-                    if (!ok) break;
-                    tc_fence_after();
-                    issue_pv(i, j);
-                    tc_commit(&pv_done[i]);
-                }
-#endif
-                if (!ok) break;
                 tc_commit(&kv_empty[j % kStagesKV]);
             }
             // All MMAs this thread issued complete before tensor memory is freed.
