@@ -13,16 +13,17 @@
 // query rows, so both heads share every K/V tile and have the same causal
 // extent.  Warp roles (12 warps):
 //   warp 0      TMA producer: Q tiles once, then K/V tiles into a 4-stage ring
-//   warp 1      tensor-memory allocator and single-thread MMA issuer
-//   warps 2-3   idle
+//   warp 1      tensor-memory allocator and the score-MMA issuer (one thread)
+//   warp 2      the PV-MMA issuer (one thread)
+//   warp 3      idle
 //   warps 4-7   softmax warpgroup for head slot 0 (TMEM lanes 0-127)
 //   warps 8-11  softmax warpgroup for head slot 1
 // Tensor memory (512 columns): S0 S1 (128 fp32 columns each), P0 P1 (128 bf16
 // packed in 64 columns each), O0 O1 (64 fp32 columns each).
-// The MMA thread keeps the scores one tile ahead of the softmax: when P_0(j)
-// and P_1(j) are in tensor memory (barrier p_full) it issues S0(j+2) and
-// S1(j+2) (each once softmax i has copied S_i(j+1) into registers, barrier
-// s_free), then PV0(j) and PV1(j).  A commit after PV_i(j) (pv_done) tells
+// Two issuing threads keep the tensor core fed: one issues S_i(j) as soon as
+// softmax i has copied S_i(j-1) out of tensor memory (barrier s_free), the
+// other PV_i(j) as soon as P_i(j) is in tensor memory (p_full), so neither
+// waits behind the other's queue.  A commit after PV_i(j) (pv_done) tells
 // softmax i that P_i may be overwritten and that O_i is current, so it can
 // rescale O_i in place before it releases P_i(j+1).
 #include <atomic>
@@ -495,7 +496,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CU
     uint8_t *sV = sK + kStagesKV * kTileBytes;    // kStagesKV tiles
 
     __shared__ __align__(8) uint64_t q_full, kv_full[kStagesKV], kv_empty[kStagesKV];
-    __shared__ __align__(8) uint64_t s_full[2], s_free[2], p_full[2], pv_done[2], mma_done;
+    __shared__ __align__(8) uint64_t s_full[2], s_free[2], p_full[2], pv_done[2], mma_done[2];
     __shared__ uint32_t tmem_base_sh;
     // kSplit == 2: per-row partial statistics of the upper key half
     // (m_raw, S1, S2, l, l2), handed to the lower half for the epilogue.
@@ -518,7 +519,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CU
         mbar_init(&q_full, 1);
         for (int st = 0; st < kStagesKV; ++st) {
             mbar_init(&kv_full[st], 1);
-            mbar_init(&kv_empty[st], 1);
+            mbar_init(&kv_empty[st], 2);  // one commit from each MMA issuer
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&s_full[i], 1);
@@ -526,7 +527,8 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CU
             mbar_init(&p_full[i], kBM * kSplit);
             mbar_init(&pv_done[i], 1);
         }
-        mbar_init(&mma_done, 1);
+        mbar_init(&mma_done[0], 1);
+        mbar_init(&mma_done[1], 1);
         fence_barrier_init();
     }
     if (warp == 1) tmem_alloc_512(&tmem_base_sh);
@@ -562,14 +564,18 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CU
             for (int j = (issued > kStagesKV ? issued - kStagesKV : 0); j < issued; ++j)
                 mbar_wait(&kv_full[j % kStagesKV], (j / kStagesKV) & 1, a.status);
         }
-    } else if (warp == 1) {
-        // ------------------------------------------------------- MMA issuer
+    } else if (warp == 1 || warp == 2) {
+        // ------------------------------------------ MMA issuers (one thread each)
+        // Warp 1 issues the score MMAs S_i(j) as soon as the K tile of j has landed
+        // and softmax i has copied S_i(j-1) out of tensor memory; warp 2 issues the
+        // PV MMAs as soon as P_i(j) is in tensor memory.  Neither waits behind the
+        // other's backlog.  Each commits only the barriers that track its own MMAs
+        // (a commit covers the issuing thread's MMAs); a K/V stage is free after
+        // one commit from each.
         if (lane == 0) {
             constexpr uint32_t idesc_qk = idesc_bf16(kBM, kBN, false);
             constexpr uint32_t idesc_pv = idesc_bf16(kBM, kHeadDim, true);
             const uint32_t sQa = smem_u32(sQ), sKa = smem_u32(sK), sVa = smem_u32(sV);
-            const uint32_t colS[2] = {kColS0, kColS1}, colP[2] = {kColP0, kColP1},
-                           colO[2] = {kColO0, kColO1};
             // Descriptor halves: low = (address >> 4) | (LBO >> 4) << 16, high =
             // (SBO >> 4) | version 1 << 14 | SWIZZLE_128B << 29.  Q and K are
             // K-major (LBO 16, SBO 1024); V is MN-major (LBO 8192, SBO 1024).
@@ -580,7 +586,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CU
             constexpr uint32_t kStage = kTileBytes >> 4;
             auto issue_s = [&](int i, int j) {
                 const uint32_t qa = q_lo0 + i * kStage, ka = k_lo0 + (j % kStagesKV) * kStage;
-                const uint32_t d = tmem + colS[i];
+                const uint32_t d = tmem + (i ? kColS1 : kColS0);
                 mma_ss2<0>(d, qa, hi, ka, hi, idesc_qk);
                 mma_ss2<1>(d, qa + 2, hi, ka + 2, hi, idesc_qk);
                 mma_ss2<1>(d, qa + 4, hi, ka + 4, hi, idesc_qk);
@@ -589,44 +595,42 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CU
             };
             auto issue_pv = [&](int i, int j) {
                 const uint32_t va = v_lo0 + (j % kStagesKV) * kStage;
-                const uint32_t d = tmem + colO[i], pa = tmem + colP[i];
+                const uint32_t d = tmem + (i ? kColO1 : kColO0), pa = tmem + (i ? kColP1 : kColP0);
                 const uint32_t acc0 = j > 0;
                 mma_ts2(d, pa, va, hi, idesc_pv, acc0);
 #pragma unroll
                 for (int kk = 1; kk < kBN / 16; ++kk)
                     mma_ts2(d, pa + 8 * kk, va + 128 * kk, hi, idesc_pv, 1u);
             };
-            // Waits for S_i(jn)'s K tile and for softmax i to have copied S_i(jn-1)
-            // out of tensor memory, then issues S_i(jn) for both heads.
-            auto next_scores = [&](int jn) -> bool {
-                if (!mbar_wait(&kv_full[jn % kStagesKV], (jn / kStagesKV) & 1, a.status)) return false;
-                for (int i = 0; i < 2; ++i) {
-                    if (jn > 0 && !mbar_wait(&s_free[i], (jn - 1) & 1, a.status)) return false;
-                    tc_fence_after();
-                    issue_s(i, jn);
+            bool ok = true;
+            if (warp == 1) {
+                ok = mbar_wait(&q_full, 0, a.status);
+#pragma unroll 1
+                for (int j = 0; j < nkv && ok; ++j) {
+                    if (!(ok = mbar_wait(&kv_full[j % kStagesKV], (j / kStagesKV) & 1, a.status))) break;
+#pragma unroll 1
+                    for (int i = 0; i < 2 && ok; ++i) {
+                        if (j > 0 && !(ok = mbar_wait(&s_free[i], (j - 1) & 1, a.status))) break;
+                        tc_fence_after();
+                        issue_s(i, j);
+                    }
+                    if (ok) tc_commit(&kv_empty[j % kStagesKV]);
                 }
-                return true;
-            };
-            bool ok = mbar_wait(&q_full, 0, a.status) && next_scores(0);
-            if (ok && nkv > 1) ok = next_scores(1);
-            for (int j = 0; j < nkv && ok; ++j) {
-                // P_0(j) and P_1(j) are in tensor memory.  The scores two tiles ahead
-                // go first: S_i(j+2) may overwrite S_i once softmax i has loaded
-                // S_i(j+1), which it does right after releasing P_i(j).  PV(j) is
-                // needed only at the end of softmax tile j+1, so it can wait behind.
-                ok = mbar_wait(&p_full[0], j & 1, a.status) && mbar_wait(&p_full[1], j & 1, a.status);
-                if (!ok) break;
-                if (j + 2 < nkv && !(ok = next_scores(j + 2))) break;
-                tc_fence_after();
-                issue_pv(0, j);
-                tc_commit(&pv_done[0]);
-                issue_pv(1, j);
-                tc_commit(&pv_done[1]);
-                tc_commit(&kv_empty[j % kStagesKV]);
+            } else {
+                for (int j = 0; j < nkv && ok; ++j) {
+                    if (!(ok = mbar_wait(&kv_full[j % kStagesKV], (j / kStagesKV) & 1, a.status))) break;
+                    for (int i = 0; i < 2 && ok; ++i) {
+                        if (!(ok = mbar_wait(&p_full[i], j & 1, a.status))) break;
+                        tc_fence_after();
+                        issue_pv(i, j);
+                        tc_commit(&pv_done[i]);
+                    }
+                    if (ok) tc_commit(&kv_empty[j % kStagesKV]);
+                }
             }
             // All MMAs this thread issued complete before tensor memory is freed.
-            tc_commit(&mma_done);
-            mbar_wait(&mma_done, 0, a.status);
+            tc_commit(&mma_done[warp - 1]);
+            mbar_wait(&mma_done[warp - 1], 0, a.status);
         }
       }
     } else if constexpr (kSplit == 2) {
