@@ -261,6 +261,8 @@ def run_ours(args):
         xp = W.prefill_inputs(PREFILL, dev, seed=seed)
         out_p = torch.empty_like(xp["q"])
         neff_p = torch.empty((PREFILL.B, PREFILL.Hq, PREFILL.T), device=dev)
+        ws_p = torch.empty(pa.fwd_workspace_size(PREFILL.B, PREFILL.T, PREFILL.Hq, PREFILL.Hkv),
+                           device=dev, dtype=torch.uint8)
     kv_bytes, tokens = 0.0, 0
     if do_dec:
         xd = W.decode_inputs(DECODE, dev, seed=seed)
@@ -275,7 +277,7 @@ def run_ours(args):
     def prefill():
         if not do_pre:
             return
-        pa.fwd(xp["q"], xp["k"], xp["v"], xp["u"], out_p, neff_p, stream=stream, **p)
+        pa.fwd(xp["q"], xp["k"], xp["v"], xp["u"], out_p, neff_p, ws_p, stream=stream, **p)
 
     def decode():
         if not do_dec:
@@ -370,7 +372,7 @@ def run_ours(args):
         dec_launch_s = t_dec / K
         tf = PREFILL.flops / pre_launch_s / 1e12 if do_pre else 0.0
         gbs = kv_bytes / dec_launch_s / 1e9 if do_dec else 0.0
-        sha_p = source_sha("fwd_tc.cu", "polar_common.cuh")
+        sha_p = source_sha("fwd_tc.cu", "fwd_moments.cu", "polar_common.cuh")
         sha_d = source_sha("decode.cu", "polar_common.cuh")
         value = aggregate_throughput(PREFILL.flops * K, world, t_pre_max) / 1e12 if do_pre else 0.0
         dec_value = aggregate_throughput(kv_bytes * K, world, t_dec_max) / 1e9 if do_dec else 0.0
@@ -397,12 +399,13 @@ def run_ours(args):
                        "pct_hbm_peak": 100 * gbs / peaks["hbm_gbs"],
                        "tokens_per_s": aggregate_throughput(DECODE.num_seqs * K, world,
                                                             t_dec_max) if do_dec else 0.0},
-            "roofline": {"bound": "tensor", "kernel": "fwd_tc_kernel", "achieved": tf,
+            "roofline": {"bound": "tensor", "kernel": "fwd_moments_kernel+fwd_tc_kernel",
+                         "achieved": tf,
                          "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                          "frac": tf / peaks["bf16_tflops"],
                          "frac_of_sustained": tf / peaks.get("bf16_tflops_sustained",
                                                               peaks["bf16_tflops"]),
-                         "traffic": profiled_traffic("fwd_tc_kernel", sha_p),
+                         "traffic": profiled_traffic("prefill", sha_p),
                          "peak_source": f"{peak_src} (burst cuBLAS bf16)"},
             "roofline_decode": {"bound": "hbm", "kernel": "decode_split_kernel+decode_merge_kernel",
                                 "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",

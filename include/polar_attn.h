@@ -95,19 +95,30 @@ void polar_attn_default_params(polar_params_t *p, int B, int T, int Hq, int Hkv,
  * online with O(block) memory from streaming accumulators with squared
  * correction factors; no T x T score matrix is stored).
  *
- *  q        [B, T, Hq,  64] dtype, device
- *  k, v     [B, T, Hkv, 64] dtype, device
- *  u        [Hq, 64] float32, device: the per-head count vectors u_h
- *  out      [B, T, Hq, 64] dtype, device: content + count
- *  neff_out [B, Hq, T] float32, device: n_eff per row (may be NULL)
+ *  q         [B, T, Hq,  64] dtype, device
+ *  k, v      [B, T, Hkv, 64] dtype, device
+ *  u         [Hq, 64] float32, device: the per-head count vectors u_h
+ *  out       [B, T, Hq, 64] dtype, device: content + count
+ *  neff_out  [B, Hq, T] float32, device: n_eff per row (may be NULL)
+ *  workspace device scratch of at least polar_attn_fwd_workspace_size()
+ *            bytes, or NULL (then ws_bytes is ignored).  With it, the raw
+ *            logit sums of the null floor over the key tiles left of a query
+ *            tile come from key moments (sum k, sum k k^T) that a pre-pass
+ *            writes here, instead of from every score: the same quantities,
+ *            computed faster.  Contents on entry are ignored; calls that
+ *            share a workspace must not overlap.  A non-NULL workspace smaller
+ *            than required returns POLAR_ERR_WORKSPACE.
  *
  * Returns POLAR_OK once the work is enqueued.  B = 0 or T = 0 is a no-op.
  */
+size_t polar_attn_fwd_workspace_size(const polar_params_t *params);
+
 polar_status_t polar_attn_fwd(const void *q, const void *k, const void *v, const float *u,
                               const polar_params_t *params, void *out, float *neff_out,
-                              void *stream);
+                              void *workspace, size_t ws_bytes, void *stream);
 
-/* Bytes of device staging that polar_attn_fwd_host needs for this shape. */
+/* Bytes of device staging that polar_attn_fwd_host needs for this shape
+ * (inputs, outputs and the workspace). */
 size_t polar_attn_fwd_staging_size(const polar_params_t *params);
 
 /*

@@ -6,9 +6,10 @@ the C ABI of include/polar_attn.h); ``native`` is its thin ctypes binding and
 and a missing build raises: there is no CPU or PyTorch fallback.
 """
 from .native import (decode_paged, decode_paged_host, decode_staging_size,  # noqa: F401
-                     decode_workspace_size, fwd, fwd_host, fwd_staging_size, get_status,
+                     decode_workspace_size, fwd, fwd_host, fwd_staging_size,
+                     fwd_workspace_size, get_status,
                      launch_count, PolarError)
 
-__all__ = ["fwd", "fwd_host", "fwd_staging_size", "decode_paged", "decode_paged_host",
+__all__ = ["fwd", "fwd_host", "fwd_staging_size", "fwd_workspace_size", "decode_paged", "decode_paged_host",
            "decode_staging_size", "decode_workspace_size", "get_status", "launch_count",
            "PolarError"]

@@ -83,7 +83,7 @@ FwdLaunch make_fwd(const void *q, const void *k, const void *v, const float *u,
     a.q = q; a.k = k; a.v = v; a.u = u; a.out = out; a.neff = neff;
     a.B = p->B; a.T = p->T; a.Hq = p->Hq; a.Hkv = p->Hkv; a.dtype = p->dtype;
     a.s = p->logit_scale; a.alpha = p->alpha; a.beta = p->beta; a.L = p->L_train;
-    a.status = status; a.stream = stream;
+    a.status = status; a.moments = nullptr; a.stream = stream;
     return a;
 }
 
@@ -126,20 +126,30 @@ void polar_attn_default_params(polar_params_t *p, int B, int T, int Hq, int Hkv,
     p->causal = 1; p->impl = POLAR_IMPL_AUTO;
 }
 
+size_t polar_attn_fwd_workspace_size(const polar_params_t *p) {
+    if (check_fwd(p) != POLAR_OK) return 0;
+    return fwd_moments_bytes(p->B, p->T, p->Hkv);
+}
+
 polar_status_t polar_attn_fwd(const void *q, const void *k, const void *v, const float *u,
                               const polar_params_t *params, void *out, float *neff_out,
-                              void *stream) {
+                              void *workspace, size_t ws_bytes, void *stream) {
     polar_status_t st = check_fwd(params);
     if (st != POLAR_OK) return st;
     if (params->B == 0 || params->T == 0) return POLAR_OK;
     if (!q || !k || !v || !u || !out) return POLAR_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(u) || !aligned16(out) ||
-        (neff_out && (reinterpret_cast<uintptr_t>(neff_out) & 3u)))
+        (neff_out && (reinterpret_cast<uintptr_t>(neff_out) & 3u)) ||
+        (workspace && !aligned16(workspace)))
         return POLAR_ERR_INVALID_ARG;
+    if (workspace && ws_bytes < fwd_moments_bytes(params->B, params->T, params->Hkv))
+        return POLAR_ERR_WORKSPACE;
     int *status = status_ptr();
     if (!status) return POLAR_ERR_CUDA;
     FwdLaunch a = make_fwd(q, k, v, u, params, out, neff_out, status,
                            static_cast<cudaStream_t>(stream));
+    // Key moments only where they are used: the tensor-core kernel, beyond one tile.
+    a.moments = fwd_moment_records(params->T) > 0 ? static_cast<float *>(workspace) : nullptr;
     // The tensor-core kernel pairs two query heads of one key/value group per
     // CTA, so it needs an even group size; fp32 inputs use the CUDA-core kernel.
     const bool tc_ok = params->dtype == POLAR_BF16 && (params->Hq / params->Hkv) % 2 == 0;
@@ -161,6 +171,7 @@ size_t polar_attn_fwd_staging_size(const polar_params_t *p) {
     n += round_up(static_cast<size_t>(p->Hq) * kHeadDim * 4, 256);  // u
     n += round_up(rows * p->Hq * kHeadDim * e, 256);       // out
     n += round_up(rows * p->Hq * 4, 256);                  // neff
+    n += round_up(fwd_moments_bytes(p->B, p->T, p->Hkv), 256);  // workspace
     return n;
 }
 
@@ -186,13 +197,16 @@ polar_status_t polar_attn_fwd_host(const void *q_h, const void *k_h, const void 
     char *du = dv + round_up(kb, 256);
     char *dout = du + round_up(ub, 256);
     char *dne = dout + round_up(qb, 256);
+    char *dws = dne + round_up(nb, 256);
+    const size_t wsb = fwd_moments_bytes(p->B, p->T, p->Hkv);
     if (cudaMemcpyAsync(dq, q_h, qb, cudaMemcpyHostToDevice, s) != cudaSuccess ||
         cudaMemcpyAsync(dk, k_h, kb, cudaMemcpyHostToDevice, s) != cudaSuccess ||
         cudaMemcpyAsync(dv, v_h, kb, cudaMemcpyHostToDevice, s) != cudaSuccess ||
         cudaMemcpyAsync(du, u_h, ub, cudaMemcpyHostToDevice, s) != cudaSuccess)
         return POLAR_ERR_CUDA;
     st = polar_attn_fwd(dq, dk, dv, reinterpret_cast<float *>(du), p, dout,
-                        neff_h ? reinterpret_cast<float *>(dne) : nullptr, stream);
+                        neff_h ? reinterpret_cast<float *>(dne) : nullptr,
+                        wsb ? dws : nullptr, wsb, stream);
     if (st != POLAR_OK) return st;
     if (cudaMemcpyAsync(out_h, dout, qb, cudaMemcpyDeviceToHost, s) != cudaSuccess) return POLAR_ERR_CUDA;
     if (neff_h && cudaMemcpyAsync(neff_h, dne, nb, cudaMemcpyDeviceToHost, s) != cudaSuccess)

@@ -11,13 +11,15 @@
 //
 // CTA work unit: two query heads of one key/value group over the same 128
 // query rows, so both heads share every K/V tile and have the same causal
-// extent.  Warp roles (12 warps):
+// extent.  Warp roles:
 //   warp 0      TMA producer: Q tiles once, then K/V tiles into a 4-stage ring
 //   warp 1      tensor-memory allocator and the score-MMA issuer (one thread)
 //   warp 2      the PV-MMA issuer (one thread)
-//   warp 3      idle
-//   warps 4-7   softmax warpgroup for head slot 0 (TMEM lanes 0-127)
-//   warps 8-11  softmax warpgroup for head slot 1
+//   warp 3      key moments of the keys left of the query tile (kMoments), else idle
+//   softmax     one warpgroup per head slot (warps 4-7, 8-11; TMEM lanes 0-127),
+//               or with split rows two per head slot (warps 4-11 for slot 0, the
+//               first four on keys 0-63 of each tile, the next four on 64-127;
+//               warps 12-19 for slot 1)
 // Tensor memory (512 columns): S0 S1 (128 fp32 columns each), P0 P1 (128 bf16
 // packed in 64 columns each), O0 O1 (64 fp32 columns each).
 // Two issuing threads keep the tensor core fed: one issues S_i(j) as soon as
@@ -39,7 +41,11 @@ constexpr int kBM = 128;               // query rows per head slot
 constexpr int kBN = 128;               // keys per tile
 constexpr int kStagesKV = 4;           // K/V ring depth
 constexpr int kTileBytes = 128 * 128;  // 128 rows x 64 bf16
-constexpr int kSmemBytes = (2 + 2 * kStagesKV) * kTileBytes + 1024;
+constexpr int kGramBytes = 64 * 128;   // 64 x 64 bf16, 128B-swizzled, K-major
+// The key moments pay off from this many query tiles on: below it the
+// pre-pass and the per-CTA moment epilogue cost more than they save.
+constexpr int kMomMinTiles = 32;
+constexpr int kSmemBytes = (2 + 2 * kStagesKV) * kTileBytes + 2 * kGramBytes + 256 + 1024;
 
 // Tensor-memory column map.
 constexpr uint32_t kColS0 = 0, kColS1 = 128, kColP0 = 256, kColP1 = 320, kColO0 = 384,
@@ -129,6 +135,16 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
         "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
         "%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
         : POLAR_R32(r)
+        : "r"(taddr));
+}
+
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
+        "%14,%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+          "=r"(r[14]), "=r"(r[15])
         : "r"(taddr));
 }
 
@@ -376,7 +392,7 @@ __device__ __forceinline__ void fused_tile(const uint32_t (&sr)[4][32], int t, f
 // fused_tile for a half row: 64 keys (keys 64*half .. 64*half + 63 of the
 // tile, in sr[0..1][0..31]) of one row, used when two softmax threads share a
 // row.  tlim = t - 64*half: key c of this half is visible iff c <= tlim.
-template <bool kDiag>
+template <bool kDiag, bool kMoments>
 __device__ __forceinline__ void fused_half(const uint32_t (&sr)[2][32], int tlim, float2 sc2,
                                            float neg_m, uint32_t (&pk)[2][16], float &tmax,
                                            float &ts1, float &ts2, float &tl, float &tl2) {
@@ -402,8 +418,10 @@ __device__ __forceinline__ void fused_half(const uint32_t (&sr)[2][32], int tlim
                 mx[e & 1] = max3(mx[e & 1], sv.x, sv.y);
                 x = f2_fma(sv, sc2, nm);
             }
-            a1 = f2_add(a1, sv);
-            a2 = f2_fma(sv, sv, a2);
+            if (kDiag || !kMoments) {  // full tiles: from the key moments instead
+                a1 = f2_add(a1, sv);
+                a2 = f2_fma(sv, sv, a2);
+            }
             float2 p;
             if (!kDiag && ((POLAR_TC_SPLIT_POLY_MASK >> e) & 1)) {
                 p = exp2_poly2(make_float2(fmaxf(x.x, -126.f), fmaxf(x.y, -126.f)));
@@ -433,6 +451,7 @@ struct TcArgs {
     __nv_bfloat16 *out;
     float *neff;
     int *status;
+    const float *mom;  // key-moment records (kMoments only)
     int B, T, Hq, Hkv, nqt, npairs;
     float s, alpha, L, beta, inv_ln_L;
 };
@@ -484,7 +503,15 @@ __device__ __forceinline__ void store_row(const uint32_t (&o)[2][32], float l, f
 // kSplit: softmax warpgroups per head slot.  1: one thread per row (128
 // columns; any reference).  2: two threads per row, each with 64 of the keys
 // (fixed reference only: the halves need no exchange until the epilogue).
-template <bool kFixedRef, int kSplit>
+// kMoments (split rows only): the raw sums S1, S2 of the null floor over the
+// full key tiles come from the key moments of those tiles (sum k, sum k k^T;
+// written by the moments pre-pass) instead of from every score: warp 3 adds the
+// moment records up into shared memory during the main loop, and after the last
+// score tile the score issuer computes Y_i = Q_i G on the tensor cores into the
+// free score columns, so that S2_i = <Y_i, q_i> and S1_i = <sum k, q_i>.  The
+// diagonal tile still sums its visible scores one by one.  The host uses this
+// variant from kMomMinTiles query tiles on.
+template <bool kFixedRef, int kSplit, bool kMoments>
 __global__ void __launch_bounds__(128 + 256 * kSplit, 1)
 fwd_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
               const __grid_constant__ CUtensorMap tv, const TcArgs a) {
@@ -494,14 +521,18 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CU
     uint8_t *sQ = smem;                           // 2 tiles
     uint8_t *sK = smem + 2 * kTileBytes;          // kStagesKV tiles
     uint8_t *sV = sK + kStagesKV * kTileBytes;    // kStagesKV tiles
+    uint8_t *sG = sV + kStagesKV * kTileBytes;    // key Gram, bf16 high part then low part
+    float *sKs = reinterpret_cast<float *>(sG + 2 * kGramBytes);  // key sums, 64 fp32
 
     __shared__ __align__(8) uint64_t q_full, kv_full[kStagesKV], kv_empty[kStagesKV];
     __shared__ __align__(8) uint64_t s_full[2], s_free[2], p_full[2], pv_done[2], mma_done[2];
+    __shared__ __align__(8) uint64_t g_full, y_full[2];
     __shared__ uint32_t tmem_base_sh;
     // kSplit == 2: per-row partial statistics of the upper key half
     // (m_raw, S1, S2, l, l2), handed to the lower half for the epilogue.
     __shared__ float part[kSplit == 2 ? 2 : 1][kSplit == 2 ? kBM : 1][5];
     static_assert(kSplit == 1 || kFixedRef, "split rows need the fixed reference");
+    static_assert(!kMoments || kSplit == 2, "key moments are used by the split rows only");
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -529,6 +560,9 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CU
         }
         mbar_init(&mma_done[0], 1);
         mbar_init(&mma_done[1], 1);
+        mbar_init(&g_full, 1);
+        mbar_init(&y_full[0], 1);
+        mbar_init(&y_full[1], 1);
         fence_barrier_init();
     }
     if (warp == 1) tmem_alloc_512(&tmem_base_sh);
@@ -616,6 +650,30 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CU
                     }
                     if (ok) tc_commit(&kv_empty[j % kStagesKV]);
                 }
+                if constexpr (kMoments) {
+                    // Y_i = Q_i (G_hi + G_lo) into S_i's first 64 columns, once
+                    // softmax i has copied out its last score tile.
+                    if (ok && qt >= 1) {
+                        constexpr uint32_t idesc_y = idesc_bf16(kBM, kHeadDim, false);
+                        const uint32_t gh = ((smem_u32(sG) & 0x3FFFFu) >> 4) | (1u << 16);
+                        const uint32_t gl = gh + (kGramBytes >> 4);
+                        ok = mbar_wait(&g_full, 0, a.status);
+                        for (int i = 0; i < 2 && ok; ++i) {
+                            if (!(ok = mbar_wait(&s_free[i], (nkv - 1) & 1, a.status))) break;
+                            tc_fence_after();
+                            const uint32_t qa = q_lo0 + i * kStage;
+                            const uint32_t d = tmem + (i ? kColS1 : kColS0);
+                            mma_ss2<0>(d, qa, hi, gh, hi, idesc_y);
+#pragma unroll
+                            for (int kk = 1; kk < 4; ++kk)
+                                mma_ss2<1>(d, qa + 2 * kk, hi, gh + 2 * kk, hi, idesc_y);
+#pragma unroll
+                            for (int kk = 0; kk < 4; ++kk)
+                                mma_ss2<1>(d, qa + 2 * kk, hi, gl + 2 * kk, hi, idesc_y);
+                            tc_commit(&y_full[i]);
+                        }
+                    }
+                }
             } else {
                 for (int j = 0; j < nkv && ok; ++j) {
                     if (!(ok = mbar_wait(&kv_full[j % kStagesKV], (j / kStagesKV) & 1, a.status))) break;
@@ -631,6 +689,44 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CU
             // All MMAs this thread issued complete before tensor memory is freed.
             tc_commit(&mma_done[warp - 1]);
             mbar_wait(&mma_done[warp - 1], 0, a.status);
+        }
+      } else if constexpr (kMoments) {
+        // ----------------------------------------- warp 3: key moments
+        // Moments of keys 0 .. q0-1: the records closing every chunk before
+        // tile qt-1's, plus tile qt-1's own record.  The Gram goes to shared
+        // memory as an MMA B operand (K-major, 128B-swizzled, one row of 64
+        // bf16 per d) split into a bf16 high part and the bf16 of the remainder,
+        // so that Q G_hi + Q G_lo carries the Gram to ~2^-16 relative; the key
+        // sums stay fp32.
+        if (qt >= 1) {
+            constexpr int kRec4 = kMomFloats / 4;
+            const int last = qt - 1, nclose = last / kMomChunk;
+            const float4 *rec = reinterpret_cast<const float4 *>(a.mom) +
+                                (static_cast<size_t>(b) * a.Hkv + g) * (a.nqt - 1) * kRec4;
+            for (int i = lane; i < kRec4; i += 32) {
+                float4 v = rec[static_cast<size_t>(last) * kRec4 + i];
+#pragma unroll 4
+                for (int c = 0; c < nclose; ++c) {
+                    const float4 w = rec[static_cast<size_t>((c + 1) * kMomChunk - 1) * kRec4 + i];
+                    v.x += w.x; v.y += w.y; v.z += w.z; v.w += w.w;
+                }
+                if (i < kHeadDim * kHeadDim / 4) {
+                    const int d = i >> 4, e0 = (i & 15) * 4;
+                    const uint32_t off = d * 128 + ((((e0 >> 3) ^ (d & 7))) << 4) + (e0 & 7) * 2;
+                    const uint32_t h01 = pack_bf16(v.x, v.y), h23 = pack_bf16(v.z, v.w);
+                    const uint32_t l01 = pack_bf16(v.x - __uint_as_float(h01 << 16),
+                                                   v.y - __uint_as_float(h01 & 0xFFFF0000u));
+                    const uint32_t l23 = pack_bf16(v.z - __uint_as_float(h23 << 16),
+                                                   v.w - __uint_as_float(h23 & 0xFFFF0000u));
+                    *reinterpret_cast<uint2 *>(sG + off) = make_uint2(h01, h23);
+                    *reinterpret_cast<uint2 *>(sG + kGramBytes + off) = make_uint2(l01, l23);
+                } else {
+                    reinterpret_cast<float4 *>(sKs)[i - kHeadDim * kHeadDim / 4] = v;
+                }
+            }
+            fence_proxy_async_smem();  // the tensor core reads sG through the async proxy
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&g_full);
         }
       }
     } else if constexpr (kSplit == 2) {
@@ -667,9 +763,9 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CU
             uint32_t pk[2][16];
             float tmax, ts1, ts2, tl, tl2;
             if (j == nkv - 1)
-                fused_half<true>(sr, t - 64 * half, sc2, -m_ref, pk, tmax, ts1, ts2, tl, tl2);
+                fused_half<true, kMoments>(sr, t - 64 * half, sc2, -m_ref, pk, tmax, ts1, ts2, tl, tl2);
             else
-                fused_half<false>(sr, t - 64 * half, sc2, -m_ref, pk, tmax, ts1, ts2, tl, tl2);
+                fused_half<false, kMoments>(sr, t - 64 * half, sc2, -m_ref, pk, tmax, ts1, ts2, tl, tl2);
             s1 += ts1;
             s2 += ts2;
             l += tl;
@@ -686,6 +782,47 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CU
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(&p_full[slot]);
+        }
+        if constexpr (kMoments) {
+            // Null-floor sums over the full tiles, from the key moments: this
+            // thread's 32 of the 64 components of S1 = <sum k, q>, S2 = <G q, q>.
+            if (ok && nkv > 1) {
+                // g_full orders warp 3's key-sum stores before the reads below.
+                ok = mbar_wait(&y_full[slot], 0, a.status) && mbar_wait(&g_full, 0, a.status);
+                if (__all_sync(0xffffffffu, ok)) {
+                    tc_fence_after();
+                    const uint8_t *qrow = sQ + slot * kTileBytes + t * 128;
+                    float m1 = 0.f, m2 = 0.f;
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh) {  // 16 columns at a time
+                        uint32_t y[16];
+                        tmem_ld16(lane_base + (slot ? kColS1 : kColS0) + 32 * half + 16 * hh, y);
+                        tmem_wait_ld();
+                        const float *ks = sKs + 32 * half + 16 * hh;
+#pragma unroll
+                        for (int cc = 0; cc < 2; ++cc) {
+                            const int ch = 4 * half + 2 * hh + cc;
+                            const uint4 w =
+                                *reinterpret_cast<const uint4 *>(qrow + ((ch ^ (t & 7)) << 4));
+                            const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                            for (int x = 0; x < 4; ++x) {
+                                const float qa = __uint_as_float(ww[x] << 16);
+                                const float qb = __uint_as_float(ww[x] & 0xFFFF0000u);
+                                const int e = 8 * cc + 2 * x;
+                                m2 = fmaf(__uint_as_float(y[e]), qa, m2);
+                                m2 = fmaf(__uint_as_float(y[e + 1]), qb, m2);
+                                m1 = fmaf(ks[e], qa, m1);
+                                m1 = fmaf(ks[e + 1], qb, m1);
+                            }
+                        }
+                    }
+                    s1 += m1;
+                    s2 += m2;
+                } else {
+                    ok = false;
+                }
+            }
         }
         // Combine the two halves of every row; the lower half runs the epilogue.
         if (half == 1) {
@@ -855,19 +992,26 @@ cudaError_t launch_fwd_tc(const FwdLaunch &a) {
     if (e != cudaSuccess) return e;
     const uint64_t bit = 1ull << (dev & 63);
     if (!(configured.load() & bit)) {
-        e = cudaFuncSetAttribute(fwd_tc_kernel<true, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 kSmemBytes);
+        e = cudaFuncSetAttribute(fwd_tc_kernel<true, 2, true>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
         if (e == cudaSuccess)
-            e = cudaFuncSetAttribute(fwd_tc_kernel<false, 1>,
+            e = cudaFuncSetAttribute(fwd_tc_kernel<true, 2, false>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(fwd_tc_kernel<false, 1, false>,
                                      cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
         if (e != cudaSuccess) return e;
         // setmaxnreg can only hand out the registers the block was launched with:
         // 64 for the producer/MMA warpgroup plus 104 for each of the four softmax
         // warpgroups must fit in (registers per thread at launch) x 640.
-        cudaFuncAttributes fa;
-        e = cudaFuncGetAttributes(&fa, fwd_tc_kernel<true, 2>);
+        cudaFuncAttributes fa, fb;
+        e = cudaFuncGetAttributes(&fa, fwd_tc_kernel<true, 2, true>);
+        if (e == cudaSuccess) e = cudaFuncGetAttributes(&fb, fwd_tc_kernel<true, 2, false>);
         if (e != cudaSuccess) return e;
-        if (static_cast<long long>(fa.numRegs) * 640 >= 64ll * 128 + 104ll * 512) split_ok.fetch_or(bit);
+        const long long need = 64ll * 128 + 104ll * 512;
+        if (static_cast<long long>(fa.numRegs) * 640 >= need &&
+            static_cast<long long>(fb.numRegs) * 640 >= need)
+            split_ok.fetch_or(bit);
         configured.fetch_or(bit);
     }
     // [B, T, H, 64] bf16 as a 4-D tensor (d, head, t, b); tiles of 128 rows x 64.
@@ -896,6 +1040,7 @@ cudaError_t launch_fwd_tc(const FwdLaunch &a) {
     ta.out = static_cast<__nv_bfloat16 *>(a.out);
     ta.neff = a.neff;
     ta.status = a.status;
+    ta.mom = a.moments;
     ta.B = a.B; ta.T = a.T; ta.Hq = a.Hq; ta.Hkv = a.Hkv;
     ta.nqt = (a.T + kBM - 1) / kBM;
     ta.npairs = a.Hq / 2;
@@ -909,10 +1054,18 @@ cudaError_t launch_fwd_tc(const FwdLaunch &a) {
     const float cl2_max = a.s *
                           (a.T > a.L ? 1.0f + a.alpha * logf(static_cast<float>(a.T) / a.L) : 1.0f) *
                           1.4426950408889634f;
-    if (cl2_max <= 28.0f && (split_ok.load() & bit))
-        fwd_tc_kernel<true, 2><<<static_cast<unsigned>(ctas), 640, kSmemBytes, a.stream>>>(tq, tk, tv, ta);
-    else
-        fwd_tc_kernel<false, 1><<<static_cast<unsigned>(ctas), 384, kSmemBytes, a.stream>>>(tq, tk, tv, ta);
+    const unsigned grid = static_cast<unsigned>(ctas);
+    if (cl2_max <= 28.0f && (split_ok.load() & bit)) {
+        if (a.moments && ta.nqt >= kMomMinTiles) {
+            e = launch_fwd_moments(a.k, a.B, a.T, a.Hkv, a.moments, a.stream);
+            if (e != cudaSuccess) return e;
+            fwd_tc_kernel<true, 2, true><<<grid, 640, kSmemBytes, a.stream>>>(tq, tk, tv, ta);
+        } else {
+            fwd_tc_kernel<true, 2, false><<<grid, 640, kSmemBytes, a.stream>>>(tq, tk, tv, ta);
+        }
+    } else {
+        fwd_tc_kernel<false, 1, false><<<grid, 384, kSmemBytes, a.stream>>>(tq, tk, tv, ta);
+    }
     count_launches(1);
     return cudaGetLastError();
 }

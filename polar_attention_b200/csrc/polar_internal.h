@@ -19,6 +19,7 @@ struct FwdLaunch {
     float s, alpha, beta;
     int L;
     int *status;  // device status word
+    float *moments;  // key-moment records (fwd_moments_bytes), or null
     cudaStream_t stream;
 };
 
@@ -44,6 +45,16 @@ struct DecodeLaunch {
 cudaError_t launch_fwd_simt(const FwdLaunch &a);
 cudaError_t launch_fwd_tc(const FwdLaunch &a);
 cudaError_t launch_decode(const DecodeLaunch &a);
+
+// Key moments of causal prefill (fwd_moments.cu): one record of kMomFloats
+// fp32 (the 64 x 64 key Gram, then the 64 key sums) per (batch, kv head, full
+// key tile), running sums within chunks of kMomChunk tiles.
+constexpr int kMomChunk = 8;
+constexpr int kMomFloats = 64 * 64 + 64;
+int fwd_moment_records(int T);
+size_t fwd_moments_bytes(int B, int T, int Hkv);
+cudaError_t launch_fwd_moments(const void *k, int B, int T, int Hkv, float *rec,
+                               cudaStream_t stream);
 
 // Decode work split: pages per split and the partial-state bytes it needs.
 int decode_pages_per_split(int num_seqs, int max_pages, int Hkv);

@@ -22,7 +22,8 @@ STATUS = {0: "POLAR_OK", 1: "POLAR_ERR_INVALID_ARG", 2: "POLAR_ERR_UNSUPPORTED",
           6: "POLAR_ERR_CUDA", 7: "POLAR_ERR_BAD_SEQLEN"}
 
 # Every entry point include/polar_attn.h declares.
-EXPORTS = ["polar_attn_default_params", "polar_attn_fwd", "polar_attn_fwd_staging_size",
+EXPORTS = ["polar_attn_default_params", "polar_attn_fwd_workspace_size", "polar_attn_fwd",
+           "polar_attn_fwd_staging_size",
            "polar_attn_fwd_host", "polar_attn_decode_workspace_size", "polar_attn_decode_paged",
            "polar_attn_decode_staging_size", "polar_attn_decode_paged_host",
            "polar_attn_get_status", "polar_attn_status_string", "polar_attn_launch_count",
@@ -63,7 +64,9 @@ def lib() -> ctypes.CDLL:
             PP = ctypes.POINTER(Params)
             L.polar_attn_default_params.argtypes = [PP, I, I, I, I, I]
             L.polar_attn_default_params.restype = None
-            L.polar_attn_fwd.argtypes = [P, P, P, P, PP, P, P, P]
+            L.polar_attn_fwd_workspace_size.argtypes = [PP]
+            L.polar_attn_fwd_workspace_size.restype = Z
+            L.polar_attn_fwd.argtypes = [P, P, P, P, PP, P, P, P, Z, P]
             L.polar_attn_fwd_staging_size.argtypes = [PP]
             L.polar_attn_fwd_staging_size.restype = Z
             L.polar_attn_fwd_host.argtypes = [P, P, P, P, PP, P, P, P, Z, P]
@@ -126,10 +129,17 @@ def _check(code: int, where: str):
         raise PolarError(code, where)
 
 
-def fwd(q, k, v, u, out=None, neff=None, *, s=8.0, alpha=0.3, L=2048, beta=1.0, impl="auto",
-        stream=None, want_neff=True):
+def fwd_workspace_size(B: int, T: int, Hq: int, Hkv: int) -> int:
+    p = make_params(B, T, Hq, Hkv, POLAR_BF16)
+    return int(lib().polar_attn_fwd_workspace_size(ctypes.byref(p)))
+
+
+def fwd(q, k, v, u, out=None, neff=None, workspace=None, *, s=8.0, alpha=0.3, L=2048, beta=1.0,
+        impl="auto", stream=None, want_neff=True, moments=True):
     """Causal prefill.  q [B,T,Hq,64], k/v [B,T,Hkv,64] (bf16 or fp32, CUDA,
-    contiguous), u [Hq,64] fp32.  Returns (out [B,T,Hq,64], neff [B,Hq,T])."""
+    contiguous), u [Hq,64] fp32.  Returns (out [B,T,Hq,64], neff [B,Hq,T]).
+    moments=True passes a workspace for the key-moment pre-pass (allocated
+    here when `workspace` is None); moments=False passes none."""
     B, T, Hq, D = q.shape
     Hkv = k.shape[2]
     for t in (q, k, v, u):
@@ -143,8 +153,18 @@ def fwd(q, k, v, u, out=None, neff=None, *, s=8.0, alpha=0.3, L=2048, beta=1.0, 
         neff = torch.empty((B, Hq, T), device=q.device, dtype=torch.float32)
     p = make_params(B, T, Hq, Hkv, _dt(q), s, alpha, L, beta, impl)
     p.head_dim = D
+    ws_bytes = 0
+    if moments:
+        ws_bytes = int(lib().polar_attn_fwd_workspace_size(ctypes.byref(p)))
+        if workspace is None:
+            workspace = torch.empty(max(ws_bytes, 16), device=q.device, dtype=torch.uint8)
+        else:
+            ws_bytes = workspace.numel() * workspace.element_size()
+    else:
+        workspace = None
     _check(lib().polar_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(u), ctypes.byref(p), _ptr(out),
-                                _ptr(neff), _stream(stream)), "polar_attn_fwd")
+                                _ptr(neff), _ptr(workspace), ws_bytes, _stream(stream)),
+           "polar_attn_fwd")
     return out, neff
 
 

@@ -10,11 +10,11 @@ from polar_attention_b200 import workloads as W
 pytestmark = pytest.mark.gpu
 
 
-def _run(w, x=None, impl="tc"):
+def _run(w, x=None, impl="tc", moments=True):
     x = W.prefill_inputs(w, "cpu") if x is None else x
     xd = PT.to_device(x)
     out, neff = pa.fwd(xd["q"], xd["k"], xd["v"], xd["u"], s=w.s, alpha=w.alpha, L=w.L,
-                       beta=w.beta, impl=impl)
+                       beta=w.beta, impl=impl, moments=moments)
     torch.cuda.synchronize()
     assert pa.get_status() == 0
     return x, out, neff
@@ -32,6 +32,85 @@ def test_small_all_rows(cuda_ok, T, G):
     rows = np.arange(w.B * w.Hq * w.T)
     o, n, grp = PT.gpu_rows_prefill(out, neff, rows, w.B, w.T, w.Hq)
     PT.compare(o, n, ref, grp, PT.OUT_TOL_BF16, what=f"tc T={T} G={G}")
+
+
+@pytest.mark.parametrize("T,G", [(4097, 2), (4500, 4), (4200, 8)])
+def test_moment_chunks_all_rows(cuda_ok, T, G):
+    """From 32 query tiles on, the null-floor sums over the full key tiles come
+    from the key moments, whose records run in chunks of 8 tiles: query tiles
+    1-8 read one running record, later ones add the records closing up to
+    four chunks; T=4097 ends on a one-row tile, T=4500 on a ragged chunk.
+    Every row against the oracle, GQA groups 2/4/8."""
+    w = W.small_prefill(B=1, T=T, Hq=2 * G, Hkv=2, dtype="bf16", seed=T + G, plant="frac",
+                        plant_frac=0.02, L=512)
+    x, out, neff = _run(w)
+    ref = PT.oracle_prefill(w, x)
+    rows = np.arange(w.B * w.Hq * w.T)
+    o, n, grp = PT.gpu_rows_prefill(out, neff, rows, w.B, w.T, w.Hq)
+    PT.compare(o, n, ref, grp, PT.OUT_TOL_BF16, what=f"moment chunks T={T}")
+
+
+def test_moments_agree_with_in_loop_sums(cuda_ok):
+    """The two ways of forming the null-floor sums give the same rows: n_eff
+    does not depend on them, and out moves only by their rounding."""
+    w = W.small_prefill(B=2, T=4500, Hq=4, Hkv=2, dtype="bf16", seed=5, plant="frac",
+                        plant_frac=0.01, L=512)
+    x = W.prefill_inputs(w, "cpu")
+    _, oa, na = _run(w, x, moments=True)
+    _, ob, nb = _run(w, x, moments=False)
+    assert ((na - nb).abs() / nb).amax() < 1e-6
+    err = (oa.float() - ob.float()).abs().amax() / ob.float().abs().amax()
+    assert err < 2e-3
+
+
+def test_moment_records_are_key_moments(cuda_ok):
+    """After a call the workspace holds, per (batch, kv head, full key tile t),
+    the Gram sum k k^T and the sum of k over the keys from the start of t's
+    chunk of 8 tiles through tile t (fp32, checked against fp64 sums of the
+    same bf16 keys)."""
+    w = W.small_prefill(B=2, T=4500, Hq=4, Hkv=2, dtype="bf16", seed=8)
+    x = W.prefill_inputs(w, "cpu")
+    xd = PT.to_device(x)
+    nbytes = pa.fwd_workspace_size(w.B, w.T, w.Hq, w.Hkv)
+    nrec = (w.T + 127) // 128 - 1
+    assert nbytes == w.B * w.Hkv * nrec * 4160 * 4
+    ws = torch.empty(nbytes, device="cuda", dtype=torch.uint8)
+    pa.fwd(xd["q"], xd["k"], xd["v"], xd["u"], workspace=ws, impl="tc")
+    torch.cuda.synchronize()
+    assert pa.get_status() == 0
+    rec = ws.view(torch.float32).view(w.B, w.Hkv, nrec, 4160).double().cpu().numpy()
+    k = x["k"].float().double().numpy()  # [B, T, Hkv, 64]
+    for b in range(w.B):
+        for g in range(w.Hkv):
+            for t in range(nrec):
+                lo = (t // 8) * 8 * 128
+                kk = k[b, lo:(t + 1) * 128, g, :]
+                gram = kk.T @ kk
+                scale = np.abs(gram).max()
+                assert np.abs(rec[b, g, t, :4096].reshape(64, 64) - gram).max() < 1e-5 * scale
+                ks = kk.sum(0)
+                assert np.abs(rec[b, g, t, 4096:] - ks).max() < 1e-5 * max(1.0, np.abs(ks).max())
+
+
+def test_workspace_unused_below_32_tiles(cuda_ok):
+    """Below 32 query tiles the moments do not pay off: a call with a workspace
+    gives bit-identical rows to one without."""
+    w = W.small_prefill(B=1, T=3000, Hq=4, Hkv=2, dtype="bf16", seed=6, plant="frac",
+                        plant_frac=0.01, L=512)
+    x = W.prefill_inputs(w, "cpu")
+    _, oa, na = _run(w, x, moments=True)
+    _, ob, nb = _run(w, x, moments=False)
+    assert torch.equal(oa, ob) and torch.equal(na, nb)
+
+
+def test_small_workspace_is_rejected(cuda_ok):
+    w = W.small_prefill(B=1, T=300, Hq=4, Hkv=2, dtype="bf16", seed=1)
+    xd = PT.to_device(W.prefill_inputs(w, "cpu"))
+    need = pa.fwd_workspace_size(w.B, w.T, w.Hq, w.Hkv)
+    ws = torch.empty(need - 16, device="cuda", dtype=torch.uint8)
+    with pytest.raises(pa.PolarError) as e:
+        pa.fwd(xd["q"], xd["k"], xd["v"], xd["u"], workspace=ws, impl="tc")
+    assert e.value.code == 3  # POLAR_ERR_WORKSPACE
 
 
 def test_matches_cuda_core_kernel(cuda_ok):
