@@ -166,6 +166,37 @@ polar_status_t polar_attn_decode_paged(const void *q, const void *kv_pages, int 
                                        const polar_params_t *params, void *out, float *neff_out,
                                        void *workspace, size_t ws_bytes, void *stream);
 
+/*
+ * Multi-token paged decode: `chunk` query tokens per sequence, for speculative
+ * verification or chunked prefill against the paged cache (the pages'
+ * evaluation decodes against 256K-token caches; this extends the grouped
+ * decode of section 2.2 to several queries per sequence).
+ *
+ *  q        [num_seqs, chunk, Hq, 64] dtype, device: token t of sequence s is
+ *           the query at cache position seqlen[s] - chunk + t (the chunk's own
+ *           keys and values must already be in the cache)
+ *  out      [num_seqs, chunk, Hq, 64] dtype, device
+ *  neff_out [num_seqs, chunk, Hq] float32, device (may be NULL)
+ *  other arguments as polar_attn_decode_paged.
+ *
+ * Token t sees the cache positions below n_t = seqlen - chunk + t + 1 (causal
+ * within the chunk), with the length temperature of n_t; each token's row
+ * equals polar_attn_decode_paged with seqlen n_t.  Every key/value page is read
+ * once for all chunk x (Hq/Hkv) queries of its group.  Requires chunk >= 1,
+ * (Hq/Hkv) * chunk <= 16 (else POLAR_ERR_UNSUPPORTED) and chunk <= seqlen <=
+ * 64 * max_pages per sequence (else POLAR_ERR_BAD_SEQLEN on the device, and the
+ * sequence is skipped).  chunk = 1 is polar_attn_decode_paged.
+ */
+size_t polar_attn_decode_chunk_workspace_size(int num_seqs, int max_pages, int chunk,
+                                              const polar_params_t *params);
+
+polar_status_t polar_attn_decode_paged_chunk(const void *q, const void *kv_pages, int num_pages,
+                                             const int32_t *page_table, int max_pages,
+                                             const int32_t *seqlens, int num_seqs, int chunk,
+                                             const float *u, const polar_params_t *params,
+                                             void *out, float *neff_out, void *workspace,
+                                             size_t ws_bytes, void *stream);
+
 /* Bytes of device staging that polar_attn_decode_paged_host needs. */
 size_t polar_attn_decode_staging_size(int num_seqs, int max_pages, const polar_params_t *params);
 

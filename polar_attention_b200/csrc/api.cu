@@ -74,6 +74,18 @@ polar_status_t check_decode(const polar_params_t *p, int num_seqs, int max_pages
     return POLAR_OK;
 }
 
+// Multi-token decode: every row of the mma tile is a (chunk token, query head)
+// pair of one kv group, so G * chunk rows must fit the 16 of one tile; the
+// merge grid's second dimension is num_seqs * chunk.
+polar_status_t check_decode_chunk(const polar_params_t *p, int num_seqs, int max_pages, int chunk) {
+    polar_status_t st = check_decode(p, num_seqs, max_pages);
+    if (st != POLAR_OK) return st;
+    if (chunk < 1) return POLAR_ERR_INVALID_ARG;
+    if ((p->Hq / p->Hkv) * chunk > 16) return POLAR_ERR_UNSUPPORTED;
+    if (static_cast<long long>(num_seqs) * chunk > 65535) return POLAR_ERR_UNSUPPORTED;
+    return POLAR_OK;
+}
+
 polar_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? POLAR_OK : POLAR_ERR_CUDA; }
 
 FwdLaunch make_fwd(const void *q, const void *k, const void *v, const float *u,
@@ -216,7 +228,13 @@ polar_status_t polar_attn_fwd_host(const void *q_h, const void *k_h, const void 
 
 size_t polar_attn_decode_workspace_size(int num_seqs, int max_pages, const polar_params_t *p) {
     if (check_decode(p, num_seqs, max_pages) != POLAR_OK) return 0;
-    return decode_partials_bytes(num_seqs, max_pages, p->Hq, p->Hkv);
+    return decode_partials_bytes(num_seqs, max_pages, p->Hq, p->Hkv, 1);
+}
+
+size_t polar_attn_decode_chunk_workspace_size(int num_seqs, int max_pages, int chunk,
+                                              const polar_params_t *p) {
+    if (check_decode_chunk(p, num_seqs, max_pages, chunk) != POLAR_OK) return 0;
+    return decode_partials_bytes(num_seqs, max_pages, p->Hq, p->Hkv, chunk);
 }
 
 polar_status_t polar_attn_decode_paged(const void *q, const void *kv_pages, int num_pages,
@@ -224,7 +242,18 @@ polar_status_t polar_attn_decode_paged(const void *q, const void *kv_pages, int 
                                        const int32_t *seqlens, int num_seqs, const float *u,
                                        const polar_params_t *p, void *out, float *neff_out,
                                        void *workspace, size_t ws_bytes, void *stream) {
-    polar_status_t st = check_decode(p, num_seqs, max_pages);
+    return polar_attn_decode_paged_chunk(q, kv_pages, num_pages, page_table, max_pages, seqlens,
+                                         num_seqs, 1, u, p, out, neff_out, workspace, ws_bytes,
+                                         stream);
+}
+
+polar_status_t polar_attn_decode_paged_chunk(const void *q, const void *kv_pages, int num_pages,
+                                             const int32_t *page_table, int max_pages,
+                                             const int32_t *seqlens, int num_seqs, int chunk,
+                                             const float *u, const polar_params_t *p, void *out,
+                                             float *neff_out, void *workspace, size_t ws_bytes,
+                                             void *stream) {
+    polar_status_t st = check_decode_chunk(p, num_seqs, max_pages, chunk);
     if (st != POLAR_OK) return st;
     if (num_seqs == 0) return POLAR_OK;
     if (num_pages < 1 || static_cast<long long>(num_pages) * 2 * p->Hkv * kPage > (1ll << 31) - 1)
@@ -236,11 +265,12 @@ polar_status_t polar_attn_decode_paged(const void *q, const void *kv_pages, int 
         (reinterpret_cast<uintptr_t>(seqlens) & 3u) ||
         (neff_out && (reinterpret_cast<uintptr_t>(neff_out) & 3u)))
         return POLAR_ERR_INVALID_ARG;
-    if (ws_bytes < decode_partials_bytes(num_seqs, max_pages, p->Hq, p->Hkv))
+    if (ws_bytes < decode_partials_bytes(num_seqs, max_pages, p->Hq, p->Hkv, chunk))
         return POLAR_ERR_WORKSPACE;
     int *status = status_ptr();
     if (!status) return POLAR_ERR_CUDA;
     DecodeLaunch a;
+    a.chunk = chunk;
     a.q = q; a.kv_pages = kv_pages; a.num_pages = num_pages; a.page_table = page_table;
     a.max_pages = max_pages; a.seqlens = seqlens; a.num_seqs = num_seqs; a.u = u; a.out = out;
     a.neff = neff_out; a.Hq = p->Hq; a.Hkv = p->Hkv; a.s = p->logit_scale; a.alpha = p->alpha;
@@ -259,7 +289,7 @@ size_t polar_attn_decode_staging_size(int num_seqs, int max_pages, const polar_p
     n += round_up(static_cast<size_t>(p->Hq) * kHeadDim * 4, 256);             // u
     n += round_up(static_cast<size_t>(num_seqs) * p->Hq * kHeadDim * e, 256);  // out
     n += round_up(static_cast<size_t>(num_seqs) * p->Hq * 4, 256);             // neff
-    n += round_up(decode_partials_bytes(num_seqs, max_pages, p->Hq, p->Hkv), 256);
+    n += round_up(decode_partials_bytes(num_seqs, max_pages, p->Hq, p->Hkv, 1), 256);
     return n;
 }
 
@@ -284,7 +314,7 @@ polar_status_t polar_attn_decode_paged_host(const void *q_h, const void *kv_page
     const size_t slb = static_cast<size_t>(num_seqs) * 4;
     const size_t ub = static_cast<size_t>(p->Hq) * kHeadDim * 4;
     const size_t nb = static_cast<size_t>(num_seqs) * p->Hq * 4;
-    const size_t wsb = decode_partials_bytes(num_seqs, max_pages, p->Hq, p->Hkv);
+    const size_t wsb = decode_partials_bytes(num_seqs, max_pages, p->Hq, p->Hkv, 1);
     char *dq = static_cast<char *>(staging);
     char *dpt = dq + round_up(qb, 256);
     char *dsl = dpt + round_up(ptb, 256);

@@ -42,6 +42,7 @@ struct SplitArgs {
     float *partials;
     int *status;
     int num_pages, max_pages, Hq, Hkv, pages_per_split, max_splits;
+    int chunk;  // query tokens per sequence (the last `chunk` cache positions)
     float s, alpha, L;
 };
 
@@ -62,15 +63,15 @@ __device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t (&r)[4]) {
                  : "r"(addr));
 }
 
-// d += A(16x16, rows g and g+8 of the lane) * B(16x8), bf16 in, fp32 accumulate.
-// Rows g+8 (a1, a3) are the zero padding of the query-head dimension.
-__device__ __forceinline__ void mma_bf16(float (&d)[4], uint32_t a0, uint32_t a2, uint32_t b0,
-                                         uint32_t b1) {
+// d += A(16x16; a0/a2 row g of the lane, a1/a3 row g+8) * B(16x8), bf16 in,
+// fp32 accumulate.
+__device__ __forceinline__ void mma_bf16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                         uint32_t a3, uint32_t b0, uint32_t b1) {
     asm volatile(
         "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
         "{%8,%9}, {%0,%1,%2,%3};"
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-        : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1));
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
@@ -85,30 +86,42 @@ __device__ __forceinline__ uint32_t mask_pair(uint32_t x, bool lo_ok, bool hi_ok
 }
 
 // Split kernel: CTA (split, kv head g, sequence), 4 warps.  Warp w owns tokens
-// 16w .. 16w+15 of every page and keeps, for each query head of the group
-// (mma rows; rows >= G are zero padding), the streaming state of the method:
-// reference max m_ref (log2 units), l, l2 (rescaled by r, r^2 when m_ref
-// moves past the lazy threshold), the raw-dot sums S1, S2 and max, and the
-// value accumulator O (mma accumulator fragments).  The scores S = Q K^T and
-// O += P V run on mma.sync (bf16 in, fp32 accumulate); the S fragments are
-// reused as the P operand in registers.  At the end the four warps' states are
-// merged exactly in shared memory into one partial per (split, query head).
-template <int G>
+// 16w .. 16w+15 of every page.  The mma rows carry the R = G * chunk queries of
+// the sequence that belong to kv head g: row r is query token r / G (of the
+// chunk's `chunk` tokens, the last cache positions) for query head g*G + r % G;
+// rows >= R are zero padding.  kTwo: R > 8, so rows 8-15 of the m16 tile carry
+// queries too and each lane keeps two rows' state.  Each row keeps the
+// streaming state of the method: reference max m_ref (log2 units), l, l2
+// (rescaled by r, r^2 when m_ref moves past the lazy threshold), the raw-dot
+// sums S1, S2 and max, and the value accumulator O (mma accumulator fragments).
+// Row r sees the cache positions below n_r = seqlen - chunk + r / G + 1, so a
+// chunk is causal within itself; its length temperature uses n_r.  The scores
+// S = Q K^T and O += P V run on mma.sync (bf16 in, fp32 accumulate); the S
+// fragments are reused as the P operand in registers.  At the end the four
+// warps' states are merged exactly in shared memory into one partial per
+// (split, row).
+template <int G, bool kTwo>
 __global__ void __launch_bounds__(128)
 decode_split_kernel(const __grid_constant__ CUtensorMap kv_map, const SplitArgs a) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    constexpr int kHR = kTwo ? 2 : 1;       // row sets per lane: g and g + 8
+    constexpr int kRows = 8 * kHR;
     __shared__ __align__(8) uint64_t full_bar[kStages];
-    __shared__ float mst[4][G][6];          // per warp, head: m_ref, m_raw, l, l2, S1, S2
-    __shared__ float macc[4][G][kHeadDim];  // per warp, head: O row
+    __shared__ float mst[4][kRows][6];          // per warp, row: m_ref, m_raw, l, l2, S1, S2
+    // Per warp, row: the O row, in the page ring once every page is consumed
+    // (so that three CTAs still fit per SM).
+    static_assert(4 * kRows * kHeadDim * sizeof(float) <= kStages * kStageBytes, "ring too small");
+    float(*macc)[kRows][kHeadDim] = reinterpret_cast<float(*)[kRows][kHeadDim]>(smem);
 
     const int split = blockIdx.x, g = blockIdx.y, seq = blockIdx.z;
     const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int gq = lane >> 2, tq = lane & 3;  // mma row (query head) and column pair
+    const int gq = lane >> 2, tq = lane & 3;  // mma row and column pair
+    const int C = a.chunk, R = G * C;
 
     const int seqlen = a.seqlens[seq];
-    if (seqlen < 1 || seqlen > a.max_pages * kPage) {
+    if (seqlen < C || seqlen > a.max_pages * kPage) {
         if (split == 0 && g == 0 && threadIdx.x == 0) record_error(a.status, POLAR_ERR_BAD_SEQLEN);
         return;
     }
@@ -145,22 +158,33 @@ decode_split_kernel(const __grid_constant__ CUtensorMap kv_map, const SplitArgs 
     if (threadIdx.x == 0)
         for (int kk = 0; kk < min(kStages, np); ++kk) issue(kk);
 
-    // Query fragments (A operand of S = Q K^T): row gq = query head g*G + gq.
-    const bool real = gq < G;
-    uint32_t qa[4][2];
-    {
+    // Per row set: query fragments (A operand of S = Q K^T), the visible
+    // positions n_r and the row's exponent scale.
+    uint32_t qa[kHR][4][2];
+    int lim[kHR];
+    float cl2[kHR];
+#pragma unroll
+    for (int hr = 0; hr < kHR; ++hr) {
+        const int r = gq + 8 * hr;
+        const bool real = r < R;
+        const int t = real ? r / G : 0, hh = real ? r % G : 0;
         const uint32_t *qrow = reinterpret_cast<const uint32_t *>(
-            a.q + (static_cast<size_t>(seq) * a.Hq + g * G + (real ? gq : 0)) * kHeadDim);
+            a.q + ((static_cast<size_t>(seq) * C + t) * a.Hq + g * G + hh) * kHeadDim);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
-            qa[kk][0] = real ? __ldg(qrow + 8 * kk + tq) : 0u;
-            qa[kk][1] = real ? __ldg(qrow + 8 * kk + 4 + tq) : 0u;
+            qa[hr][kk][0] = real ? __ldg(qrow + 8 * kk + tq) : 0u;
+            qa[hr][kk][1] = real ? __ldg(qrow + 8 * kk + 4 + tq) : 0u;
         }
+        lim[hr] = seqlen - C + t + 1;
+        cl2[hr] = a.s * length_temperature(static_cast<float>(lim[hr]), a.alpha, a.L) * kLog2e;
     }
-    const float n = static_cast<float>(seqlen);
-    const float cl2 = a.s * length_temperature(n, a.alpha, a.L) * kLog2e;
 
-    float m_ref = -INFINITY, m_raw = -INFINITY, l = 0.f, l2 = 0.f, s1 = 0.f, s2 = 0.f;
+    float m_ref[kHR], m_raw[kHR], l[kHR], l2[kHR], s1[kHR], s2[kHR];
+#pragma unroll
+    for (int hr = 0; hr < kHR; ++hr) {
+        m_ref[hr] = m_raw[hr] = -INFINITY;
+        l[hr] = l2[hr] = s1[hr] = s2[hr] = 0.f;
+    }
     float acc[8][4];
 #pragma unroll
     for (int i = 0; i < 8; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
@@ -190,51 +214,59 @@ decode_split_kernel(const __grid_constant__ CUtensorMap kv_map, const SplitArgs 
                 ldsm_x4(kb + swz(tok, 4 + (lane >> 3)), b[1]);
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks)
-                    mma_bf16(sc[nt], qa[ks][0], qa[ks][1], b[ks >> 1][2 * (ks & 1)],
+                    mma_bf16(sc[nt], qa[0][ks][0], kTwo ? qa[kHR - 1][ks][0] : 0u, qa[0][ks][1],
+                             kTwo ? qa[kHR - 1][ks][1] : 0u, b[ks >> 1][2 * (ks & 1)],
                              b[ks >> 1][2 * (ks & 1) + 1]);
             }
-            // Streaming statistics of the valid tokens (rows gq; c0/c1 of each n-tile).
-            bool vld[2][2];
-            float tmax = -INFINITY, ts1 = 0.f, ts2 = 0.f;
+            // Streaming statistics of each row's visible positions (elements
+            // 2hr, 2hr+1 of each n-tile belong to row set hr).
+            uint32_t pa[kHR][2];
 #pragma unroll
-            for (int nt = 0; nt < 2; ++nt)
+            for (int hr = 0; hr < kHR; ++hr) {
+                const int pos0 = page * kPage + 16 * w + 2 * tq;
+                bool vld[2][2];
+                float tmax = -INFINITY, ts1 = 0.f, ts2 = 0.f;
 #pragma unroll
-                for (int e = 0; e < 2; ++e) {
-                    vld[nt][e] = 16 * w + 8 * nt + 2 * tq + e < ntok;
-                    const float x = sc[nt][e];
-                    tmax = fmaxf(tmax, vld[nt][e] ? x : -INFINITY);
-                    ts1 += vld[nt][e] ? x : 0.f;
-                    ts2 += vld[nt][e] ? x * x : 0.f;
+                for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        vld[nt][e] = pos0 + 8 * nt + e < lim[hr];
+                        const float x = sc[nt][2 * hr + e];
+                        tmax = fmaxf(tmax, vld[nt][e] ? x : -INFINITY);
+                        ts1 += vld[nt][e] ? x : 0.f;
+                        ts2 += vld[nt][e] ? x * x : 0.f;
+                    }
+                tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 1));
+                tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 2));
+                s1[hr] += ts1;
+                s2[hr] += ts2;
+                m_raw[hr] = fmaxf(m_raw[hr], tmax);
+                const float zmax = tmax * cl2[hr];
+                if (zmax > m_ref[hr] + kRescaleThreshold) {  // uniform over the quad of the row
+                    const float r = exp2f(m_ref[hr] - zmax);
+                    l[hr] *= r;
+                    l2[hr] *= r * r;
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        acc[i][2 * hr] *= r;
+                        acc[i][2 * hr + 1] *= r;
+                    }
+                    m_ref[hr] = zmax;
                 }
-            tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 1));
-            tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 2));
-            s1 += ts1;
-            s2 += ts2;
-            m_raw = fmaxf(m_raw, tmax);
-            const float zmax = tmax * cl2;
-            if (zmax > m_ref + kRescaleThreshold) {  // uniform over the quad of row gq
-                const float r = exp2f(m_ref - zmax);
-                l *= r;
-                l2 *= r * r;
+                float pv[2][2];
 #pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    acc[i][0] *= r;
-                    acc[i][1] *= r;
-                }
-                m_ref = zmax;
+                for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        const float pp =
+                            vld[nt][e] ? exp2f(fmaf(sc[nt][2 * hr + e], cl2[hr], -m_ref[hr])) : 0.f;
+                        pv[nt][e] = pp;
+                        l[hr] += pp;
+                        l2[hr] = fmaf(pp, pp, l2[hr]);
+                    }
+                pa[hr][0] = pack_bf16x2(pv[0][0], pv[0][1]);
+                pa[hr][1] = pack_bf16x2(pv[1][0], pv[1][1]);
             }
-            float pv[2][2];
-#pragma unroll
-            for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-                for (int e = 0; e < 2; ++e) {
-                    const float pp = vld[nt][e] ? exp2f(fmaf(sc[nt][e], cl2, -m_ref)) : 0.f;
-                    pv[nt][e] = pp;
-                    l += pp;
-                    l2 = fmaf(pp, pp, l2);
-                }
-            const uint32_t pa0 = pack_bf16x2(pv[0][0], pv[0][1]);
-            const uint32_t pa2 = pack_bf16x2(pv[1][0], pv[1][1]);
             // O += P V: V^T fragments by transposed ldmatrix; tokens past the end
             // of the sequence are zeroed so no stale value can enter the sum.
             const bool last = ntok < kPage;
@@ -250,8 +282,10 @@ decode_split_kernel(const __grid_constant__ CUtensorMap kv_map, const SplitArgs 
                     v[2] = mask_pair(v[2], t0 < ntok, t0 + 1 < ntok);
                     v[3] = mask_pair(v[3], t0 + 8 < ntok, t0 + 9 < ntok);
                 }
-                mma_bf16(acc[2 * i], pa0, pa2, v[0], v[1]);
-                mma_bf16(acc[2 * i + 1], pa0, pa2, v[2], v[3]);
+                mma_bf16(acc[2 * i], pa[0][0], kTwo ? pa[kHR - 1][0] : 0u, pa[0][1],
+                         kTwo ? pa[kHR - 1][1] : 0u, v[0], v[1]);
+                mma_bf16(acc[2 * i + 1], pa[0][0], kTwo ? pa[kHR - 1][0] : 0u, pa[0][1],
+                         kTwo ? pa[kHR - 1][1] : 0u, v[2], v[3]);
             }
         }
         __syncthreads();  // every warp is done with stage st
@@ -269,51 +303,56 @@ decode_split_kernel(const __grid_constant__ CUtensorMap kv_map, const SplitArgs 
 
     // Reduce the quad of each row, then merge the four warps exactly.
 #pragma unroll
-    for (int o = 1; o <= 2; o <<= 1) {
-        l += __shfl_xor_sync(0xffffffffu, l, o);
-        l2 += __shfl_xor_sync(0xffffffffu, l2, o);
-        s1 += __shfl_xor_sync(0xffffffffu, s1, o);
-        s2 += __shfl_xor_sync(0xffffffffu, s2, o);
-        m_raw = fmaxf(m_raw, __shfl_xor_sync(0xffffffffu, m_raw, o));
-    }
-    if (real) {
-        if (tq == 0) {
-            mst[w][gq][0] = m_ref;
-            mst[w][gq][1] = m_raw;
-            mst[w][gq][2] = l;
-            mst[w][gq][3] = l2;
-            mst[w][gq][4] = s1;
-            mst[w][gq][5] = s2;
-        }
+    for (int hr = 0; hr < kHR; ++hr) {
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            macc[w][gq][8 * i + 2 * tq] = acc[i][0];
-            macc[w][gq][8 * i + 2 * tq + 1] = acc[i][1];
+        for (int o = 1; o <= 2; o <<= 1) {
+            l[hr] += __shfl_xor_sync(0xffffffffu, l[hr], o);
+            l2[hr] += __shfl_xor_sync(0xffffffffu, l2[hr], o);
+            s1[hr] += __shfl_xor_sync(0xffffffffu, s1[hr], o);
+            s2[hr] += __shfl_xor_sync(0xffffffffu, s2[hr], o);
+            m_raw[hr] = fmaxf(m_raw[hr], __shfl_xor_sync(0xffffffffu, m_raw[hr], o));
+        }
+        const int r = gq + 8 * hr;
+        if (r < R) {
+            if (tq == 0) {
+                mst[w][r][0] = m_ref[hr];
+                mst[w][r][1] = m_raw[hr];
+                mst[w][r][2] = l[hr];
+                mst[w][r][3] = l2[hr];
+                mst[w][r][4] = s1[hr];
+                mst[w][r][5] = s2[hr];
+            }
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                macc[w][r][8 * i + 2 * tq] = acc[i][2 * hr];
+                macc[w][r][8 * i + 2 * tq + 1] = acc[i][2 * hr + 1];
+            }
         }
     }
     __syncthreads();
-    for (int hh = w; hh < G; hh += 4) {
+    for (int r = w; r < R; r += 4) {
         float M = -INFINITY;
 #pragma unroll
-        for (int ww = 0; ww < 4; ++ww) M = fmaxf(M, mst[ww][hh][0]);
-        float r[4];
+        for (int ww = 0; ww < 4; ++ww) M = fmaxf(M, mst[ww][r][0]);
+        float rr[4];
 #pragma unroll
-        for (int ww = 0; ww < 4; ++ww) r[ww] = M == -INFINITY ? 0.f : exp2f(mst[ww][hh][0] - M);
+        for (int ww = 0; ww < 4; ++ww) rr[ww] = M == -INFINITY ? 0.f : exp2f(mst[ww][r][0] - M);
         float2 o = make_float2(0.f, 0.f);
         float ml = 0.f, ml2 = 0.f, ms1 = 0.f, ms2 = 0.f, mraw = -INFINITY;
 #pragma unroll
         for (int ww = 0; ww < 4; ++ww) {
-            o.x = fmaf(macc[ww][hh][2 * lane], r[ww], o.x);
-            o.y = fmaf(macc[ww][hh][2 * lane + 1], r[ww], o.y);
-            ml = fmaf(mst[ww][hh][2], r[ww], ml);
-            ml2 = fmaf(mst[ww][hh][3], r[ww] * r[ww], ml2);
-            ms1 += mst[ww][hh][4];
-            ms2 += mst[ww][hh][5];
-            mraw = fmaxf(mraw, mst[ww][hh][1]);
+            o.x = fmaf(macc[ww][r][2 * lane], rr[ww], o.x);
+            o.y = fmaf(macc[ww][r][2 * lane + 1], rr[ww], o.y);
+            ml = fmaf(mst[ww][r][2], rr[ww], ml);
+            ml2 = fmaf(mst[ww][r][3], rr[ww] * rr[ww], ml2);
+            ms1 += mst[ww][r][4];
+            ms2 += mst[ww][r][5];
+            mraw = fmaxf(mraw, mst[ww][r][1]);
         }
-        const int h = g * G + hh;
+        const int t = r / G, h = g * G + r % G;
         float *dst = a.partials +
-                     ((static_cast<size_t>(seq) * a.Hq + h) * a.max_splits + split) * kPartialFloats;
+                     (((static_cast<size_t>(seq) * C + t) * a.Hq + h) * a.max_splits + split) *
+                         kPartialFloats;
         reinterpret_cast<float2 *>(dst)[lane] = o;
         if (lane == 0) {
             reinterpret_cast<float4 *>(dst + 64)[0] = make_float4(M, mraw, ml, ml2);
@@ -322,19 +361,21 @@ decode_split_kernel(const __grid_constant__ CUtensorMap kv_map, const SplitArgs 
     }
 }
 
-// Exact merge of the split partials of one (sequence, query head) and the
-// epilogue.  One warp; lane owns columns 2*lane and 2*lane + 1.
+// Exact merge of the split partials of one (sequence, chunk token, query head)
+// and the epilogue.  One warp; lane owns columns 2*lane and 2*lane + 1.
 __global__ void __launch_bounds__(32)
 decode_merge_kernel(const float *__restrict__ partials, const int32_t *__restrict__ seqlens,
                     const float *__restrict__ u, __nv_bfloat16 *__restrict__ out,
-                    float *__restrict__ neff_out, int Hq, int max_pages, int pages_per_split,
-                    int max_splits, float s, float alpha, float L, float beta, float inv_ln_L) {
-    const int h = blockIdx.x, seq = blockIdx.y, lane = threadIdx.x;
+                    float *__restrict__ neff_out, int Hq, int chunk, int max_pages,
+                    int pages_per_split, int max_splits, float s, float alpha, float L, float beta,
+                    float inv_ln_L) {
+    const int h = blockIdx.x, row = blockIdx.y, lane = threadIdx.x;  // row = seq * chunk + token
+    const int seq = row / chunk, tok = row % chunk;
     const int seqlen = seqlens[seq];
-    if (seqlen < 1 || seqlen > max_pages * kPage) return;  // reported by the split kernel
+    if (seqlen < chunk || seqlen > max_pages * kPage) return;  // reported by the split kernel
     const int npg = (seqlen + kPage - 1) / kPage;
     const int nsplit = (npg + pages_per_split - 1) / pages_per_split;
-    const float *base = partials + (static_cast<size_t>(seq) * Hq + h) * max_splits * kPartialFloats;
+    const float *base = partials + (static_cast<size_t>(row) * Hq + h) * max_splits * kPartialFloats;
 
     float M = -INFINITY;
     for (int sp = lane; sp < nsplit; sp += 32) M = fmaxf(M, base[sp * kPartialFloats + 64]);
@@ -355,7 +396,7 @@ decode_merge_kernel(const float *__restrict__ partials, const int32_t *__restric
         s2 += ss.y;
         m_raw = fmaxf(m_raw, st.y);
     }
-    const float n = static_cast<float>(seqlen);
+    const float n = static_cast<float>(seqlen - chunk + tok + 1);  // positions this token sees
     const float c = s * length_temperature(n, alpha, L);
     float ne;
     const float mag = polar_magnitude(l, l2, m_raw, s1, s2, c, n, beta, inv_ln_L, &ne);
@@ -363,11 +404,11 @@ decode_merge_kernel(const float *__restrict__ partials, const int32_t *__restric
     const float inv = 1.0f / fmaxf(nrm, 1e-30f);
     const float2 uu = reinterpret_cast<const float2 *>(u + static_cast<size_t>(h) * kHeadDim)[lane];
     const __nv_bfloat162 o = __floats2bfloat162_rn(fmaf(mag, uu.x, a0 * inv), fmaf(mag, uu.y, a1 * inv));
-    reinterpret_cast<__nv_bfloat162 *>(out + (static_cast<size_t>(seq) * Hq + h) * kHeadDim)[lane] = o;
-    if (neff_out && lane == 0) neff_out[static_cast<size_t>(seq) * Hq + h] = ne;
+    reinterpret_cast<__nv_bfloat162 *>(out + (static_cast<size_t>(row) * Hq + h) * kHeadDim)[lane] = o;
+    if (neff_out && lane == 0) neff_out[static_cast<size_t>(row) * Hq + h] = ne;
 }
 
-template <int G>
+template <int G, bool kTwo>
 cudaError_t launch_split(const CUtensorMap &map, const SplitArgs &sa, int num_seqs,
                          cudaStream_t stream) {
     static std::atomic<uint64_t> configured{0};  // one bit per device
@@ -376,14 +417,21 @@ cudaError_t launch_split(const CUtensorMap &map, const SplitArgs &sa, int num_se
     if (e != cudaSuccess) return e;
     const uint64_t bit = 1ull << (dev & 63);
     if (!(configured.load() & bit)) {
-        e = cudaFuncSetAttribute(decode_split_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 kSplitSmem);
+        e = cudaFuncSetAttribute(decode_split_kernel<G, kTwo>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, kSplitSmem);
         if (e != cudaSuccess) return e;
         configured.fetch_or(bit);
     }
     dim3 grid(sa.max_splits, sa.Hkv, num_seqs);
-    decode_split_kernel<G><<<grid, 128, kSplitSmem, stream>>>(map, sa);
+    decode_split_kernel<G, kTwo><<<grid, 128, kSplitSmem, stream>>>(map, sa);
     return cudaGetLastError();
+}
+
+template <int G>
+cudaError_t launch_split_rows(const CUtensorMap &map, const SplitArgs &sa, int num_seqs,
+                              cudaStream_t stream) {
+    return G * sa.chunk > 8 ? launch_split<G, true>(map, sa, num_seqs, stream)
+                            : launch_split<G, false>(map, sa, num_seqs, stream);
 }
 
 }  // namespace
@@ -398,10 +446,10 @@ int decode_pages_per_split(int num_seqs, int max_pages, int Hkv) {
     return pps;
 }
 
-size_t decode_partials_bytes(int num_seqs, int max_pages, int Hq, int Hkv) {
+size_t decode_partials_bytes(int num_seqs, int max_pages, int Hq, int Hkv, int chunk) {
     const int pps = decode_pages_per_split(num_seqs, max_pages, Hkv);
     const size_t max_splits = (static_cast<size_t>(max_pages) + pps - 1) / pps;
-    return static_cast<size_t>(num_seqs) * Hq * max_splits * kPartialFloats * sizeof(float);
+    return static_cast<size_t>(num_seqs) * chunk * Hq * max_splits * kPartialFloats * sizeof(float);
 }
 
 cudaError_t launch_decode(const DecodeLaunch &a) {
@@ -420,21 +468,22 @@ cudaError_t launch_decode(const DecodeLaunch &a) {
 
     SplitArgs sa{a.page_table, a.seqlens, static_cast<const __nv_bfloat16 *>(a.q),
                  static_cast<float *>(a.workspace), a.status, a.num_pages, a.max_pages, a.Hq, a.Hkv,
-                 pps, max_splits, a.s, a.alpha, static_cast<float>(a.L)};
+                 pps, max_splits, a.chunk, a.s, a.alpha, static_cast<float>(a.L)};
+    if (a.chunk < 1 || G * a.chunk > 16) return cudaErrorInvalidValue;
     cudaError_t e;
     switch (G) {
-        case 1: e = launch_split<1>(map, sa, a.num_seqs, a.stream); break;
-        case 2: e = launch_split<2>(map, sa, a.num_seqs, a.stream); break;
-        case 4: e = launch_split<4>(map, sa, a.num_seqs, a.stream); break;
-        case 8: e = launch_split<8>(map, sa, a.num_seqs, a.stream); break;
+        case 1: e = launch_split_rows<1>(map, sa, a.num_seqs, a.stream); break;
+        case 2: e = launch_split_rows<2>(map, sa, a.num_seqs, a.stream); break;
+        case 4: e = launch_split_rows<4>(map, sa, a.num_seqs, a.stream); break;
+        case 8: e = launch_split_rows<8>(map, sa, a.num_seqs, a.stream); break;
         default: return cudaErrorInvalidValue;
     }
     if (e != cudaSuccess) return e;
-    dim3 mgrid(a.Hq, a.num_seqs);
+    dim3 mgrid(a.Hq, a.num_seqs * a.chunk);
     decode_merge_kernel<<<mgrid, 32, 0, a.stream>>>(
         static_cast<const float *>(a.workspace), a.seqlens, a.u, static_cast<__nv_bfloat16 *>(a.out),
-        a.neff, a.Hq, a.max_pages, pps, max_splits, a.s, a.alpha, static_cast<float>(a.L), a.beta,
-        1.0f / logf(static_cast<float>(a.L)));
+        a.neff, a.Hq, a.chunk, a.max_pages, pps, max_splits, a.s, a.alpha,
+        static_cast<float>(a.L), a.beta, 1.0f / logf(static_cast<float>(a.L)));
     count_launches(2);
     return cudaGetLastError();
 }

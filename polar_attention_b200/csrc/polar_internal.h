@@ -37,6 +37,7 @@ struct DecodeLaunch {
     float s, alpha, beta;
     int L;
     void *workspace;
+    int chunk;  // query tokens per sequence (1 for plain decode)
     int *status;
     cudaStream_t stream;
 };
@@ -58,7 +59,7 @@ cudaError_t launch_fwd_moments(const void *k, int B, int T, int Hkv, float *rec,
 
 // Decode work split: pages per split and the partial-state bytes it needs.
 int decode_pages_per_split(int num_seqs, int max_pages, int Hkv);
-size_t decode_partials_bytes(int num_seqs, int max_pages, int Hq, int Hkv);
+size_t decode_partials_bytes(int num_seqs, int max_pages, int Hq, int Hkv, int chunk);
 
 // Bookkeeping shared by the launchers.
 void count_launches(int n);

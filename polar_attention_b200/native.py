@@ -27,7 +27,8 @@ EXPORTS = ["polar_attn_default_params", "polar_attn_fwd_workspace_size", "polar_
            "polar_attn_fwd_host", "polar_attn_decode_workspace_size", "polar_attn_decode_paged",
            "polar_attn_decode_staging_size", "polar_attn_decode_paged_host",
            "polar_attn_get_status", "polar_attn_status_string", "polar_attn_launch_count",
-           "polar_attn_decode_paged_noalloc", "polar_attn_selftest_exp2"]
+           "polar_attn_decode_paged_noalloc", "polar_attn_selftest_exp2",
+           "polar_attn_decode_chunk_workspace_size", "polar_attn_decode_paged_chunk"]
 
 
 class PolarError(RuntimeError):
@@ -73,6 +74,9 @@ def lib() -> ctypes.CDLL:
             L.polar_attn_decode_workspace_size.argtypes = [I, I, PP]
             L.polar_attn_decode_workspace_size.restype = Z
             L.polar_attn_decode_paged.argtypes = [P, P, I, P, I, P, I, P, PP, P, P, P, Z, P]
+            L.polar_attn_decode_chunk_workspace_size.argtypes = [I, I, I, PP]
+            L.polar_attn_decode_chunk_workspace_size.restype = Z
+            L.polar_attn_decode_paged_chunk.argtypes = [P, P, I, P, I, P, I, I, P, PP, P, P, P, Z, P]
             L.polar_attn_decode_staging_size.argtypes = [I, I, PP]
             L.polar_attn_decode_staging_size.restype = Z
             L.polar_attn_decode_paged_host.argtypes = [P, P, I, P, I, P, I, P, PP, P, P, P, Z, P]
@@ -84,7 +88,8 @@ def lib() -> ctypes.CDLL:
             L.polar_attn_launch_count.restype = ctypes.c_uint64
             for name in ("polar_attn_fwd", "polar_attn_fwd_host", "polar_attn_decode_paged",
                          "polar_attn_decode_paged_host", "polar_attn_get_status",
-                         "polar_attn_decode_paged_noalloc", "polar_attn_selftest_exp2"):
+                         "polar_attn_decode_paged_noalloc", "polar_attn_selftest_exp2",
+                         "polar_attn_decode_paged_chunk"):
                 getattr(L, name).restype = I
             _lib = L
     return _lib
@@ -196,6 +201,39 @@ def decode_paged(q, kv_pages, page_table, seqlens, u, out=None, neff=None, works
         _ptr(q), _ptr(kv_pages), P_, _ptr(page_table), max_pages, _ptr(seqlens), N, _ptr(u),
         ctypes.byref(p), _ptr(out), _ptr(neff), _ptr(workspace), workspace.numel(),
         _stream(stream)), "polar_attn_decode_paged")
+    return out, neff
+
+
+def decode_chunk_workspace_size(num_seqs: int, max_pages: int, chunk: int, Hq: int,
+                                Hkv: int) -> int:
+    p = make_params(0, 0, Hq, Hkv, POLAR_BF16)
+    return int(lib().polar_attn_decode_chunk_workspace_size(num_seqs, max_pages, chunk,
+                                                            ctypes.byref(p)))
+
+
+def decode_paged_chunk(q, kv_pages, page_table, seqlens, u, out=None, neff=None, workspace=None,
+                       *, s=8.0, alpha=0.3, L=2048, beta=1.0, stream=None, want_neff=True):
+    """Multi-token paged decode.  q [N,C,Hq,64] bf16: token t of sequence n is
+    the query at cache position seqlens[n] - C + t.  Returns (out [N,C,Hq,64],
+    neff [N,C,Hq])."""
+    N, C, Hq, D = q.shape
+    P_, _, Hkv, _, _ = kv_pages.shape
+    max_pages = page_table.shape[1]
+    if page_table.dtype != torch.int32 or seqlens.dtype != torch.int32:
+        raise TypeError("page_table and seqlens must be int32")
+    p = make_params(0, 0, Hq, Hkv, _dt(q), s, alpha, L, beta)
+    p.head_dim = D
+    ws_need = int(lib().polar_attn_decode_chunk_workspace_size(N, max_pages, C, ctypes.byref(p)))
+    if workspace is None:
+        workspace = torch.empty(max(ws_need, 16), device=q.device, dtype=torch.uint8)
+    if out is None:
+        out = torch.empty_like(q)
+    if neff is None and want_neff:
+        neff = torch.empty((N, C, Hq), device=q.device, dtype=torch.float32)
+    _check(lib().polar_attn_decode_paged_chunk(
+        _ptr(q), _ptr(kv_pages), P_, _ptr(page_table), max_pages, _ptr(seqlens), N, C, _ptr(u),
+        ctypes.byref(p), _ptr(out), _ptr(neff), _ptr(workspace), workspace.numel(),
+        _stream(stream)), "polar_attn_decode_paged_chunk")
     return out, neff
 
 

@@ -209,6 +209,20 @@ def decode_inputs(w: DecodeWorkload, device="cpu", seed: int | None = None,
             "u": u, "num_pages": P, "max_pages": max_pages}
 
 
+def decode_chunk_queries(w: DecodeWorkload, x: dict, chunk: int, seed: int | None = None) -> torch.Tensor:
+    """Queries of a multi-token decode: q [N, chunk, Hq, D], unit rows.  The
+    last token of each sequence is the single-token decode query x["q"] (whose
+    planted keys sit in the cache); the earlier tokens are fresh random rows."""
+    q1 = x["q"]
+    N = q1.shape[0]
+    g = _gen(q1.device, (w.seed if seed is None else seed) + 7)
+    fresh = _unit(torch.randn((N, chunk, w.Hq, w.D), generator=g, device=q1.device,
+                              dtype=torch.float32))
+    q = _cast(fresh, w.dtype).clone()
+    q[:, chunk - 1] = q1
+    return q.contiguous()
+
+
 def small_prefill(B=1, T=300, Hq=4, Hkv=2, D=64, dtype="fp32", seed=0, **kw) -> PrefillWorkload:
     return PrefillWorkload(f"custom_B{B}_T{T}_H{Hq}x{Hkv}", B=B, T=T, Hq=Hq, Hkv=Hkv, D=D,
                            dtype=dtype, seed=seed, **kw)

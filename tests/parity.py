@@ -37,6 +37,20 @@ def oracle_decode(w, x, rows=None):
                                x["u"].detach().cpu().numpy(), oracle_params(w), rows=rows)
 
 
+def oracle_decode_chunk(w, x, q, rows=None):
+    """Oracle of a multi-token decode: token t of sequence n is a single-token
+    decode of its own query with seqlen n_t = seqlens[n] - C + t + 1 over the
+    same page table (one virtual sequence per token).  Rows are flat
+    ((n*C + t)*Hq + h), matching out.reshape(-1, D)."""
+    N, C = q.shape[0], q.shape[1]
+    lens = x["seqlens"].cpu().numpy().astype(np.int64)
+    vlens = (lens[:, None] - C + np.arange(C)[None, :] + 1).reshape(-1).astype(np.int32)
+    vpt = np.repeat(x["page_table"].cpu().numpy(), C, axis=0)
+    qv = W.to_host_bits(q.reshape(N * C, q.shape[2], q.shape[3]))
+    return oracle.polar_decode(qv, W.to_host_bits(x["kv_pages"]), vpt, vlens,
+                               x["u"].detach().cpu().numpy(), oracle_params(w), rows=rows)
+
+
 def gpu_rows_prefill(out, neff, rows, B, T, Hq):
     """Gather flat oracle rows ((b*Hq + h)*T + i) from GPU out [B,T,Hq,D] and
     neff [B,Hq,T]."""
