@@ -62,6 +62,9 @@ def parse_args(argv=None):
                     help="prefill workload (profiling runs use a smaller one)")
     ap.add_argument("--decode-seqs", type=int, default=W.DECODE.num_seqs,
                     help="decode sequences (profiling runs use fewer)")
+    ap.add_argument("--chunk", type=int, default=4,
+                    help="query tokens per sequence of the separately timed multi-token decode "
+                         "(0 skips it)")
     return ap.parse_args(argv)
 
 
@@ -318,6 +321,38 @@ def run_ours(args):
 
     t_pre = sum(ev[i][0].elapsed_time(ev[i][1]) for i in range(K)) / 1e3
     t_dec = sum(ev[i][1].elapsed_time(ev[i][2]) for i in range(K)) / 1e3
+
+    # ---- multi-token decode (chunk query tokens per sequence), timed on its own ----
+    chunk_res = None
+    if do_dec and args.chunk > 1:
+        C = args.chunk
+        qc = W.decode_chunk_queries(DECODE, xd, C, seed=seed)
+        out_c = torch.empty_like(qc)
+        neff_c = torch.empty((DECODE.num_seqs, C, DECODE.Hq), device=dev)
+        ws_c = torch.empty(pa.decode_chunk_workspace_size(DECODE.num_seqs, xd["max_pages"], C,
+                                                          DECODE.Hq, DECODE.Hkv),
+                           device=dev, dtype=torch.uint8)
+
+        def chunk_decode():
+            pa.decode_paged_chunk(qc, xd["kv_pages"], xd["page_table"], xd["seqlens"], xd["u"],
+                                  out_c, neff_c, ws_c, stream=stream, **p)
+
+        for _ in range(Wm):
+            chunk_decode()
+        torch.cuda.synchronize(dev)
+        ec = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
+        barrier(world, dev)
+        torch.cuda.synchronize(dev)
+        for i in range(K):
+            ec[i][0].record(stream)
+            chunk_decode()
+            ec[i][1].record(stream)
+        torch.cuda.synchronize(dev)
+        barrier(world, dev)
+        if pa.get_status() != 0:
+            raise RuntimeError("device status after the multi-token decode")
+        t_chunk = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in ec) / 1e3, world, dev)
+        chunk_res = (C, t_chunk)
     t_all = outer[0].elapsed_time(outer[1]) / 1e3
     t_pre_max = max_over_ranks(t_pre, world, dev)
     t_dec_max = max_over_ranks(t_dec, world, dev)
@@ -416,6 +451,21 @@ def run_ours(args):
             "clocks": clk.summary(),
             "e2e": e2e,
         }
+        if chunk_res is not None:
+            C, t_chunk = chunk_res
+            c_launch = t_chunk / K
+            c_gbs = kv_bytes / c_launch / 1e9
+            result["decode_chunk"] = {
+                "chunk": C, "value": c_gbs, "unit": "GB/s", "ms_per_launch": c_launch * 1e3,
+                "query_tokens_per_s": aggregate_throughput(DECODE.num_seqs * C * K, world, t_chunk),
+                "pct_hbm_peak": 100 * c_gbs / peaks["hbm_gbs"],
+                "note": "multi-token paged decode (polar_attn_decode_paged_chunk) on the same "
+                        "32-sequence cache, timed separately after the step loop; not part of value"}
+            result["roofline_decode_chunk"] = {
+                "bound": "hbm", "kernel": "decode_split_kernel<4,16 rows>+decode_merge_kernel",
+                "achieved": c_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": c_gbs / peaks["hbm_gbs"], "traffic": profiled_traffic("decode_chunk", sha_d),
+                "peak_source": f"{peak_src} (copy bandwidth)"}
     if world > 1:
         import torch.distributed as dist
         dist.barrier(device_ids=[dev.index])
