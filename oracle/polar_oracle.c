@@ -23,6 +23,13 @@
  *           | T (non-causal)           temperature is the number of keys the
  *           | seqlen (decode)          row can see, so row i never depends on
  *                                      the future (len_mode 1 uses total T).
+ *   window W > 0 (sliding window, the ablation the results section names):
+ *                                      the visible keys are the last W of
+ *                                      those, j in [i - W + 1, i] (prefill) or
+ *                                      [seqlen - W, seqlen) (decode), and n is
+ *                                      their count, min(i + 1, W) / min(seqlen,
+ *                                      W); every statistic below runs over
+ *                                      that range.
  *   tau   = 1 + alpha*ln(n/L)  if n > L, else 1     length temperature,
  *                                      "sharpen distributions as context
  *                                      grows" (section 2.1, direction channel).
@@ -85,6 +92,7 @@ typedef struct {
     double beta;   /* gate slope */
     int causal;    /* prefill: 1 = row i sees keys 0..i */
     int len_mode;  /* 0: n = visible keys; 1: n = total length T (ablation) */
+    int window;    /* 0: all of them; W > 0: only the last W visible keys */
 } oracle_cfg;
 
 /* ---- input decoding (not method arithmetic) ------------------------------ */
@@ -105,9 +113,11 @@ typedef struct {
     int64_t dense_off;    /* dense: element offset of (b, j=0, g, d=0) */
     int64_t dense_stride; /* dense: elements between consecutive j */
     const int32_t *pt;    /* paged: page-table row of this sequence */
+    int64_t j0;           /* position of the first visible key (row index j = 0) */
 } key_src;
 
 static inline int64_t kv_off(const key_src *ks, int64_t j, int which) {
+    j += ks->j0;
     if (!ks->paged) return ks->dense_off + j * ks->dense_stride;
     int64_t page = ks->pt[j / ORACLE_PAGE];
     return (((page * 2 + which) * ks->Hkv + ks->g) * ORACLE_PAGE + (j % ORACLE_PAGE)) * ks->D;
@@ -364,13 +374,18 @@ int oracle_polar_fwd(const oracle_cfg *cfg, const void *q, const void *k, const 
         int g = kv_head_of(h, cfg->Hq, cfg->Hkv);
         double qrow[256];
         for (int d = 0; d < D; ++d) qrow[d] = ld(q, dtype, (((int64_t)b * T + i) * cfg->Hq + h) * D + d);
-        key_src ks = {k, v, dtype, D, cfg->Hkv, g, 0,
-                      ((int64_t)b * T * cfg->Hkv + g) * D, (int64_t)cfg->Hkv * D, NULL};
 #if ORACLE_MUTANT == 4
         int64_t n = cfg->causal ? (i > 0 ? i : 1) : T;
 #else
         int64_t n = cfg->causal ? i + 1 : T;
 #endif
+        int64_t lo = 0; /* first visible key */
+        if (cfg->causal && cfg->window > 0 && n > cfg->window) {
+            lo = n - cfg->window;
+            n = cfg->window;
+        }
+        key_src ks = {k, v, dtype, D, cfg->Hkv, g, 0,
+                      ((int64_t)b * T * cfg->Hkv + g) * D, (int64_t)cfg->Hkv * D, NULL, lo};
         int64_t n_len = cfg->len_mode == 1 ? T : n;
         double *zbuf = (double *)malloc(sizeof(double) * (size_t)(n > block ? n : block) + 8);
         if (!zbuf) { bad = 1; continue; }
@@ -389,7 +404,8 @@ int oracle_polar_fwd(const oracle_cfg *cfg, const void *q, const void *k, const 
 /*
  * Paged GQA decode.  q: [N,Hq,D]; kv_pages: [num_pages][2][Hkv][64][D] (K then
  * V, head-major, 64 tokens per page); page_table: [N][max_pages] int32;
- * seqlens: [N] (>= 1).  Query of sequence s sees its keys 0..seqlens[s]-1.
+ * seqlens: [N] (>= 1).  Query of sequence s sees its keys 0..seqlens[s]-1
+ * (the last cfg->window of them when window > 0).
  * rows: flat (s*Hq + h) or NULL for all.  Outputs as for oracle_polar_fwd.
  * Returns 0, -1 on invalid arguments, -2 on a page id out of range.
  */
@@ -421,7 +437,12 @@ int oracle_polar_decode(const oracle_cfg *cfg, const void *q, const void *kv_pag
         int g = kv_head_of(h, cfg->Hq, cfg->Hkv);
         double qrow[256];
         for (int d = 0; d < D; ++d) qrow[d] = ld(q, dtype, ((int64_t)sq * cfg->Hq + h) * D + d);
-        key_src ks = {kv_pages, kv_pages, dtype, D, cfg->Hkv, g, 1, 0, 0, pt};
+        int64_t lo = 0; /* first visible position */
+        if (cfg->window > 0 && n > cfg->window) {
+            lo = n - cfg->window;
+            n = cfg->window;
+        }
+        key_src ks = {kv_pages, kv_pages, dtype, D, cfg->Hkv, g, 1, 0, 0, pt, lo};
         double *zbuf = (double *)malloc(sizeof(double) * (size_t)(n > block ? n : block) + 8);
         if (!zbuf) { bad |= 1; continue; }
         eval_row(mode, block, theta, qrow, &ks, n, n, cfg, u + (int64_t)h * D, zbuf, out + r * D,

@@ -317,6 +317,47 @@ def pin_decode_matches_prefill(mutant=0, bd=None):
     _close(dc.neff, pf.neff[last], rtol=0, atol=0, what="decode vs prefill n_eff")
 
 
+# --------------------------------------------------------------------------
+# 10. sliding window W: a window no shorter than the sequence changes nothing;
+#     W = 1 leaves each row only its own key (out = v_i / |v_i|, n_eff = 1,
+#     gate 1/2, count 0); row i >= W-1 equals the unwindowed last row of the
+#     slice of keys i-W+1 .. i taken as a sequence of its own (same keys, same
+#     count n = W, so the same temperature), bit for bit, and earlier rows
+#     equal their unwindowed selves; a windowed decode equals the windowed
+#     prefill's last row.
+# --------------------------------------------------------------------------
+def pin_window(mutant=0, bd=None):
+    rng = np.random.default_rng(14)
+    T, W = 150, 37
+    q, k, v, u = _rand_inputs(rng, B=1, T=T, Hq=2, Hkv=1)
+    full = oracle.polar_fwd(q, k, v, u, Params(L=16), mutant=mutant, build_dir=bd)
+    big = oracle.polar_fwd(q, k, v, u, Params(L=16, window=T), mutant=mutant, build_dir=bd)
+    _close(big.out, full.out, rtol=0, atol=0, what="window >= T")
+    one = oracle.polar_fwd(q, k, v, u, Params(L=16, window=1), mutant=mutant, build_dir=bd)
+    vv = v[0, :, 0].astype(np.float64)
+    for h in range(2):
+        _close(one.out[h * T:(h + 1) * T], vv / np.linalg.norm(vv, axis=1, keepdims=True),
+               rtol=1e-14, atol=1e-15, what="window 1 = v_i")
+    assert np.all(one.neff == 1.0)
+    win = oracle.polar_fwd(q, k, v, u, Params(L=16, window=W), mutant=mutant, build_dir=bd)
+    for h in range(2):
+        r = [h * T + i for i in range(W - 1)]
+        _close(win.out[r], full.out[r], rtol=0, atol=0, what="rows inside the first window")
+    for i in (W - 1, W, 90, T - 1):
+        sl = slice(i - W + 1, i + 1)
+        qs, ks, vs = (np.ascontiguousarray(x[:, sl]) for x in (q, k, v))
+        ref = oracle.polar_fwd(qs, ks, vs, u, Params(L=16), mutant=mutant, build_dir=bd,
+                               rows=[h * W + W - 1 for h in range(2)])
+        got = [h * T + i for h in range(2)]
+        _close(win.out[got], ref.out, rtol=0, atol=0, what=f"window row {i} vs slice")
+        _close(win.neff[got], ref.neff, rtol=0, atol=0, what=f"window n_eff {i} vs slice")
+    pool, pt = _paged_from_dense(k, v, 0, perm_seed=6)
+    dc = oracle.polar_decode(np.ascontiguousarray(q[:, T - 1]), pool, pt,
+                             np.array([T], np.int32), u, Params(L=16, window=W),
+                             mutant=mutant, build_dir=bd)
+    _close(dc.out, win.out[[T - 1, 2 * T - 1]], rtol=0, atol=0, what="windowed decode")
+
+
 ALL_PINS = [pin_modes_agree, pin_uniform, pin_uniform_train_length_constant, pin_closed_form,
             pin_temperature_constants, pin_unit_norm_and_bounded, pin_duplication,
-            pin_causality, pin_gqa, pin_decode_matches_prefill]
+            pin_causality, pin_gqa, pin_decode_matches_prefill, pin_window]
