@@ -62,6 +62,8 @@ def parse_args(argv=None):
                     help="prefill workload (profiling runs use a smaller one)")
     ap.add_argument("--decode-seqs", type=int, default=W.DECODE.num_seqs,
                     help="decode sequences (profiling runs use fewer)")
+    ap.add_argument("--window", type=int, default=4096,
+                    help="sliding window of the separately timed windowed prefill (0 skips it)")
     ap.add_argument("--chunk", type=int, default=4,
                     help="query tokens per sequence of the separately timed multi-token decode "
                          "(0 skips it)")
@@ -322,6 +324,32 @@ def run_ours(args):
     t_pre = sum(ev[i][0].elapsed_time(ev[i][1]) for i in range(K)) / 1e3
     t_dec = sum(ev[i][1].elapsed_time(ev[i][2]) for i in range(K)) / 1e3
 
+    # ---- sliding-window prefill on the same inputs, timed on its own ----
+    window_res = None
+    if do_pre and 0 < args.window < PREFILL.T:
+        wp = dataclasses.replace(PREFILL, window=args.window)
+
+        def prefill_window():
+            pa.fwd(xp["q"], xp["k"], xp["v"], xp["u"], out_p, neff_p, ws_p, stream=stream,
+                   window=args.window, **p)
+
+        for _ in range(Wm):
+            prefill_window()
+        torch.cuda.synchronize(dev)
+        ew = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
+        barrier(world, dev)
+        torch.cuda.synchronize(dev)
+        for i in range(K):
+            ew[i][0].record(stream)
+            prefill_window()
+            ew[i][1].record(stream)
+        torch.cuda.synchronize(dev)
+        barrier(world, dev)
+        if pa.get_status() != 0:
+            raise RuntimeError("device status after the windowed prefill")
+        t_win = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in ew) / 1e3, world, dev)
+        window_res = (wp, t_win)
+
     # ---- multi-token decode (chunk query tokens per sequence), timed on its own ----
     chunk_res = None
     if do_dec and args.chunk > 1:
@@ -451,6 +479,17 @@ def run_ours(args):
             "clocks": clk.summary(),
             "e2e": e2e,
         }
+        if window_res is not None:
+            wp, t_win = window_res
+            w_launch = t_win / K
+            w_tf = wp.flops / w_launch / 1e12
+            result["prefill_window"] = {
+                "window": wp.window, "value": w_tf, "unit": "TFLOP/s",
+                "ms_per_launch": w_launch * 1e3, "flops_per_launch": wp.flops,
+                "pct_bf16_peak": 100 * w_tf / peaks["bf16_tflops"],
+                "note": "sliding-window prefill on the same T=16384 inputs, flops of the visible "
+                        "(query, key) pairs; timed separately after the step loop, L2 warm from "
+                        "the previous launch; not part of value"}
         if chunk_res is not None:
             C, t_chunk = chunk_res
             c_launch = t_chunk / K

@@ -84,9 +84,14 @@ typedef struct {
     float beta;       /* gate slope; typical 1.0 */
     int causal;       /* prefill: must be 1 (row i sees keys 0..i) */
     int impl;         /* polar_impl_t, prefill only */
+    int window;       /* 0: every causal key; W > 0: sliding window, only the last W
+                         visible keys (prefill i-W+1..i, decode seqlen-W..seqlen-1);
+                         n, and with it the length temperature and the null floor,
+                         is then the windowed count.  The pages' results section
+                         names the window as an ablation. */
 } polar_params_t;
 
-/* Fills *p with the typical constants above for the given shape. */
+/* Fills *p with the typical constants above for the given shape (window 0). */
 void polar_attn_default_params(polar_params_t *p, int B, int T, int Hq, int Hkv, int dtype);
 
 /*

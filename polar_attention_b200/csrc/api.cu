@@ -50,6 +50,7 @@ polar_status_t check_common(const polar_params_t *p) {
     if (!(p->alpha >= 0.0f) || !std::isfinite(p->alpha)) return POLAR_ERR_INVALID_ARG;
     if (!std::isfinite(p->beta)) return POLAR_ERR_INVALID_ARG;
     if (p->L_train < 2) return POLAR_ERR_INVALID_ARG;
+    if (p->window < 0) return POLAR_ERR_INVALID_ARG;
     return POLAR_OK;
 }
 
@@ -95,6 +96,7 @@ FwdLaunch make_fwd(const void *q, const void *k, const void *v, const float *u,
     a.q = q; a.k = k; a.v = v; a.u = u; a.out = out; a.neff = neff;
     a.B = p->B; a.T = p->T; a.Hq = p->Hq; a.Hkv = p->Hkv; a.dtype = p->dtype;
     a.s = p->logit_scale; a.alpha = p->alpha; a.beta = p->beta; a.L = p->L_train;
+    a.window = p->window;
     a.status = status; a.moments = nullptr; a.stream = stream;
     return a;
 }
@@ -160,8 +162,11 @@ polar_status_t polar_attn_fwd(const void *q, const void *k, const void *v, const
     if (!status) return POLAR_ERR_CUDA;
     FwdLaunch a = make_fwd(q, k, v, u, params, out, neff_out, status,
                            static_cast<cudaStream_t>(stream));
-    // Key moments only where they are used: the tensor-core kernel, beyond one tile.
-    a.moments = fwd_moment_records(params->T) > 0 ? static_cast<float *>(workspace) : nullptr;
+    // Key moments only where they are used: the tensor-core kernel, beyond one
+    // tile, without a window (a window bounds every row's work anyway).
+    a.moments = fwd_moment_records(params->T) > 0 && params->window == 0
+                    ? static_cast<float *>(workspace)
+                    : nullptr;
     // The tensor-core kernel pairs two query heads of one key/value group per
     // CTA, so it needs an even group size; fp32 inputs use the CUDA-core kernel.
     const bool tc_ok = params->dtype == POLAR_BF16 && (params->Hq / params->Hkv) % 2 == 0;
@@ -274,7 +279,8 @@ polar_status_t polar_attn_decode_paged_chunk(const void *q, const void *kv_pages
     a.q = q; a.kv_pages = kv_pages; a.num_pages = num_pages; a.page_table = page_table;
     a.max_pages = max_pages; a.seqlens = seqlens; a.num_seqs = num_seqs; a.u = u; a.out = out;
     a.neff = neff_out; a.Hq = p->Hq; a.Hkv = p->Hkv; a.s = p->logit_scale; a.alpha = p->alpha;
-    a.beta = p->beta; a.L = p->L_train; a.workspace = workspace; a.status = status;
+    a.beta = p->beta; a.L = p->L_train; a.window = p->window; a.workspace = workspace;
+    a.status = status;
     a.stream = static_cast<cudaStream_t>(stream);
     return from_cuda(launch_decode(a));
 }

@@ -43,8 +43,15 @@ struct SplitArgs {
     int *status;
     int num_pages, max_pages, Hq, Hkv, pages_per_split, max_splits;
     int chunk;  // query tokens per sequence (the last `chunk` cache positions)
+    int window; // 0: every cached position; W > 0: each row's last W
     float s, alpha, L;
 };
+
+// Page of the earliest cache position any query row of a sequence sees.
+__host__ __device__ __forceinline__ int first_visible_page(int seqlen, int chunk, int window) {
+    const int lo = window > 0 ? seqlen - chunk + 1 - window : 0;
+    return lo > 0 ? lo / kPage : 0;
+}
 
 // Byte offset of logical 16-byte chunk c of row t inside a 128B-swizzled tile.
 __device__ __forceinline__ uint32_t swz(int t, int c) {
@@ -126,7 +133,8 @@ decode_split_kernel(const __grid_constant__ CUtensorMap kv_map, const SplitArgs 
         return;
     }
     const int npg = (seqlen + kPage - 1) / kPage;
-    const int p0 = split * a.pages_per_split;
+    // Splits start at the page of the earliest position any row sees.
+    const int p0 = first_visible_page(seqlen, C, a.window) + split * a.pages_per_split;
     if (p0 >= npg) return;
     const int np = min(npg, p0 + a.pages_per_split) - p0;
     const int32_t *pt = a.page_table + static_cast<size_t>(seq) * a.max_pages + p0;
@@ -161,7 +169,7 @@ decode_split_kernel(const __grid_constant__ CUtensorMap kv_map, const SplitArgs 
     // Per row set: query fragments (A operand of S = Q K^T), the visible
     // positions n_r and the row's exponent scale.
     uint32_t qa[kHR][4][2];
-    int lim[kHR];
+    int lim[kHR], lo[kHR];  // row r sees positions lo <= pos < lim
     float cl2[kHR];
 #pragma unroll
     for (int hr = 0; hr < kHR; ++hr) {
@@ -176,7 +184,9 @@ decode_split_kernel(const __grid_constant__ CUtensorMap kv_map, const SplitArgs 
             qa[hr][kk][1] = real ? __ldg(qrow + 8 * kk + 4 + tq) : 0u;
         }
         lim[hr] = seqlen - C + t + 1;
-        cl2[hr] = a.s * length_temperature(static_cast<float>(lim[hr]), a.alpha, a.L) * kLog2e;
+        lo[hr] = a.window > 0 ? max(0, lim[hr] - a.window) : 0;
+        cl2[hr] = a.s * length_temperature(static_cast<float>(lim[hr] - lo[hr]), a.alpha, a.L) *
+                  kLog2e;
     }
 
     float m_ref[kHR], m_raw[kHR], l[kHR], l2[kHR], s1[kHR], s2[kHR];
@@ -230,7 +240,8 @@ decode_split_kernel(const __grid_constant__ CUtensorMap kv_map, const SplitArgs 
                 for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
                     for (int e = 0; e < 2; ++e) {
-                        vld[nt][e] = pos0 + 8 * nt + e < lim[hr];
+                        const int pos = pos0 + 8 * nt + e;
+                        vld[nt][e] = pos < lim[hr] && pos >= lo[hr];
                         const float x = sc[nt][2 * hr + e];
                         tmax = fmaxf(tmax, vld[nt][e] ? x : -INFINITY);
                         ts1 += vld[nt][e] ? x : 0.f;
@@ -366,7 +377,7 @@ decode_split_kernel(const __grid_constant__ CUtensorMap kv_map, const SplitArgs 
 __global__ void __launch_bounds__(32)
 decode_merge_kernel(const float *__restrict__ partials, const int32_t *__restrict__ seqlens,
                     const float *__restrict__ u, __nv_bfloat16 *__restrict__ out,
-                    float *__restrict__ neff_out, int Hq, int chunk, int max_pages,
+                    float *__restrict__ neff_out, int Hq, int chunk, int window, int max_pages,
                     int pages_per_split, int max_splits, float s, float alpha, float L, float beta,
                     float inv_ln_L) {
     const int h = blockIdx.x, row = blockIdx.y, lane = threadIdx.x;  // row = seq * chunk + token
@@ -374,7 +385,8 @@ decode_merge_kernel(const float *__restrict__ partials, const int32_t *__restric
     const int seqlen = seqlens[seq];
     if (seqlen < chunk || seqlen > max_pages * kPage) return;  // reported by the split kernel
     const int npg = (seqlen + kPage - 1) / kPage;
-    const int nsplit = (npg + pages_per_split - 1) / pages_per_split;
+    const int nsplit =
+        (npg - first_visible_page(seqlen, chunk, window) + pages_per_split - 1) / pages_per_split;
     const float *base = partials + (static_cast<size_t>(row) * Hq + h) * max_splits * kPartialFloats;
 
     float M = -INFINITY;
@@ -396,7 +408,8 @@ decode_merge_kernel(const float *__restrict__ partials, const int32_t *__restric
         s2 += ss.y;
         m_raw = fmaxf(m_raw, st.y);
     }
-    const float n = static_cast<float>(seqlen - chunk + tok + 1);  // positions this token sees
+    const int lim = seqlen - chunk + tok + 1;  // positions below lim, the last `window` of them
+    const float n = static_cast<float>(window > 0 ? min(lim, window) : lim);
     const float c = s * length_temperature(n, alpha, L);
     float ne;
     const float mag = polar_magnitude(l, l2, m_raw, s1, s2, c, n, beta, inv_ln_L, &ne);
@@ -468,7 +481,7 @@ cudaError_t launch_decode(const DecodeLaunch &a) {
 
     SplitArgs sa{a.page_table, a.seqlens, static_cast<const __nv_bfloat16 *>(a.q),
                  static_cast<float *>(a.workspace), a.status, a.num_pages, a.max_pages, a.Hq, a.Hkv,
-                 pps, max_splits, a.chunk, a.s, a.alpha, static_cast<float>(a.L)};
+                 pps, max_splits, a.chunk, a.window, a.s, a.alpha, static_cast<float>(a.L)};
     if (a.chunk < 1 || G * a.chunk > 16) return cudaErrorInvalidValue;
     cudaError_t e;
     switch (G) {
@@ -482,7 +495,7 @@ cudaError_t launch_decode(const DecodeLaunch &a) {
     dim3 mgrid(a.Hq, a.num_seqs * a.chunk);
     decode_merge_kernel<<<mgrid, 32, 0, a.stream>>>(
         static_cast<const float *>(a.workspace), a.seqlens, a.u, static_cast<__nv_bfloat16 *>(a.out),
-        a.neff, a.Hq, a.chunk, a.max_pages, pps, max_splits, a.s, a.alpha,
+        a.neff, a.Hq, a.chunk, a.window, a.max_pages, pps, max_splits, a.s, a.alpha,
         static_cast<float>(a.L), a.beta, 1.0f / logf(static_cast<float>(a.L)));
     count_launches(2);
     return cudaGetLastError();

@@ -22,7 +22,7 @@ __global__ void __launch_bounds__(kRows)
 fwd_simt_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v,
                 const float *__restrict__ u, T *__restrict__ out, float *__restrict__ neff_out,
                 int Tlen, int Hq, int Hkv, float s, float alpha, float L, float beta,
-                float inv_ln_L) {
+                float inv_ln_L, int window) {
     __shared__ __align__(16) float Ks[kKeyTile][kHeadDim];
     __shared__ __align__(16) float Vs[kKeyTile][kHeadDim];
 
@@ -38,7 +38,9 @@ fwd_simt_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__res
 #pragma unroll
         for (int d = 0; d < kHeadDim; ++d) qr[d] = live ? to_f32(qp[d]) : 0.0f;
     }
-    const int n = i + 1;  // causal: keys 0..i are visible
+    // Causal keys 0..i; with a sliding window only the last `window` of them.
+    const int lo = window > 0 ? max(0, i - window + 1) : 0;
+    const int n = i + 1 - lo;
     const float c = s * length_temperature(static_cast<float>(n), alpha, L);
     const float cl2 = c * kLog2e;
 
@@ -48,7 +50,8 @@ fwd_simt_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__res
     float m_ref = -INFINITY, m_raw = -INFINITY, l = 0.0f, l2 = 0.0f, s1 = 0.0f, s2 = 0.0f;
 
     const int kend = min(Tlen, row0 + kRows);  // keys any row of the block can see
-    for (int j0 = 0; j0 < kend; j0 += kKeyTile) {
+    const int kbeg = window > 0 ? max(0, row0 - window + 1) / kKeyTile * kKeyTile : 0;
+    for (int j0 = kbeg; j0 < kend; j0 += kKeyTile) {
         __syncthreads();
         for (int e = threadIdx.x; e < kKeyTile * kHeadDim; e += kRows) {
             const int jj = e / kHeadDim, d = e % kHeadDim, j = j0 + jj;
@@ -63,8 +66,8 @@ fwd_simt_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__res
         }
         __syncthreads();
         if (!live) continue;
-        const int jn = min(kKeyTile, n - j0);
-        for (int jj = 0; jj < jn; ++jj) {
+        const int jn = min(kKeyTile, i + 1 - j0);
+        for (int jj = max(0, lo - j0); jj < jn; ++jj) {
             float sd = 0.0f;
 #pragma unroll
             for (int d = 0; d < kHeadDim; d += 4) {
@@ -124,12 +127,13 @@ cudaError_t launch_fwd_simt(const FwdLaunch &a) {
         fwd_simt_kernel<float><<<grid, kRows, 0, a.stream>>>(
             static_cast<const float *>(a.q), static_cast<const float *>(a.k),
             static_cast<const float *>(a.v), a.u, static_cast<float *>(a.out), a.neff, a.T, a.Hq,
-            a.Hkv, a.s, a.alpha, static_cast<float>(a.L), a.beta, inv_ln_L);
+            a.Hkv, a.s, a.alpha, static_cast<float>(a.L), a.beta, inv_ln_L, a.window);
     } else {
         fwd_simt_kernel<__nv_bfloat16><<<grid, kRows, 0, a.stream>>>(
             static_cast<const __nv_bfloat16 *>(a.q), static_cast<const __nv_bfloat16 *>(a.k),
             static_cast<const __nv_bfloat16 *>(a.v), a.u, static_cast<__nv_bfloat16 *>(a.out),
-            a.neff, a.T, a.Hq, a.Hkv, a.s, a.alpha, static_cast<float>(a.L), a.beta, inv_ln_L);
+            a.neff, a.T, a.Hq, a.Hkv, a.s, a.alpha, static_cast<float>(a.L), a.beta, inv_ln_L,
+            a.window);
     }
     count_launches(1);
     return cudaGetLastError();

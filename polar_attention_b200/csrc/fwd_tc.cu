@@ -28,6 +28,7 @@
 // waits behind the other's queue.  A commit after PV_i(j) (pv_done) tells
 // softmax i that P_i may be overwritten and that O_i is current, so it can
 // rescale O_i in place before it releases P_i(j+1).
+#include <algorithm>
 #include <atomic>
 
 #include "polar_attn_selftest.h"
@@ -259,11 +260,13 @@ __device__ __forceinline__ float2 exp2_poly2(float2 x) {
 
 // Row statistics of one 128-key tile of S (raw dots, one row per thread):
 // max, sum and sum of squares over the visible keys.  Independent partial
-// accumulators keep the dependency chains short.  kDiag: the tile holds the
-// row's own position t; keys after it are invisible and are set to -inf in sr.
+// accumulators keep the dependency chains short.  kDiag: some keys of the
+// tile are invisible to the row (key e is visible iff tlo <= e <= thi: after
+// the row's own position, or before its sliding window); they are set to -inf
+// in sr.
 template <bool kDiag>
-__device__ __forceinline__ void row_stats(uint32_t (&sr)[4][32], int t, float &tmax, float &ts1,
-                                          float &ts2) {
+__device__ __forceinline__ void row_stats(uint32_t (&sr)[4][32], int thi, int tlo, float &tmax,
+                                          float &ts1, float &ts2) {
     if (!kDiag) {
         float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
         float2 a1[4], a2[4];
@@ -288,7 +291,7 @@ __device__ __forceinline__ void row_stats(uint32_t (&sr)[4][32], int t, float &t
         float a1[4] = {0.f, 0.f, 0.f, 0.f}, a2[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int e = 0; e < 128; ++e) {
-            const bool vis = e <= t;
+            const bool vis = e <= thi && e >= tlo;
             const float x = __uint_as_float(sr[e >> 5][e & 31]);
             const float xv = vis ? x : 0.f;
             sr[e >> 5][e & 31] = __float_as_uint(vis ? x : -INFINITY);
@@ -341,11 +344,13 @@ __device__ __forceinline__ void row_weights(const uint32_t (&sr)[4][32], float2 
 // no wait for the tile max, and returned packed as bf16 pairs in pk; the max,
 // sum and sum of squares of the raw dots (for the gate and the null floor) and
 // the sums of p and p^2 (l, l2) accumulate alongside.  kDiag masks the keys
-// after the row's own position t (p = 0, excluded from every sum).
+// outside tlo .. thi (after the row's own position or before its sliding
+// window: p = 0, excluded from every sum).
 template <bool kDiag, bool kPoly>
-__device__ __forceinline__ void fused_tile(const uint32_t (&sr)[4][32], int t, float2 sc2,
-                                           float neg_m, uint32_t (&pk)[4][16], float &tmax,
-                                           float &ts1, float &ts2, float &tl, float &tl2) {
+__device__ __forceinline__ void fused_tile(const uint32_t (&sr)[4][32], int thi, int tlo,
+                                           float2 sc2, float neg_m, uint32_t (&pk)[4][16],
+                                           float &tmax, float &ts1, float &ts2, float &tl,
+                                           float &tl2) {
     const float2 nm = make_float2(neg_m, neg_m);
     float mx[2] = {-INFINITY, -INFINITY};
     float2 a1 = make_float2(0.f, 0.f), a2 = a1, la = a1, l2a = a1;
@@ -357,7 +362,7 @@ __device__ __forceinline__ void fused_tile(const uint32_t (&sr)[4][32], int t, f
             float2 x;
             if (kDiag) {
                 const int col = 32 * cc + 2 * e;
-                const bool v0 = col <= t, v1 = col + 1 <= t;
+                const bool v0 = col <= thi && col >= tlo, v1 = col + 1 <= thi && col + 1 >= tlo;
                 mx[e & 1] = max3(mx[e & 1], v0 ? sv.x : -INFINITY, v1 ? sv.y : -INFINITY);
                 x = f2_fma(sv, sc2, nm);
                 x.x = v0 ? x.x : -INFINITY;
@@ -391,9 +396,10 @@ __device__ __forceinline__ void fused_tile(const uint32_t (&sr)[4][32], int t, f
 
 // fused_tile for a half row: 64 keys (keys 64*half .. 64*half + 63 of the
 // tile, in sr[0..1][0..31]) of one row, used when two softmax threads share a
-// row.  tlim = t - 64*half: key c of this half is visible iff c <= tlim.
+// row.  Key c of this half is visible iff tlo <= c <= thi (both in the half's
+// own coordinates).
 template <bool kDiag, bool kMoments>
-__device__ __forceinline__ void fused_half(const uint32_t (&sr)[2][32], int tlim, float2 sc2,
+__device__ __forceinline__ void fused_half(const uint32_t (&sr)[2][32], int thi, int tlo, float2 sc2,
                                            float neg_m, uint32_t (&pk)[2][16], float &tmax,
                                            float &ts1, float &ts2, float &tl, float &tl2) {
     const float2 nm = make_float2(neg_m, neg_m);
@@ -407,7 +413,7 @@ __device__ __forceinline__ void fused_half(const uint32_t (&sr)[2][32], int tlim
             float2 x;
             if (kDiag) {
                 const int col = 32 * cc + 2 * e;
-                const bool v0 = col <= tlim, v1 = col + 1 <= tlim;
+                const bool v0 = col <= thi && col >= tlo, v1 = col + 1 <= thi && col + 1 >= tlo;
                 mx[e & 1] = max3(mx[e & 1], v0 ? sv.x : -INFINITY, v1 ? sv.y : -INFINITY);
                 x = f2_fma(sv, sc2, nm);
                 x.x = v0 ? x.x : -INFINITY;
@@ -453,6 +459,7 @@ struct TcArgs {
     int *status;
     const float *mom;  // key-moment records (kMoments only)
     int B, T, Hq, Hkv, nqt, npairs;
+    int window;  // 0: all causal keys; W > 0: the last W of each row's
     float s, alpha, L, beta, inv_ln_L;
 };
 
@@ -511,7 +518,9 @@ __device__ __forceinline__ void store_row(const uint32_t (&o)[2][32], float l, f
 // free score columns, so that S2_i = <Y_i, q_i> and S1_i = <sum k, q_i>.  The
 // diagonal tile still sums its visible scores one by one.  The host uses this
 // variant from kMomMinTiles query tiles on.
-template <bool kFixedRef, int kSplit, bool kMoments>
+// kWindow: a sliding window shorter than the sequence (a.window); false
+// compiles every window test away.
+template <bool kFixedRef, int kSplit, bool kMoments, bool kWindow>
 __global__ void __launch_bounds__(128 + 256 * kSplit, 1)
 fwd_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
               const __grid_constant__ CUtensorMap tv, const TcArgs a) {
@@ -544,7 +553,21 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CU
     const int h0 = 2 * pair;
     const int g = h0 / (a.Hq / a.Hkv);
     const int q0 = qt * kBM;
-    const int nkv = qt + 1;  // key tiles 0..qt are (partly) visible
+    // Key tiles jt0..qt are (partly) visible to some row of the tile; with a
+    // sliding window the first is the one holding key q0 - window + 1.
+    const int window = kWindow ? a.window : 0;
+    const int jt0 = window > 0 ? max(0, q0 - window + 1) / kBN : 0;
+    const int nkv = qt - jt0 + 1;
+    // Loop tile j (key tile jt0 + j) needs masking if it is the diagonal tile
+    // or starts before the window of the tile's last row (min(q0 + 127, T - 1)).
+    auto masked_tile = [&](int j) {
+        return j == nkv - 1 || (window > 0 && (jt0 + j) * kBN < min(q0 + kBM, a.T) - window);
+    };
+    // Visible key range of row t in loop tile j, in the tile's coordinates.
+    auto vis_hi = [&](int j, int t) { return q0 + t - (jt0 + j) * kBN; };
+    auto vis_lo = [&](int j, int t) {
+        return window > 0 ? q0 + t - window + 1 - (jt0 + j) * kBN : -(1 << 30);
+    };
 
     if (warp == 0 && lane == 0) {
         mbar_init(&q_full, 1);
@@ -589,8 +612,8 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CU
                 if (j >= kStagesKV) ok = mbar_wait(&kv_empty[st], ((j / kStagesKV) - 1) & 1, a.status);
                 if (!ok) break;
                 mbar_arrive_expect_tx(&kv_full[st], 2 * kTileBytes);
-                tma_load_4d(sK + st * kTileBytes, &tk, 0, g, j * kBN, b, &kv_full[st]);
-                tma_load_4d(sV + st * kTileBytes, &tv, 0, g, j * kBN, b, &kv_full[st]);
+                tma_load_4d(sK + st * kTileBytes, &tk, 0, g, (jt0 + j) * kBN, b, &kv_full[st]);
+                tma_load_4d(sV + st * kTileBytes, &tv, 0, g, (jt0 + j) * kBN, b, &kv_full[st]);
                 ++issued;
             }
             // Every copy this thread started lands before shared memory is released.
@@ -743,7 +766,8 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CU
         const uint32_t tP = lane_base + (slot ? kColP1 : kColP0) + 32 * half;
         const uint32_t tO = lane_base + (slot ? kColO1 : kColO0);
         const int row = q0 + t;
-        const float n = static_cast<float>(row + 1);
+        // Visible keys of the row: row + 1, or the window.
+        const float n = static_cast<float>(window > 0 ? min(row + 1, window) : row + 1);
         const float c = a.s * length_temperature(n, a.alpha, a.L);
         const float cl2 = c * kLog2e;
         const float m_ref = cl2;
@@ -762,10 +786,11 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CU
             mbar_arrive(&s_free[slot]);
             uint32_t pk[2][16];
             float tmax, ts1, ts2, tl, tl2;
-            if (j == nkv - 1)
-                fused_half<true, kMoments>(sr, t - 64 * half, sc2, -m_ref, pk, tmax, ts1, ts2, tl, tl2);
+            if (masked_tile(j))
+                fused_half<true, kMoments>(sr, vis_hi(j, t) - 64 * half, vis_lo(j, t) - 64 * half,
+                                           sc2, -m_ref, pk, tmax, ts1, ts2, tl, tl2);
             else
-                fused_half<false, kMoments>(sr, t - 64 * half, sc2, -m_ref, pk, tmax, ts1, ts2, tl, tl2);
+                fused_half<false, kMoments>(sr, 0, 0, sc2, -m_ref, pk, tmax, ts1, ts2, tl, tl2);
             s1 += ts1;
             s2 += ts2;
             l += tl;
@@ -861,11 +886,16 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CU
         const uint32_t tP = lane_base + (slot ? kColP1 : kColP0);
         const uint32_t tO = lane_base + (slot ? kColO1 : kColO0);
         const int row = q0 + t;
-        const float n = static_cast<float>(row + 1);
+        // Visible keys of the row: row + 1, or the window.
+        const float n = static_cast<float>(window > 0 ? min(row + 1, window) : row + 1);
         const float c = a.s * length_temperature(n, a.alpha, a.L);
         const float cl2 = c * kLog2e;
 
-        float m_ref = kFixedRef ? cl2 : -INFINITY;
+        // Running reference: a finite floor rather than -inf, so that a tile with
+        // no visible key (a sliding window can start past the first loaded
+        // tile) gives weights 2^(-inf) = 0 instead of -inf + inf; the first real
+        // max still rescales by 2^(floor - max) = 0.
+        float m_ref = kFixedRef ? cl2 : -1e30f;
         float m_raw = -INFINITY, l = 0.f, l2 = 0.f, s1 = 0.f, s2 = 0.f;
         const float2 sc2 = make_float2(cl2, cl2);
         // O_i *= r for this thread's row (a warp-collective TMEM round trip).
@@ -894,16 +924,17 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CU
             // S_i(j) is in registers: the MMA thread may overwrite it with S_i(j+1).
             tc_fence_before();
             mbar_arrive(&s_free[slot]);
-            const bool diag = (j == nkv - 1);
+            const bool diag = masked_tile(j);
+            const int thi = vis_hi(j, t), tlo = vis_lo(j, t);
             uint32_t pk[4][16];
             float r = 1.f;
             bool need = false;
             if (kFixedRef) {
                 float tmax, ts1, ts2, tl, tl2;
                 if (diag)
-                    fused_tile<true, false>(sr, t, sc2, -m_ref, pk, tmax, ts1, ts2, tl, tl2);
+                    fused_tile<true, false>(sr, thi, tlo, sc2, -m_ref, pk, tmax, ts1, ts2, tl, tl2);
                 else
-                    fused_tile<false, true>(sr, t, sc2, -m_ref, pk, tmax, ts1, ts2, tl, tl2);
+                    fused_tile<false, true>(sr, thi, tlo, sc2, -m_ref, pk, tmax, ts1, ts2, tl, tl2);
                 s1 += ts1;
                 s2 += ts2;
                 l += tl;
@@ -915,9 +946,9 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CU
             } else {
                 float tmax, ts1, ts2;
                 if (diag)
-                    row_stats<true>(sr, t, tmax, ts1, ts2);
+                    row_stats<true>(sr, thi, tlo, tmax, ts1, ts2);
                 else
-                    row_stats<false>(sr, t, tmax, ts1, ts2);
+                    row_stats<false>(sr, thi, tlo, tmax, ts1, ts2);
                 s1 += ts1;
                 s2 += ts2;
                 m_raw = fmaxf(m_raw, tmax);
@@ -992,26 +1023,28 @@ cudaError_t launch_fwd_tc(const FwdLaunch &a) {
     if (e != cudaSuccess) return e;
     const uint64_t bit = 1ull << (dev & 63);
     if (!(configured.load() & bit)) {
-        e = cudaFuncSetAttribute(fwd_tc_kernel<true, 2, true>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-        if (e == cudaSuccess)
-            e = cudaFuncSetAttribute(fwd_tc_kernel<true, 2, false>,
-                                     cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-        if (e == cudaSuccess)
-            e = cudaFuncSetAttribute(fwd_tc_kernel<false, 1, false>,
-                                     cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-        if (e != cudaSuccess) return e;
+        const void *all[] = {reinterpret_cast<const void *>(fwd_tc_kernel<true, 2, true, false>),
+                             reinterpret_cast<const void *>(fwd_tc_kernel<true, 2, false, false>),
+                             reinterpret_cast<const void *>(fwd_tc_kernel<false, 1, false, false>),
+                             reinterpret_cast<const void *>(fwd_tc_kernel<true, 2, false, true>),
+                             reinterpret_cast<const void *>(fwd_tc_kernel<false, 1, false, true>)};
+        for (const void *f : all) {
+            e = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+            if (e != cudaSuccess) return e;
+        }
         // setmaxnreg can only hand out the registers the block was launched with:
         // 64 for the producer/MMA warpgroup plus 104 for each of the four softmax
         // warpgroups must fit in (registers per thread at launch) x 640.
-        cudaFuncAttributes fa, fb;
-        e = cudaFuncGetAttributes(&fa, fwd_tc_kernel<true, 2, true>);
-        if (e == cudaSuccess) e = cudaFuncGetAttributes(&fb, fwd_tc_kernel<true, 2, false>);
-        if (e != cudaSuccess) return e;
         const long long need = 64ll * 128 + 104ll * 512;
-        if (static_cast<long long>(fa.numRegs) * 640 >= need &&
-            static_cast<long long>(fb.numRegs) * 640 >= need)
-            split_ok.fetch_or(bit);
+        bool fits = true;
+        for (int i = 0; i < 5; ++i) {
+            if (i == 2 || i == 4) continue;  // the one-warpgroup-per-head kernels
+            cudaFuncAttributes fa;
+            e = cudaFuncGetAttributes(&fa, all[i]);
+            if (e != cudaSuccess) return e;
+            fits = fits && static_cast<long long>(fa.numRegs) * 640 >= need;
+        }
+        if (fits) split_ok.fetch_or(bit);
         configured.fetch_or(bit);
     }
     // [B, T, H, 64] bf16 as a 4-D tensor (d, head, t, b); tiles of 128 rows x 64.
@@ -1043,6 +1076,9 @@ cudaError_t launch_fwd_tc(const FwdLaunch &a) {
     ta.mom = a.moments;
     ta.B = a.B; ta.T = a.T; ta.Hq = a.Hq; ta.Hkv = a.Hkv;
     ta.nqt = (a.T + kBM - 1) / kBM;
+    // A window no shorter than the sequence changes nothing.
+    const bool windowed = a.window > 0 && a.window < a.T;
+    ta.window = windowed ? a.window : 0;
     ta.npairs = a.Hq / 2;
     ta.s = a.s; ta.alpha = a.alpha; ta.L = static_cast<float>(a.L); ta.beta = a.beta;
     ta.inv_ln_L = 1.0f / logf(static_cast<float>(a.L));
@@ -1051,20 +1087,25 @@ cudaError_t launch_fwd_tc(const FwdLaunch &a) {
     if (ctas > 0x7fffffffll) return cudaErrorInvalidValue;
     // Fixed exponential reference while the smallest weight squared, 2^(-4 c_max log2e)
     // with c_max the largest logit scale of any row, stays well inside fp32.
+    const int n_max = windowed ? a.window : a.T;  // longest visible range
     const float cl2_max = a.s *
-                          (a.T > a.L ? 1.0f + a.alpha * logf(static_cast<float>(a.T) / a.L) : 1.0f) *
+                          (n_max > a.L ? 1.0f + a.alpha * logf(static_cast<float>(n_max) / a.L) : 1.0f) *
                           1.4426950408889634f;
     const unsigned grid = static_cast<unsigned>(ctas);
     if (cl2_max <= 28.0f && (split_ok.load() & bit)) {
-        if (a.moments && ta.nqt >= kMomMinTiles) {
+        if (windowed) {
+            fwd_tc_kernel<true, 2, false, true><<<grid, 640, kSmemBytes, a.stream>>>(tq, tk, tv, ta);
+        } else if (a.moments && ta.nqt >= kMomMinTiles) {
             e = launch_fwd_moments(a.k, a.B, a.T, a.Hkv, a.moments, a.stream);
             if (e != cudaSuccess) return e;
-            fwd_tc_kernel<true, 2, true><<<grid, 640, kSmemBytes, a.stream>>>(tq, tk, tv, ta);
+            fwd_tc_kernel<true, 2, true, false><<<grid, 640, kSmemBytes, a.stream>>>(tq, tk, tv, ta);
         } else {
-            fwd_tc_kernel<true, 2, false><<<grid, 640, kSmemBytes, a.stream>>>(tq, tk, tv, ta);
+            fwd_tc_kernel<true, 2, false, false><<<grid, 640, kSmemBytes, a.stream>>>(tq, tk, tv, ta);
         }
+    } else if (windowed) {
+        fwd_tc_kernel<false, 1, false, true><<<grid, 384, kSmemBytes, a.stream>>>(tq, tk, tv, ta);
     } else {
-        fwd_tc_kernel<false, 1, false><<<grid, 384, kSmemBytes, a.stream>>>(tq, tk, tv, ta);
+        fwd_tc_kernel<false, 1, false, false><<<grid, 384, kSmemBytes, a.stream>>>(tq, tk, tv, ta);
     }
     count_launches(1);
     return cudaGetLastError();

@@ -18,6 +18,7 @@ struct FwdLaunch {
     int dtype;    // POLAR_BF16 / POLAR_FP32
     float s, alpha, beta;
     int L;
+    int window;   // 0: all causal keys; W > 0: the last W
     int *status;  // device status word
     float *moments;  // key-moment records (fwd_moments_bytes), or null
     cudaStream_t stream;
@@ -36,6 +37,7 @@ struct DecodeLaunch {
     int Hq, Hkv;
     float s, alpha, beta;
     int L;
+    int window;  // 0: all cached positions; W > 0: the last W of each row's
     void *workspace;
     int chunk;  // query tokens per sequence (1 for plain decode)
     int *status;

@@ -43,7 +43,7 @@ class Params(ctypes.Structure):
                 ("Hkv", ctypes.c_int), ("head_dim", ctypes.c_int), ("dtype", ctypes.c_int),
                 ("logit_scale", ctypes.c_float), ("alpha", ctypes.c_float),
                 ("L_train", ctypes.c_int), ("beta", ctypes.c_float), ("causal", ctypes.c_int),
-                ("impl", ctypes.c_int)]
+                ("impl", ctypes.c_int), ("window", ctypes.c_int)]
 
 
 _lib = None
@@ -103,10 +103,11 @@ def status_string(code: int) -> str:
 
 
 def make_params(B=0, T=0, Hq=16, Hkv=4, dtype=POLAR_BF16, s=8.0, alpha=0.3, L=2048, beta=1.0,
-                impl="auto") -> Params:
+                impl="auto", window=0) -> Params:
     p = Params()
     lib().polar_attn_default_params(ctypes.byref(p), B, T, Hq, Hkv, dtype)
     p.logit_scale, p.alpha, p.L_train, p.beta = s, alpha, L, beta
+    p.window = int(window)
     p.impl = IMPLS[impl] if isinstance(impl, str) else int(impl)
     return p
 
@@ -140,7 +141,7 @@ def fwd_workspace_size(B: int, T: int, Hq: int, Hkv: int) -> int:
 
 
 def fwd(q, k, v, u, out=None, neff=None, workspace=None, *, s=8.0, alpha=0.3, L=2048, beta=1.0,
-        impl="auto", stream=None, want_neff=True, moments=True):
+        impl="auto", stream=None, want_neff=True, moments=True, window=0):
     """Causal prefill.  q [B,T,Hq,64], k/v [B,T,Hkv,64] (bf16 or fp32, CUDA,
     contiguous), u [Hq,64] fp32.  Returns (out [B,T,Hq,64], neff [B,Hq,T]).
     moments=True passes a workspace for the key-moment pre-pass (allocated
@@ -156,7 +157,7 @@ def fwd(q, k, v, u, out=None, neff=None, workspace=None, *, s=8.0, alpha=0.3, L=
         out = torch.empty_like(q)
     if neff is None and want_neff:
         neff = torch.empty((B, Hq, T), device=q.device, dtype=torch.float32)
-    p = make_params(B, T, Hq, Hkv, _dt(q), s, alpha, L, beta, impl)
+    p = make_params(B, T, Hq, Hkv, _dt(q), s, alpha, L, beta, impl, window)
     p.head_dim = D
     ws_bytes = 0
     if moments:
@@ -179,7 +180,7 @@ def decode_workspace_size(num_seqs: int, max_pages: int, Hq: int, Hkv: int) -> i
 
 
 def decode_paged(q, kv_pages, page_table, seqlens, u, out=None, neff=None, workspace=None, *,
-                 s=8.0, alpha=0.3, L=2048, beta=1.0, stream=None, want_neff=True):
+                 s=8.0, alpha=0.3, L=2048, beta=1.0, stream=None, want_neff=True, window=0):
     """Paged GQA decode.  q [N,Hq,64] bf16; kv_pages [P,2,Hkv,64,64] bf16;
     page_table [N,max_pages] int32; seqlens [N] int32; u [Hq,64] fp32.
     Returns (out [N,Hq,64], neff [N,Hq])."""
@@ -188,7 +189,7 @@ def decode_paged(q, kv_pages, page_table, seqlens, u, out=None, neff=None, works
     max_pages = page_table.shape[1]
     if page_table.dtype != torch.int32 or seqlens.dtype != torch.int32:
         raise TypeError("page_table and seqlens must be int32")
-    p = make_params(0, 0, Hq, Hkv, _dt(q), s, alpha, L, beta)
+    p = make_params(0, 0, Hq, Hkv, _dt(q), s, alpha, L, beta, window=window)
     p.head_dim = D
     ws_need = int(lib().polar_attn_decode_workspace_size(N, max_pages, ctypes.byref(p)))
     if workspace is None:
@@ -212,7 +213,8 @@ def decode_chunk_workspace_size(num_seqs: int, max_pages: int, chunk: int, Hq: i
 
 
 def decode_paged_chunk(q, kv_pages, page_table, seqlens, u, out=None, neff=None, workspace=None,
-                       *, s=8.0, alpha=0.3, L=2048, beta=1.0, stream=None, want_neff=True):
+                       *, s=8.0, alpha=0.3, L=2048, beta=1.0, stream=None, want_neff=True,
+                       window=0):
     """Multi-token paged decode.  q [N,C,Hq,64] bf16: token t of sequence n is
     the query at cache position seqlens[n] - C + t.  Returns (out [N,C,Hq,64],
     neff [N,C,Hq])."""
@@ -221,7 +223,7 @@ def decode_paged_chunk(q, kv_pages, page_table, seqlens, u, out=None, neff=None,
     max_pages = page_table.shape[1]
     if page_table.dtype != torch.int32 or seqlens.dtype != torch.int32:
         raise TypeError("page_table and seqlens must be int32")
-    p = make_params(0, 0, Hq, Hkv, _dt(q), s, alpha, L, beta)
+    p = make_params(0, 0, Hq, Hkv, _dt(q), s, alpha, L, beta, window=window)
     p.head_dim = D
     ws_need = int(lib().polar_attn_decode_chunk_workspace_size(N, max_pages, C, ctypes.byref(p)))
     if workspace is None:
@@ -242,13 +244,13 @@ NOALLOC_SCRATCH_BYTES = 16 << 20
 
 
 def decode_paged_noalloc(q, kv_pages, page_table, seqlens, u, out, neff=None, *, s=8.0,
-                         alpha=0.3, L=2048, beta=1.0, stream=None):
+                         alpha=0.3, L=2048, beta=1.0, stream=None, window=0):
     """polar_attn_decode_paged_noalloc: the paged decode with no workspace, for
     callers that cannot allocate device memory.  out (and neff, if given) must
     be preallocated by the caller; this wrapper allocates nothing."""
     N, Hq, D = q.shape
     P_, _, Hkv, _, _ = kv_pages.shape
-    p = make_params(0, 0, Hq, Hkv, _dt(q), s, alpha, L, beta)
+    p = make_params(0, 0, Hq, Hkv, _dt(q), s, alpha, L, beta, window=window)
     p.head_dim = D
     _check(lib().polar_attn_decode_paged_noalloc(
         _ptr(q), _ptr(kv_pages), P_, _ptr(page_table), page_table.shape[1], _ptr(seqlens), N,
@@ -263,11 +265,11 @@ def fwd_staging_size(B, T, Hq, Hkv, dtype=POLAR_BF16) -> int:
 
 
 def fwd_host(q_h, k_h, v_h, u_h, out_h, neff_h, staging, *, s=8.0, alpha=0.3, L=2048, beta=1.0,
-             impl="auto", stream=None):
+             impl="auto", stream=None, window=0):
     """polar_attn_fwd_host on (pinned) host tensors; staging is a CUDA uint8
     tensor of at least fwd_staging_size bytes.  Synchronises the stream."""
     B, T, Hq, D = q_h.shape
-    p = make_params(B, T, Hq, k_h.shape[2], _dt(q_h), s, alpha, L, beta, impl)
+    p = make_params(B, T, Hq, k_h.shape[2], _dt(q_h), s, alpha, L, beta, impl, window)
     p.head_dim = D
     _check(lib().polar_attn_fwd_host(_ptr(q_h), _ptr(k_h), _ptr(v_h), _ptr(u_h), ctypes.byref(p),
                                      _ptr(out_h), _ptr(neff_h), _ptr(staging), staging.numel(),
@@ -280,12 +282,12 @@ def decode_staging_size(num_seqs, max_pages, Hq, Hkv) -> int:
 
 
 def decode_paged_host(q_h, kv_pages, page_table_h, seqlens_h, u_h, out_h, neff_h, staging, *,
-                      s=8.0, alpha=0.3, L=2048, beta=1.0, stream=None):
+                      s=8.0, alpha=0.3, L=2048, beta=1.0, stream=None, window=0):
     """polar_attn_decode_paged_host: per-step inputs and outputs in (pinned)
     host memory, the KV pool resident on the device.  Synchronises the stream."""
     N, Hq, D = q_h.shape
     P_, _, Hkv, _, _ = kv_pages.shape
-    p = make_params(0, 0, Hq, Hkv, _dt(q_h), s, alpha, L, beta)
+    p = make_params(0, 0, Hq, Hkv, _dt(q_h), s, alpha, L, beta, window=window)
     p.head_dim = D
     _check(lib().polar_attn_decode_paged_host(
         _ptr(q_h), _ptr(kv_pages), P_, _ptr(page_table_h), page_table_h.shape[1], _ptr(seqlens_h),

@@ -42,12 +42,22 @@ class PrefillWorkload:
     L: int = 2048               # training length
     beta: float = 1.0           # gate slope
     seed: int = 0
+    window: int = 0             # sliding window (0: every causal key)
+
+    @property
+    def visible_pairs(self) -> float:
+        """(query, key) pairs a row sees, summed over the rows of one head:
+        the causal triangle, or with a window W the rows' min(i + 1, W)."""
+        T, W = self.T, self.window
+        if W <= 0 or W >= T:
+            return T * (T + 1) / 2.0
+        return W * (W + 1) / 2.0 + (T - W) * float(W)
 
     @property
     def flops(self) -> float:
-        """Algorithmic MMA flops of the visible causal triangle: 4*D per
-        visible (query, key) pair (QK^T and PV, 2 flops per MAC each)."""
-        return 4.0 * self.D * self.B * self.Hq * self.T * (self.T + 1) / 2.0
+        """Algorithmic MMA flops of the visible pairs: 4*D per visible
+        (query, key) pair (QK^T and PV, 2 flops per MAC each)."""
+        return 4.0 * self.D * self.B * self.Hq * self.visible_pairs
 
     def describe(self) -> str:
         return (f"causal prefill B={self.B} T={self.T} Hq={self.Hq} Hkv={self.Hkv} "
@@ -70,6 +80,7 @@ class DecodeWorkload:
     beta: float = 1.0
     seed: int = 0
     plant: int = 0              # near-copies of the group's first query per (seq, kv head)
+    window: int = 0             # sliding window (0: every cached position)
 
     def describe(self) -> str:
         return (f"paged GQA decode {self.num_seqs} seqs ctx {self.min_len}-{self.max_len} "

@@ -22,7 +22,7 @@ NEFF_TOL = 1e-3
 
 
 def oracle_params(w) -> oracle.Params:
-    return oracle.Params(s=w.s, alpha=w.alpha, L=w.L, beta=w.beta)
+    return oracle.Params(s=w.s, alpha=w.alpha, L=w.L, beta=w.beta, window=getattr(w, "window", 0))
 
 
 def oracle_prefill(w, x, rows=None):
