@@ -89,6 +89,9 @@ def _load(mutant: int = 0, build_dir: str | None = None) -> ctypes.CDLL:
                 ctypes.c_int, P, P, ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_double,
                 P, P, P]
             lib.oracle_polar_decode.restype = ctypes.c_int
+            lib.oracle_polar_bwd.argtypes = [
+                ctypes.POINTER(_Cfg), P, P, P, ctypes.c_int, P, P, P, P, P, P]
+            lib.oracle_polar_bwd.restype = ctypes.c_int
             lib.oracle_mutant_id.restype = ctypes.c_int
             _LIBS[key] = lib
         return _LIBS[key]
@@ -149,6 +152,35 @@ def polar_fwd(q, k, v, u, p: Params = Params(), rows=None, mode: str = "two_pass
     if rc != 0:
         raise ValueError(f"oracle_polar_fwd rejected its arguments (rc={rc})")
     return Result(out, neff, stats)
+
+
+def polar_bwd(q, k, v, u, gout, p: Params = Params(), mutant: int = 0,
+              build_dir: str | None = None):
+    """Backward of the prefill: (dq, dk, dv, du) as fp64 arrays shaped like q,
+    k, v and u, for the upstream gradient gout = dL/dout [B,T,Hq,D]."""
+    q, dt = _as_input(q)
+    k, dk_ = _as_input(k)
+    v, dv_ = _as_input(v)
+    if not (dt == dk_ == dv_):
+        raise TypeError("q, k, v must share a dtype")
+    B, T, Hq, D = q.shape
+    Hkv = k.shape[2]
+    u = np.ascontiguousarray(u, dtype=np.float32)
+    g = np.ascontiguousarray(gout, dtype=np.float64)
+    if g.shape != (B, T, Hq, D):
+        raise ValueError("gout shape mismatch")
+    cfg = _Cfg(B, T, Hq, Hkv, D, p.s, p.alpha, p.L, p.beta, int(p.causal), p.len_mode,
+               int(p.window))
+    dq = np.zeros((B, T, Hq, D), np.float64)
+    dk = np.zeros((B, T, Hkv, D), np.float64)
+    dv = np.zeros((B, T, Hkv, D), np.float64)
+    du = np.zeros((Hq, D), np.float64)
+    rc = _load(mutant, build_dir).oracle_polar_bwd(ctypes.byref(cfg), _ptr(q), _ptr(k), _ptr(v), dt,
+                                                   _ptr(u), _ptr(g), _ptr(dq), _ptr(dk), _ptr(dv),
+                                                   _ptr(du))
+    if rc != 0:
+        raise ValueError(f"oracle_polar_bwd rejected its arguments (rc={rc})")
+    return dq, dk, dv, du
 
 
 def polar_decode(q, kv_pages, page_table, seqlens, u, p: Params = Params(), rows=None,

@@ -453,5 +453,139 @@ int oracle_polar_decode(const oracle_cfg *cfg, const void *q, const void *kv_pag
     return bad ? -1 : 0;
 }
 
+/*
+ * Backward of the prefill (NEXT: the training use of the step).  Given
+ * g = dL/dout for every row, the gradients dL/dq, dL/dk, dL/dv (fp64, same
+ * layouts as q, k, v) and dL/du ([Hq][D]).  Each row is recomputed by the
+ * two-pass definition above; then, with w_j = e^{z_j - m}, A = sum w_j v_j,
+ * content = A/|A|, T = tanh(ln n_eff / ln L):
+ *   du_h   += gate*T*g
+ *   gamma   = <g, u_h>;  dgate = gamma*T;  dT = gamma*gate
+ *   dn_eff  = dT*(1 - T^2) / (n_eff ln L)
+ *   dl      = 2 l/l2 * dn_eff;  dl2 = -(l/l2)^2 * dn_eff   (n_eff = l^2/l2)
+ *   dA      = (g - content <content, g>) / |A|             (A/|A|)
+ *   dm      = beta*gate*(1 - gate)*dgate;  dz0 = -dm       (gate on m - z0)
+ *   dmu     = dz0;  dsigma = dz0*sqrt(2 ln n)              (z0 = mu + sigma sqrt(2 ln n))
+ *   dz_j    = w_j (dl + 2 dl2 w_j + <dA, v_j>) + dmu/n + dsigma (z_j - mu)/(n sigma)
+ *             + [j = argmax] dm          (the max's subgradient: its first index;
+ *                                       sigma = 0 contributes nothing)
+ *   dS_j    = c dz_j;  dq += dS_j k_j;  dk_j += dS_j q;  dv_j += w_j dA.
+ * The shift m cancels from content and n_eff (both scale-invariant), so w may
+ * be taken relative to any common reference.  Inputs as oracle_polar_fwd; g
+ * is fp64 [B,T,Hq,D].  Returns 0, or -1 on invalid arguments.
+ */
+int oracle_polar_bwd(const oracle_cfg *cfg, const void *q, const void *k, const void *v,
+                     int dtype, const float *u, const double *gout, double *dq, double *dk,
+                     double *dv, double *du) {
+    if (!cfg || cfg->D <= 0 || cfg->D > 256 || cfg->Hkv <= 0 || cfg->Hq % cfg->Hkv != 0 ||
+        cfg->L < 2 || cfg->T < 0 || cfg->B < 0 || !cfg->causal || cfg->len_mode != 0)
+        return -1;
+    const int B = cfg->B, T = cfg->T, Hq = cfg->Hq, Hkv = cfg->Hkv, D = cfg->D;
+    const int G = Hq / Hkv;
+    memset(dq, 0, sizeof(double) * (size_t)B * T * Hq * D);
+    memset(dk, 0, sizeof(double) * (size_t)B * T * Hkv * D);
+    memset(dv, 0, sizeof(double) * (size_t)B * T * Hkv * D);
+    double *du_part = (double *)calloc((size_t)B * Hq * D, sizeof(double));
+    if (!du_part) return -1;
+    int bad = 0;
+#pragma omp parallel for schedule(dynamic, 1) reduction(| : bad)
+    for (int64_t task = 0; task < (int64_t)B * Hkv; ++task) {
+        /* One (batch, kv head): every write to dk, dv of kv head g and to dq
+           of its query heads stays inside this task. */
+        const int b = (int)(task / Hkv), g = (int)(task % Hkv);
+        double *z = (double *)malloc(sizeof(double) * (size_t)(T > 0 ? T : 1));
+        double *w = (double *)malloc(sizeof(double) * (size_t)(T > 0 ? T : 1));
+        if (!z || !w) { bad = 1; free(z); free(w); continue; }
+        for (int hh = 0; hh < G; ++hh) {
+            const int h = g * G + hh;
+            for (int64_t i = 0; i < T; ++i) {
+                int64_t n = i + 1, lo = 0;
+                if (cfg->window > 0 && n > cfg->window) { lo = n - cfg->window; n = cfg->window; }
+                double qr[256], gr[256];
+                const int64_t qo = (((int64_t)b * T + i) * Hq + h) * D;
+                for (int d = 0; d < D; ++d) { qr[d] = ld(q, dtype, qo + d); gr[d] = gout[qo + d]; }
+                const double c = cfg->s * length_temperature(n, cfg);
+                /* forward, two-pass */
+                double m = -INFINITY, mu = 0.0;
+                int64_t jmax = 0;
+                for (int64_t j = 0; j < n; ++j) {
+                    const int64_t ko = (((int64_t)b * T + lo + j) * Hkv + g) * D;
+                    double sd = 0.0;
+                    for (int d = 0; d < D; ++d) sd += qr[d] * ld(k, dtype, ko + d);
+                    z[j] = c * sd;
+                    if (z[j] > m) { m = z[j]; jmax = j; }
+                    mu += z[j];
+                }
+                mu /= (double)n;
+                double var = 0.0;
+                for (int64_t j = 0; j < n; ++j) var += (z[j] - mu) * (z[j] - mu);
+                const double sigma = sqrt(var / (double)n);
+                const double kn = sqrt(2.0 * log((double)n));
+                const double z0 = mu + sigma * kn;
+                const double gate = 1.0 / (1.0 + exp(-cfg->beta * (m - z0)));
+                double l = 0.0, l2 = 0.0, A[256];
+                for (int d = 0; d < D; ++d) A[d] = 0.0;
+                for (int64_t j = 0; j < n; ++j) {
+                    const int64_t vo = (((int64_t)b * T + lo + j) * Hkv + g) * D;
+                    w[j] = exp(z[j] - m);
+                    l += w[j];
+                    l2 += w[j] * w[j];
+                    for (int d = 0; d < D; ++d) A[d] += w[j] * ld(v, dtype, vo + d);
+                }
+                double nrm = 0.0;
+                for (int d = 0; d < D; ++d) nrm += A[d] * A[d];
+                nrm = sqrt(nrm);
+                const double an = nrm > 1e-30 ? nrm : 1e-30;
+                const double neff = l * l / l2;
+                const double lnL = log((double)cfg->L);
+                const double Tm = tanh(log(neff) / lnL);
+                /* backward */
+                const float *uh = u + (int64_t)h * D;
+                double gamma = 0.0, cg = 0.0;
+                for (int d = 0; d < D; ++d) {
+                    du_part[((int64_t)b * Hq + h) * D + d] += gate * Tm * gr[d];
+                    gamma += gr[d] * (double)uh[d];
+                    cg += (A[d] / an) * gr[d];
+                }
+                const double dgate = gamma * Tm, dT = gamma * gate;
+                const double dneff = dT * (1.0 - Tm * Tm) / (neff * lnL);
+                const double dl = dneff * 2.0 * l / l2;
+#if ORACLE_MUTANT == 12
+                const double dl2 = dneff * (l / l2) * (l / l2);
+#else
+                const double dl2 = -dneff * (l / l2) * (l / l2);
+#endif
+                double dA[256];
+                for (int d = 0; d < D; ++d) dA[d] = (gr[d] - (A[d] / an) * cg) / an;
+                const double dm = cfg->beta * gate * (1.0 - gate) * dgate;
+                const double dmu = -dm, dsigma = -dm * kn;
+                for (int64_t j = 0; j < n; ++j) {
+                    const int64_t ko = (((int64_t)b * T + lo + j) * Hkv + g) * D;
+                    double av = 0.0;
+                    for (int d = 0; d < D; ++d) av += dA[d] * ld(v, dtype, ko + d);
+                    double dz = w[j] * (dl + 2.0 * dl2 * w[j] + av) + dmu / (double)n;
+#if ORACLE_MUTANT != 11
+                    if (sigma > 0.0) dz += dsigma * (z[j] - mu) / ((double)n * sigma);
+#endif
+                    if (j == jmax) dz += dm;
+                    const double dS = c * dz;
+                    for (int d = 0; d < D; ++d) {
+                        dq[qo + d] += dS * ld(k, dtype, ko + d);
+                        dk[ko + d] += dS * qr[d];
+                        dv[ko + d] += w[j] * dA[d];
+                    }
+                }
+            }
+        }
+        free(z);
+        free(w);
+    }
+    memset(du, 0, sizeof(double) * (size_t)Hq * D);
+    for (int b = 0; b < B; ++b)
+        for (int64_t e = 0; e < (int64_t)Hq * D; ++e) du[e] += du_part[(int64_t)b * Hq * D + e];
+    free(du_part);
+    return bad ? -1 : 0;
+}
+
 /* Compile-time mutant id, so a test can confirm which build it loaded. */
 int oracle_mutant_id(void) { return ORACLE_MUTANT; }

@@ -358,6 +358,52 @@ def pin_window(mutant=0, bd=None):
     _close(dc.out, win.out[[T - 1, 2 * T - 1]], rtol=0, atol=0, what="windowed decode")
 
 
+# --------------------------------------------------------------------------
+# 11. backward: the oracle's analytic gradients of L = <out, G> (G random)
+#     against central finite differences of the oracle's own forward, for
+#     coordinates of q, k, v and u, with and without a window.  The forward is
+#     pinned by 1-10, so this ties the gradient to the pages' forms.
+# --------------------------------------------------------------------------
+def pin_backward_finite_differences(mutant=0, bd=None):
+    rng = np.random.default_rng(15)
+    T, Hq, Hkv = 24, 4, 2
+    q, k, v, u = _rand_inputs(rng, B=1, T=T, Hq=Hq, Hkv=Hkv)
+    u = (0.5 * rng.standard_normal(u.shape)).astype(np.float32)  # a count large enough to matter
+    G = rng.standard_normal((1, T, Hq, 64))
+    for p in (Params(L=4, alpha=0.3), Params(L=4, alpha=0.3, window=9)):
+        dq, dk, dv, du = oracle.polar_bwd(q, k, v, u, G, p, mutant=mutant, build_dir=bd)
+
+        def loss(qq, kk, vv, uu):
+            r = oracle.polar_fwd(qq, kk, vv, uu, p, mutant=mutant, build_dir=bd)
+            out = r.out.reshape(1, Hq, T, 64).transpose(0, 2, 1, 3)
+            return float(np.sum(out * G))
+
+        def fd(arrs, which, idx, eps=1e-3):
+            a = list(arrs)
+            x = a[which]
+            xp, xm = x.copy(), x.copy()
+            xp[idx] = np.float32(x[idx] + eps)
+            xm[idx] = np.float32(x[idx] - eps)
+            step = float(xp[idx]) - float(xm[idx])  # exact: both ends are fp32 values
+            a[which] = xp
+            lp = loss(*a)
+            a[which] = xm
+            lm = loss(*a)
+            return (lp - lm) / step
+
+        arrs = (q, k, v, u)
+        grads = (dq, dk, dv, du)
+        for which in range(4):
+            for _ in range(6):
+                idx = tuple(int(rng.integers(0, n)) for n in arrs[which].shape)
+                num = fd(arrs, which, idx)
+                ana = grads[which][idx]
+                scale = max(1e-3, np.max(np.abs(grads[which])))
+                assert abs(num - ana) <= 2e-4 * scale, \
+                    f"grad {'qkvu'[which]}{idx} window={p.window}: fd {num:.6e} vs {ana:.6e}"
+
+
 ALL_PINS = [pin_modes_agree, pin_uniform, pin_uniform_train_length_constant, pin_closed_form,
             pin_temperature_constants, pin_unit_norm_and_bounded, pin_duplication,
-            pin_causality, pin_gqa, pin_decode_matches_prefill, pin_window]
+            pin_causality, pin_gqa, pin_decode_matches_prefill, pin_window,
+            pin_backward_finite_differences]

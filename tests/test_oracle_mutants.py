@@ -5,14 +5,15 @@ plants one plausible mistake: a dropped square in the l2 correction, n_eff =
 l/l2, a flipped gate sign, an off-by-one causal bound, a transposed GQA
 mapping, a sample (not population) std, a log2 temperature, a dropped factor 2
 under the null-floor root, a missing unit-sphere projection, and the wrong
-head's count vector.
+head's count vector; in the backward, a dropped null-floor spread term and a
+flipped sign on the squared-sum gradient.
 """
 import pytest
 
 import oracle
 import oracle_pins as P
 
-MUTANTS = list(range(1, 11))
+MUTANTS = list(range(1, 13))
 
 
 @pytest.fixture(scope="module")
