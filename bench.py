@@ -62,6 +62,9 @@ def parse_args(argv=None):
                     help="prefill workload (profiling runs use a smaller one)")
     ap.add_argument("--decode-seqs", type=int, default=W.DECODE.num_seqs,
                     help="decode sequences (profiling runs use fewer)")
+    ap.add_argument("--bwd-steps", type=int, default=10,
+                    help="timed launches of the prefill backward on the train-length workload "
+                         "(0 skips it)")
     ap.add_argument("--window", type=int, default=4096,
                     help="sliding window of the separately timed windowed prefill (0 skips it)")
     ap.add_argument("--chunk", type=int, default=4,
@@ -350,6 +353,42 @@ def run_ours(args):
         t_win = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in ew) / 1e3, world, dev)
         window_res = (wp, t_win)
 
+    # ---- prefill backward on the train-length workload, timed on its own ----
+    bwd_res = None
+    if do_pre and args.bwd_steps > 0:
+        wb = W.TRAIN
+        xb = W.prefill_inputs(wb, dev, seed=seed + 1)
+        gb = torch.randn(xb["q"].shape, device=dev, generator=torch.Generator(device=dev).manual_seed(seed)).to(xb["q"].dtype)
+        gq = torch.empty(xb["q"].shape, device=dev)
+        gk = torch.empty(xb["k"].shape, device=dev)
+        gv = torch.empty(xb["v"].shape, device=dev)
+        gu = torch.empty(xb["u"].shape, device=dev)
+        wsb = torch.empty(pa.bwd_workspace_size(wb.B, wb.T, wb.Hq, wb.Hkv), device=dev,
+                          dtype=torch.uint8)
+
+        def backward():
+            pa.bwd(xb["q"], xb["k"], xb["v"], xb["u"], gb, gq, gk, gv, gu, wsb, stream=stream,
+                   s=wb.s, alpha=wb.alpha, L=wb.L, beta=wb.beta)
+
+        for _ in range(min(Wm, 3)):
+            backward()
+        torch.cuda.synchronize(dev)
+        Kb = args.bwd_steps
+        eb = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(Kb)]
+        barrier(world, dev)
+        torch.cuda.synchronize(dev)
+        for i in range(Kb):
+            eb[i][0].record(stream)
+            backward()
+            eb[i][1].record(stream)
+        torch.cuda.synchronize(dev)
+        barrier(world, dev)
+        if pa.get_status() != 0:
+            raise RuntimeError("device status after the backward")
+        t_b = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in eb) / 1e3, world, dev)
+        bwd_res = (wb, Kb, t_b)
+        del xb, gb, gq, gk, gv, gu, wsb
+
     # ---- multi-token decode (chunk query tokens per sequence), timed on its own ----
     chunk_res = None
     if do_dec and args.chunk > 1:
@@ -479,6 +518,16 @@ def run_ours(args):
             "clocks": clk.summary(),
             "e2e": e2e,
         }
+        if bwd_res is not None:
+            wb, Kb, t_b = bwd_res
+            b_launch = t_b / Kb
+            b_fl = 2.5 * wb.flops
+            result["backward"] = {
+                "workload": wb.describe(), "value": b_fl / b_launch / 1e12, "unit": "TFLOP/s",
+                "ms_per_launch": b_launch * 1e3, "flops_per_launch": b_fl, "launches": Kb,
+                "note": "prefill backward (polar_attn_bwd: dq, dk, dv, du; CUDA-core fp32), flops "
+                        "counted as 2.5x the forward's visible-pair flops; timed separately; not "
+                        "part of value"}
         if window_res is not None:
             wp, t_win = window_res
             w_launch = t_win / K

@@ -122,6 +122,34 @@ polar_status_t polar_attn_fwd(const void *q, const void *k, const void *v, const
                               const polar_params_t *params, void *out, float *neff_out,
                               void *workspace, size_t ws_bytes, void *stream);
 
+/*
+ * Backward of the causal prefill: the gradients of a loss L with respect to
+ * q, k, v and u, given dout = dL/dout (the training use of the fused step).
+ * Each row's forward state is recomputed, and the chain rule runs through
+ * the direction (acc/|acc|), the participation ratio n_eff = l^2/l2, the
+ * tanh-log magnitude, the gate on max logit - null floor, and the floor's mean
+ * and spread.  The max contributes through its first index (a subgradient).
+ * The window (params->window) is honoured; the key-moment workspace of
+ * polar_attn_fwd plays no part.
+ *
+ *  q, k, v, u  as polar_attn_fwd (dtype bf16 or fp32)
+ *  dout       [B, T, Hq, 64] dtype, device
+ *  dq         [B, T, Hq, 64] float32, device
+ *  dk, dv     [B, T, Hkv, 64] float32, device (summed over the group's heads)
+ *  du         [Hq, 64] float32, device (summed over batch and rows)
+ *  workspace  device scratch of at least polar_attn_bwd_workspace_size() bytes
+ *             (per-row coefficients); contents on entry are ignored
+ *
+ * Computed on the CUDA cores in fp32; deterministic.  B = 0 or T = 0 writes
+ * du = 0 and nothing else.
+ */
+size_t polar_attn_bwd_workspace_size(const polar_params_t *params);
+
+polar_status_t polar_attn_bwd(const void *q, const void *k, const void *v, const float *u,
+                              const void *dout, const polar_params_t *params, float *dq,
+                              float *dk, float *dv, float *du, void *workspace, size_t ws_bytes,
+                              void *stream);
+
 /* Bytes of device staging that polar_attn_fwd_host needs for this shape
  * (inputs, outputs and the workspace). */
 size_t polar_attn_fwd_staging_size(const polar_params_t *params);

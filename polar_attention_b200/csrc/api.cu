@@ -178,6 +178,36 @@ polar_status_t polar_attn_fwd(const void *q, const void *k, const void *v, const
     return from_cuda(launch_fwd_simt(a));
 }
 
+size_t polar_attn_bwd_workspace_size(const polar_params_t *p) {
+    if (check_fwd(p) != POLAR_OK) return 0;
+    return bwd_workspace_bytes(p->B, p->T, p->Hq);
+}
+
+polar_status_t polar_attn_bwd(const void *q, const void *k, const void *v, const float *u,
+                              const void *dout, const polar_params_t *p, float *dq, float *dk,
+                              float *dv, float *du, void *workspace, size_t ws_bytes,
+                              void *stream) {
+    polar_status_t st = check_fwd(p);
+    if (st != POLAR_OK) return st;
+    if (!du || !aligned16(du)) return POLAR_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (p->B == 0 || p->T == 0)
+        return from_cuda(cudaMemsetAsync(du, 0, static_cast<size_t>(p->Hq) * kHeadDim * 4, s));
+    if (!q || !k || !v || !u || !dout || !dq || !dk || !dv || !workspace)
+        return POLAR_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(u) || !aligned16(dout) ||
+        !aligned16(dq) || !aligned16(dk) || !aligned16(dv) || !aligned16(workspace))
+        return POLAR_ERR_INVALID_ARG;
+    if (ws_bytes < bwd_workspace_bytes(p->B, p->T, p->Hq)) return POLAR_ERR_WORKSPACE;
+    BwdLaunch a;
+    a.q = q; a.k = k; a.v = v; a.dout = dout; a.u = u;
+    a.dq = dq; a.dk = dk; a.dv = dv; a.du = du;
+    a.B = p->B; a.T = p->T; a.Hq = p->Hq; a.Hkv = p->Hkv; a.dtype = p->dtype;
+    a.s = p->logit_scale; a.alpha = p->alpha; a.beta = p->beta; a.L = p->L_train;
+    a.window = p->window; a.workspace = workspace; a.stream = s;
+    return from_cuda(launch_bwd(a));
+}
+
 size_t polar_attn_fwd_staging_size(const polar_params_t *p) {
     if (check_fwd(p) != POLAR_OK) return 0;
     const size_t e = dtype_bytes(p->dtype);

@@ -44,10 +44,25 @@ struct DecodeLaunch {
     cudaStream_t stream;
 };
 
+struct BwdLaunch {
+    const void *q, *k, *v, *dout;  // dtype; dout like out
+    const float *u;
+    float *dq, *dk, *dv, *du;      // fp32 gradients, layouts of q, k, v, u
+    int B, T, Hq, Hkv;
+    int dtype;
+    float s, alpha, beta;
+    int L;
+    int window;
+    void *workspace;               // bwd_workspace_bytes
+    cudaStream_t stream;
+};
+
 // Launchers return cudaSuccess or the launch error.
 cudaError_t launch_fwd_simt(const FwdLaunch &a);
 cudaError_t launch_fwd_tc(const FwdLaunch &a);
 cudaError_t launch_decode(const DecodeLaunch &a);
+cudaError_t launch_bwd(const BwdLaunch &a);
+size_t bwd_workspace_bytes(int B, int T, int Hq);
 
 // Key moments of causal prefill (fwd_moments.cu): one record of kMomFloats
 // fp32 (the 64 x 64 key Gram, then the 64 key sums) per (batch, kv head, full

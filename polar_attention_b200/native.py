@@ -28,7 +28,8 @@ EXPORTS = ["polar_attn_default_params", "polar_attn_fwd_workspace_size", "polar_
            "polar_attn_decode_staging_size", "polar_attn_decode_paged_host",
            "polar_attn_get_status", "polar_attn_status_string", "polar_attn_launch_count",
            "polar_attn_decode_paged_noalloc", "polar_attn_selftest_exp2",
-           "polar_attn_decode_chunk_workspace_size", "polar_attn_decode_paged_chunk"]
+           "polar_attn_decode_chunk_workspace_size", "polar_attn_decode_paged_chunk",
+           "polar_attn_bwd_workspace_size", "polar_attn_bwd"]
 
 
 class PolarError(RuntimeError):
@@ -68,6 +69,9 @@ def lib() -> ctypes.CDLL:
             L.polar_attn_fwd_workspace_size.argtypes = [PP]
             L.polar_attn_fwd_workspace_size.restype = Z
             L.polar_attn_fwd.argtypes = [P, P, P, P, PP, P, P, P, Z, P]
+            L.polar_attn_bwd_workspace_size.argtypes = [PP]
+            L.polar_attn_bwd_workspace_size.restype = Z
+            L.polar_attn_bwd.argtypes = [P, P, P, P, P, PP, P, P, P, P, P, Z, P]
             L.polar_attn_fwd_staging_size.argtypes = [PP]
             L.polar_attn_fwd_staging_size.restype = Z
             L.polar_attn_fwd_host.argtypes = [P, P, P, P, PP, P, P, P, Z, P]
@@ -89,7 +93,7 @@ def lib() -> ctypes.CDLL:
             for name in ("polar_attn_fwd", "polar_attn_fwd_host", "polar_attn_decode_paged",
                          "polar_attn_decode_paged_host", "polar_attn_get_status",
                          "polar_attn_decode_paged_noalloc", "polar_attn_selftest_exp2",
-                         "polar_attn_decode_paged_chunk"):
+                         "polar_attn_decode_paged_chunk", "polar_attn_bwd"):
                 getattr(L, name).restype = I
             _lib = L
     return _lib
@@ -172,6 +176,39 @@ def fwd(q, k, v, u, out=None, neff=None, workspace=None, *, s=8.0, alpha=0.3, L=
                                 _ptr(neff), _ptr(workspace), ws_bytes, _stream(stream)),
            "polar_attn_fwd")
     return out, neff
+
+
+def bwd_workspace_size(B: int, T: int, Hq: int, Hkv: int) -> int:
+    p = make_params(B, T, Hq, Hkv, POLAR_BF16)
+    return int(lib().polar_attn_bwd_workspace_size(ctypes.byref(p)))
+
+
+def bwd(q, k, v, u, dout, dq=None, dk=None, dv=None, du=None, workspace=None, *, s=8.0,
+        alpha=0.3, L=2048, beta=1.0, window=0, stream=None):
+    """Backward of the causal prefill.  q, dout [B,T,Hq,64] and k, v [B,T,Hkv,64]
+    (bf16 or fp32, CUDA, contiguous), u [Hq,64] fp32.  Returns fp32
+    (dq, dk, dv, du) shaped like q, k, v, u."""
+    B, T, Hq, D = q.shape
+    Hkv = k.shape[2]
+    for t in (q, k, v, u, dout):
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError("inputs must be contiguous CUDA tensors")
+    if dout.dtype != q.dtype:
+        raise TypeError("dout must have the dtype of q")
+    p = make_params(B, T, Hq, Hkv, _dt(q), s, alpha, L, beta, "auto", window)
+    p.head_dim = D
+    f32 = torch.float32
+    dq = torch.empty(q.shape, device=q.device, dtype=f32) if dq is None else dq
+    dk = torch.empty(k.shape, device=q.device, dtype=f32) if dk is None else dk
+    dv = torch.empty(v.shape, device=q.device, dtype=f32) if dv is None else dv
+    du = torch.empty(u.shape, device=q.device, dtype=f32) if du is None else du
+    need = int(lib().polar_attn_bwd_workspace_size(ctypes.byref(p)))
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), device=q.device, dtype=torch.uint8)
+    _check(lib().polar_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(u), _ptr(dout), ctypes.byref(p),
+                                _ptr(dq), _ptr(dk), _ptr(dv), _ptr(du), _ptr(workspace),
+                                workspace.numel(), _stream(stream)), "polar_attn_bwd")
+    return dq, dk, dv, du
 
 
 def decode_workspace_size(num_seqs: int, max_pages: int, Hq: int, Hkv: int) -> int:

@@ -51,6 +51,15 @@ def oracle_decode_chunk(w, x, q, rows=None):
                                x["u"].detach().cpu().numpy(), oracle_params(w), rows=rows)
 
 
+def oracle_bwd(w, x, gout):
+    """Oracle gradients (dq, dk, dv, du) in fp64 for the upstream gradient gout
+    (a CUDA or host tensor shaped like q, any float dtype; widened exactly)."""
+    h = {k: W.to_host_bits(x[k]) for k in ("q", "k", "v")}
+    g = gout.detach().float().cpu().numpy().astype(np.float64)
+    return oracle.polar_bwd(h["q"], h["k"], h["v"], x["u"].detach().cpu().numpy(), g,
+                            oracle_params(w))
+
+
 def gpu_rows_prefill(out, neff, rows, B, T, Hq):
     """Gather flat oracle rows ((b*Hq + h)*T + i) from GPU out [B,T,Hq,D] and
     neff [B,Hq,T]."""
