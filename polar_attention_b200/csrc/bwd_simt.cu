@@ -17,7 +17,8 @@
 //   dS_j    = c dz_j;  dq += dS_j k_j;  dk_j += dS_j q;  dv_j += w_j dA.
 // (w, l, l2 and A may share any reference: content and n_eff are scale-free.)
 //
-// Four launches, all FP32 on the CUDA cores:
+// Four launches (FP32 on the CUDA cores, except that for bf16 inputs passes 2
+// and 3 run their contractions on the tensor cores, see below):
 //  1. rows: one thread per query row recomputes the row's forward state
 //     (streaming, as the CUDA-core prefill does, plus the first argmax) and
 //     writes the row's coefficients: dA, the reference and scales, dl, dl2,
@@ -31,6 +32,8 @@
 //  4. du: per head, the sum over rows of gate * T * g.
 // Each kernel recomputes S_j with the same fp32 summation order, so the argmax
 // test is an index comparison.
+#include <type_traits>
+
 #include "polar_common.cuh"
 #include "polar_internal.h"
 
@@ -214,7 +217,8 @@ bwd_rows_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__res
                         (qr[d + 3] - acc[d + 3] * inv_an * cg) * inv_an);
     *reinterpret_cast<float4 *>(rec + 64) = make_float4(m_ref, cl2, c, dl);
     *reinterpret_cast<float4 *>(rec + 68) = make_float4(dl2, cmu, csS, dm);
-    *reinterpret_cast<float4 *>(rec + 72) =
+    static_assert(kRecJmax == 72 && kRecLo == 73 && kRecGT == 74, "record layout");
+    *reinterpret_cast<float4 *>(rec + kRecJmax) =
         make_float4(__int_as_float(jmax), __int_as_float(lo), gate * Tm, 0.0f);
 }
 
@@ -420,6 +424,273 @@ bwd_dq_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restr
         *reinterpret_cast<float4 *>(dq + qo + d) = make_float4(dqr[d], dqr[d + 1], dqr[d + 2], dqr[d + 3]);
 }
 
+
+// ------------------------------------------- tensor-core (mma.sync) kernels ---
+// For bf16 inputs the contractions of the dk/dv and dq passes run on the
+// tensor cores (m16n8k16, bf16 in, fp32 accumulate): the scores and <dA, v>
+// are recomputed as tile products, dz is formed in the accumulator fragments
+// and re-packed as the A operand of the gradient products (dA, dS and w are
+// rounded to bf16 for those products).  Tiles of 64 rows x 64 dims live in
+// shared memory with a 144-byte row pitch, so that the ldmatrix reads are free
+// of bank conflicts.
+constexpr int kPitch = 72;  // bf16 per padded row (144 bytes)
+
+__device__ __forceinline__ void ldsm4(uint32_t addr, uint32_t (&r)[4]) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr));
+}
+__device__ __forceinline__ void ldsm4t(uint32_t addr, uint32_t (&r)[4]) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr));
+}
+__device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                         uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ uint32_t pk2(float lo, float hi) {
+    uint32_t r;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+// A fragments (16 rows x 64, 4 k-steps) of rows r0 + lane/4 and r0 + lane/4 + 8
+// of a bf16 [*, stride] matrix in global memory; rows at or past `rows` are 0.
+__device__ __forceinline__ void load_a_rows(const __nv_bfloat16 *base, size_t stride, int r0,
+                                            int rows, uint32_t (&fa)[4][4]) {
+    const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+    const int ra = r0 + g, rb = r0 + g + 8;
+    const uint32_t *pa = reinterpret_cast<const uint32_t *>(base + static_cast<size_t>(ra < rows ? ra : 0) * stride);
+    const uint32_t *pb = reinterpret_cast<const uint32_t *>(base + static_cast<size_t>(rb < rows ? rb : 0) * stride);
+#pragma unroll
+    for (int ks = 0; ks < 4; ++ks) {
+        fa[ks][0] = ra < rows ? pa[8 * ks + t] : 0u;
+        fa[ks][1] = rb < rows ? pb[8 * ks + t] : 0u;
+        fa[ks][2] = ra < rows ? pa[8 * ks + 4 + t] : 0u;
+        fa[ks][3] = rb < rows ? pb[8 * ks + 4 + t] : 0u;
+    }
+}
+
+// Copy 64 rows (64 bf16 each) into a padded shared tile; rows past `valid` are 0.
+__device__ __forceinline__ void stage_rows(__nv_bfloat16 (*dst)[kPitch], const __nv_bfloat16 *src,
+                                           size_t stride, int valid) {
+    for (int e = threadIdx.x; e < 64 * 8; e += blockDim.x) {
+        const int r = e >> 3, c = e & 7;
+        uint4 val = make_uint4(0u, 0u, 0u, 0u);
+        if (r < valid) val = *reinterpret_cast<const uint4 *>(src + static_cast<size_t>(r) * stride + 8 * c);
+        *reinterpret_cast<uint4 *>(&dst[r][8 * c]) = val;
+    }
+}
+
+// S-like products of a warp's 16 A rows with 64 shared rows: out[nt] holds
+// columns 8nt .. 8nt+7 (the shared rows), i.e. sum over the 64 dims of
+// A[row][d] * M[col][d].
+__device__ __forceinline__ void rows_times_tile(const uint32_t (&fa)[4][4], uint32_t tile,
+                                                float (&out)[8][4]) {
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int nt = 0; nt < 8; ++nt) {
+        out[nt][0] = out[nt][1] = out[nt][2] = out[nt][3] = 0.f;
+#pragma unroll
+        for (int kk = 0; kk < 2; ++kk) {  // 32 dims per ldmatrix.x4
+            uint32_t b[4];
+            ldsm4(tile + ((8 * nt + (lane & 7)) * kPitch + 32 * kk + 8 * (lane >> 3)) * 2, b);
+            mma16816(out[nt], fa[2 * kk], b[0], b[1]);
+            mma16816(out[nt], fa[2 * kk + 1], b[2], b[3]);
+        }
+    }
+}
+
+// acc[nt] += P (16 x 64, as 4 k-steps of A fragments) times the 64 x 64 shared
+// tile (rows = the k dimension, columns = the 64 dims): columns 8nt .. 8nt+7.
+__device__ __forceinline__ void frag_times_tile(const uint32_t (&pa)[4][4], uint32_t tile,
+                                                float (&acc)[8][4]) {
+    const int lane = threadIdx.x & 31, mi = lane >> 3;
+#pragma unroll
+    for (int ks = 0; ks < 4; ++ks)
+#pragma unroll
+        for (int p = 0; p < 4; ++p) {  // dims 16p .. 16p+15: two n-tiles
+            uint32_t b[4];
+            ldsm4t(tile + ((16 * ks + (lane & 7) + 8 * (mi & 1)) * kPitch + 16 * p + 8 * (mi >> 1)) * 2, b);
+            mma16816(acc[2 * p], pa[ks], b[0], b[1]);
+            mma16816(acc[2 * p + 1], pa[ks], b[2], b[3]);
+        }
+}
+
+// dq for bf16 inputs: a warp owns 16 query rows; keys stream in blocks of 64.
+__global__ void __launch_bounds__(128)
+bwd_dq_mma_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
+                  const __nv_bfloat16 *__restrict__ v, float *__restrict__ dq, const BwdArgs a) {
+    __shared__ __align__(16) __nv_bfloat16 Ks[64][kPitch];
+    __shared__ __align__(16) __nv_bfloat16 Vs[64][kPitch];
+    const int Tlen = a.T, G = a.Hq / a.Hkv;
+    const int row0 = blockIdx.x * 64, h = blockIdx.y, b = blockIdx.z, g = h / G;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, gq = lane >> 2, tq = lane & 3;
+    const int r0 = row0 + 16 * warp;
+    const size_t qstride = static_cast<size_t>(a.Hq) * kHeadDim;
+    const size_t kstride = static_cast<size_t>(a.Hkv) * kHeadDim;
+    uint32_t qa[4][4], da[4][4];
+    load_a_rows(q + (static_cast<size_t>(b) * Tlen * a.Hq + h) * kHeadDim, qstride, r0, Tlen, qa);
+    // dA rows from the records, rounded to bf16.
+    RowCoef cf[2];
+    int rowi[2];
+#pragma unroll
+    for (int hr = 0; hr < 2; ++hr) {
+        const int r = r0 + gq + 8 * hr;
+        rowi[hr] = r;
+        const float *rp = a.rec + ((static_cast<size_t>(b) * a.Hq + h) * Tlen + (r < Tlen ? r : 0)) * kRecWords;
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks) {
+            const float2 x0 = *reinterpret_cast<const float2 *>(rp + 16 * ks + 2 * tq);
+            const float2 x1 = *reinterpret_cast<const float2 *>(rp + 16 * ks + 8 + 2 * tq);
+            da[ks][hr] = r < Tlen ? pk2(x0.x, x0.y) : 0u;
+            da[ks][2 + hr] = r < Tlen ? pk2(x1.x, x1.y) : 0u;
+        }
+        cf[hr] = load_coef(rp);
+    }
+    float acc[8][4];
+#pragma unroll
+    for (int nt = 0; nt < 8; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
+    const uint32_t ks_addr = smem_u32(&Ks[0][0]), vs_addr = smem_u32(&Vs[0][0]);
+    const int kend = min(Tlen, row0 + 64);
+    const int kbeg = a.window > 0 ? max(0, row0 - a.window + 1) / 64 * 64 : 0;
+    for (int j0 = kbeg; j0 < kend; j0 += 64) {
+        __syncthreads();
+        stage_rows(Ks, k + ((static_cast<size_t>(b) * Tlen + j0) * a.Hkv + g) * kHeadDim, kstride, Tlen - j0);
+        stage_rows(Vs, v + ((static_cast<size_t>(b) * Tlen + j0) * a.Hkv + g) * kHeadDim, kstride, Tlen - j0);
+        __syncthreads();
+        float sc[8][4], av[8][4];
+        rows_times_tile(qa, ks_addr, sc);
+        rows_times_tile(da, vs_addr, av);
+        uint32_t pa[4][4];
+#pragma unroll
+        for (int nt = 0; nt < 8; ++nt) {
+            float ds[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int hr = e >> 1, i = rowi[hr], j = j0 + 8 * nt + 2 * tq + (e & 1);
+                const bool vis = i < Tlen && j < Tlen && j <= i && j >= cf[hr].lo;
+                float w;
+                const float x = pair_ds(cf[hr], sc[nt][e], av[nt][e], j, w);
+                ds[e] = vis ? x : 0.f;
+            }
+            pa[nt >> 1][(nt & 1) * 2] = pk2(ds[0], ds[1]);
+            pa[nt >> 1][(nt & 1) * 2 + 1] = pk2(ds[2], ds[3]);
+        }
+        frag_times_tile(pa, ks_addr, acc);
+    }
+#pragma unroll
+    for (int hr = 0; hr < 2; ++hr) {
+        const int r = rowi[hr];
+        if (r >= Tlen) continue;
+        float *dst = dq + ((static_cast<size_t>(b) * Tlen + r) * a.Hq + h) * kHeadDim;
+#pragma unroll
+        for (int nt = 0; nt < 8; ++nt)
+            *reinterpret_cast<float2 *>(dst + 8 * nt + 2 * tq) = make_float2(acc[nt][2 * hr], acc[nt][2 * hr + 1]);
+    }
+}
+
+// dk, dv for bf16 inputs: a warp owns 16 keys; the rows that see them stream
+// in blocks of 64, for every query head of the group.
+__global__ void __launch_bounds__(128)
+bwd_dkdv_mma_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
+                    const __nv_bfloat16 *__restrict__ v, float *__restrict__ dk,
+                    float *__restrict__ dv, const BwdArgs a) {
+    __shared__ __align__(16) __nv_bfloat16 Qs[64][kPitch];
+    __shared__ __align__(16) __nv_bfloat16 DAs[64][kPitch];
+    __shared__ float Cs[64][12];  // per staged row: ref cl2 c dl dl2 cmu csS dm jmax lo valid
+    const int Tlen = a.T, G = a.Hq / a.Hkv;
+    const int key0 = blockIdx.x * 64, g = blockIdx.y, b = blockIdx.z;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, gq = lane >> 2, tq = lane & 3;
+    const int k0 = key0 + 16 * warp;
+    const size_t kstride = static_cast<size_t>(a.Hkv) * kHeadDim;
+    uint32_t ka[4][4], va[4][4];
+    load_a_rows(k + (static_cast<size_t>(b) * Tlen * a.Hkv + g) * kHeadDim, kstride, k0, Tlen, ka);
+    load_a_rows(v + (static_cast<size_t>(b) * Tlen * a.Hkv + g) * kHeadDim, kstride, k0, Tlen, va);
+    float dka[8][4], dva[8][4];
+#pragma unroll
+    for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) dka[nt][e] = dva[nt][e] = 0.f;
+    const uint32_t qs_addr = smem_u32(&Qs[0][0]), da_addr = smem_u32(&DAs[0][0]);
+    const int iend = a.window > 0 ? min(Tlen, key0 + 63 + a.window) : Tlen;
+    for (int hh = 0; hh < G; ++hh) {
+        const int h = g * G + hh;
+        const size_t qstride = static_cast<size_t>(a.Hq) * kHeadDim;
+        for (int i0 = key0; i0 < iend; i0 += 64) {
+            __syncthreads();
+            stage_rows(Qs, q + ((static_cast<size_t>(b) * Tlen + i0) * a.Hq + h) * kHeadDim, qstride, Tlen - i0);
+            for (int e = threadIdx.x; e < 64 * 32; e += 128) {  // dA as bf16 pairs
+                const int r = e >> 5, c = e & 31, i = i0 + r;
+                uint32_t val = 0u;
+                if (i < Tlen) {
+                    const float2 x = *reinterpret_cast<const float2 *>(
+                        a.rec + ((static_cast<size_t>(b) * a.Hq + h) * Tlen + i) * kRecWords + 2 * c);
+                    val = pk2(x.x, x.y);
+                }
+                *reinterpret_cast<uint32_t *>(&DAs[r][2 * c]) = val;
+            }
+            for (int e = threadIdx.x; e < 64 * 11; e += 128) {
+                const int r = e / 11, c = e % 11, i = i0 + r;
+                float val = 0.f;
+                if (i < Tlen) {
+                    const float *rp = a.rec + ((static_cast<size_t>(b) * a.Hq + h) * Tlen + i) * kRecWords;
+                    val = c < 10 ? rp[kRecRef + c] : 1.f;
+                } else if (c == 9) {
+                    val = __int_as_float(0x7fffffff);  // lo past every key: the row sees nothing
+                }
+                Cs[r][c] = val;
+            }
+            __syncthreads();
+            float st[8][4], at[8][4];
+            rows_times_tile(ka, qs_addr, st);  // S^T: keys x rows
+            rows_times_tile(va, da_addr, at);  // <v_j, dA_i>
+            uint32_t ps[4][4], pw[4][4];
+#pragma unroll
+            for (int nt = 0; nt < 8; ++nt) {
+                float ds[4], ws[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int rr = 8 * nt + 2 * tq + (e & 1), i = i0 + rr;
+                    const int j = k0 + gq + 8 * (e >> 1);
+                    RowCoef cf;
+                    cf.ref = Cs[rr][0]; cf.cl2 = Cs[rr][1]; cf.c = Cs[rr][2]; cf.dl = Cs[rr][3];
+                    cf.dl2 = Cs[rr][4]; cf.cmu = Cs[rr][5]; cf.csS = Cs[rr][6]; cf.dm = Cs[rr][7];
+                    cf.jmax = __float_as_int(Cs[rr][8]);
+                    cf.lo = __float_as_int(Cs[rr][9]);
+                    const bool vis = i < Tlen && j < Tlen && j <= i && j >= cf.lo;
+                    float w;
+                    const float x = pair_ds(cf, st[nt][e], at[nt][e], j, w);
+                    ds[e] = vis ? x : 0.f;
+                    ws[e] = vis ? w : 0.f;
+                }
+                ps[nt >> 1][(nt & 1) * 2] = pk2(ds[0], ds[1]);
+                ps[nt >> 1][(nt & 1) * 2 + 1] = pk2(ds[2], ds[3]);
+                pw[nt >> 1][(nt & 1) * 2] = pk2(ws[0], ws[1]);
+                pw[nt >> 1][(nt & 1) * 2 + 1] = pk2(ws[2], ws[3]);
+            }
+            frag_times_tile(ps, qs_addr, dka);  // dK += dS^T Q
+            frag_times_tile(pw, da_addr, dva);  // dV += W^T dA
+        }
+    }
+#pragma unroll
+    for (int hr = 0; hr < 2; ++hr) {
+        const int j = k0 + gq + 8 * hr;
+        if (j >= Tlen) continue;
+        const size_t off = ((static_cast<size_t>(b) * Tlen + j) * a.Hkv + g) * kHeadDim;
+#pragma unroll
+        for (int nt = 0; nt < 8; ++nt) {
+            *reinterpret_cast<float2 *>(dk + off + 8 * nt + 2 * tq) = make_float2(dka[nt][2 * hr], dka[nt][2 * hr + 1]);
+            *reinterpret_cast<float2 *>(dv + off + 8 * nt + 2 * tq) = make_float2(dva[nt][2 * hr], dva[nt][2 * hr + 1]);
+        }
+    }
+}
+
 // -------------------------------------------------------------------- du ---
 // du_h = sum over the row blocks of their partial sums (fixed order).
 __global__ void __launch_bounds__(kHeadDim)
@@ -436,10 +707,16 @@ cudaError_t launch_all(const BwdLaunch &l, const BwdArgs &a) {
             *v = static_cast<const T *>(l.v), *go = static_cast<const T *>(l.dout);
     bwd_rows_kernel<T><<<dim3((a.T + kRowsB0 - 1) / kRowsB0, a.Hq, a.B), kRowsB0, 0, l.stream>>>(
         q, k, v, go, a);
-    bwd_dkdv_kernel<T><<<dim3((a.T + kKeyTile - 1) / kKeyTile, a.Hkv, a.B), 128, 0, l.stream>>>(
-        q, k, v, l.dk, l.dv, a);
-    bwd_dq_kernel<T><<<dim3((a.T + kKeyTile - 1) / kKeyTile, a.Hq, a.B), 128, 0, l.stream>>>(
-        q, k, v, l.dq, a);
+    if constexpr (std::is_same<T, __nv_bfloat16>::value) {
+        bwd_dkdv_mma_kernel<<<dim3((a.T + 63) / 64, a.Hkv, a.B), 128, 0, l.stream>>>(
+            q, k, v, l.dk, l.dv, a);
+        bwd_dq_mma_kernel<<<dim3((a.T + 63) / 64, a.Hq, a.B), 128, 0, l.stream>>>(q, k, v, l.dq, a);
+    } else {
+        bwd_dkdv_kernel<T><<<dim3((a.T + kKeyTile - 1) / kKeyTile, a.Hkv, a.B), 128, 0, l.stream>>>(
+            q, k, v, l.dk, l.dv, a);
+        bwd_dq_kernel<T><<<dim3((a.T + kKeyTile - 1) / kKeyTile, a.Hq, a.B), 128, 0, l.stream>>>(
+            q, k, v, l.dq, a);
+    }
     bwd_du_kernel<<<a.Hq, kHeadDim, 0, l.stream>>>(l.du, a, a.B * ((a.T + kRowsB0 - 1) / kRowsB0));
     count_launches(4);
     return cudaGetLastError();

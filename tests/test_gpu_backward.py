@@ -11,11 +11,16 @@ from polar_attention_b200 import workloads as W
 
 pytestmark = pytest.mark.gpu
 
-GRAD_TOL = 2e-3  # normwise max|gpu - oracle| / max|oracle| per slice (fp32 arithmetic)
-# Gradients here are of order 0.01-10; where the exact gradient vanishes (one
-# visible key: the direction, gate and magnitude do not depend on q), fp32
-# leaves rounding residue of order 1e-7, so the scale has this floor.
-GRAD_FLOOR = 1e-3
+# normwise max|gpu - oracle| / max|oracle| per slice: fp32 inputs run fp32
+# arithmetic; bf16 inputs run the gradient products on the tensor cores with
+# dA, dS and the weights rounded to bf16 (the forward's bf16 output tolerance).
+GRAD_TOL = {"fp32": 2e-3, "bf16": 2e-2}
+# Where the exact gradient vanishes (one visible key: the direction, gate and
+# magnitude do not depend on q), what is left is rounding residue: about 1e-7
+# in fp32, and a few 1e-3 when <dA, v> runs on bf16 operands.  The slice scale
+# therefore has a floor, in the gradients' natural units (dq, dk, dv are of
+# order 1-10 here: c = 8 times unit vectors).
+GRAD_FLOOR = {"fp32": 1e-3, "bf16": 0.5}
 
 
 def _gout(w, seed):
@@ -39,12 +44,12 @@ def _slices(a, axis_heads):
     return [a[b, :, h] for b in range(B) for h in range(H)]
 
 
-def _check(name, got, ref, tol=GRAD_TOL):
+def _check(name, got, ref, tol, floor):
     assert np.all(np.isfinite(got)), f"{name}: non-finite gradient"
     worst = 0.0
     pairs = [(got, ref)] if got.ndim == 2 else list(zip(_slices(got, 2), _slices(ref, 2)))
     for g, r in pairs:
-        scale = max(np.max(np.abs(r)), GRAD_FLOOR)
+        scale = max(np.max(np.abs(r)), floor)
         worst = max(worst, np.max(np.abs(g - r)) / scale)
     assert worst <= tol, f"{name}: normwise error {worst:.3e} > {tol}"
     return worst
@@ -55,7 +60,7 @@ def _compare(w, x, seed=0):
     got = _run(w, x, gout)
     ref = PT.oracle_bwd(w, x, gout)
     for name, g, r in zip(("dq", "dk", "dv", "du"), got, ref):
-        _check(f"{name} T={w.T} window={w.window}", g, r)
+        _check(f"{name} T={w.T} window={w.window}", g, r, GRAD_TOL[w.dtype], GRAD_FLOOR[w.dtype])
 
 
 CASES = [(1, 2, 0, "bf16"), (77, 2, 0, "bf16"), (300, 4, 0, "bf16"), (300, 2, 64, "bf16"),
