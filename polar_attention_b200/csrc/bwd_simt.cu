@@ -17,8 +17,9 @@
 //   dS_j    = c dz_j;  dq += dS_j k_j;  dk_j += dS_j q;  dv_j += w_j dA.
 // (w, l, l2 and A may share any reference: content and n_eff are scale-free.)
 //
-// Four launches (FP32 on the CUDA cores, except that for bf16 inputs passes 2
-// and 3 run their contractions on the tensor cores, see below):
+// Four launches.  For fp32 inputs they run on the CUDA cores in fp32; for bf16
+// inputs passes 1-3 run their contractions on the tensor cores (mma.sync,
+// below):
 //  1. rows: one thread per query row recomputes the row's forward state
 //     (streaming, as the CUDA-core prefill does, plus the first argmax) and
 //     writes the row's coefficients: dA, the reference and scales, dl, dl2,
@@ -522,6 +523,212 @@ __device__ __forceinline__ void frag_times_tile(const uint32_t (&pa)[4][4], uint
         }
 }
 
+
+// Rows pass for bf16 inputs on the tensor cores: a warp owns 16 query rows
+// (two per lane: rows lane/4 and lane/4 + 8); key blocks of 64 stream through
+// shared memory.  S = Q K^T and O += P V are tile products; the row statistics
+// (first argmax, S1, S2, l, l2 under a lazy reference) come from the
+// accumulator fragments with quad shuffles.  The epilogue writes the same
+// record as bwd_rows_kernel, and a du partial per 64-row block.
+__global__ void __launch_bounds__(128)
+bwd_rows_mma_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
+                    const __nv_bfloat16 *__restrict__ v, const __nv_bfloat16 *__restrict__ gout,
+                    const BwdArgs a) {
+    __shared__ __align__(16) __nv_bfloat16 Ks[64][kPitch];
+    __shared__ __align__(16) __nv_bfloat16 Vs[64][kPitch];
+    __shared__ float red[4][kHeadDim];
+    const int Tlen = a.T, G = a.Hq / a.Hkv;
+    const int row0 = blockIdx.x * 64, h = blockIdx.y, b = blockIdx.z, g = h / G;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, gq = lane >> 2, tq = lane & 3;
+    const int r0 = row0 + 16 * warp;
+    const size_t qstride = static_cast<size_t>(a.Hq) * kHeadDim;
+    const size_t kstride = static_cast<size_t>(a.Hkv) * kHeadDim;
+    uint32_t qa[4][4];
+    load_a_rows(q + (static_cast<size_t>(b) * Tlen * a.Hq + h) * kHeadDim, qstride, r0, Tlen, qa);
+    int rowi[2], lo[2];
+    float cl2[2], cc[2];
+    float m_ref[2], m_raw[2], l[2], l2[2], s1[2], s2[2];
+    int jmax[2];
+#pragma unroll
+    for (int hr = 0; hr < 2; ++hr) {
+        const int i = r0 + gq + 8 * hr;
+        rowi[hr] = i;
+        lo[hr] = a.window > 0 ? max(0, i - a.window + 1) : 0;
+        const float n = static_cast<float>(i + 1 - lo[hr]);
+        cc[hr] = a.s * length_temperature(n, a.alpha, a.L);
+        cl2[hr] = cc[hr] * kLog2e;
+        m_ref[hr] = m_raw[hr] = -INFINITY;
+        l[hr] = l2[hr] = s1[hr] = s2[hr] = 0.f;
+        jmax[hr] = lo[hr];
+    }
+    float acc[8][4];
+#pragma unroll
+    for (int nt = 0; nt < 8; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
+    const uint32_t ks_addr = smem_u32(&Ks[0][0]), vs_addr = smem_u32(&Vs[0][0]);
+    const int kend = min(Tlen, row0 + 64);
+    const int kbeg = a.window > 0 ? max(0, row0 - a.window + 1) / 64 * 64 : 0;
+    for (int j0 = kbeg; j0 < kend; j0 += 64) {
+        __syncthreads();
+        stage_rows(Ks, k + ((static_cast<size_t>(b) * Tlen + j0) * a.Hkv + g) * kHeadDim, kstride, Tlen - j0);
+        stage_rows(Vs, v + ((static_cast<size_t>(b) * Tlen + j0) * a.Hkv + g) * kHeadDim, kstride, Tlen - j0);
+        __syncthreads();
+        float sc[8][4];
+        rows_times_tile(qa, ks_addr, sc);
+        float pw[8][4];
+#pragma unroll
+        for (int hr = 0; hr < 2; ++hr) {
+            const int i = rowi[hr];
+            float tmax = -INFINITY, ts1 = 0.f, ts2 = 0.f;
+            int tidx = 0x7fffffff;
+#pragma unroll
+            for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const int j = j0 + 8 * nt + 2 * tq + e;
+                    const bool vis = i < Tlen && j <= i && j >= lo[hr];
+                    const float x = sc[nt][2 * hr + e];
+                    if (vis && x > tmax) { tmax = x; tidx = j; }  // columns ascend within a lane
+                    ts1 += vis ? x : 0.f;
+                    ts2 += vis ? x * x : 0.f;
+                }
+#pragma unroll
+            for (int off = 1; off <= 2; off <<= 1) {
+                const float ov = __shfl_xor_sync(0xffffffffu, tmax, off);
+                const int oi = __shfl_xor_sync(0xffffffffu, tidx, off);
+                if (ov > tmax || (ov == tmax && oi < tidx)) { tmax = ov; tidx = oi; }
+            }
+            if (tmax > m_raw[hr]) { m_raw[hr] = tmax; jmax[hr] = tidx; }  // strict: first index
+            s1[hr] += ts1;
+            s2[hr] += ts2;
+            const float zmax = tmax * cl2[hr];
+            if (zmax > m_ref[hr] + kRescaleThreshold) {  // uniform over the quad
+                const float r = exp2f(m_ref[hr] - zmax);
+                l[hr] *= r;
+                l2[hr] *= r * r;
+#pragma unroll
+                for (int nt = 0; nt < 8; ++nt) {
+                    acc[nt][2 * hr] *= r;
+                    acc[nt][2 * hr + 1] *= r;
+                }
+                m_ref[hr] = zmax;
+            }
+#pragma unroll
+            for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const int j = j0 + 8 * nt + 2 * tq + e;
+                    const bool vis = i < Tlen && j <= i && j >= lo[hr];
+                    const float pp = vis ? exp2f(fmaf(sc[nt][2 * hr + e], cl2[hr], -m_ref[hr])) : 0.f;
+                    pw[nt][2 * hr + e] = pp;
+                    l[hr] += pp;
+                    l2[hr] = fmaf(pp, pp, l2[hr]);
+                }
+        }
+        uint32_t pa[4][4];
+#pragma unroll
+        for (int nt = 0; nt < 8; ++nt) {
+            pa[nt >> 1][(nt & 1) * 2] = pk2(pw[nt][0], pw[nt][1]);
+            pa[nt >> 1][(nt & 1) * 2 + 1] = pk2(pw[nt][2], pw[nt][3]);
+        }
+        frag_times_tile(pa, vs_addr, acc);  // O += P V
+    }
+
+    // Epilogue per row: quad sums of the partial statistics and dot products.
+    float dupart[8][2];
+#pragma unroll
+    for (int nt = 0; nt < 8; ++nt) dupart[nt][0] = dupart[nt][1] = 0.f;
+#pragma unroll
+    for (int hr = 0; hr < 2; ++hr) {
+        const int i = rowi[hr];
+        const bool live = i < Tlen;
+        float gr[8][2], nrm = 0.f, gamma = 0.f, cgr = 0.f;
+        const __nv_bfloat16 *gp = gout + ((static_cast<size_t>(b) * Tlen + (live ? i : 0)) * a.Hq + h) * kHeadDim;
+        const float *uh = a.u + static_cast<size_t>(h) * kHeadDim;
+#pragma unroll
+        for (int nt = 0; nt < 8; ++nt) {
+            const int d = 8 * nt + 2 * tq;
+            const __nv_bfloat162 gg = *reinterpret_cast<const __nv_bfloat162 *>(gp + d);
+            gr[nt][0] = live ? __low2float(gg) : 0.f;
+            gr[nt][1] = live ? __high2float(gg) : 0.f;
+            const float o0 = acc[nt][2 * hr], o1 = acc[nt][2 * hr + 1];
+            nrm = fmaf(o0, o0, fmaf(o1, o1, nrm));
+            gamma = fmaf(gr[nt][0], uh[d], fmaf(gr[nt][1], uh[d + 1], gamma));
+            cgr = fmaf(o0, gr[nt][0], fmaf(o1, gr[nt][1], cgr));
+        }
+        float ll = l[hr], ll2 = l2[hr], ss1 = s1[hr], ss2 = s2[hr];
+#pragma unroll
+        for (int off = 1; off <= 2; off <<= 1) {
+            nrm += __shfl_xor_sync(0xffffffffu, nrm, off);
+            gamma += __shfl_xor_sync(0xffffffffu, gamma, off);
+            cgr += __shfl_xor_sync(0xffffffffu, cgr, off);
+            ll += __shfl_xor_sync(0xffffffffu, ll, off);
+            ll2 += __shfl_xor_sync(0xffffffffu, ll2, off);
+            ss1 += __shfl_xor_sync(0xffffffffu, ss1, off);
+            ss2 += __shfl_xor_sync(0xffffffffu, ss2, off);
+        }
+        const float nf = static_cast<float>(live ? i + 1 - lo[hr] : 1);
+        const float c = cc[hr];
+        const float mean_s = ss1 / nf;
+        const float sig_s = sqrtf(fmaxf(ss2 / nf - mean_s * mean_s, 0.0f));
+        const float mu = c * mean_s, sigma = c * sig_s;
+        const float kn = sqrtf(2.0f * logf(nf));
+        const float z0 = mu + sigma * kn;
+        const float gate = 1.0f / (1.0f + expf(-a.beta * (c * m_raw[hr] - z0)));
+        const float ne_raw = (ll * ll) / ll2;
+        const float ne = fminf(fmaxf(ne_raw, 1.0f), nf);
+        const bool clamped = ne != ne_raw;
+        const float Tm = tanhf(logf(ne) * a.inv_ln_L);
+        const float an = fmaxf(sqrtf(nrm), 1e-30f), inv_an = 1.0f / an;
+        const float cg = cgr * inv_an;  // <content, g>
+        const float dgate = gamma * Tm, dT = gamma * gate;
+        const float dneff = clamped ? 0.0f : dT * (1.0f - Tm * Tm) * a.inv_ln_L / ne;
+        const float dl = 2.0f * dneff * ll / ll2;
+        const float dl2 = -dneff * (ll / ll2) * (ll / ll2);
+        const float dm = a.beta * gate * (1.0f - gate) * dgate;
+        const float dmu = -dm, dsigma = -dm * kn;
+        const float cmu = dmu / nf - (sigma > 0.0f ? dsigma * mu / (nf * sigma) : 0.0f);
+        const float csS = sigma > 0.0f ? dsigma * c / (nf * sigma) : 0.0f;
+        const float gt = live ? gate * Tm : 0.0f;
+#pragma unroll
+        for (int nt = 0; nt < 8; ++nt) {
+            dupart[nt][0] = fmaf(gt, gr[nt][0], dupart[nt][0]);
+            dupart[nt][1] = fmaf(gt, gr[nt][1], dupart[nt][1]);
+        }
+        if (!live) continue;
+        float *rec = a.rec + ((static_cast<size_t>(b) * a.Hq + h) * Tlen + i) * kRecWords;
+#pragma unroll
+        for (int nt = 0; nt < 8; ++nt) {
+            const int d = 8 * nt + 2 * tq;
+            const float o0 = acc[nt][2 * hr] * inv_an, o1 = acc[nt][2 * hr + 1] * inv_an;
+            *reinterpret_cast<float2 *>(rec + kRecDA + d) =
+                make_float2((gr[nt][0] - o0 * cg) * inv_an, (gr[nt][1] - o1 * cg) * inv_an);
+        }
+        if (tq == 0) {
+            *reinterpret_cast<float4 *>(rec + 64) = make_float4(m_ref[hr], cl2[hr], c, dl);
+            *reinterpret_cast<float4 *>(rec + 68) = make_float4(dl2, cmu, csS, dm);
+            *reinterpret_cast<float4 *>(rec + kRecJmax) =
+                make_float4(__int_as_float(jmax[hr]), __int_as_float(lo[hr]), gt, 0.0f);
+        }
+    }
+    // du: sum over the warp's 16 rows (lanes of equal tq), then over the warps.
+#pragma unroll
+    for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            float x = dupart[nt][e];
+            x += __shfl_xor_sync(0xffffffffu, x, 4);
+            x += __shfl_xor_sync(0xffffffffu, x, 8);
+            x += __shfl_xor_sync(0xffffffffu, x, 16);
+            if (gq == 0) red[warp][8 * nt + 2 * tq + e] = x;
+        }
+    __syncthreads();
+    if (threadIdx.x < kHeadDim) {
+        const int d = threadIdx.x;
+        a.du_part[((static_cast<size_t>(b) * gridDim.x + blockIdx.x) * a.Hq + h) * kHeadDim + d] =
+            (red[0][d] + red[1][d]) + (red[2][d] + red[3][d]);
+    }
+}
+
 // dq for bf16 inputs: a warp owns 16 query rows; keys stream in blocks of 64.
 __global__ void __launch_bounds__(128)
 bwd_dq_mma_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
@@ -705,19 +912,23 @@ template <typename T>
 cudaError_t launch_all(const BwdLaunch &l, const BwdArgs &a) {
     const T *q = static_cast<const T *>(l.q), *k = static_cast<const T *>(l.k),
             *v = static_cast<const T *>(l.v), *go = static_cast<const T *>(l.dout);
-    bwd_rows_kernel<T><<<dim3((a.T + kRowsB0 - 1) / kRowsB0, a.Hq, a.B), kRowsB0, 0, l.stream>>>(
-        q, k, v, go, a);
+    int nparts;
     if constexpr (std::is_same<T, __nv_bfloat16>::value) {
+        nparts = a.B * ((a.T + 63) / 64);
+        bwd_rows_mma_kernel<<<dim3((a.T + 63) / 64, a.Hq, a.B), 128, 0, l.stream>>>(q, k, v, go, a);
         bwd_dkdv_mma_kernel<<<dim3((a.T + 63) / 64, a.Hkv, a.B), 128, 0, l.stream>>>(
             q, k, v, l.dk, l.dv, a);
         bwd_dq_mma_kernel<<<dim3((a.T + 63) / 64, a.Hq, a.B), 128, 0, l.stream>>>(q, k, v, l.dq, a);
     } else {
+        nparts = a.B * ((a.T + kRowsB0 - 1) / kRowsB0);
+        bwd_rows_kernel<T><<<dim3((a.T + kRowsB0 - 1) / kRowsB0, a.Hq, a.B), kRowsB0, 0, l.stream>>>(
+            q, k, v, go, a);
         bwd_dkdv_kernel<T><<<dim3((a.T + kKeyTile - 1) / kKeyTile, a.Hkv, a.B), 128, 0, l.stream>>>(
             q, k, v, l.dk, l.dv, a);
         bwd_dq_kernel<T><<<dim3((a.T + kKeyTile - 1) / kKeyTile, a.Hq, a.B), 128, 0, l.stream>>>(
             q, k, v, l.dq, a);
     }
-    bwd_du_kernel<<<a.Hq, kHeadDim, 0, l.stream>>>(l.du, a, a.B * ((a.T + kRowsB0 - 1) / kRowsB0));
+    bwd_du_kernel<<<a.Hq, kHeadDim, 0, l.stream>>>(l.du, a, nparts);
     count_launches(4);
     return cudaGetLastError();
 }
@@ -726,8 +937,8 @@ cudaError_t launch_all(const BwdLaunch &l, const BwdArgs &a) {
 
 size_t bwd_workspace_bytes(int B, int T, int Hq) {
     const size_t rec = static_cast<size_t>(B) * Hq * T * kRecWords * sizeof(float);
-    const size_t part =
-        static_cast<size_t>(B) * ((T + kRowsB0 - 1) / kRowsB0) * Hq * kHeadDim * sizeof(float);
+    const size_t part =  // per 64-row block (the bf16 rows pass; the fp32 one uses 128-row blocks)
+        static_cast<size_t>(B) * ((T + 63) / 64) * Hq * kHeadDim * sizeof(float);
     return rec + part;
 }
 
