@@ -6,6 +6,9 @@ code.  The arithmetic lives in ``polar_oracle.c``; this module only compiles
 it with gcc (``-O2 -fopenmp -ffp-contract=off``, no fast-math) and marshals numpy
 arrays through ctypes.
 
+The memory channel (a gated-delta associative memory, the third additive
+stream) lives in ``gdelta_oracle.c``, compiled into the same library.
+
 Method source: "ATMA: Length-Invariant Language Modeling via Polar Attention
 and Gated-Delta Compression Memory" (gist.science technical summary, section
 2.1 "Polar Attention: A Three-Channel Decomposition"; section 2.2, "Fused Polar
@@ -24,6 +27,7 @@ import numpy as np
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "polar_oracle.c")
+_SRC_GD = os.path.join(_HERE, "gdelta_oracle.c")
 _BUILD = os.path.join(_HERE, "_build")
 _LOCK = threading.Lock()
 _LIBS: dict = {}
@@ -39,6 +43,10 @@ class _Cfg(ctypes.Structure):
         ("L", ctypes.c_int), ("beta", ctypes.c_double), ("causal", ctypes.c_int),
         ("len_mode", ctypes.c_int), ("window", ctypes.c_int),
     ]
+
+
+class _GdCfg(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("T", ctypes.c_int), ("H", ctypes.c_int), ("D", ctypes.c_int)]
 
 
 @dataclass
@@ -64,11 +72,11 @@ def build(mutant: int = 0, build_dir: str | None = None, force: bool = False) ->
     out = lib_path(mutant, build_dir)
     os.makedirs(os.path.dirname(out), exist_ok=True)
     if (not force and os.path.exists(out)
-            and os.path.getmtime(out) >= os.path.getmtime(_SRC)):
+            and os.path.getmtime(out) >= max(os.path.getmtime(_SRC), os.path.getmtime(_SRC_GD))):
         return out
     tmp = out + f".tmp{os.getpid()}"
     cmd = ["gcc", "-O2", "-std=c11", "-fopenmp", "-ffp-contract=off", "-fPIC", "-shared",
-           f"-DORACLE_MUTANT={int(mutant)}", "-o", tmp, _SRC, "-lm"]
+           f"-DORACLE_MUTANT={int(mutant)}", "-o", tmp, _SRC, _SRC_GD, "-lm"]
     subprocess.run(cmd, check=True, capture_output=True)
     os.replace(tmp, out)
     return out
@@ -92,6 +100,9 @@ def _load(mutant: int = 0, build_dir: str | None = None) -> ctypes.CDLL:
             lib.oracle_polar_bwd.argtypes = [
                 ctypes.POINTER(_Cfg), P, P, P, ctypes.c_int, P, P, P, P, P, P]
             lib.oracle_polar_bwd.restype = ctypes.c_int
+            lib.oracle_gdelta.argtypes = [ctypes.POINTER(_GdCfg), P, P, P, ctypes.c_int, P, P, P,
+                                          P, ctypes.c_int]
+            lib.oracle_gdelta.restype = ctypes.c_int
             lib.oracle_mutant_id.restype = ctypes.c_int
             _LIBS[key] = lib
         return _LIBS[key]
@@ -218,6 +229,39 @@ def polar_decode(q, kv_pages, page_table, seqlens, u, p: Params = Params(), rows
     if rc != 0:
         raise ValueError(f"oracle_polar_decode rejected its arguments (rc={rc})")
     return Result(out, neff, stats)
+
+
+def gdelta(q, k, v, alpha, beta, state=None, literal: bool = False, mutant: int = 0,
+           build_dir: str | None = None):
+    """Gated-delta memory channel over whole sequences.
+
+    q, k, v: [B,T,H,D] float32 or bf16 bits (uint16); alpha, beta: [B,T,H]
+    (any float dtype, widened exactly); state: [B,H,D,D] initial state S_0
+    (row = value dim, column = key dim), None for zeros.  Returns (o, S_T):
+    o [B,T,H,D] and the final state [B,H,D,D], both fp64."""
+    q, dt = _as_input(q)
+    k, dk_ = _as_input(k)
+    v, dv_ = _as_input(v)
+    if not (dt == dk_ == dv_):
+        raise TypeError("q, k, v must share a dtype")
+    B, T, H, D = q.shape
+    if k.shape != q.shape or v.shape != q.shape:
+        raise ValueError("q, k, v must share a shape")
+    a = np.ascontiguousarray(alpha, dtype=np.float64)
+    b = np.ascontiguousarray(beta, dtype=np.float64)
+    if a.shape != (B, T, H) or b.shape != (B, T, H):
+        raise ValueError("alpha and beta must be [B, T, H]")
+    S = (np.zeros((B, H, D, D), np.float64) if state is None
+         else np.array(state, dtype=np.float64, copy=True, order="C"))
+    if S.shape != (B, H, D, D):
+        raise ValueError("state must be [B, H, D, D]")
+    out = np.zeros((B, T, H, D), np.float64)
+    cfg = _GdCfg(B, T, H, D)
+    rc = _load(mutant, build_dir).oracle_gdelta(ctypes.byref(cfg), _ptr(q), _ptr(k), _ptr(v), dt,
+                                                _ptr(a), _ptr(b), _ptr(S), _ptr(out), int(literal))
+    if rc != 0:
+        raise ValueError(f"oracle_gdelta rejected its arguments (rc={rc})")
+    return out, S
 
 
 def mutant_id(mutant: int = 0, build_dir: str | None = None) -> int:

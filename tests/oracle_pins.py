@@ -403,7 +403,173 @@ def pin_backward_finite_differences(mutant=0, bd=None):
                     f"grad {'qkvu'[which]}{idx} window={p.window}: fd {num:.6e} vs {ana:.6e}"
 
 
+# ---- memory channel (gated-delta associative memory) ---------------------
+# The pages name the rule (ATMA technical summary, section 2.1, "Recurrent
+# Memory Channel": gated-delta memory with L2-normalised keys and queries);
+# the facts below follow from the delta rule itself, not from the oracle.
+
+def _gd_rand(rng, B, T, H, D=64, scale_rows=True):
+    q = rng.standard_normal((B, T, H, D))
+    k = rng.standard_normal((B, T, H, D))
+    if scale_rows:  # rows of arbitrary length: the channel normalises them
+        q *= rng.uniform(0.2, 5.0, (B, T, H, 1))
+        k *= rng.uniform(0.2, 5.0, (B, T, H, 1))
+    v = rng.standard_normal((B, T, H, D))
+    return q.astype(np.float32), k.astype(np.float32), v.astype(np.float32)
+
+
+def pin_gdelta_orders_agree(mutant=0, bd=None):
+    """The literal update S (alpha (I - beta k k^T)) + beta v k^T with the
+    matrix built, and its rank-one expansion, agree to rounding."""
+    rng = np.random.default_rng(31)
+    B, T, H = 2, 40, 2
+    q, k, v = _gd_rand(rng, B, T, H)
+    a = rng.uniform(0.3, 1.0, (B, T, H))
+    b = rng.uniform(0.0, 1.0, (B, T, H))
+    S0 = rng.standard_normal((B, H, 64, 64)) * 0.3
+    o1, S1 = oracle.gdelta(q, k, v, a, b, S0, literal=True, mutant=mutant, build_dir=bd)
+    o0, S0_ = oracle.gdelta(q, k, v, a, b, S0, literal=False, mutant=mutant, build_dir=bd)
+    _close(o0, o1, rtol=1e-10, atol=1e-11, what="gdelta orders: o")
+    _close(S0_, S1, rtol=1e-10, atol=1e-11, what="gdelta orders: state")
+
+
+def pin_gdelta_last_write_retrieved(mutant=0, bd=None):
+    """With beta = 1 the write replaces whatever the memory returned for the
+    (unit) key: S_t k_t = alpha S (k - k (k.k)) + v (k.k) = v_t, whatever the
+    history, the decay or S_0.  So a query equal to the key reads v_t back."""
+    rng = np.random.default_rng(32)
+    B, T, H = 1, 50, 2
+    q, k, v = _gd_rand(rng, B, T, H)
+    q = (k * 2.0 ** rng.integers(-2, 3, (B, T, H, 1))).astype(np.float32)  # exact rescale
+    a = rng.uniform(0.5, 1.0, (B, T, H))
+    b = np.ones((B, T, H))
+    S0 = rng.standard_normal((B, H, 64, 64))
+    for literal in (False, True):
+        o, _ = oracle.gdelta(q, k, v, a, b, S0, literal=literal, mutant=mutant, build_dir=bd)
+        _close(o, v, rtol=1e-10, atol=1e-10, what=f"gdelta last write (literal={literal})")
+
+
+def pin_gdelta_orthonormal_store(mutant=0, bd=None):
+    """alpha = beta = 1 and keys drawn from a scaled orthonormal basis: the
+    memory is a key -> value table.  A query along basis vector e returns the
+    value last written under e (an overwrite, not a sum), or zero."""
+    rng = np.random.default_rng(33)
+    T, D = 60, 64
+    basis, _ = np.linalg.qr(rng.standard_normal((D, D)))
+    slots = rng.integers(0, 12, size=T)       # repeated slots: overwrites
+    qslots = rng.integers(0, 16, size=T)      # 12..15 are never written
+    k = (basis[:, slots].T * rng.uniform(0.3, 3.0, (T, 1)))[None, :, None]
+    q = (basis[:, qslots].T * rng.uniform(0.3, 3.0, (T, 1)))[None, :, None]
+    v = rng.standard_normal((1, T, 1, D))
+    ones = np.ones((1, T, 1))
+    expect = np.zeros((T, D))
+    last = {}
+    for t in range(T):
+        last[int(slots[t])] = v[0, t, 0]
+        expect[t] = last.get(int(qslots[t]), np.zeros(D))
+    for literal in (False, True):
+        o, _ = oracle.gdelta(q.astype(np.float32), k.astype(np.float32), v.astype(np.float32),
+                             ones, ones, literal=literal, mutant=mutant, build_dir=bd)
+        _close(o[0, :, 0], expect.astype(np.float32).astype(np.float64), rtol=1e-6, atol=1e-6,
+               what=f"gdelta orthonormal store (literal={literal})")
+
+
+def pin_gdelta_partial_writes(mutant=0, bd=None):
+    """alpha = 1, beta = 1/2, the same key and value written n times from an
+    empty memory: S_n = (1 - 2^-n) v k^T (each write closes half of the gap),
+    so the read with q = k is (1 - 2^-n) v."""
+    rng = np.random.default_rng(34)
+    T, D = 10, 64
+    kk = rng.standard_normal(D)
+    vv = rng.standard_normal(D)
+    k = np.tile(kk, (1, T, 1, 1)).astype(np.float32)
+    v = np.tile(vv, (1, T, 1, 1)).astype(np.float32)
+    o, _ = oracle.gdelta(k, k, v, np.ones((1, T, 1)), np.full((1, T, 1), 0.5), mutant=mutant,
+                         build_dir=bd)
+    vf = vv.astype(np.float32).astype(np.float64)
+    for n in range(1, T + 1):
+        _close(o[0, n - 1, 0], (1 - 0.5 ** n) * vf, rtol=1e-10, atol=1e-12,
+               what=f"gdelta partial write n={n}")
+
+
+def pin_gdelta_decay_and_reset(mutant=0, bd=None):
+    """beta = 0: nothing is written, the state only decays, S_t = (prod alpha)
+    S_0 and o_t = (prod_{s<=t} alpha_s) S_0 q_t/|q_t|.  alpha = 0: everything
+    is forgotten before the write, S_t = beta_t v_t k_t^T/|k_t|, so
+    o_t = beta_t v_t <k_t, q_t>/(|k_t||q_t|)."""
+    rng = np.random.default_rng(35)
+    B, T, H = 1, 30, 2
+    q, k, v = _gd_rand(rng, B, T, H)
+    a = rng.uniform(0.7, 1.0, (B, T, H))
+    S0 = rng.standard_normal((B, H, 64, 64))
+    o, S = oracle.gdelta(q, k, v, a, np.zeros((B, T, H)), S0, mutant=mutant, build_dir=bd)
+    qn = q.astype(np.float64) / np.linalg.norm(q.astype(np.float64), axis=-1, keepdims=True)
+    cum = np.cumprod(a, axis=1)
+    for h in range(H):
+        exp = cum[0, :, h, None] * (qn[0, :, h] @ S0[0, h].T)
+        _close(o[0, :, h], exp, rtol=1e-10, atol=1e-11, what="gdelta decay only")
+        _close(S[0, h], cum[0, -1, h] * S0[0, h], rtol=1e-10, atol=1e-12, what="gdelta decay state")
+    b = rng.uniform(0.1, 1.0, (B, T, H))
+    o, _ = oracle.gdelta(q, k, v, np.zeros((B, T, H)), b, S0, mutant=mutant, build_dir=bd)
+    kn = k.astype(np.float64) / np.linalg.norm(k.astype(np.float64), axis=-1, keepdims=True)
+    exp = b[..., None] * v.astype(np.float64) * np.sum(kn * qn, axis=-1, keepdims=True)
+    _close(o, exp, rtol=1e-10, atol=1e-12, what="gdelta reset")
+
+
+def pin_gdelta_invariances(mutant=0, bd=None):
+    """The channel sees only the directions of q and k (it normalises them):
+    rescaling their rows changes nothing, a common rotation R of every q and k
+    leaves o unchanged and turns the final state into S R^T, and the output is
+    linear in v (from an empty memory)."""
+    rng = np.random.default_rng(36)
+    B, T, H = 1, 24, 2
+    q, k, v = _gd_rand(rng, B, T, H, scale_rows=False)
+    a = rng.uniform(0.5, 1.0, (B, T, H))
+    b = rng.uniform(0.0, 1.0, (B, T, H))
+    o, S = oracle.gdelta(q, k, v, a, b, mutant=mutant, build_dir=bd)
+    sq = rng.uniform(0.1, 10.0, (B, T, H, 1))
+    sk = rng.uniform(0.1, 10.0, (B, T, H, 1))
+    # powers of two keep the rescaled fp32 rows exact
+    sq, sk = 2.0 ** np.round(np.log2(sq)), 2.0 ** np.round(np.log2(sk))
+    o2, _ = oracle.gdelta((q * sq).astype(np.float32), (k * sk).astype(np.float32), v, a, b,
+                          mutant=mutant, build_dir=bd)
+    _close(o2, o, rtol=1e-12, atol=1e-13, what="gdelta row scale")
+    R, _ = np.linalg.qr(rng.standard_normal((64, 64)))
+    qr = (q.astype(np.float64) @ R.T)
+    kr = (k.astype(np.float64) @ R.T)
+    # the rotated rows are not fp32-exact: compare against the unrotated run on
+    # the same rounded inputs rotated back, within fp32 input rounding
+    o3, S3 = oracle.gdelta(qr.astype(np.float32), kr.astype(np.float32), v, a, b,
+                           mutant=mutant, build_dir=bd)
+    _close(o3, o, rtol=1e-5, atol=1e-5, what="gdelta rotation: o")
+    _close(S3, S @ R.T, rtol=1e-5, atol=1e-5, what="gdelta rotation: state")
+    o4, _ = oracle.gdelta(q, k, (4.0 * v).astype(np.float32), a, b, mutant=mutant, build_dir=bd)
+    _close(o4, 4.0 * o, rtol=1e-12, atol=1e-13, what="gdelta linear in v")
+
+
+def pin_gdelta_state_carries(mutant=0, bd=None):
+    """Running T tokens equals running the first T1 and then the rest from
+    the returned state (the state is the whole of the channel's memory)."""
+    rng = np.random.default_rng(37)
+    B, T, H, T1 = 2, 33, 2, 14
+    q, k, v = _gd_rand(rng, B, T, H)
+    a = rng.uniform(0.5, 1.0, (B, T, H))
+    b = rng.uniform(0.0, 1.0, (B, T, H))
+    o, S = oracle.gdelta(q, k, v, a, b, mutant=mutant, build_dir=bd)
+    oa, Sa = oracle.gdelta(q[:, :T1], k[:, :T1], v[:, :T1], a[:, :T1], b[:, :T1], mutant=mutant,
+                           build_dir=bd)
+    ob, Sb = oracle.gdelta(q[:, T1:], k[:, T1:], v[:, T1:], a[:, T1:], b[:, T1:], Sa,
+                           mutant=mutant, build_dir=bd)
+    _close(np.concatenate([oa, ob], axis=1), o, rtol=1e-12, atol=1e-13, what="gdelta split: o")
+    _close(Sb, S, rtol=1e-12, atol=1e-13, what="gdelta split: state")
+
+
+GDELTA_PINS = [pin_gdelta_orders_agree, pin_gdelta_last_write_retrieved,
+               pin_gdelta_orthonormal_store, pin_gdelta_partial_writes,
+               pin_gdelta_decay_and_reset, pin_gdelta_invariances, pin_gdelta_state_carries]
+
+
 ALL_PINS = [pin_modes_agree, pin_uniform, pin_uniform_train_length_constant, pin_closed_form,
             pin_temperature_constants, pin_unit_norm_and_bounded, pin_duplication,
             pin_causality, pin_gqa, pin_decode_matches_prefill, pin_window,
-            pin_backward_finite_differences]
+            pin_backward_finite_differences] + GDELTA_PINS

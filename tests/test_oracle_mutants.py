@@ -6,14 +6,16 @@ l/l2, a flipped gate sign, an off-by-one causal bound, a transposed GQA
 mapping, a sample (not population) std, a log2 temperature, a dropped factor 2
 under the null-floor root, a missing unit-sphere projection, and the wrong
 head's count vector; in the backward, a dropped null-floor spread term and a
-flipped sign on the squared-sum gradient.
+flipped sign on the squared-sum gradient; in the memory channel, the decay gate
+left off the erase term, the key/query normalisation skipped, and a read taken
+before the write.
 """
 import pytest
 
 import oracle
 import oracle_pins as P
 
-MUTANTS = list(range(1, 13))
+MUTANTS = list(range(1, 16))
 
 
 @pytest.fixture(scope="module")
