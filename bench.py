@@ -65,6 +65,8 @@ def parse_args(argv=None):
     ap.add_argument("--bwd-steps", type=int, default=10,
                     help="timed launches of the prefill backward on the train-length workload "
                          "(0 skips it)")
+    ap.add_argument("--gdelta-steps", type=int, default=20,
+                    help="timed launches of the memory channel (prefill and decode step); 0 skips")
     ap.add_argument("--window", type=int, default=4096,
                     help="sliding window of the separately timed windowed prefill (0 skips it)")
     ap.add_argument("--chunk", type=int, default=4,
@@ -389,6 +391,54 @@ def run_ours(args):
         bwd_res = (wb, Kb, t_b)
         del xb, gb, gq, gk, gv, gu, wsb
 
+    # ---- memory channel: chunked prefill and in-place decode step, timed on their own ----
+    gd_res = None
+    if args.gdelta_steps > 0:
+        wg, wst = W.GD_TRAIN, W.GD_STEP
+        xg = W.gdelta_inputs(wg, dev, seed=seed + 2)
+        og = torch.empty_like(xg["q"])
+        sg = torch.empty((wg.B, wg.H, wg.D, wg.D), device=dev)
+        wsg = torch.empty(pa.gdelta_workspace_size(wg.B, wg.T, wg.H), device=dev,
+                          dtype=torch.uint8)
+        xs = W.gdelta_step_inputs(wst, dev, seed=seed + 3)
+        os_ = torch.empty_like(xs["q"])
+
+        def gd_prefill():
+            sg.zero_()  # not timed: outside the events below
+            pa.gdelta_prefill(xg["q"], xg["k"], xg["v"], xg["alpha"], xg["beta"], sg, og, wsg,
+                              stream=stream)
+
+        def gd_step():
+            pa.gdelta_step(xs["q"], xs["k"], xs["v"], xs["alpha"], xs["beta"], xs["state_pool"],
+                           xs["slots"], os_, stream=stream)
+
+        Kg = args.gdelta_steps
+        times = []
+        for fn in (gd_prefill, gd_step):
+            for _ in range(max(Wm, 3)):
+                fn()
+            torch.cuda.synchronize(dev)
+            eg = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(Kg)]
+            barrier(world, dev)
+            torch.cuda.synchronize(dev)
+            for i in range(Kg):
+                if fn is gd_prefill:
+                    sg.zero_()
+                eg[i][0].record(stream)
+                if fn is gd_prefill:
+                    pa.gdelta_prefill(xg["q"], xg["k"], xg["v"], xg["alpha"], xg["beta"], sg, og,
+                                      wsg, stream=stream)
+                else:
+                    fn()
+                eg[i][1].record(stream)
+            torch.cuda.synchronize(dev)
+            barrier(world, dev)
+            if pa.get_status() != 0:
+                raise RuntimeError("device status after the memory channel")
+            times.append(max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in eg) / 1e3, world, dev))
+        gd_res = (wg, wst, Kg, times[0], times[1])
+        del xg, og, sg, wsg, xs, os_
+
     # ---- multi-token decode (chunk query tokens per sequence), timed on its own ----
     chunk_res = None
     if do_dec and args.chunk > 1:
@@ -525,9 +575,48 @@ def run_ours(args):
             result["backward"] = {
                 "workload": wb.describe(), "value": b_fl / b_launch / 1e12, "unit": "TFLOP/s",
                 "ms_per_launch": b_launch * 1e3, "flops_per_launch": b_fl, "launches": Kb,
-                "note": "prefill backward (polar_attn_bwd: dq, dk, dv, du; CUDA-core fp32), flops "
+                "note": "prefill backward (polar_attn_bwd: dq, dk, dv, du; mma.sync tensor cores for "
+                        "bf16 inputs), flops "
                         "counted as 2.5x the forward's visible-pair flops; timed separately; not "
                         "part of value"}
+        if gd_res is not None:
+            wg, wst, Kg, t_gp, t_gs = gd_res
+            gp_launch, gs_launch = t_gp / Kg, t_gs / Kg
+            tok = wg.B * wg.T
+            nch = (wg.T + 63) // 64
+            # FMAs the two prefill kernels execute per (chunk, head): the chunk
+            # kernel's lower-triangle key-key and query-key products (136 tiles of
+            # 4 x 4 x 64, twice) and its 128-column forward substitution (sum over
+            # rows of 4 ceil(t/4) per column); the scan kernel's four products
+            # over its four 16-row state slices.
+            chunk_fma = 2 * 136 * 16 * 64 + 128 * sum(4 * ((t + 3) // 4) for t in range(1, 64))
+            scan_fma = 4 * (2 * 1024 * 64 + 64 * sum(4 * (g + 1) for g in range(16)) + 1024 * 64)
+            exec_flops = 2.0 * (chunk_fma + scan_fma) * wg.B * wg.H * nch
+            gp_tf = exec_flops / gp_launch / 1e12
+            alu_peak = 2 * 148 * 128 * 1.965e9 / 1e12
+            step_bytes = wst.state_bytes + wst.num_seqs * wst.H * wst.D * (4 * 2) + \
+                wst.num_seqs * wst.H * 8 + wst.num_seqs * 4
+            gs_gbs = step_bytes / gs_launch / 1e9
+            result["gdelta"] = {
+                "workload": wg.describe(), "ms_per_launch": gp_launch * 1e3,
+                "tokens_per_s": aggregate_throughput(tok * Kg, world, t_gp),
+                "recurrence_tflops": wg.flops / gp_launch / 1e12,
+                "note": "memory channel prefill (polar_gdelta_prefill: chunk kernel + scan kernel, "
+                        "fp32 CUDA cores), timed separately; not part of value"}
+            result["roofline_gdelta"] = {
+                "bound": "alu", "kernel": "gd_chunk_kernel+gd_scan_kernel", "achieved": gp_tf,
+                "peak": alu_peak, "unit": "TFLOP/s", "frac": gp_tf / alu_peak,
+                "flops_per_launch": exec_flops, "traffic": None,
+                "peak_source": "fp32 FMA: 148 SMs x 128 lanes x 2 flops x 1965 MHz (max SM clock)"}
+            result["gdelta_step"] = {
+                "workload": wst.describe(), "ms_per_launch": gs_launch * 1e3,
+                "tokens_per_s": aggregate_throughput(wst.num_seqs * Kg, world, t_gs),
+                "note": "in-place decode step (polar_gdelta_step), timed separately"}
+            result["roofline_gdelta_step"] = {
+                "bound": "hbm", "kernel": "gd_step_kernel", "achieved": gs_gbs,
+                "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": gs_gbs / peaks["hbm_gbs"],
+                "bytes_per_launch": step_bytes, "traffic": None,
+                "peak_source": f"{peak_src} (copy bandwidth)"}
         if window_res is not None:
             wp, t_win = window_res
             w_launch = t_win / K

@@ -60,7 +60,8 @@ typedef enum {
     POLAR_ERR_BAD_PAGE = 4,    /* device: page id outside [0, num_pages) */
     POLAR_ERR_TIMEOUT = 5,     /* device: a bounded wait ran out */
     POLAR_ERR_CUDA = 6,        /* a CUDA runtime call failed */
-    POLAR_ERR_BAD_SEQLEN = 7   /* device: seqlen outside [1, max_pages*64] */
+    POLAR_ERR_BAD_SEQLEN = 7,  /* device: seqlen outside [1, max_pages*64] */
+    POLAR_ERR_BAD_SLOT = 8     /* device: memory state slot >= num_slots (polar_gdelta.h) */
 } polar_status_t;
 
 typedef enum { POLAR_BF16 = 0, POLAR_FP32 = 1 } polar_dtype_t;

@@ -1,7 +1,8 @@
-"""B200 (sm_100a) Polar Attention: fused causal prefill and GQA paged decode.
+"""B200 (sm_100a) Polar Attention: fused causal prefill, GQA paged decode and
+the gated-delta memory channel.
 
 The computation lives in libpolar_attn.so (hand-written CUDA for sm_100a behind
-the C ABI of include/polar_attn.h); ``native`` is its thin ctypes binding and
+the C ABI of include/polar_attn.h and include/polar_gdelta.h); ``native`` is its thin ctypes binding and
 ``workloads`` the seeded synthetic inputs.  The library is loaded on first use,
 and a missing build raises: there is no CPU or PyTorch fallback.
 """
@@ -9,10 +10,12 @@ from .native import (bwd, bwd_workspace_size, decode_chunk_workspace_size,  # no
                      decode_paged, decode_paged_chunk,
                      decode_paged_host, decode_staging_size,
                      decode_workspace_size, fwd, fwd_host, fwd_staging_size,
-                     fwd_workspace_size, get_status,
+                     fwd_workspace_size, gdelta_prefill, gdelta_step,
+                     gdelta_workspace_size, get_status,
                      launch_count, PolarError)
 
 __all__ = ["fwd", "bwd", "bwd_workspace_size", "fwd_host", "fwd_staging_size", "fwd_workspace_size", "decode_paged",
            "decode_paged_chunk", "decode_chunk_workspace_size", "decode_paged_host",
-           "decode_staging_size", "decode_workspace_size", "get_status", "launch_count",
+           "decode_staging_size", "decode_workspace_size", "gdelta_prefill", "gdelta_step",
+           "gdelta_workspace_size", "get_status", "launch_count",
            "PolarError"]

@@ -8,6 +8,7 @@
 #include <cudaTypedefs.h>
 
 #include "polar_common.cuh"
+#include "polar_gdelta.h"
 #include "polar_internal.h"
 
 namespace polar {
@@ -86,6 +87,28 @@ polar_status_t check_decode_chunk(const polar_params_t *p, int num_seqs, int max
     if (static_cast<long long>(num_seqs) * chunk > 65535) return POLAR_ERR_UNSUPPORTED;
     return POLAR_OK;
 }
+
+// Memory channel: shape and flag checks shared by prefill and step.
+polar_status_t check_gdelta(const polar_gdelta_params_t *p) {
+    if (!p) return POLAR_ERR_INVALID_ARG;
+    if (p->head_dim != kHeadDim) return POLAR_ERR_UNSUPPORTED;
+    if (p->dtype != POLAR_BF16 && p->dtype != POLAR_FP32) return POLAR_ERR_INVALID_ARG;
+    if (p->H <= 0) return POLAR_ERR_INVALID_ARG;
+    if ((p->zero_init != 0 && p->zero_init != 1) || (p->accumulate != 0 && p->accumulate != 1))
+        return POLAR_ERR_INVALID_ARG;
+    return POLAR_OK;
+}
+
+// Prefill: the scan grid's second dimension is B * H.
+polar_status_t check_gdelta_prefill(const polar_gdelta_params_t *p) {
+    polar_status_t st = check_gdelta(p);
+    if (st != POLAR_OK) return st;
+    if (p->B < 0 || p->T < 0) return POLAR_ERR_INVALID_ARG;
+    if (static_cast<long long>(p->B) * p->H > 65535) return POLAR_ERR_UNSUPPORTED;
+    return POLAR_OK;
+}
+
+bool aligned4(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
 
 polar_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? POLAR_OK : POLAR_ERR_CUDA; }
 
@@ -397,10 +420,62 @@ const char *polar_attn_status_string(polar_status_t s) {
         case POLAR_ERR_TIMEOUT: return "a bounded device wait timed out";
         case POLAR_ERR_CUDA: return "CUDA runtime error";
         case POLAR_ERR_BAD_SEQLEN: return "sequence length outside [1, 64*max_pages]";
+        case POLAR_ERR_BAD_SLOT: return "memory state slot outside the state pool";
     }
     return "unknown status";
 }
 
 uint64_t polar_attn_launch_count(void) { return g_launches.load(); }
+
+size_t polar_gdelta_prefill_workspace_size(const polar_gdelta_params_t *p) {
+    if (check_gdelta_prefill(p) != POLAR_OK) return 0;
+    return gdelta_workspace_bytes(p->B, p->T, p->H);
+}
+
+polar_status_t polar_gdelta_prefill(const void *q, const void *k, const void *v,
+                                    const float *alpha, const float *beta, float *state,
+                                    const polar_gdelta_params_t *p, void *out, void *workspace,
+                                    size_t ws_bytes, void *stream) {
+    polar_status_t st = check_gdelta_prefill(p);
+    if (st != POLAR_OK) return st;
+    if (p->B == 0 || p->T == 0) return POLAR_OK;
+    if (!q || !k || !v || !alpha || !beta || !state || !out || !workspace)
+        return POLAR_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(state) || !aligned16(out) ||
+        !aligned16(workspace) || !aligned4(alpha) || !aligned4(beta))
+        return POLAR_ERR_INVALID_ARG;
+    if (ws_bytes < gdelta_workspace_bytes(p->B, p->T, p->H)) return POLAR_ERR_WORKSPACE;
+    GdeltaLaunch a;
+    a.q = q; a.k = k; a.v = v; a.alpha = alpha; a.beta = beta; a.state = state; a.out = out;
+    a.B = p->B; a.T = p->T; a.H = p->H; a.dtype = p->dtype; a.zero_init = p->zero_init;
+    a.accumulate = p->accumulate; a.workspace = workspace;
+    a.stream = static_cast<cudaStream_t>(stream);
+    return from_cuda(launch_gdelta_prefill(a));
+}
+
+polar_status_t polar_gdelta_step(const void *q, const void *k, const void *v,
+                                 const float *alpha, const float *beta, float *state_pool,
+                                 int num_slots, const int32_t *slots, int num_seqs,
+                                 const polar_gdelta_params_t *p, void *out, void *stream) {
+    polar_status_t st = check_gdelta(p);
+    if (st != POLAR_OK) return st;
+    if (num_seqs < 0 || num_slots < 0) return POLAR_ERR_INVALID_ARG;
+    if (static_cast<long long>(num_seqs) * p->H > (1ll << 31) - 1) return POLAR_ERR_UNSUPPORTED;
+    if (num_seqs == 0) return POLAR_OK;
+    if (!q || !k || !v || !alpha || !beta || !slots || !out || (num_slots > 0 && !state_pool))
+        return POLAR_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) ||
+        (state_pool && !aligned16(state_pool)) || !aligned4(alpha) || !aligned4(beta) ||
+        !aligned4(slots))
+        return POLAR_ERR_INVALID_ARG;
+    int *status = status_ptr();
+    if (!status) return POLAR_ERR_CUDA;
+    GdeltaStepLaunch a;
+    a.q = q; a.k = k; a.v = v; a.alpha = alpha; a.beta = beta; a.pool = state_pool;
+    a.num_slots = num_slots; a.slots = slots; a.num_seqs = num_seqs; a.H = p->H;
+    a.dtype = p->dtype; a.accumulate = p->accumulate; a.out = out; a.status = status;
+    a.stream = static_cast<cudaStream_t>(stream);
+    return from_cuda(launch_gdelta_step(a));
+}
 
 }  // extern "C"

@@ -57,12 +57,39 @@ struct BwdLaunch {
     cudaStream_t stream;
 };
 
+struct GdeltaLaunch {              // memory channel over whole sequences
+    const void *q, *k, *v;         // [B, T, H, 64] dtype
+    const float *alpha, *beta;     // [B, T, H]
+    float *state;                  // [B, H, 64, 64], in place
+    void *out;                     // [B, T, H, 64] dtype
+    int B, T, H;
+    int dtype, zero_init, accumulate;
+    void *workspace;               // gdelta_workspace_bytes
+    cudaStream_t stream;
+};
+
+struct GdeltaStepLaunch {          // one decode token per sequence, in place
+    const void *q, *k, *v;         // [num_seqs, H, 64] dtype
+    const float *alpha, *beta;     // [num_seqs, H]
+    float *pool;                   // [num_slots, H, 64, 64]
+    int num_slots;
+    const int32_t *slots;          // [num_seqs]
+    int num_seqs, H;
+    int dtype, accumulate;
+    void *out;                     // [num_seqs, H, 64] dtype
+    int *status;
+    cudaStream_t stream;
+};
+
 // Launchers return cudaSuccess or the launch error.
 cudaError_t launch_fwd_simt(const FwdLaunch &a);
 cudaError_t launch_fwd_tc(const FwdLaunch &a);
 cudaError_t launch_decode(const DecodeLaunch &a);
 cudaError_t launch_bwd(const BwdLaunch &a);
 size_t bwd_workspace_bytes(int B, int T, int Hq);
+cudaError_t launch_gdelta_prefill(const GdeltaLaunch &a);
+cudaError_t launch_gdelta_step(const GdeltaStepLaunch &a);
+size_t gdelta_workspace_bytes(int B, int T, int H);
 
 // Key moments of causal prefill (fwd_moments.cu): one record of kMomFloats
 // fp32 (the 64 x 64 key Gram, then the 64 key sums) per (batch, kv head, full

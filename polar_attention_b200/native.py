@@ -1,4 +1,5 @@
-"""ctypes binding of libpolar_attn.so, the C ABI of include/polar_attn.h.
+"""ctypes binding of libpolar_attn.so, the C ABI of include/polar_attn.h and
+include/polar_gdelta.h.
 
 Argument marshalling only: torch tensors supply device memory and streams, and
 every step of the computation runs in the library's CUDA kernels.  There is no
@@ -19,9 +20,9 @@ POLAR_BF16, POLAR_FP32 = 0, 1
 IMPLS = {"auto": 0, "simt": 1, "tc": 2}
 STATUS = {0: "POLAR_OK", 1: "POLAR_ERR_INVALID_ARG", 2: "POLAR_ERR_UNSUPPORTED",
           3: "POLAR_ERR_WORKSPACE", 4: "POLAR_ERR_BAD_PAGE", 5: "POLAR_ERR_TIMEOUT",
-          6: "POLAR_ERR_CUDA", 7: "POLAR_ERR_BAD_SEQLEN"}
+          6: "POLAR_ERR_CUDA", 7: "POLAR_ERR_BAD_SEQLEN", 8: "POLAR_ERR_BAD_SLOT"}
 
-# Every entry point include/polar_attn.h declares.
+# Every entry point include/polar_attn.h and include/polar_gdelta.h declare.
 EXPORTS = ["polar_attn_default_params", "polar_attn_fwd_workspace_size", "polar_attn_fwd",
            "polar_attn_fwd_staging_size",
            "polar_attn_fwd_host", "polar_attn_decode_workspace_size", "polar_attn_decode_paged",
@@ -29,7 +30,8 @@ EXPORTS = ["polar_attn_default_params", "polar_attn_fwd_workspace_size", "polar_
            "polar_attn_get_status", "polar_attn_status_string", "polar_attn_launch_count",
            "polar_attn_decode_paged_noalloc", "polar_attn_selftest_exp2",
            "polar_attn_decode_chunk_workspace_size", "polar_attn_decode_paged_chunk",
-           "polar_attn_bwd_workspace_size", "polar_attn_bwd"]
+           "polar_attn_bwd_workspace_size", "polar_attn_bwd",
+           "polar_gdelta_prefill_workspace_size", "polar_gdelta_prefill", "polar_gdelta_step"]
 
 
 class PolarError(RuntimeError):
@@ -45,6 +47,13 @@ class Params(ctypes.Structure):
                 ("logit_scale", ctypes.c_float), ("alpha", ctypes.c_float),
                 ("L_train", ctypes.c_int), ("beta", ctypes.c_float), ("causal", ctypes.c_int),
                 ("impl", ctypes.c_int), ("window", ctypes.c_int)]
+
+
+class GdeltaParams(ctypes.Structure):
+    """polar_gdelta_params_t."""
+    _fields_ = [("B", ctypes.c_int), ("T", ctypes.c_int), ("H", ctypes.c_int),
+                ("head_dim", ctypes.c_int), ("dtype", ctypes.c_int), ("zero_init", ctypes.c_int),
+                ("accumulate", ctypes.c_int)]
 
 
 _lib = None
@@ -86,6 +95,11 @@ def lib() -> ctypes.CDLL:
             L.polar_attn_decode_paged_host.argtypes = [P, P, I, P, I, P, I, P, PP, P, P, P, Z, P]
             L.polar_attn_decode_paged_noalloc.argtypes = [P, P, I, P, I, P, I, P, PP, P, P, P]
             L.polar_attn_selftest_exp2.argtypes = [P, P, P, I, P]
+            GP = ctypes.POINTER(GdeltaParams)
+            L.polar_gdelta_prefill_workspace_size.argtypes = [GP]
+            L.polar_gdelta_prefill_workspace_size.restype = Z
+            L.polar_gdelta_prefill.argtypes = [P, P, P, P, P, P, GP, P, P, Z, P]
+            L.polar_gdelta_step.argtypes = [P, P, P, P, P, P, I, P, I, GP, P, P]
             L.polar_attn_get_status.argtypes = [P]
             L.polar_attn_status_string.argtypes = [I]
             L.polar_attn_status_string.restype = ctypes.c_char_p
@@ -93,7 +107,8 @@ def lib() -> ctypes.CDLL:
             for name in ("polar_attn_fwd", "polar_attn_fwd_host", "polar_attn_decode_paged",
                          "polar_attn_decode_paged_host", "polar_attn_get_status",
                          "polar_attn_decode_paged_noalloc", "polar_attn_selftest_exp2",
-                         "polar_attn_decode_paged_chunk", "polar_attn_bwd"):
+                         "polar_attn_decode_paged_chunk", "polar_attn_bwd",
+                         "polar_gdelta_prefill", "polar_gdelta_step"):
                 getattr(L, name).restype = I
             _lib = L
     return _lib
@@ -339,6 +354,69 @@ def selftest_exp2(x, stream=None):
     _check(lib().polar_attn_selftest_exp2(_ptr(x), _ptr(poly), _ptr(mufu), x.numel(),
                                           _stream(stream)), "polar_attn_selftest_exp2")
     return poly, mufu
+
+
+def _gd_params(B, T, H, dtype, zero_init, accumulate) -> GdeltaParams:
+    return GdeltaParams(int(B), int(T), int(H), 64, int(dtype), int(bool(zero_init)),
+                        int(bool(accumulate)))
+
+
+def gdelta_workspace_size(B: int, T: int, H: int) -> int:
+    p = _gd_params(B, T, H, POLAR_BF16, 0, 0)
+    return int(lib().polar_gdelta_prefill_workspace_size(ctypes.byref(p)))
+
+
+def gdelta_prefill(q, k, v, alpha, beta, state=None, out=None, workspace=None, *,
+                   accumulate=False, stream=None):
+    """Memory channel over whole sequences.  q, k, v [B,T,H,64] (bf16 or fp32,
+    CUDA, contiguous), alpha, beta [B,T,H] fp32.  ``state`` [B,H,64,64] fp32 is
+    updated in place (S_0 in, final state out); None starts from zero and
+    returns a fresh final-state tensor.  With accumulate, ``out`` (required)
+    gets the memory read added to it.  Returns (out, state)."""
+    B, T, H, D = q.shape
+    for t in (q, k, v, alpha, beta):
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError("inputs must be contiguous CUDA tensors")
+    zero_init = state is None
+    if state is None:
+        state = torch.empty((B, H, D, D), device=q.device, dtype=torch.float32)
+    if out is None:
+        if accumulate:
+            raise ValueError("accumulate needs the output tensor to add into")
+        out = torch.empty_like(q)
+    p = _gd_params(B, T, H, _dt(q), zero_init, accumulate)
+    p.head_dim = D
+    need = int(lib().polar_gdelta_prefill_workspace_size(ctypes.byref(p)))
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), device=q.device, dtype=torch.uint8)
+    _check(lib().polar_gdelta_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta),
+                                      _ptr(state), ctypes.byref(p), _ptr(out), _ptr(workspace),
+                                      workspace.numel(), _stream(stream)), "polar_gdelta_prefill")
+    return out, state
+
+
+def gdelta_step(q, k, v, alpha, beta, state_pool, slots, out=None, *, accumulate=False,
+                stream=None):
+    """One decode token per sequence with the states updated in place in their
+    pool slots.  q, k, v [N,H,64]; alpha, beta [N,H] fp32; state_pool
+    [num_slots,H,64,64] fp32; slots [N] int32 (negative: skip).  Returns out."""
+    N, H, D = q.shape
+    for t in (q, k, v, alpha, beta, state_pool, slots):
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError("inputs must be contiguous CUDA tensors")
+    if slots.dtype != torch.int32:
+        raise TypeError("slots must be int32")
+    if out is None:
+        if accumulate:
+            raise ValueError("accumulate needs the output tensor to add into")
+        out = torch.empty_like(q)
+    p = _gd_params(0, 0, H, _dt(q), 0, accumulate)
+    p.head_dim = D
+    _check(lib().polar_gdelta_step(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta),
+                                   _ptr(state_pool), state_pool.shape[0], _ptr(slots), N,
+                                   ctypes.byref(p), _ptr(out), _stream(stream)),
+           "polar_gdelta_step")
+    return out
 
 
 def get_status(stream=None) -> int:

@@ -234,6 +234,102 @@ def decode_chunk_queries(w: DecodeWorkload, x: dict, chunk: int, seed: int | Non
     return q.contiguous()
 
 
+@dataclass(frozen=True)
+class GdeltaWorkload:
+    """The memory channel (gated-delta memory, one state per (sequence, head)).
+
+    Inputs: q, k ~ N(0, 1) rows of arbitrary length (the channel normalises
+    them itself), v unit rows, decay gates alpha = 1 - 10^U(lg_lo, lg_hi)
+    (between 0.9 and 0.999 by default: memories from about ten to about a
+    thousand tokens), write strengths beta = sigmoid(N(0, 1))."""
+    name: str
+    B: int
+    T: int
+    H: int = 16
+    D: int = 64
+    dtype: str = "bf16"
+    seed: int = 0
+    lg_lo: float = -3.0
+    lg_hi: float = -1.0
+
+    @property
+    def flops(self) -> float:
+        """Flops of the token-by-token recurrence: S k, the rank-one write and
+        S q, 2 D^2 each (2 flops per multiply-add), per (token, head)."""
+        return 6.0 * self.D * self.D * self.B * self.T * self.H
+
+    def describe(self) -> str:
+        return f"gated-delta memory B={self.B} T={self.T} H={self.H} d={self.D} {self.dtype}"
+
+
+@dataclass(frozen=True)
+class GdeltaStepWorkload:
+    """One decode token per sequence against a pool of state slots (random
+    distinct slots, states ~ N(0, 0.1^2))."""
+    name: str
+    num_seqs: int
+    num_slots: int
+    H: int = 16
+    D: int = 64
+    dtype: str = "bf16"
+    seed: int = 0
+
+    @property
+    def state_bytes(self) -> int:
+        """Bytes the step must move: every state read once and written once."""
+        return 2 * self.num_seqs * self.H * self.D * self.D * 4
+
+    def describe(self) -> str:
+        return (f"gated-delta step {self.num_seqs} seqs x {self.H} heads, pool of "
+                f"{self.num_slots} slots, {self.dtype}")
+
+
+GD_TRAIN = GdeltaWorkload("gdelta_train_T2048", B=8, T=2048, H=16)
+GD_STEP = GdeltaStepWorkload("gdelta_step_1024seqs", num_seqs=1024, num_slots=1024, H=16)
+
+
+def gdelta_inputs(w: GdeltaWorkload, device="cpu", seed: int | None = None) -> dict:
+    """q, k, v [B,T,H,D] (dtype), alpha, beta [B,T,H] fp32."""
+    device = torch.device(device)
+    g = _gen(device, w.seed if seed is None else seed)
+    f32 = torch.float32
+    shp = (w.B, w.T, w.H, w.D)
+    q = torch.randn(shp, generator=g, device=device, dtype=f32)
+    k = torch.randn(shp, generator=g, device=device, dtype=f32)
+    v = _unit(torch.randn(shp, generator=g, device=device, dtype=f32))
+    u = torch.rand((w.B, w.T, w.H), generator=g, device=device, dtype=f32)
+    alpha = 1.0 - torch.pow(10.0, w.lg_lo + (w.lg_hi - w.lg_lo) * u)
+    beta = torch.sigmoid(torch.randn((w.B, w.T, w.H), generator=g, device=device, dtype=f32))
+    return {"q": _cast(q, w.dtype), "k": _cast(k, w.dtype), "v": _cast(v, w.dtype),
+            "alpha": alpha.contiguous(), "beta": beta.contiguous()}
+
+
+def gdelta_step_inputs(w: GdeltaStepWorkload, device="cpu", seed: int | None = None) -> dict:
+    """q, k, v [N,H,D], alpha, beta [N,H], state_pool [num_slots,H,D,D] fp32,
+    slots [N] int32 (distinct)."""
+    device = torch.device(device)
+    s = w.seed if seed is None else seed
+    g = _gen(device, s)
+    f32 = torch.float32
+    shp = (w.num_seqs, w.H, w.D)
+    q = torch.randn(shp, generator=g, device=device, dtype=f32)
+    k = torch.randn(shp, generator=g, device=device, dtype=f32)
+    v = _unit(torch.randn(shp, generator=g, device=device, dtype=f32))
+    u = torch.rand((w.num_seqs, w.H), generator=g, device=device, dtype=f32)
+    alpha = 1.0 - torch.pow(10.0, -3.0 + 2.0 * u)
+    beta = torch.sigmoid(torch.randn((w.num_seqs, w.H), generator=g, device=device, dtype=f32))
+    pool = 0.1 * torch.randn((w.num_slots, w.H, w.D, w.D), generator=g, device=device, dtype=f32)
+    perm = np.random.default_rng(s + 1).permutation(w.num_slots)[:w.num_seqs].astype(np.int32)
+    return {"q": _cast(q, w.dtype), "k": _cast(k, w.dtype), "v": _cast(v, w.dtype),
+            "alpha": alpha.contiguous(), "beta": beta.contiguous(), "state_pool": pool.contiguous(),
+            "slots": torch.from_numpy(perm).to(device)}
+
+
+def small_gdelta(B=1, T=300, H=2, dtype="bf16", seed=0, **kw) -> GdeltaWorkload:
+    return GdeltaWorkload(f"custom_gdelta_B{B}_T{T}_H{H}", B=B, T=T, H=H, dtype=dtype, seed=seed,
+                          **kw)
+
+
 def small_prefill(B=1, T=300, Hq=4, Hkv=2, D=64, dtype="fp32", seed=0, **kw) -> PrefillWorkload:
     return PrefillWorkload(f"custom_B{B}_T{T}_H{Hq}x{Hkv}", B=B, T=T, Hq=Hq, Hkv=Hkv, D=D,
                            dtype=dtype, seed=seed, **kw)

@@ -15,7 +15,7 @@ def declared_functions():
     for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
         src = open(h).read()
         src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
-        for m in re.finditer(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\s*\*?\s*(polar_attn_[A-Za-z0-9_]+)\s*\(",
+        for m in re.finditer(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\s*\*?\s*(polar_(?:attn|gdelta)_[A-Za-z0-9_]+)\s*\(",
                              src, flags=re.M):
             names.add(m.group(1))
     return sorted(names)
@@ -23,7 +23,8 @@ def declared_functions():
 
 def test_header_declares_the_boundary():
     names = declared_functions()
-    for must in ("polar_attn_fwd", "polar_attn_decode_paged", "polar_attn_get_status"):
+    for must in ("polar_attn_fwd", "polar_attn_decode_paged", "polar_attn_get_status",
+                 "polar_gdelta_prefill", "polar_gdelta_step"):
         assert must in names
 
 
