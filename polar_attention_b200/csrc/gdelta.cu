@@ -20,12 +20,22 @@
 //   S_C = b_last S_0 + U^T diag(e^{g_last-g_j}) Kh
 // Kernel 1 (one CTA per chunk, all chunks in parallel) forms A, the masked
 // query-key matrix P, solves for W and Ut, and stores them with the row scales.
-// Kernel 2 (one CTA per (sequence, head, 16 value rows); state rows evolve
-// independently) walks the chunks in order and applies the three products to
-// its slice of the state.  All arithmetic is fp32 on the CUDA cores.
+// Kernel 2 walks the chunks in order for one slice of value rows of one
+// (sequence, head) -- state rows evolve independently -- and applies the
+// products to its slice of the state:
+//  - bf16 inputs: on the tensor cores (mma.sync m16n8k16, fp32 accumulate),
+//    32 value rows a CTA.  The raw bf16 queries and keys are exact operands;
+//    every fp32 operand (W, the state, U) is split into bf16 hi + lo, and each
+//    product sums the hi*hi, hi*lo and lo*hi terms (or hi and lo against an
+//    exact operand), so the state path keeps about 16 more bits than bf16.
+//    P, which only reaches the output, is one bf16 operand.
+//  - fp32 inputs: fp32 on the CUDA cores, 16 value rows a CTA.
+// Kernel 1 is fp32 on the CUDA cores for both.
 //
 // The decode step updates S in place in its pool slot: one read and one write
 // of the 16 KB state per (sequence, head), the rank-one form of the update.
+#include <type_traits>
+
 #include "polar_common.cuh"
 #include "polar_gdelta.h"
 #include "polar_internal.h"
@@ -37,6 +47,10 @@ constexpr int kC = 64;                 // tokens per chunk
 constexpr int kPitch = 68;             // fp32 row pitch in shared memory (272 B)
 constexpr int kSlice = 16;             // value rows of the state per scan CTA
 constexpr int kWsFloats = 3 * 4096 + 192;  // W, Ut, P, then qs[64], ks[64], b_last
+// Workspace of one (sequence x head, chunk), in floats: W at 0 (fp32, or for
+// the tensor-core scan -W as bf16 hi then lo planes), Ut at kWsUt (fp32), P at
+// kWsP (fp32, or bf16), then the row scales.
+constexpr int kWsUt = 4096, kWsP = 2 * 4096;
 constexpr int kWsQs = 3 * 4096, kWsKs = kWsQs + 64, kWsBlast = kWsKs + 64;
 constexpr float kMinLogAlpha = -87.0f;  // alpha below e^-87 (1.6e-38) acts as e^-87
 
@@ -96,6 +110,49 @@ __device__ __forceinline__ float dot4(float4 a, float4 b, float acc) {
     return fmaf(a.w, b.w, acc);
 }
 
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t (&r)[4]) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr));
+}
+__device__ __forceinline__ void mma_bf16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                         uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+// Two fp32 values as a bf16 pair, the first in the low half.
+__device__ __forceinline__ uint32_t pack_bf16(float x, float y) {
+    uint32_t r;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(y), "f"(x));
+    return r;
+}
+// x = hi + lo with hi = bf16(x) and lo = bf16(x - hi), for a pair.
+__device__ __forceinline__ void split_bf16(float x, float y, uint32_t &hi, uint32_t &lo) {
+    hi = pack_bf16(x, y);
+    const float hx = __uint_as_float(hi << 16), hy = __uint_as_float(hi & 0xffff0000u);
+    lo = pack_bf16(x - hx, y - hy);
+}
+__device__ __forceinline__ void st_shared_u32(uint32_t addr, uint32_t v) {
+    asm volatile("st.shared.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+// 16-byte asynchronous copy; src_bytes = 0 fills the destination with zeros.
+__device__ __forceinline__ void cp_async_16(uint32_t dst, const void *src, int src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
+                 "r"(src_bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit_wait_all() {
+    asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+}
+
 // Normalises rows [8w, 8w + 8) of a [64][kPitch] tile in place (warp w of 8)
 // and stores 1/|row| (0 for a zero row) in inv[].
 __device__ __forceinline__ void normalise_rows(float *tile, float *inv) {
@@ -121,7 +178,7 @@ struct GdArgs {
     int B, T, H, nchunks, zero_init, accumulate;
 };
 
-// Kernel 1: one CTA per (chunk, sequence x head).
+// Kernel 1 for fp32 inputs: one CTA per (chunk, sequence x head), fp32 FMA.
 template <typename Tin>
 __global__ void __launch_bounds__(256) gd_chunk_kernel(GdArgs a) {
     extern __shared__ __align__(16) float sm[];
@@ -209,7 +266,7 @@ __global__ void __launch_bounds__(256) gd_chunk_kernel(GdArgs a) {
             }
             *reinterpret_cast<float4 *>(As + t * kPitch + 4 * tc) =
                 make_float4(av[0], av[1], av[2], av[3]);
-            *reinterpret_cast<float4 *>(ws + 2 * 4096 + t * 64 + 4 * tc) =
+            *reinterpret_cast<float4 *>(ws + kWsP + t * 64 + 4 * tc) =
                 make_float4(pv[0], pv[1], pv[2], pv[3]);
         }
     }
@@ -224,18 +281,19 @@ __global__ void __launch_bounds__(256) gd_chunk_kernel(GdArgs a) {
             x[t] = c < 64 ? bb[t] * Ks[t * kPitch + c] : bet[t] * Vs[t * kPitch + c - 64];
 #pragma unroll
         for (int t = 1; t < kC; ++t) {
-            float acc = x[t];
+            // four partial sums: a dependency chain of t/4 instead of t
+            float a0 = 0.0f, a1 = 0.0f, a2 = 0.0f, a3 = 0.0f;
 #pragma unroll
             for (int g = 0; g < (t + 3) / 4; ++g) {
                 const float4 av = *reinterpret_cast<const float4 *>(As + t * kPitch + 4 * g);
-                acc = fmaf(-av.x, x[4 * g], acc);
-                acc = fmaf(-av.y, x[4 * g + 1], acc);
-                acc = fmaf(-av.z, x[4 * g + 2], acc);
-                acc = fmaf(-av.w, x[4 * g + 3], acc);
+                a0 = fmaf(av.x, x[4 * g], a0);
+                a1 = fmaf(av.y, x[4 * g + 1], a1);
+                a2 = fmaf(av.z, x[4 * g + 2], a2);
+                a3 = fmaf(av.w, x[4 * g + 3], a3);
             }
-            x[t] = acc;
+            x[t] -= (a0 + a1) + (a2 + a3);
         }
-        float *dst = c < 64 ? ws + c : ws + 4096 + (c - 64);
+        float *dst = c < 64 ? ws + c : ws + kWsUt + (c - 64);
 #pragma unroll
         for (int t = 0; t < kC; ++t) dst[t * 64] = x[t];
     } else if (tid < 192) {
@@ -285,12 +343,12 @@ __global__ void __launch_bounds__(256) gd_scan_kernel(GdArgs a) {
             *reinterpret_cast<float4 *>(Wsm + t * kPitch + c) =
                 *reinterpret_cast<const float4 *>(ws + t * 64 + c);
             *reinterpret_cast<float4 *>(Psm + t * kPitch + c) =
-                *reinterpret_cast<const float4 *>(ws + 2 * 4096 + t * 64 + c);
+                *reinterpret_cast<const float4 *>(ws + kWsP + t * 64 + c);
         }
         float u[4], oi[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-            u[i] = ws[4096 + (4 * tg + i) * 64 + r0 + r];
+            u[i] = ws[kWsUt + (4 * tg + i) * 64 + r0 + r];
             oi[i] = 0.0f;
         }
         const float blast = ws[kWsBlast];
@@ -360,6 +418,387 @@ __global__ void __launch_bounds__(256) gd_scan_kernel(GdArgs a) {
         const int rr = i >> 6, c = i & 63;
         state[rr * 64 + c] = Ssm[rr * kPitch + c];
     }
+}
+
+// Kernel 1 for bf16 inputs: one CTA of 4 warps per (chunk, sequence x head).
+// The key-key and query-key products run on the tensor cores from the raw bf16
+// rows (exact products, fp32 accumulate) and are scaled by the row norms
+// afterwards; the triangular solve runs on the CUDA cores, one thread per
+// right-hand-side column.  Writes -W as bf16 hi/lo planes, Ut (fp32), P (bf16)
+// and the row scales.
+constexpr int kTPc = 144;                              // bytes per row of a [64][64] bf16 tile
+constexpr int kTBc = 64 * kTPc;
+constexpr size_t kChunkMmaSmem = 3 * kTBc + (kC * kPitch + 5 * kC) * sizeof(float);
+
+__global__ void __launch_bounds__(128, 4) gd_chunk_mma_kernel(GdArgs a) {
+    extern __shared__ __align__(128) uint8_t smb[];
+    const uint32_t sb = smem_u32(smb);
+    const uint8_t *Kb = smb + kTBc, *Vb = smb + 2 * kTBc;
+    float *As = reinterpret_cast<float *>(smb + 3 * kTBc);
+    float *gam = As + kC * kPitch, *bet = gam + kC, *rho = bet + kC, *kap = rho + kC, *bb = kap + kC;
+
+    const int ch = blockIdx.x, bh = blockIdx.y;
+    const int b = bh / a.H, h = bh % a.H;
+    const int t0 = ch * kC, n = min(kC, a.T - t0);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int g = lane >> 2, q2 = 2 * (lane & 3);
+    const size_t row0 = static_cast<size_t>(b) * a.T + t0;
+    float *ws = a.ws + (static_cast<size_t>(bh) * a.nchunks + ch) * kWsFloats;
+    __nv_bfloat16 *wsh = reinterpret_cast<__nv_bfloat16 *>(ws);
+
+    // Raw rows of q, k, v (rows >= n zero).
+    for (int p = tid; p < 3 * 512; p += 128) {
+        const int tile = p >> 9, row = (p & 511) >> 3, c8 = 8 * (p & 7);
+        const __nv_bfloat16 *base = static_cast<const __nv_bfloat16 *>(
+                                        tile == 0 ? a.q : tile == 1 ? a.k : a.v) +
+                                    h * kHeadDim;
+        const int rr = row < n ? row : 0;
+        cp_async_16(sb + tile * kTBc + row * kTPc + 2 * c8,
+                    base + (row0 + rr) * a.H * static_cast<size_t>(kHeadDim) + c8,
+                    row < n ? 16 : 0);
+    }
+    if (warp == 0) {
+        float la[2], be[2];
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+            const int t = 2 * lane + i;
+            const size_t idx = (row0 + t) * a.H + h;
+            la[i] = t < n ? fmaxf(logf(a.alpha[idx]), kMinLogAlpha) : 0.0f;
+            be[i] = t < n ? a.beta[idx] : 0.0f;
+        }
+        const float pair = la[0] + la[1];
+        float incl = pair;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const float y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
+        }
+        const float excl = incl - pair;
+        gam[2 * lane] = excl + la[0];
+        gam[2 * lane + 1] = incl;
+        bet[2 * lane] = be[0];
+        bet[2 * lane + 1] = be[1];
+        bb[2 * lane] = be[0] * expf(excl + la[0]);
+        bb[2 * lane + 1] = be[1] * expf(incl);
+    }
+    cp_async_commit_wait_all();
+    __syncthreads();
+
+    // Row norms: warp w takes rows 16w .. 16w + 15 of q and of k.
+#pragma unroll 4
+    for (int i = 0; i < 16; ++i) {
+        const int t = 16 * warp + i;
+        const uint32_t qq = *reinterpret_cast<const uint32_t *>(smb + t * kTPc + 4 * lane);
+        const uint32_t kk = *reinterpret_cast<const uint32_t *>(Kb + t * kTPc + 4 * lane);
+        const float q0 = __uint_as_float(qq << 16), q1 = __uint_as_float(qq & 0xffff0000u);
+        const float k0 = __uint_as_float(kk << 16), k1 = __uint_as_float(kk & 0xffff0000u);
+        const float sq = warp_sum(fmaf(q0, q0, q1 * q1));
+        const float sk = warp_sum(fmaf(k0, k0, k1 * k1));
+        if (lane == 0) {
+            rho[t] = sq > 0.0f ? 1.0f / sqrtf(sq) : 0.0f;
+            kap[t] = sk > 0.0f ? 1.0f / sqrtf(sk) : 0.0f;
+        }
+    }
+    __syncthreads();
+    if (tid < 64) {
+        const int t = tid;
+        const float glast = gam[kC - 1];
+        ws[kWsQs + t] = rho[t] * expf(gam[t]);
+        ws[kWsKs + t] = kap[t] * expf(glast - gam[t]);
+        if (t == 0) ws[kWsBlast] = expf(glast);
+    }
+
+    // K K^T and Q K^T for rows 16w .. 16w + 15, columns up to the diagonal block.
+    {
+        const int a_row = (lane & 7) + 8 * ((lane >> 3) & 1), a_col = 8 * (lane >> 4);
+        const int bn_row = (lane & 7) + 8 * (lane >> 4), bn_col = 8 * ((lane >> 3) & 1);
+        float gk[8][4], gq[8][4];
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) gk[i][j] = gq[i][j] = 0.0f;
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks) {
+            const uint32_t ao = (16 * warp + a_row) * kTPc + 2 * (16 * ks + a_col);
+            uint32_t ak[4], aq[4];
+            ldsm_x4(sb + kTBc + ao, ak);
+            ldsm_x4(sb + ao, aq);
+#pragma unroll
+            for (int np = 0; np < 4; ++np) {
+                if (np > warp) break;
+                uint32_t bk[4];
+                ldsm_x4(sb + kTBc + (16 * np + bn_row) * kTPc + 2 * (16 * ks + bn_col), bk);
+                mma_bf16(gk[2 * np], ak, bk[0], bk[1]);
+                mma_bf16(gk[2 * np + 1], ak, bk[2], bk[3]);
+                mma_bf16(gq[2 * np], aq, bk[0], bk[1]);
+                mma_bf16(gq[2 * np + 1], aq, bk[2], bk[3]);
+            }
+        }
+#pragma unroll
+        for (int nt = 0; nt < 8; ++nt) {
+            if (nt > 2 * warp + 1) break;
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf) {
+                const int t = 16 * warp + g + 8 * hf, j = 8 * nt + q2;
+                float av[2], pv[2];
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const int jj = j + e;
+                    const float d = jj <= t ? expf(gam[t] - gam[jj]) * kap[jj] : 0.0f;
+                    av[e] = jj < t ? bet[t] * kap[t] * d * gk[nt][2 * hf + e] : 0.0f;
+                    pv[e] = rho[t] * d * gq[nt][2 * hf + e];
+                }
+                *reinterpret_cast<float2 *>(As + t * kPitch + j) = make_float2(av[0], av[1]);
+                *reinterpret_cast<uint32_t *>(wsh + 2 * kWsP + t * 64 + j) = pack_bf16(pv[0], pv[1]);
+            }
+        }
+    }
+    __syncthreads();
+
+    // Forward substitution, column c of [diag(beta b kap) K | diag(beta) V].
+    {
+        const int c = tid;
+        float x[kC];
+#pragma unroll
+        for (int t = 0; t < kC; ++t) {
+            const __nv_bfloat16 e = c < 64 ? *reinterpret_cast<const __nv_bfloat16 *>(
+                                                 Kb + t * kTPc + 2 * c)
+                                           : *reinterpret_cast<const __nv_bfloat16 *>(
+                                                 Vb + t * kTPc + 2 * (c - 64));
+            x[t] = (c < 64 ? bb[t] * kap[t] : bet[t]) * __bfloat162float(e);
+        }
+#pragma unroll
+        for (int t = 1; t < kC; ++t) {
+            float a0 = 0.0f, a1 = 0.0f, a2 = 0.0f, a3 = 0.0f;
+#pragma unroll
+            for (int gg = 0; gg < (t + 3) / 4; ++gg) {
+                const float4 av = *reinterpret_cast<const float4 *>(As + t * kPitch + 4 * gg);
+                a0 = fmaf(av.x, x[4 * gg], a0);
+                a1 = fmaf(av.y, x[4 * gg + 1], a1);
+                a2 = fmaf(av.z, x[4 * gg + 2], a2);
+                a3 = fmaf(av.w, x[4 * gg + 3], a3);
+            }
+            x[t] -= (a0 + a1) + (a2 + a3);
+        }
+        if (c < 64) {
+#pragma unroll
+            for (int t = 0; t < kC; ++t) {
+                const __nv_bfloat16 h16 = __float2bfloat16(-x[t]);
+                wsh[t * 64 + c] = h16;
+                wsh[4096 + t * 64 + c] = __float2bfloat16(-x[t] - __bfloat162float(h16));
+            }
+        } else {
+#pragma unroll
+            for (int t = 0; t < kC; ++t) ws[kWsUt + t * 64 + (c - 64)] = x[t];
+        }
+    }
+}
+
+// Kernel 2 for bf16 inputs, on the tensor cores: one CTA per (32 value rows,
+// sequence x head).  The CTA's 32 x 64 slice of the state lives in the
+// accumulator fragments of the state product (warp w: rows 16 (w/4) .. +16,
+// columns 16 (w%4) .. +16).  Per chunk:
+//   U  (64 t x 32 r) = Ut + (-W) S^T          3 terms: W hi/lo x S hi/lo
+//   O  (64 t x 32 r) = qs_t Q S^T + P U       Q exact; S, U hi/lo; P bf16
+//   S' (32 r x 64 c) = b_last S + (ks U)^T K  K exact; ks U hi/lo
+// where Q, K are the raw bf16 rows and qs, ks their norm-and-decay scales.
+constexpr int kMmaRows = 32;                          // value rows per CTA
+constexpr int kTP = 144;                              // bytes per row of a [*][64] bf16 tile
+constexpr int kTB = 64 * kTP;                         // one [64][64] bf16 tile
+constexpr int kUP = 80;                               // bytes per row of a [64][32] bf16 tile
+constexpr int kUB = 64 * kUP;
+constexpr int kSB = kMmaRows * kTP;                   // [32][64] bf16 state plane
+constexpr int kOffW = 0, kOffP = 2 * kTB, kOffQ = 3 * kTB, kOffK = 4 * kTB;
+constexpr int kOffS = 5 * kTB, kOffU = kOffS + 2 * kSB, kOffUK = kOffU + 2 * kUB;
+constexpr int kOffScal = kOffUK + 2 * kUB;            // qs[64], ks[64], b_last, 3 pad
+constexpr size_t kScanMmaSmem = kOffScal + 132 * sizeof(float);
+
+__global__ void __launch_bounds__(256, 2) gd_scan_mma_kernel(GdArgs a) {
+    extern __shared__ __align__(128) uint8_t smb[];
+    const uint32_t sb = smem_u32(smb);
+    const float *scal = reinterpret_cast<const float *>(smb + kOffScal);
+
+    const int slice = blockIdx.x, bh = blockIdx.y;
+    const int b = bh / a.H, h = bh % a.H;
+    const int r0 = slice * kMmaRows;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int g = lane >> 2, q2 = 2 * (lane & 3);
+    const int mt = warp >> 1, nh = warp & 1;   // U and O tiles: t rows 16 mt, r cols 16 nh
+    const int rm = warp >> 2, cn = warp & 3;   // state tiles: r rows 16 rm, c cols 16 cn
+    float *state = a.state + (static_cast<size_t>(bh) * 64 + r0) * 64;
+    const __nv_bfloat16 *qsrc = static_cast<const __nv_bfloat16 *>(a.q) + h * kHeadDim;
+    const __nv_bfloat16 *ksrc = static_cast<const __nv_bfloat16 *>(a.k) + h * kHeadDim;
+    __nv_bfloat16 *out = static_cast<__nv_bfloat16 *>(a.out);
+
+    float sacc[2][4];
+#pragma unroll
+    for (int n = 0; n < 2; ++n)
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+            const int r = 16 * rm + g + 8 * hf, c = 16 * cn + 8 * n + q2;
+            float2 v = make_float2(0.0f, 0.0f);
+            if (!a.zero_init) v = *reinterpret_cast<const float2 *>(state + r * 64 + c);
+            sacc[n][2 * hf] = v.x;
+            sacc[n][2 * hf + 1] = v.y;
+        }
+
+    // ldmatrix lane offsets (bytes within a tile)
+    const int a_row = (lane & 7) + 8 * ((lane >> 3) & 1), a_col = 8 * (lane >> 4);
+    const int bn_row = (lane & 7) + 8 * (lane >> 4), bn_col = 8 * ((lane >> 3) & 1);
+    const int bt_row = (lane & 7) + 8 * ((lane >> 3) & 1), bt_col = 8 * (lane >> 4);
+    const int at_row = (lane & 7) + 8 * (lane >> 4), at_col = 8 * ((lane >> 3) & 1);
+
+    for (int ch = 0; ch < a.nchunks; ++ch) {
+        const int t0 = ch * kC, n = min(kC, a.T - t0);
+        const size_t row0 = static_cast<size_t>(b) * a.T + t0;
+        const float *ws = a.ws + (static_cast<size_t>(bh) * a.nchunks + ch) * kWsFloats;
+        const __nv_bfloat16 *wsh = reinterpret_cast<const __nv_bfloat16 *>(ws);
+
+        // -W hi, -W lo, P (workspace) and the raw Q, K rows; rows >= n zero.
+        for (int p = tid; p < 5 * 512; p += 256) {
+            const int tile = p >> 9, row = (p & 511) >> 3, c8 = 8 * (p & 7);
+            const void *src;
+            int bytes = 16;
+            if (tile < 2) {
+                src = wsh + tile * 4096 + row * 64 + c8;
+            } else if (tile == 2) {
+                src = wsh + 2 * kWsP + row * 64 + c8;
+            } else {
+                const __nv_bfloat16 *base = tile == 3 ? qsrc : ksrc;
+                const int rr = row < n ? row : 0;
+                bytes = row < n ? 16 : 0;
+                src = base + (row0 + rr) * a.H * static_cast<size_t>(kHeadDim) + c8;
+            }
+            cp_async_16(sb + tile * kTB + row * kTP + 2 * c8, src, bytes);
+        }
+        if (tid < 33) cp_async_16(sb + kOffScal + 16 * tid, ws + kWsQs + 4 * tid, 16);
+
+        // The state slice as bf16 hi/lo planes [r][c].
+#pragma unroll
+        for (int n2 = 0; n2 < 2; ++n2)
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf) {
+                const int r = 16 * rm + g + 8 * hf, c = 16 * cn + 8 * n2 + q2;
+                uint32_t hi, lo;
+                split_bf16(sacc[n2][2 * hf], sacc[n2][2 * hf + 1], hi, lo);
+                st_shared_u32(sb + kOffS + r * kTP + 2 * c, hi);
+                st_shared_u32(sb + kOffS + kSB + r * kTP + 2 * c, lo);
+            }
+
+        float uacc[2][4], oacc[2][4];
+#pragma unroll
+        for (int n2 = 0; n2 < 2; ++n2)
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf) {
+                const int t = 16 * mt + g + 8 * hf, r = 16 * nh + 8 * n2 + q2;
+                const float2 u2 = *reinterpret_cast<const float2 *>(ws + kWsUt + t * 64 + r0 + r);
+                uacc[n2][2 * hf] = u2.x;
+                uacc[n2][2 * hf + 1] = u2.y;
+                oacc[n2][2 * hf] = oacc[n2][2 * hf + 1] = 0.0f;
+            }
+        cp_async_commit_wait_all();
+        __syncthreads();
+
+        // U = Ut + (-W) S^T ;  O = Q S^T
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks) {
+            const uint32_t ao = (16 * mt + a_row) * kTP + 2 * (16 * ks + a_col);
+            uint32_t wh[4], wl[4], aq[4], bh4[4], bl4[4];
+            ldsm_x4(sb + kOffW + ao, wh);
+            ldsm_x4(sb + kOffW + kTB + ao, wl);
+            ldsm_x4(sb + kOffQ + ao, aq);
+            const uint32_t bo = (16 * nh + bn_row) * kTP + 2 * (16 * ks + bn_col);
+            ldsm_x4(sb + kOffS + bo, bh4);
+            ldsm_x4(sb + kOffS + kSB + bo, bl4);
+#pragma unroll
+            for (int n2 = 0; n2 < 2; ++n2) {
+                mma_bf16(uacc[n2], wh, bh4[2 * n2], bh4[2 * n2 + 1]);
+                mma_bf16(uacc[n2], wh, bl4[2 * n2], bl4[2 * n2 + 1]);
+                mma_bf16(uacc[n2], wl, bh4[2 * n2], bh4[2 * n2 + 1]);
+                mma_bf16(oacc[n2], aq, bh4[2 * n2], bh4[2 * n2 + 1]);
+                mma_bf16(oacc[n2], aq, bl4[2 * n2], bl4[2 * n2 + 1]);
+            }
+        }
+        // U and ks U as hi/lo planes [t][r]; O's inter-chunk part times qs_t.
+#pragma unroll
+        for (int n2 = 0; n2 < 2; ++n2)
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf) {
+                const int t = 16 * mt + g + 8 * hf, r = 16 * nh + 8 * n2 + q2;
+                const float u0 = uacc[n2][2 * hf], u1 = uacc[n2][2 * hf + 1];
+                const float kst = scal[64 + t], qst = scal[t];
+                uint32_t hi, lo;
+                split_bf16(u0, u1, hi, lo);
+                st_shared_u32(sb + kOffU + t * kUP + 2 * r, hi);
+                st_shared_u32(sb + kOffU + kUB + t * kUP + 2 * r, lo);
+                split_bf16(kst * u0, kst * u1, hi, lo);
+                st_shared_u32(sb + kOffUK + t * kUP + 2 * r, hi);
+                st_shared_u32(sb + kOffUK + kUB + t * kUP + 2 * r, lo);
+                oacc[n2][2 * hf] *= qst;
+                oacc[n2][2 * hf + 1] *= qst;
+            }
+        __syncthreads();
+
+        // O += P U  (P is zero above the diagonal: k-steps up to the row tile)
+        for (int ks = 0; ks <= mt; ++ks) {
+            uint32_t ap[4], bh4[4], bl4[4];
+            ldsm_x4(sb + kOffP + (16 * mt + a_row) * kTP + 2 * (16 * ks + a_col), ap);
+            const uint32_t bo = (16 * ks + bt_row) * kUP + 2 * (16 * nh + bt_col);
+            ldsm_x4_t(sb + kOffU + bo, bh4);
+            ldsm_x4_t(sb + kOffU + kUB + bo, bl4);
+#pragma unroll
+            for (int n2 = 0; n2 < 2; ++n2) {
+                mma_bf16(oacc[n2], ap, bh4[2 * n2], bh4[2 * n2 + 1]);
+                mma_bf16(oacc[n2], ap, bl4[2 * n2], bl4[2 * n2 + 1]);
+            }
+        }
+#pragma unroll
+        for (int n2 = 0; n2 < 2; ++n2)
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf) {
+                const int t = 16 * mt + g + 8 * hf, r = 16 * nh + 8 * n2 + q2;
+                if (t < n) {
+                    uint32_t *dst = reinterpret_cast<uint32_t *>(
+                        out + ((row0 + t) * a.H + h) * static_cast<size_t>(kHeadDim) + r0 + r);
+                    float v0 = oacc[n2][2 * hf], v1 = oacc[n2][2 * hf + 1];
+                    if (a.accumulate) {
+                        const uint32_t old = *dst;
+                        v0 += __uint_as_float(old << 16);
+                        v1 += __uint_as_float(old & 0xffff0000u);
+                    }
+                    *dst = pack_bf16(v0, v1);
+                }
+            }
+
+        // S = b_last S + (ks U)^T K
+        const float blast = scal[128];
+#pragma unroll
+        for (int n2 = 0; n2 < 2; ++n2)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) sacc[n2][i] *= blast;
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks) {
+            uint32_t ah[4], al[4], bk[4];
+            const uint32_t ao = (16 * ks + at_row) * kUP + 2 * (16 * rm + at_col);
+            ldsm_x4_t(sb + kOffUK + ao, ah);
+            ldsm_x4_t(sb + kOffUK + kUB + ao, al);
+            ldsm_x4_t(sb + kOffK + (16 * ks + bt_row) * kTP + 2 * (16 * cn + bt_col), bk);
+#pragma unroll
+            for (int n2 = 0; n2 < 2; ++n2) {
+                mma_bf16(sacc[n2], ah, bk[2 * n2], bk[2 * n2 + 1]);
+                mma_bf16(sacc[n2], al, bk[2 * n2], bk[2 * n2 + 1]);
+            }
+        }
+        __syncthreads();  // every read of this chunk's tiles and planes is done
+    }
+#pragma unroll
+    for (int n2 = 0; n2 < 2; ++n2)
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+            const int r = 16 * rm + g + 8 * hf, c = 16 * cn + 8 * n2 + q2;
+            *reinterpret_cast<float2 *>(state + r * 64 + c) =
+                make_float2(sacc[n2][2 * hf], sacc[n2][2 * hf + 1]);
+        }
 }
 
 // Decode step: one CTA per (sequence, head); thread owns S[tid/4][16 (tid%4) .. +16).
@@ -435,22 +874,39 @@ constexpr size_t kScanSmem = (4 * kC * kPitch + 2 * kSlice * kPitch + 2 * kC) * 
 
 template <typename Tin>
 cudaError_t launch_prefill_t(const GdArgs &g, cudaStream_t stream) {
+    constexpr bool kMma = std::is_same<Tin, __nv_bfloat16>::value;
     static bool configured = false;
+    cudaError_t e = cudaSuccess;
     if (!configured) {
-        cudaError_t e = cudaFuncSetAttribute(gd_chunk_kernel<Tin>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             static_cast<int>(kChunkSmem));
-        if (e != cudaSuccess) return e;
-        e = cudaFuncSetAttribute(gd_scan_kernel<Tin>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 static_cast<int>(kScanSmem));
+        if constexpr (kMma) {
+            e = cudaFuncSetAttribute(gd_chunk_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     static_cast<int>(kChunkMmaSmem));
+            if (e == cudaSuccess)
+                e = cudaFuncSetAttribute(gd_scan_mma_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(kScanMmaSmem));
+        } else {
+            e = cudaFuncSetAttribute(gd_chunk_kernel<Tin>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     static_cast<int>(kChunkSmem));
+            if (e == cudaSuccess)
+                e = cudaFuncSetAttribute(gd_scan_kernel<Tin>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(kScanSmem));
+        }
         if (e != cudaSuccess) return e;
         configured = true;
     }
     const unsigned bh = static_cast<unsigned>(g.B * g.H);
-    gd_chunk_kernel<Tin><<<dim3(g.nchunks, bh), 256, kChunkSmem, stream>>>(g);
-    cudaError_t e = cudaGetLastError();
+    if constexpr (kMma)
+        gd_chunk_mma_kernel<<<dim3(g.nchunks, bh), 128, kChunkMmaSmem, stream>>>(g);
+    else
+        gd_chunk_kernel<Tin><<<dim3(g.nchunks, bh), 256, kChunkSmem, stream>>>(g);
+    e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    gd_scan_kernel<Tin><<<dim3(64 / kSlice, bh), 256, kScanSmem, stream>>>(g);
+    if constexpr (kMma)
+        gd_scan_mma_kernel<<<dim3(64 / kMmaRows, bh), 256, kScanMmaSmem, stream>>>(g);
+    else
+        gd_scan_kernel<Tin><<<dim3(64 / kSlice, bh), 256, kScanSmem, stream>>>(g);
     count_launches(2);
     return cudaGetLastError();
 }
