@@ -583,16 +583,11 @@ def run_ours(args):
             wg, wst, Kg, t_gp, t_gs = gd_res
             gp_launch, gs_launch = t_gp / Kg, t_gs / Kg
             tok = wg.B * wg.T
-            nch = (wg.T + 63) // 64
-            # FMAs the two prefill kernels execute per (chunk, head): the chunk
-            # kernel's lower-triangle key-key and query-key products (136 tiles of
-            # 4 x 4 x 64, twice) and its 128-column forward substitution (sum over
-            # rows of 4 ceil(t/4) per column); the scan kernel's four products
-            # over its four 16-row state slices.
-            chunk_fma = 2 * 136 * 16 * 64 + 128 * sum(4 * ((t + 3) // 4) for t in range(1, 64))
-            scan_fma = 4 * (2 * 1024 * 64 + 64 * sum(4 * (g + 1) for g in range(16)) + 1024 * 64)
-            exec_flops = 2.0 * (chunk_fma + scan_fma) * wg.B * wg.H * nch
-            gp_tf = exec_flops / gp_launch / 1e12
+            # The recurrence's own arithmetic (S k, the rank-one write, S q:
+            # 6 D^2 flops per token and head) against the fp32 CUDA-core peak;
+            # the chunked kernels execute more (the triangular solve, hi/lo
+            # splits) to expose parallelism, partly on the tensor cores.
+            gp_tf = wg.flops / gp_launch / 1e12
             alu_peak = 2 * 148 * 128 * 1.965e9 / 1e12
             step_bytes = wst.state_bytes + wst.num_seqs * wst.H * wst.D * (4 * 2) + \
                 wst.num_seqs * wst.H * 8 + wst.num_seqs * 4
@@ -600,13 +595,13 @@ def run_ours(args):
             result["gdelta"] = {
                 "workload": wg.describe(), "ms_per_launch": gp_launch * 1e3,
                 "tokens_per_s": aggregate_throughput(tok * Kg, world, t_gp),
-                "recurrence_tflops": wg.flops / gp_launch / 1e12,
-                "note": "memory channel prefill (polar_gdelta_prefill: chunk kernel + scan kernel, "
-                        "fp32 CUDA cores), timed separately; not part of value"}
+                "note": "memory channel prefill (polar_gdelta_prefill: chunk kernel + scan kernel; "
+                        "bf16 inputs, products on mma.sync with hi/lo-split fp32 operands), timed "
+                        "separately; not part of value"}
             result["roofline_gdelta"] = {
-                "bound": "alu", "kernel": "gd_chunk_kernel+gd_scan_kernel", "achieved": gp_tf,
-                "peak": alu_peak, "unit": "TFLOP/s", "frac": gp_tf / alu_peak,
-                "flops_per_launch": exec_flops, "traffic": None,
+                "bound": "alu", "kernel": "gd_chunk_mma_kernel+gd_scan_mma_kernel",
+                "achieved": gp_tf, "peak": alu_peak, "unit": "TFLOP/s", "frac": gp_tf / alu_peak,
+                "flops_per_launch": wg.flops, "traffic": None,
                 "peak_source": "fp32 FMA: 148 SMs x 128 lanes x 2 flops x 1965 MHz (max SM clock)"}
             result["gdelta_step"] = {
                 "workload": wst.describe(), "ms_per_launch": gs_launch * 1e3,
