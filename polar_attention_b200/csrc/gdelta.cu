@@ -648,30 +648,76 @@ __global__ void __launch_bounds__(256, 2) gd_scan_mma_kernel(GdArgs a) {
     const int bt_row = (lane & 7) + 8 * ((lane >> 3) & 1), bt_col = 8 * (lane >> 4);
     const int at_row = (lane & 7) + 8 * (lane >> 4), at_col = 8 * ((lane >> 3) & 1);
 
+    // Two cp.async groups per chunk, each landing one phase ahead of its use:
+    // (-W hi, -W lo, Q, scales) for the first products and (P, K) for the rest.
+    auto chunk_ws = [&](int c) {
+        return a.ws + (static_cast<size_t>(bh) * a.nchunks + c) * kWsFloats;
+    };
+    auto issue_wq = [&](int c) {
+        if (c < a.nchunks) {
+            const int nc = min(kC, a.T - c * kC);
+            const size_t r0c = static_cast<size_t>(b) * a.T + c * kC;
+            const float *wsc = chunk_ws(c);
+            const __nv_bfloat16 *wshc = reinterpret_cast<const __nv_bfloat16 *>(wsc);
+            for (int p = tid; p < 3 * 512; p += 256) {
+                const int tile = p >> 9, row = (p & 511) >> 3, c8 = 8 * (p & 7);
+                if (tile < 2) {
+                    cp_async_16(sb + kOffW + tile * kTB + row * kTP + 2 * c8,
+                                wshc + tile * 4096 + row * 64 + c8, 16);
+                } else {
+                    const int rr = row < nc ? row : 0;
+                    cp_async_16(sb + kOffQ + row * kTP + 2 * c8,
+                                qsrc + (r0c + rr) * a.H * static_cast<size_t>(kHeadDim) + c8,
+                                row < nc ? 16 : 0);
+                }
+            }
+            if (tid < 33) cp_async_16(sb + kOffScal + 16 * tid, wsc + kWsQs + 4 * tid, 16);
+        }
+        asm volatile("cp.async.commit_group;" ::: "memory");
+    };
+    auto issue_pk = [&](int c) {
+        if (c < a.nchunks) {
+            const int nc = min(kC, a.T - c * kC);
+            const size_t r0c = static_cast<size_t>(b) * a.T + c * kC;
+            const __nv_bfloat16 *wshc = reinterpret_cast<const __nv_bfloat16 *>(chunk_ws(c));
+            for (int p = tid; p < 2 * 512; p += 256) {
+                const int tile = p >> 9, row = (p & 511) >> 3, c8 = 8 * (p & 7);
+                if (tile == 0) {
+                    cp_async_16(sb + kOffP + row * kTP + 2 * c8, wshc + 2 * kWsP + row * 64 + c8,
+                                16);
+                } else {
+                    const int rr = row < nc ? row : 0;
+                    cp_async_16(sb + kOffK + row * kTP + 2 * c8,
+                                ksrc + (r0c + rr) * a.H * static_cast<size_t>(kHeadDim) + c8,
+                                row < nc ? 16 : 0);
+                }
+            }
+        }
+        asm volatile("cp.async.commit_group;" ::: "memory");
+    };
+    // This thread's Ut entries of chunk c (the initial value of U).
+    auto load_ut = [&](int c, float (&u)[2][4]) {
+        if (c >= a.nchunks) return;
+        const float *wsc = chunk_ws(c);
+#pragma unroll
+        for (int n2 = 0; n2 < 2; ++n2)
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf) {
+                const int t = 16 * mt + g + 8 * hf, r = 16 * nh + 8 * n2 + q2;
+                const float2 u2 = *reinterpret_cast<const float2 *>(wsc + kWsUt + t * 64 + r0 + r);
+                u[n2][2 * hf] = u2.x;
+                u[n2][2 * hf + 1] = u2.y;
+            }
+    };
+
+    float unext[2][4];
+    issue_wq(0);
+    issue_pk(0);
+    load_ut(0, unext);
+
     for (int ch = 0; ch < a.nchunks; ++ch) {
         const int t0 = ch * kC, n = min(kC, a.T - t0);
         const size_t row0 = static_cast<size_t>(b) * a.T + t0;
-        const float *ws = a.ws + (static_cast<size_t>(bh) * a.nchunks + ch) * kWsFloats;
-        const __nv_bfloat16 *wsh = reinterpret_cast<const __nv_bfloat16 *>(ws);
-
-        // -W hi, -W lo, P (workspace) and the raw Q, K rows; rows >= n zero.
-        for (int p = tid; p < 5 * 512; p += 256) {
-            const int tile = p >> 9, row = (p & 511) >> 3, c8 = 8 * (p & 7);
-            const void *src;
-            int bytes = 16;
-            if (tile < 2) {
-                src = wsh + tile * 4096 + row * 64 + c8;
-            } else if (tile == 2) {
-                src = wsh + 2 * kWsP + row * 64 + c8;
-            } else {
-                const __nv_bfloat16 *base = tile == 3 ? qsrc : ksrc;
-                const int rr = row < n ? row : 0;
-                bytes = row < n ? 16 : 0;
-                src = base + (row0 + rr) * a.H * static_cast<size_t>(kHeadDim) + c8;
-            }
-            cp_async_16(sb + tile * kTB + row * kTP + 2 * c8, src, bytes);
-        }
-        if (tid < 33) cp_async_16(sb + kOffScal + 16 * tid, ws + kWsQs + 4 * tid, 16);
 
         // The state slice as bf16 hi/lo planes [r][c].
 #pragma unroll
@@ -689,14 +735,11 @@ __global__ void __launch_bounds__(256, 2) gd_scan_mma_kernel(GdArgs a) {
 #pragma unroll
         for (int n2 = 0; n2 < 2; ++n2)
 #pragma unroll
-            for (int hf = 0; hf < 2; ++hf) {
-                const int t = 16 * mt + g + 8 * hf, r = 16 * nh + 8 * n2 + q2;
-                const float2 u2 = *reinterpret_cast<const float2 *>(ws + kWsUt + t * 64 + r0 + r);
-                uacc[n2][2 * hf] = u2.x;
-                uacc[n2][2 * hf + 1] = u2.y;
-                oacc[n2][2 * hf] = oacc[n2][2 * hf + 1] = 0.0f;
+            for (int i = 0; i < 4; ++i) {
+                uacc[n2][i] = unext[n2][i];
+                oacc[n2][i] = 0.0f;
             }
-        cp_async_commit_wait_all();
+        asm volatile("cp.async.wait_group 1;" ::: "memory");  // this chunk's W, Q, scales
         __syncthreads();
 
         // U = Ut + (-W) S^T ;  O = Q S^T
@@ -737,6 +780,11 @@ __global__ void __launch_bounds__(256, 2) gd_scan_mma_kernel(GdArgs a) {
                 oacc[n2][2 * hf] *= qst;
                 oacc[n2][2 * hf + 1] *= qst;
             }
+        const float blast = scal[128];
+        __syncthreads();  // W, Q and the scales are consumed; U planes are visible
+        issue_wq(ch + 1);
+        load_ut(ch + 1, unext);
+        asm volatile("cp.async.wait_group 1;" ::: "memory");  // this chunk's P, K
         __syncthreads();
 
         // O += P U  (P is zero above the diagonal: k-steps up to the row tile)
@@ -771,7 +819,6 @@ __global__ void __launch_bounds__(256, 2) gd_scan_mma_kernel(GdArgs a) {
             }
 
         // S = b_last S + (ks U)^T K
-        const float blast = scal[128];
 #pragma unroll
         for (int n2 = 0; n2 < 2; ++n2)
 #pragma unroll
@@ -790,7 +837,9 @@ __global__ void __launch_bounds__(256, 2) gd_scan_mma_kernel(GdArgs a) {
             }
         }
         __syncthreads();  // every read of this chunk's tiles and planes is done
+        issue_pk(ch + 1);
     }
+    asm volatile("cp.async.wait_group 0;" ::: "memory");
 #pragma unroll
     for (int n2 = 0; n2 < 2; ++n2)
 #pragma unroll
@@ -801,15 +850,43 @@ __global__ void __launch_bounds__(256, 2) gd_scan_mma_kernel(GdArgs a) {
         }
 }
 
-// Decode step: one CTA per (sequence, head); thread owns S[tid/4][16 (tid%4) .. +16).
+// 16 consecutive elements of a row as fp32 (two or four 16-byte loads).
 template <typename Tin>
-__global__ void __launch_bounds__(256) gd_step_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
+__device__ __forceinline__ void load16(const Tin *src, float (&x)[16]);
+template <>
+__device__ __forceinline__ void load16<float>(const float *src, float (&x)[16]) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float4 v = reinterpret_cast<const float4 *>(src)[i];
+        x[4 * i] = v.x; x[4 * i + 1] = v.y; x[4 * i + 2] = v.z; x[4 * i + 3] = v.w;
+    }
+}
+template <>
+__device__ __forceinline__ void load16<__nv_bfloat16>(const __nv_bfloat16 *src, float (&x)[16]) {
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        const uint4 v = reinterpret_cast<const uint4 *>(src)[i];
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            x[8 * i + 2 * j] = __uint_as_float(w[j] << 16);
+            x[8 * i + 2 * j + 1] = __uint_as_float(w[j] & 0xffff0000u);
+        }
+    }
+}
+
+// Decode step: one CTA per (sequence, head); thread owns S[tid/4][16 (tid%4) .. +16).
+// Every warp takes the query and key norms itself (two elements a lane and a
+// warp sum) and each thread reads its own 16 columns of q and k, so the warps
+// never wait for one another.
+template <typename Tin>
+__global__ void __launch_bounds__(256, sizeof(Tin) == 2 ? 4 : 3)
+gd_step_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
                                                       const Tin *__restrict__ v,
                                                       const float *__restrict__ alpha,
                                                       const float *__restrict__ beta, float *pool,
                                                       int num_slots, const int32_t *__restrict__ slots,
                                                       int H, Tin *out, int accumulate, int *status) {
-    __shared__ float qh[64], kh[64], vv[64];
     const int seq = blockIdx.x / H, h = blockIdx.x % H;
     const int slot = slots[seq];
     if (slot < 0) return;
@@ -817,48 +894,45 @@ __global__ void __launch_bounds__(256) gd_step_kernel(const Tin *__restrict__ q,
         if (threadIdx.x == 0) record_error(status, POLAR_ERR_BAD_SLOT);
         return;
     }
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int tid = threadIdx.x, lane = tid & 31;
     const int r = tid >> 2, c0 = 16 * (tid & 3);
     float *S = pool + ((static_cast<size_t>(slot) * H + h) * 64 + r) * 64 + c0;
     float4 s[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) s[i] = reinterpret_cast<const float4 *>(S)[i];
     const size_t row = static_cast<size_t>(seq) * H + h;
-    if (warp < 3) {
-        const Tin *src = (warp == 0 ? q : warp == 1 ? k : v) + row * kHeadDim;
-        float x0 = to_f<Tin>(src[lane]), x1 = to_f<Tin>(src[lane + 32]);
-        if (warp < 2) {
-            const float ss = warp_sum(fmaf(x0, x0, x1 * x1));
-            const float inv = ss > 0.0f ? 1.0f / sqrtf(ss) : 0.0f;
-            x0 *= inv;
-            x1 *= inv;
-        }
-        float *dst = warp == 0 ? qh : warp == 1 ? kh : vv;
-        dst[lane] = x0;
-        dst[lane + 32] = x1;
-    }
+    const Tin *qr = q + row * kHeadDim, *kr = k + row * kHeadDim;
+    const float q0 = to_f<Tin>(qr[lane]), q1 = to_f<Tin>(qr[lane + 32]);
+    const float k0 = to_f<Tin>(kr[lane]), k1 = to_f<Tin>(kr[lane + 32]);
+    float qc[16], kc[16];
+    load16<Tin>(qr + c0, qc);
+    load16<Tin>(kr + c0, kc);
+    const float vr = to_f<Tin>(v[row * kHeadDim + r]);
     const float al = alpha[row], be = beta[row];
-    __syncthreads();
+    const float sq = warp_sum(fmaf(q0, q0, q1 * q1)), sk2 = warp_sum(fmaf(k0, k0, k1 * k1));
+    const float iq = sq > 0.0f ? 1.0f / sqrtf(sq) : 0.0f;
+    const float ik = sk2 > 0.0f ? 1.0f / sqrtf(sk2) : 0.0f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        qc[i] *= iq;
+        kc[i] *= ik;
+    }
 
     float sk = 0.0f;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const float4 k4 = *reinterpret_cast<const float4 *>(kh + c0 + 4 * i);
-        sk = dot4(s[i], k4, sk);
-    }
+    for (int i = 0; i < 4; ++i)
+        sk = dot4(s[i], make_float4(kc[4 * i], kc[4 * i + 1], kc[4 * i + 2], kc[4 * i + 3]), sk);
     sk += __shfl_xor_sync(0xffffffffu, sk, 1);
     sk += __shfl_xor_sync(0xffffffffu, sk, 2);
-    const float w = be * (vv[r] - al * sk);
+    const float w = be * (vr - al * sk);
     float o = 0.0f;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-        const float4 k4 = *reinterpret_cast<const float4 *>(kh + c0 + 4 * i);
-        const float4 q4 = *reinterpret_cast<const float4 *>(qh + c0 + 4 * i);
-        s[i].x = fmaf(al, s[i].x, w * k4.x);
-        s[i].y = fmaf(al, s[i].y, w * k4.y);
-        s[i].z = fmaf(al, s[i].z, w * k4.z);
-        s[i].w = fmaf(al, s[i].w, w * k4.w);
-        o = dot4(s[i], q4, o);
+        s[i].x = fmaf(al, s[i].x, w * kc[4 * i]);
+        s[i].y = fmaf(al, s[i].y, w * kc[4 * i + 1]);
+        s[i].z = fmaf(al, s[i].z, w * kc[4 * i + 2]);
+        s[i].w = fmaf(al, s[i].w, w * kc[4 * i + 3]);
+        o = dot4(s[i], make_float4(qc[4 * i], qc[4 * i + 1], qc[4 * i + 2], qc[4 * i + 3]), o);
         reinterpret_cast<float4 *>(S)[i] = s[i];
     }
     o += __shfl_xor_sync(0xffffffffu, o, 1);
