@@ -425,7 +425,7 @@ __global__ void __launch_bounds__(256) gd_scan_kernel(GdArgs a) {
 // rows (exact products, fp32 accumulate) and are scaled by the row norms
 // afterwards; the triangular solve runs on the CUDA cores, one thread per
 // right-hand-side column.  Writes -W as bf16 hi/lo planes, Ut (fp32), P (bf16)
-// and the row scales.
+// and the row scales.  The cumulative log-gates are kept in log2 units here.
 constexpr int kTPc = 144;                              // bytes per row of a [64][64] bf16 tile
 constexpr int kTBc = 64 * kTPc;
 constexpr size_t kChunkMmaSmem = 3 * kTBc + (kC * kPitch + 5 * kC) * sizeof(float);
@@ -463,7 +463,7 @@ __global__ void __launch_bounds__(128, 4) gd_chunk_mma_kernel(GdArgs a) {
         for (int i = 0; i < 2; ++i) {
             const int t = 2 * lane + i;
             const size_t idx = (row0 + t) * a.H + h;
-            la[i] = t < n ? fmaxf(logf(a.alpha[idx]), kMinLogAlpha) : 0.0f;
+            la[i] = t < n ? fmaxf(log2f(a.alpha[idx]), kMinLogAlpha * kLog2e) : 0.0f;
             be[i] = t < n ? a.beta[idx] : 0.0f;
         }
         const float pair = la[0] + la[1];
@@ -478,34 +478,36 @@ __global__ void __launch_bounds__(128, 4) gd_chunk_mma_kernel(GdArgs a) {
         gam[2 * lane + 1] = incl;
         bet[2 * lane] = be[0];
         bet[2 * lane + 1] = be[1];
-        bb[2 * lane] = be[0] * expf(excl + la[0]);
-        bb[2 * lane + 1] = be[1] * expf(incl);
+        bb[2 * lane] = be[0] * exp2f(excl + la[0]);
+        bb[2 * lane + 1] = be[1] * exp2f(incl);
     }
     cp_async_commit_wait_all();
     __syncthreads();
 
-    // Row norms: warp w takes rows 16w .. 16w + 15 of q and of k.
-#pragma unroll 4
-    for (int i = 0; i < 16; ++i) {
-        const int t = 16 * warp + i;
-        const uint32_t qq = *reinterpret_cast<const uint32_t *>(smb + t * kTPc + 4 * lane);
-        const uint32_t kk = *reinterpret_cast<const uint32_t *>(Kb + t * kTPc + 4 * lane);
-        const float q0 = __uint_as_float(qq << 16), q1 = __uint_as_float(qq & 0xffff0000u);
-        const float k0 = __uint_as_float(kk << 16), k1 = __uint_as_float(kk & 0xffff0000u);
-        const float sq = warp_sum(fmaf(q0, q0, q1 * q1));
-        const float sk = warp_sum(fmaf(k0, k0, k1 * k1));
-        if (lane == 0) {
-            rho[t] = sq > 0.0f ? 1.0f / sqrtf(sq) : 0.0f;
-            kap[t] = sk > 0.0f ? 1.0f / sqrtf(sk) : 0.0f;
+    // Row norms: thread t < 64 takes query row t, thread 64 + t key row t.
+    {
+        const int t = tid & 63;
+        const uint8_t *rowp = (tid < 64 ? smb : Kb) + t * kTPc;
+        float ss = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const uint4 v4 = *reinterpret_cast<const uint4 *>(rowp + 16 * i);
+            const uint32_t w[4] = {v4.x, v4.y, v4.z, v4.w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const float x0 = __uint_as_float(w[j] << 16), x1 = __uint_as_float(w[j] & 0xffff0000u);
+                ss = fmaf(x0, x0, fmaf(x1, x1, ss));
+            }
         }
+        (tid < 64 ? rho : kap)[t] = ss > 0.0f ? 1.0f / sqrtf(ss) : 0.0f;
     }
     __syncthreads();
     if (tid < 64) {
         const int t = tid;
         const float glast = gam[kC - 1];
-        ws[kWsQs + t] = rho[t] * expf(gam[t]);
-        ws[kWsKs + t] = kap[t] * expf(glast - gam[t]);
-        if (t == 0) ws[kWsBlast] = expf(glast);
+        ws[kWsQs + t] = rho[t] * exp2f(gam[t]);
+        ws[kWsKs + t] = kap[t] * exp2f(glast - gam[t]);
+        if (t == 0) ws[kWsBlast] = exp2f(glast);
     }
 
     // K K^T and Q K^T for rows 16w .. 16w + 15, columns up to the diagonal block.
@@ -544,7 +546,7 @@ __global__ void __launch_bounds__(128, 4) gd_chunk_mma_kernel(GdArgs a) {
 #pragma unroll
                 for (int e = 0; e < 2; ++e) {
                     const int jj = j + e;
-                    const float d = jj <= t ? expf(gam[t] - gam[jj]) * kap[jj] : 0.0f;
+                    const float d = jj <= t ? exp2f(gam[t] - gam[jj]) * kap[jj] : 0.0f;
                     av[e] = jj < t ? bet[t] * kap[t] * d * gk[nt][2 * hf + e] : 0.0f;
                     pv[e] = rho[t] * d * gq[nt][2 * hf + e];
                 }
