@@ -56,8 +56,9 @@ def parse_args(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="CPU work budget of the oracle baseline sample")
-    ap.add_argument("--only", choices=["both", "prefill", "decode"], default="both",
-                    help="time one half of the step (profiling runs)")
+    ap.add_argument("--only", choices=["both", "prefill", "decode", "gdelta"], default="both",
+                    help="time one half of the step, or only the memory-channel legs "
+                         "(profiling runs)")
     ap.add_argument("--prefill", choices=sorted(W.PREFILL_WORKLOADS), default=W.EXTRAP.name,
                     help="prefill workload (profiling runs use a smaller one)")
     ap.add_argument("--decode-seqs", type=int, default=W.DECODE.num_seqs,
@@ -689,7 +690,9 @@ def main(argv=None):
         res = run_ours(args)
         rank, world, _ = dist_env()
         if res is not None and args.only != "both":
-            res["partial_step"] = f"only the {args.only} half was timed (profiling run)"
+            res["partial_step"] = (f"only the {args.only} legs were timed (profiling run)"
+                                   if args.only == "gdelta" else
+                                   f"only the {args.only} half was timed (profiling run)")
         if res is not None and world == 1 and not args.no_cpu_baseline and args.only == "both":
             res["cpu_baseline"] = cpu_baseline(args.cpu_seconds)
         elif res is not None:

@@ -582,17 +582,29 @@ __global__ void __launch_bounds__(128, 4) gd_chunk_mma_kernel(GdArgs a) {
             }
             x[t] -= (a0 + a1) + (a2 + a3);
         }
-        if (c < 64) {
-#pragma unroll
-            for (int t = 0; t < kC; ++t) {
-                const __nv_bfloat16 h16 = __float2bfloat16(-x[t]);
-                wsh[t * 64 + c] = h16;
-                wsh[4096 + t * 64 + c] = __float2bfloat16(-x[t] - __bfloat162float(h16));
-            }
-        } else {
+        if (c >= 64) {
 #pragma unroll
             for (int t = 0; t < kC; ++t) ws[kWsUt + t * 64 + (c - 64)] = x[t];
         }
+        __syncthreads();  // every read of A is done: its area takes W
+        if (c < 64) {
+#pragma unroll
+            for (int t = 0; t < kC; ++t) As[t * kPitch + c] = -x[t];
+        }
+    }
+    __syncthreads();
+    // -W as bf16 hi and lo planes, 16-byte stores: thread (row t, 8 columns).
+    for (int e = tid; e < 64 * 8; e += 128) {
+        const int t = e >> 3, c8 = 8 * (e & 7);
+        const float4 x0 = *reinterpret_cast<const float4 *>(As + t * kPitch + c8);
+        const float4 x1 = *reinterpret_cast<const float4 *>(As + t * kPitch + c8 + 4);
+        uint4 hi, lo;
+        split_bf16(x0.x, x0.y, hi.x, lo.x);
+        split_bf16(x0.z, x0.w, hi.y, lo.y);
+        split_bf16(x1.x, x1.y, hi.z, lo.z);
+        split_bf16(x1.z, x1.w, hi.w, lo.w);
+        *reinterpret_cast<uint4 *>(wsh + t * 64 + c8) = hi;
+        *reinterpret_cast<uint4 *>(wsh + 4096 + t * 64 + c8) = lo;
     }
 }
 
