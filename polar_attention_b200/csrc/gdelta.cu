@@ -122,7 +122,7 @@ __device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t (&r)[4]) {
 }
 __device__ __forceinline__ void mma_bf16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
                                          uint32_t b1) {
-    asm volatile(
+    asm(
         "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
         "{%8,%9}, {%0,%1,%2,%3};"
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
@@ -664,61 +664,59 @@ __global__ void __launch_bounds__(256, 2) gd_scan_mma_kernel(GdArgs a) {
 
     // Two cp.async groups per chunk, each landing one phase ahead of its use:
     // (-W hi, -W lo, Q, scales) for the first products and (P, K) for the rest.
+    // Thread tid copies rows tid/8 and tid/8 + 32, 16 bytes at column 8 (tid%8),
+    // of every tile; the offsets below do not change from chunk to chunk.
+    const int cp_row = tid >> 3, cp_c8 = 8 * (tid & 7);
+    const uint32_t cp_dst = cp_row * kTP + 2 * cp_c8;                // + tile base, + 32 rows
+    const int cp_ws = cp_row * 64 + cp_c8;                           // bf16 elements, + 32 rows
+    const size_t row_stride = static_cast<size_t>(a.H) * kHeadDim;   // elements between tokens
     auto chunk_ws = [&](int c) {
         return a.ws + (static_cast<size_t>(bh) * a.nchunks + c) * kWsFloats;
     };
+    auto issue_rows = [&](uint32_t tile, const __nv_bfloat16 *src0, int nc) {
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+            const int row = cp_row + 32 * i;
+            cp_async_16(sb + tile + cp_dst + 32 * i * kTP,
+                        src0 + (row < nc ? row : 0) * row_stride + cp_c8, row < nc ? 16 : 0);
+        }
+    };
     auto issue_wq = [&](int c) {
         if (c < a.nchunks) {
-            const int nc = min(kC, a.T - c * kC);
-            const size_t r0c = static_cast<size_t>(b) * a.T + c * kC;
             const float *wsc = chunk_ws(c);
             const __nv_bfloat16 *wshc = reinterpret_cast<const __nv_bfloat16 *>(wsc);
-            for (int p = tid; p < 3 * 512; p += 256) {
-                const int tile = p >> 9, row = (p & 511) >> 3, c8 = 8 * (p & 7);
-                if (tile < 2) {
-                    cp_async_16(sb + kOffW + tile * kTB + row * kTP + 2 * c8,
-                                wshc + tile * 4096 + row * 64 + c8, 16);
-                } else {
-                    const int rr = row < nc ? row : 0;
-                    cp_async_16(sb + kOffQ + row * kTP + 2 * c8,
-                                qsrc + (r0c + rr) * a.H * static_cast<size_t>(kHeadDim) + c8,
-                                row < nc ? 16 : 0);
-                }
-            }
+#pragma unroll
+            for (int i = 0; i < 4; ++i)  // -W hi (rows, rows + 32), then -W lo
+                cp_async_16(sb + kOffW + (i >> 1) * kTB + cp_dst + 32 * (i & 1) * kTP,
+                            wshc + (i >> 1) * 4096 + cp_ws + 32 * 64 * (i & 1), 16);
+            issue_rows(kOffQ, qsrc + (static_cast<size_t>(b) * a.T + c * kC) * row_stride,
+                       min(kC, a.T - c * kC));
             if (tid < 33) cp_async_16(sb + kOffScal + 16 * tid, wsc + kWsQs + 4 * tid, 16);
         }
         asm volatile("cp.async.commit_group;" ::: "memory");
     };
     auto issue_pk = [&](int c) {
         if (c < a.nchunks) {
-            const int nc = min(kC, a.T - c * kC);
-            const size_t r0c = static_cast<size_t>(b) * a.T + c * kC;
             const __nv_bfloat16 *wshc = reinterpret_cast<const __nv_bfloat16 *>(chunk_ws(c));
-            for (int p = tid; p < 2 * 512; p += 256) {
-                const int tile = p >> 9, row = (p & 511) >> 3, c8 = 8 * (p & 7);
-                if (tile == 0) {
-                    cp_async_16(sb + kOffP + row * kTP + 2 * c8, wshc + 2 * kWsP + row * 64 + c8,
-                                16);
-                } else {
-                    const int rr = row < nc ? row : 0;
-                    cp_async_16(sb + kOffK + row * kTP + 2 * c8,
-                                ksrc + (r0c + rr) * a.H * static_cast<size_t>(kHeadDim) + c8,
-                                row < nc ? 16 : 0);
-                }
-            }
+#pragma unroll
+            for (int i = 0; i < 2; ++i)
+                cp_async_16(sb + kOffP + cp_dst + 32 * i * kTP,
+                            wshc + 2 * kWsP + cp_ws + 32 * 64 * i, 16);
+            issue_rows(kOffK, ksrc + (static_cast<size_t>(b) * a.T + c * kC) * row_stride,
+                       min(kC, a.T - c * kC));
         }
         asm volatile("cp.async.commit_group;" ::: "memory");
     };
     // This thread's Ut entries of chunk c (the initial value of U).
+    const int ut_off = (16 * mt + g) * 64 + r0 + 16 * nh + q2;
     auto load_ut = [&](int c, float (&u)[2][4]) {
         if (c >= a.nchunks) return;
-        const float *wsc = chunk_ws(c);
+        const float *src = chunk_ws(c) + kWsUt + ut_off;
 #pragma unroll
         for (int n2 = 0; n2 < 2; ++n2)
 #pragma unroll
             for (int hf = 0; hf < 2; ++hf) {
-                const int t = 16 * mt + g + 8 * hf, r = 16 * nh + 8 * n2 + q2;
-                const float2 u2 = *reinterpret_cast<const float2 *>(wsc + kWsUt + t * 64 + r0 + r);
+                const float2 u2 = *reinterpret_cast<const float2 *>(src + 8 * hf * 64 + 8 * n2);
                 u[n2][2 * hf] = u2.x;
                 u[n2][2 * hf + 1] = u2.y;
             }
@@ -767,14 +765,17 @@ __global__ void __launch_bounds__(256, 2) gd_scan_mma_kernel(GdArgs a) {
             const uint32_t bo = (16 * nh + bn_row) * kTP + 2 * (16 * ks + bn_col);
             ldsm_x4(sb + kOffS + bo, bh4);
             ldsm_x4(sb + kOffS + kSB + bo, bl4);
+            // consecutive MMAs go to different accumulators
 #pragma unroll
-            for (int n2 = 0; n2 < 2; ++n2) {
-                mma_bf16(uacc[n2], wh, bh4[2 * n2], bh4[2 * n2 + 1]);
-                mma_bf16(uacc[n2], wh, bl4[2 * n2], bl4[2 * n2 + 1]);
-                mma_bf16(uacc[n2], wl, bh4[2 * n2], bh4[2 * n2 + 1]);
-                mma_bf16(oacc[n2], aq, bh4[2 * n2], bh4[2 * n2 + 1]);
-                mma_bf16(oacc[n2], aq, bl4[2 * n2], bl4[2 * n2 + 1]);
-            }
+            for (int n2 = 0; n2 < 2; ++n2) mma_bf16(uacc[n2], wh, bh4[2 * n2], bh4[2 * n2 + 1]);
+#pragma unroll
+            for (int n2 = 0; n2 < 2; ++n2) mma_bf16(oacc[n2], aq, bh4[2 * n2], bh4[2 * n2 + 1]);
+#pragma unroll
+            for (int n2 = 0; n2 < 2; ++n2) mma_bf16(uacc[n2], wh, bl4[2 * n2], bl4[2 * n2 + 1]);
+#pragma unroll
+            for (int n2 = 0; n2 < 2; ++n2) mma_bf16(oacc[n2], aq, bl4[2 * n2], bl4[2 * n2 + 1]);
+#pragma unroll
+            for (int n2 = 0; n2 < 2; ++n2) mma_bf16(uacc[n2], wl, bh4[2 * n2], bh4[2 * n2 + 1]);
         }
         // U and ks U as hi/lo planes [t][r]; O's inter-chunk part times qs_t.
 #pragma unroll
@@ -809,10 +810,9 @@ __global__ void __launch_bounds__(256, 2) gd_scan_mma_kernel(GdArgs a) {
             ldsm_x4_t(sb + kOffU + bo, bh4);
             ldsm_x4_t(sb + kOffU + kUB + bo, bl4);
 #pragma unroll
-            for (int n2 = 0; n2 < 2; ++n2) {
-                mma_bf16(oacc[n2], ap, bh4[2 * n2], bh4[2 * n2 + 1]);
-                mma_bf16(oacc[n2], ap, bl4[2 * n2], bl4[2 * n2 + 1]);
-            }
+            for (int n2 = 0; n2 < 2; ++n2) mma_bf16(oacc[n2], ap, bh4[2 * n2], bh4[2 * n2 + 1]);
+#pragma unroll
+            for (int n2 = 0; n2 < 2; ++n2) mma_bf16(oacc[n2], ap, bl4[2 * n2], bl4[2 * n2 + 1]);
         }
 #pragma unroll
         for (int n2 = 0; n2 < 2; ++n2)
@@ -845,10 +845,9 @@ __global__ void __launch_bounds__(256, 2) gd_scan_mma_kernel(GdArgs a) {
             ldsm_x4_t(sb + kOffUK + kUB + ao, al);
             ldsm_x4_t(sb + kOffK + (16 * ks + bt_row) * kTP + 2 * (16 * cn + bt_col), bk);
 #pragma unroll
-            for (int n2 = 0; n2 < 2; ++n2) {
-                mma_bf16(sacc[n2], ah, bk[2 * n2], bk[2 * n2 + 1]);
-                mma_bf16(sacc[n2], al, bk[2 * n2], bk[2 * n2 + 1]);
-            }
+            for (int n2 = 0; n2 < 2; ++n2) mma_bf16(sacc[n2], ah, bk[2 * n2], bk[2 * n2 + 1]);
+#pragma unroll
+            for (int n2 = 0; n2 < 2; ++n2) mma_bf16(sacc[n2], al, bk[2 * n2], bk[2 * n2 + 1]);
         }
         __syncthreads();  // every read of this chunk's tiles and planes is done
         issue_pk(ch + 1);
