@@ -582,6 +582,7 @@ def run_ours(args):
                         "part of value"}
         if gd_res is not None:
             wg, wst, Kg, t_gp, t_gs = gd_res
+            sha_g = source_sha("gdelta.cu", "polar_common.cuh")
             gp_launch, gs_launch = t_gp / Kg, t_gs / Kg
             tok = wg.B * wg.T
             # The recurrence's own arithmetic (S k, the rank-one write, S q:
@@ -602,7 +603,7 @@ def run_ours(args):
             result["roofline_gdelta"] = {
                 "bound": "alu", "kernel": "gd_chunk_mma_kernel+gd_scan_mma_kernel",
                 "achieved": gp_tf, "peak": alu_peak, "unit": "TFLOP/s", "frac": gp_tf / alu_peak,
-                "flops_per_launch": wg.flops, "traffic": None,
+                "flops_per_launch": wg.flops, "traffic": profiled_traffic("gdelta", sha_g),
                 "peak_source": "fp32 FMA: 148 SMs x 128 lanes x 2 flops x 1965 MHz (max SM clock)"}
             result["gdelta_step"] = {
                 "workload": wst.describe(), "ms_per_launch": gs_launch * 1e3,
@@ -611,7 +612,7 @@ def run_ours(args):
             result["roofline_gdelta_step"] = {
                 "bound": "hbm", "kernel": "gd_step_kernel", "achieved": gs_gbs,
                 "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": gs_gbs / peaks["hbm_gbs"],
-                "bytes_per_launch": step_bytes, "traffic": None,
+                "bytes_per_launch": step_bytes, "traffic": profiled_traffic("gdelta_step", sha_g),
                 "peak_source": f"{peak_src} (copy bandwidth)"}
         if window_res is not None:
             wp, t_win = window_res
