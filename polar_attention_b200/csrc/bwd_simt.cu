@@ -64,6 +64,7 @@ struct BwdArgs {
     const float *u;
     float *rec;
     float *du_part;  // [B * row blocks][Hq][64]: per-block sums of gate * T * g
+    __nv_bfloat16 *dab;  // [B][Hq][T][64]: dA rounded to bf16 once (bf16 inputs only)
     int B, T, Hq, Hkv, window;
     float s, alpha, L, beta, inv_ln_L;
 };
@@ -700,8 +701,10 @@ bwd_rows_mma_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__
         for (int nt = 0; nt < 8; ++nt) {
             const int d = 8 * nt + 2 * tq;
             const float o0 = acc[nt][2 * hr] * inv_an, o1 = acc[nt][2 * hr + 1] * inv_an;
-            *reinterpret_cast<float2 *>(rec + kRecDA + d) =
-                make_float2((gr[nt][0] - o0 * cg) * inv_an, (gr[nt][1] - o1 * cg) * inv_an);
+            const float da0 = (gr[nt][0] - o0 * cg) * inv_an, da1 = (gr[nt][1] - o1 * cg) * inv_an;
+            *reinterpret_cast<float2 *>(rec + kRecDA + d) = make_float2(da0, da1);
+            *reinterpret_cast<uint32_t *>(
+                a.dab + ((static_cast<size_t>(b) * a.Hq + h) * Tlen + i) * kHeadDim + d) = pk2(da0, da1);
         }
         if (tq == 0) {
             *reinterpret_cast<float4 *>(rec + 64) = make_float4(m_ref[hr], cl2[hr], c, dl);
@@ -803,14 +806,15 @@ bwd_dq_mma_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__re
 }
 
 // dk, dv for bf16 inputs: a warp owns 16 keys; the rows that see them stream
-// in blocks of 64, for every query head of the group.
-__global__ void __launch_bounds__(128)
+// in blocks of 64, for every query head of the group.  Three CTAs per SM (a
+// small register spill) measured faster than two without one.
+__global__ void __launch_bounds__(128, 3)
 bwd_dkdv_mma_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
                     const __nv_bfloat16 *__restrict__ v, float *__restrict__ dk,
                     float *__restrict__ dv, const BwdArgs a) {
     __shared__ __align__(16) __nv_bfloat16 Qs[64][kPitch];
     __shared__ __align__(16) __nv_bfloat16 DAs[64][kPitch];
-    __shared__ float Cs[64][12];  // per staged row: ref cl2 c dl dl2 cmu csS dm jmax lo valid
+    __shared__ __align__(16) float Cs[64][12];  // per staged row: ref cl2 c dl dl2 cmu csS dm jmax lo valid
     const int Tlen = a.T, G = a.Hq / a.Hkv;
     const int key0 = blockIdx.x * 64, g = blockIdx.y, b = blockIdx.z;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, gq = lane >> 2, tq = lane & 3;
@@ -832,16 +836,8 @@ bwd_dkdv_mma_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__
         for (int i0 = key0; i0 < iend; i0 += 64) {
             __syncthreads();
             stage_rows(Qs, q + ((static_cast<size_t>(b) * Tlen + i0) * a.Hq + h) * kHeadDim, qstride, Tlen - i0);
-            for (int e = threadIdx.x; e < 64 * 32; e += 128) {  // dA as bf16 pairs
-                const int r = e >> 5, c = e & 31, i = i0 + r;
-                uint32_t val = 0u;
-                if (i < Tlen) {
-                    const float2 x = *reinterpret_cast<const float2 *>(
-                        a.rec + ((static_cast<size_t>(b) * a.Hq + h) * Tlen + i) * kRecWords + 2 * c);
-                    val = pk2(x.x, x.y);
-                }
-                *reinterpret_cast<uint32_t *>(&DAs[r][2 * c]) = val;
-            }
+            stage_rows(DAs, a.dab + ((static_cast<size_t>(b) * a.Hq + h) * Tlen + i0) * kHeadDim,
+                       kHeadDim, Tlen - i0);
             for (int e = threadIdx.x; e < 64 * 11; e += 128) {
                 const int r = e / 11, c = e % 11, i = i0 + r;
                 float val = 0.f;
@@ -865,11 +861,14 @@ bwd_dkdv_mma_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__
                 for (int e = 0; e < 4; ++e) {
                     const int rr = 8 * nt + 2 * tq + (e & 1), i = i0 + rr;
                     const int j = k0 + gq + 8 * (e >> 1);
+                    const float4 c0 = *reinterpret_cast<const float4 *>(&Cs[rr][0]);
+                    const float4 c1 = *reinterpret_cast<const float4 *>(&Cs[rr][4]);
+                    const float4 c2 = *reinterpret_cast<const float4 *>(&Cs[rr][8]);
                     RowCoef cf;
-                    cf.ref = Cs[rr][0]; cf.cl2 = Cs[rr][1]; cf.c = Cs[rr][2]; cf.dl = Cs[rr][3];
-                    cf.dl2 = Cs[rr][4]; cf.cmu = Cs[rr][5]; cf.csS = Cs[rr][6]; cf.dm = Cs[rr][7];
-                    cf.jmax = __float_as_int(Cs[rr][8]);
-                    cf.lo = __float_as_int(Cs[rr][9]);
+                    cf.ref = c0.x; cf.cl2 = c0.y; cf.c = c0.z; cf.dl = c0.w;
+                    cf.dl2 = c1.x; cf.cmu = c1.y; cf.csS = c1.z; cf.dm = c1.w;
+                    cf.jmax = __float_as_int(c2.x);
+                    cf.lo = __float_as_int(c2.y);
                     const bool vis = i < Tlen && j < Tlen && j <= i && j >= cf.lo;
                     float w;
                     const float x = pair_ds(cf, st[nt][e], at[nt][e], j, w);
@@ -939,7 +938,8 @@ size_t bwd_workspace_bytes(int B, int T, int Hq) {
     const size_t rec = static_cast<size_t>(B) * Hq * T * kRecWords * sizeof(float);
     const size_t part =  // per 64-row block (the bf16 rows pass; the fp32 one uses 128-row blocks)
         static_cast<size_t>(B) * ((T + 63) / 64) * Hq * kHeadDim * sizeof(float);
-    return rec + part;
+    const size_t dab = static_cast<size_t>(B) * Hq * T * kHeadDim * sizeof(__nv_bfloat16);
+    return rec + part + dab;
 }
 
 cudaError_t launch_bwd(const BwdLaunch &l) {
@@ -947,6 +947,8 @@ cudaError_t launch_bwd(const BwdLaunch &l) {
     a.u = l.u;
     a.rec = static_cast<float *>(l.workspace);
     a.du_part = a.rec + static_cast<size_t>(l.B) * l.Hq * l.T * kRecWords;
+    a.dab = reinterpret_cast<__nv_bfloat16 *>(
+        a.du_part + static_cast<size_t>(l.B) * ((l.T + 63) / 64) * l.Hq * kHeadDim);
     a.B = l.B; a.T = l.T; a.Hq = l.Hq; a.Hkv = l.Hkv; a.window = l.window;
     a.s = l.s; a.alpha = l.alpha; a.L = static_cast<float>(l.L); a.beta = l.beta;
     a.inv_ln_L = 1.0f / logf(static_cast<float>(l.L));
