@@ -34,6 +34,7 @@
 //
 // The decode step updates S in place in its pool slot: one read and one write
 // of the 16 KB state per (sequence, head), the rank-one form of the update.
+#include <atomic>
 #include <type_traits>
 
 #include "polar_common.cuh"
@@ -962,9 +963,12 @@ constexpr size_t kScanSmem = (4 * kC * kPitch + 2 * kSlice * kPitch + 2 * kC) * 
 template <typename Tin>
 cudaError_t launch_prefill_t(const GdArgs &g, cudaStream_t stream) {
     constexpr bool kMma = std::is_same<Tin, __nv_bfloat16>::value;
-    static bool configured = false;
-    cudaError_t e = cudaSuccess;
-    if (!configured) {
+    static std::atomic<uint64_t> configured{0};  // one bit per device
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const uint64_t bit = 1ull << (dev & 63);
+    if (!(configured.load() & bit)) {
         if constexpr (kMma) {
             e = cudaFuncSetAttribute(gd_chunk_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      static_cast<int>(kChunkMmaSmem));
@@ -981,7 +985,7 @@ cudaError_t launch_prefill_t(const GdArgs &g, cudaStream_t stream) {
                                          static_cast<int>(kScanSmem));
         }
         if (e != cudaSuccess) return e;
-        configured = true;
+        configured.fetch_or(bit);
     }
     const unsigned bh = static_cast<unsigned>(g.B * g.H);
     if constexpr (kMma)
