@@ -33,3 +33,15 @@ def test_tiny_workload_has_planted_signal():
     assert neff.min() >= 1.0
     assert (neff[np.r_[64:256, 320:512]] < 3).any()
     assert (neff > 20).any()
+
+
+def test_memory_oracle_matches_golden_fixture():
+    with open(os.path.join(HERE, "golden", "oracle_gdelta_fp32_T130.json")) as f:
+        g = json.load(f)
+    w = W.small_gdelta(B=1, T=130, H=2, dtype="fp32", seed=5)
+    x = W.gdelta_inputs(w, "cpu")
+    o, S = oracle.gdelta(x["q"].numpy(), x["k"].numpy(), x["v"].numpy(),
+                         x["alpha"].numpy().astype(np.float64), x["beta"].numpy().astype(np.float64))
+    np.testing.assert_allclose(o[0, g["sample_tokens"]], g["out_sample"], rtol=1e-12, atol=1e-14)
+    np.testing.assert_allclose(S[0, :, 0], g["state_row0"], rtol=1e-12, atol=1e-14)
+    np.testing.assert_allclose(np.sqrt((S[0] ** 2).sum(axis=(1, 2))), g["state_fro"], rtol=1e-12)
