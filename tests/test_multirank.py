@@ -37,8 +37,9 @@ def _worker(rank, world, port, q):
         m = bench.max_over_ranks(t, w, cpu)
         seed = bench.rank_seed(0, r)
         x = W.prefill_inputs(W.small_prefill(B=1, T=64, Hq=4, Hkv=2, dtype="bf16"), "cpu", seed=seed)
+        xg = W.gdelta_inputs(W.small_gdelta(B=1, T=64, H=2), "cpu", seed=seed + 2)
         q.put((r, w, local, seed, m, bench.aggregate_throughput(10.0, w, m),
-               float(x["q"].float().sum())))
+               float(x["q"].float().sum()), float(xg["k"].float().sum() + xg["alpha"].sum())))
         bench.barrier(w, cpu)
     finally:
         dist.destroy_process_group()
@@ -55,10 +56,11 @@ def test_two_gloo_ranks_weak_scaling():
     for p in procs:
         p.join(timeout=60)
         assert p.exitcode == 0
-    (r0, w0, l0, s0, m0, v0, q0), (r1, w1, l1, s1, m1, v1, q1) = res
+    (r0, w0, l0, s0, m0, v0, q0, g0), (r1, w1, l1, s1, m1, v1, q1, g1) = res
     assert (r0, r1) == (0, 1) and w0 == w1 == 2 and (l0, l1) == (0, 1)
     assert s0 != s1, "each rank must draw its own batch"
     assert q0 != q1, "the two ranks' inputs must differ"
+    assert g0 != g1, "the two ranks' memory-channel inputs must differ"
     assert m0 == m1 == 1.5, "every rank sees the slowest rank's time"
     assert v0 == v1 == pytest.approx(10.0 * 2 / 1.5), "whole-job work over the max time"
 
