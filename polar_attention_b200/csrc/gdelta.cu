@@ -10,7 +10,7 @@
 //
 // Prefill runs chunk-parallel (64 tokens a chunk).  Inside a chunk, with
 // g_t = sum_{s<=t} ln alpha_s (chunk-local, inclusive) and b_t = exp(g_t), the
-// rank-one writes u_t = S_t - alpha_t S_{t-1} applied to kh_t satisfy
+// rank-one writes u_t, defined by S_t = alpha_t S_{t-1} + u_t kh_t^T, satisfy
 //   u_t + beta_t sum_{j<t} e^{g_t-g_j} <kh_t,kh_j> u_j = beta_t (v_t - b_t S_0 kh_t),
 // a unit lower-triangular system (I + A) U = diag(beta) V - diag(beta b) Kh S_0^T.
 // Writing W = (I+A)^-1 diag(beta b) Kh and Ut = (I+A)^-1 diag(beta) V (both
@@ -30,7 +30,10 @@
 //    exact operand), so the state path keeps about 16 more bits than bf16.
 //    P, which only reaches the output, is one bf16 operand.
 //  - fp32 inputs: fp32 on the CUDA cores, 16 value rows a CTA.
-// Kernel 1 is fp32 on the CUDA cores for both.
+// Kernel 1 forms the key-key and query-key products on the tensor cores for
+// bf16 inputs (exact products of the raw rows, scaled by the row norms after)
+// and in fp32 FMA for fp32 inputs; its triangular solve is fp32 on the CUDA
+// cores in both.
 //
 // The decode step updates S in place in its pool slot: one read and one write
 // of the 16 KB state per (sequence, head), the rank-one form of the update.
