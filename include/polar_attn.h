@@ -4,10 +4,13 @@
  * The library computes the Polar Attention mixing step of "ATMA: Length-
  * Invariant Language Modeling via Polar Attention and Gated-Delta Compression
  * Memory" (H. Akbar; gist.science technical summary, section 2.1 "Polar
- * Attention: A Three-Channel Decomposition") without its recurrent-memory
- * stream:
+ * Attention: A Three-Channel Decomposition"):
  *
  *     out = content + count
+ *
+ * The third stream, the recurrent gated-delta memory, has its own entry
+ * points in polar_gdelta.h; they can add their read into an output written
+ * here (out = content + count + memory).
  *
  * For query row i of head h with visible keys j < n (n = i + 1 in causal
  * prefill, n = seqlen in decode) and kv head g = h / (Hq / Hkv):
