@@ -54,8 +54,8 @@
  *                                      detection" (section 2.1).
  *   count = gate * tanh(ln(n_eff) / ln(L)) * u_h    "bounded, saturating
  *                                      monotonic function (tanh of log)".
- *   out   = content + count            three-channel sum without the memory
- *                                      stream (out of scope here).
+ *   out   = content + count            the first two channels; the memory
+ *                                      stream's oracle is gdelta_oracle.c.
  *
  * Modes (all fp64; inputs are the exact fp32 values or the exact bf16 bits
  * widened to fp64):
