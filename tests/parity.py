@@ -1,7 +1,7 @@
 """Shared helpers of the GPU parity tests: oracle runs on the exact input bits
 and the comparison rules.
 
-Tolerances (stated by the method's specification for this build):
+Tolerances, as the method's specification fixes them:
   * out: normwise relative error max|gpu - ref| / max|ref| <= 2e-2 per
     (batch, head) slice for bf16 outputs (element-relative error is
     meaningless for content entries near zero); fp32 outputs from the fp32
