@@ -96,7 +96,7 @@ __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap *map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
 
-// 2D tiled TMA load into this CTA's own shared memory.
+// 2D tiled TMA load (no multicast) into this CTA's shared memory.
 __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, int x, int y,
                                             uint64_t *bar) {
     asm volatile(
@@ -106,7 +106,7 @@ __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, i
         : "memory");
 }
 
-// 4D tiled TMA load into this CTA's own shared memory.
+// 4D tiled TMA load (no multicast).
 __device__ __forceinline__ void tma_load_4d(void *dst, const CUtensorMap *map, int x, int y,
                                             int z, int w, uint64_t *bar) {
     asm volatile(
