@@ -21,6 +21,16 @@ extern "C" {
 polar_status_t polar_attn_selftest_exp2(const float *x, float *poly, float *mufu, int n,
                                         void *stream);
 
+/*
+ * Failure detection: launches one CTA whose single mbarrier wait can never
+ * complete (nothing arrives on the barrier).  The wait is the kernels' own
+ * bounded wait: after its cycle budget (about a second) it records
+ * POLAR_ERR_TIMEOUT in the device status word and the kernel exits normally,
+ * so polar_attn_get_status then returns POLAR_ERR_TIMEOUT and the context
+ * stays usable.  Asynchronous on `stream`.
+ */
+polar_status_t polar_attn_selftest_timeout(void *stream);
+
 #ifdef __cplusplus
 }
 #endif

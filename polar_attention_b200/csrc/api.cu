@@ -7,6 +7,7 @@
 
 #include <cudaTypedefs.h>
 
+#include "polar_attn_selftest.h"
 #include "polar_common.cuh"
 #include "polar_gdelta.h"
 #include "polar_internal.h"
@@ -127,6 +128,17 @@ FwdLaunch make_fwd(const void *q, const void *k, const void *v, const float *u,
 }  // namespace
 
 void count_launches(int n) { g_launches.fetch_add(static_cast<uint64_t>(n)); }
+
+// One bounded wait on a barrier that no thread or copy ever completes.
+__global__ void selftest_timeout_kernel(int *status) {
+    __shared__ __align__(8) uint64_t bar;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        fence_barrier_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) mbar_wait(&bar, 0, status);
+}
 
 CUresult encode_tiled(CUtensorMap *map, CUtensorMapDataType dtype, uint32_t rank, void *base,
                       const uint64_t *dims, const uint64_t *strides_bytes, const uint32_t *box,
@@ -426,6 +438,14 @@ const char *polar_attn_status_string(polar_status_t s) {
 }
 
 uint64_t polar_attn_launch_count(void) { return g_launches.load(); }
+
+polar_status_t polar_attn_selftest_timeout(void *stream) {
+    int *status = status_ptr();
+    if (!status) return POLAR_ERR_CUDA;
+    selftest_timeout_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(status);
+    count_launches(1);
+    return from_cuda(cudaGetLastError());
+}
 
 size_t polar_gdelta_prefill_workspace_size(const polar_gdelta_params_t *p) {
     if (check_gdelta_prefill(p) != POLAR_OK) return 0;

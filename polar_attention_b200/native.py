@@ -31,7 +31,8 @@ EXPORTS = ["polar_attn_default_params", "polar_attn_fwd_workspace_size", "polar_
            "polar_attn_decode_paged_noalloc", "polar_attn_selftest_exp2",
            "polar_attn_decode_chunk_workspace_size", "polar_attn_decode_paged_chunk",
            "polar_attn_bwd_workspace_size", "polar_attn_bwd",
-           "polar_gdelta_prefill_workspace_size", "polar_gdelta_prefill", "polar_gdelta_step"]
+           "polar_gdelta_prefill_workspace_size", "polar_gdelta_prefill", "polar_gdelta_step",
+           "polar_attn_selftest_timeout"]
 
 
 class PolarError(RuntimeError):
@@ -95,6 +96,7 @@ def lib() -> ctypes.CDLL:
             L.polar_attn_decode_paged_host.argtypes = [P, P, I, P, I, P, I, P, PP, P, P, P, Z, P]
             L.polar_attn_decode_paged_noalloc.argtypes = [P, P, I, P, I, P, I, P, PP, P, P, P]
             L.polar_attn_selftest_exp2.argtypes = [P, P, P, I, P]
+            L.polar_attn_selftest_timeout.argtypes = [P]
             GP = ctypes.POINTER(GdeltaParams)
             L.polar_gdelta_prefill_workspace_size.argtypes = [GP]
             L.polar_gdelta_prefill_workspace_size.restype = Z
@@ -108,7 +110,8 @@ def lib() -> ctypes.CDLL:
                          "polar_attn_decode_paged_host", "polar_attn_get_status",
                          "polar_attn_decode_paged_noalloc", "polar_attn_selftest_exp2",
                          "polar_attn_decode_paged_chunk", "polar_attn_bwd",
-                         "polar_gdelta_prefill", "polar_gdelta_step"):
+                         "polar_gdelta_prefill", "polar_gdelta_step",
+                         "polar_attn_selftest_timeout"):
                 getattr(L, name).restype = I
             _lib = L
     return _lib
@@ -417,6 +420,12 @@ def gdelta_step(q, k, v, alpha, beta, state_pool, slots, out=None, *, accumulate
                                    ctypes.byref(p), _ptr(out), _stream(stream)),
            "polar_gdelta_step")
     return out
+
+
+def selftest_timeout(stream=None):
+    """Launches one bounded wait that can never complete; afterwards
+    get_status() returns POLAR_ERR_TIMEOUT (5)."""
+    _check(lib().polar_attn_selftest_timeout(_stream(stream)), "polar_attn_selftest_timeout")
 
 
 def get_status(stream=None) -> int:
