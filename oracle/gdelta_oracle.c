@@ -34,7 +34,7 @@
  *                S[r][c] <- alpha S[r][c] + beta (v[r] - alpha (S kh)[r]) kh[c]
  *                (O(D^2) a token), for full-length sequences.
  *
- * ORACLE_MUTANT 13-15 plant mistakes that the memory pins must catch.
+ * ORACLE_MUTANT 13-17 plant mistakes that the memory pins must catch.
  */
 #include <math.h>
 #include <stdint.h>
@@ -122,7 +122,12 @@ int oracle_gdelta(const gdelta_cfg *cfg, const void *q, const void *k, const voi
                     for (int r = 0; r < D; ++r)
                         for (int c = 0; c < D; ++c) {
                             double acc = 0.0;
+#if ORACLE_MUTANT == 16
+                            /* mistake: the operands of the product swapped, M S */
+                            for (int i = 0; i < D; ++i) acc += M[r * D + i] * S[i * D + c];
+#else
                             for (int i = 0; i < D; ++i) acc += S[r * D + i] * M[i * D + c];
+#endif
                             SM[r * D + c] = acc;
                         }
                     for (int r = 0; r < D; ++r)
@@ -147,7 +152,12 @@ int oracle_gdelta(const gdelta_cfg *cfg, const void *q, const void *k, const voi
 #if ORACLE_MUTANT != 15
                 for (int r = 0; r < D; ++r) {
                     double acc = 0.0;
+#if ORACLE_MUTANT == 17
+                    /* mistake: the read takes the transposed state, S^T q */
+                    for (int c = 0; c < D; ++c) acc += S[c * D + r] * qh[c];
+#else
                     for (int c = 0; c < D; ++c) acc += S[r * D + c] * qh[c];
+#endif
                     o[r] = acc;
                 }
 #endif

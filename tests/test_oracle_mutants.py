@@ -7,15 +7,16 @@ mapping, a sample (not population) std, a log2 temperature, a dropped factor 2
 under the null-floor root, a missing unit-sphere projection, and the wrong
 head's count vector; in the backward, a dropped null-floor spread term and a
 flipped sign on the squared-sum gradient; in the memory channel, the decay gate
-left off the erase term, the key/query normalisation skipped, and a read taken
-before the write.
+left off the erase term, the key/query normalisation skipped, a read taken
+before the write, the operands of the update's matrix product swapped, and a
+read through the transposed state.
 """
 import pytest
 
 import oracle
 import oracle_pins as P
 
-MUTANTS = list(range(1, 16))
+MUTANTS = list(range(1, 18))
 
 
 @pytest.fixture(scope="module")
