@@ -567,12 +567,19 @@ int oracle_polar_bwd(const oracle_cfg *cfg, const void *q, const void *k, const 
 #if ORACLE_MUTANT != 11
                     if (sigma > 0.0) dz += dsigma * (z[j] - mu) / ((double)n * sigma);
 #endif
+#if ORACLE_MUTANT != 19
                     if (j == jmax) dz += dm;
+#endif
                     const double dS = c * dz;
                     for (int d = 0; d < D; ++d) {
                         dq[qo + d] += dS * ld(k, dtype, ko + d);
                         dk[ko + d] += dS * qr[d];
+#if ORACLE_MUTANT == 18
+                        /* mistake: the direction's projection left out of dv */
+                        dv[ko + d] += w[j] * gr[d] / an;
+#else
                         dv[ko + d] += w[j] * dA[d];
+#endif
                     }
                 }
             }

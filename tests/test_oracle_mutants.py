@@ -5,8 +5,9 @@ plants one plausible mistake: a dropped square in the l2 correction, n_eff =
 l/l2, a flipped gate sign, an off-by-one causal bound, a transposed GQA
 mapping, a sample (not population) std, a log2 temperature, a dropped factor 2
 under the null-floor root, a missing unit-sphere projection, and the wrong
-head's count vector; in the backward, a dropped null-floor spread term and a
-flipped sign on the squared-sum gradient; in the memory channel, the decay gate
+head's count vector; in the backward, a dropped null-floor spread term, a
+flipped sign on the squared-sum gradient, dv taken without the direction's
+projection, and a dropped argmax term of the gate; in the memory channel, the decay gate
 left off the erase term, the key/query normalisation skipped, a read taken
 before the write, the operands of the update's matrix product swapped, and a
 read through the transposed state.
@@ -16,7 +17,7 @@ import pytest
 import oracle
 import oracle_pins as P
 
-MUTANTS = list(range(1, 18))
+MUTANTS = list(range(1, 20))
 
 
 @pytest.fixture(scope="module")
