@@ -120,6 +120,9 @@ static inline int64_t kv_off(const key_src *ks, int64_t j, int which) {
     j += ks->j0;
     if (!ks->paged) return ks->dense_off + j * ks->dense_stride;
     int64_t page = ks->pt[j / ORACLE_PAGE];
+#if ORACLE_MUTANT == 20
+    which = 1 - which; /* mistake: the page's key and value planes swapped */
+#endif
     return (((page * 2 + which) * ks->Hkv + ks->g) * ORACLE_PAGE + (j % ORACLE_PAGE)) * ks->D;
 }
 

@@ -1,7 +1,8 @@
 """Planted mistakes in the oracle must each fail at least one pin.
 
 Each mutant is the oracle's C source compiled with ORACLE_MUTANT=k, which
-plants one plausible mistake: a dropped square in the l2 correction, n_eff =
+plants one plausible mistake (mutant 20: the paged cache's key and value planes
+swapped): a dropped square in the l2 correction, n_eff =
 l/l2, a flipped gate sign, an off-by-one causal bound, a transposed GQA
 mapping, a sample (not population) std, a log2 temperature, a dropped factor 2
 under the null-floor root, a missing unit-sphere projection, and the wrong
@@ -17,7 +18,7 @@ import pytest
 import oracle
 import oracle_pins as P
 
-MUTANTS = list(range(1, 20))
+MUTANTS = list(range(1, 21))
 
 
 @pytest.fixture(scope="module")
