@@ -384,8 +384,13 @@ int oracle_polar_fwd(const oracle_cfg *cfg, const void *q, const void *k, const 
 #endif
         int64_t lo = 0; /* first visible key */
         if (cfg->causal && cfg->window > 0 && n > cfg->window) {
+#if ORACLE_MUTANT == 21
+            lo = n - cfg->window + 1; /* mistake: the window one key short */
+            n = cfg->window - 1;
+#else
             lo = n - cfg->window;
             n = cfg->window;
+#endif
         }
         key_src ks = {k, v, dtype, D, cfg->Hkv, g, 0,
                       ((int64_t)b * T * cfg->Hkv + g) * D, (int64_t)cfg->Hkv * D, NULL, lo};

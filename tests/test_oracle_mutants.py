@@ -2,7 +2,7 @@
 
 Each mutant is the oracle's C source compiled with ORACLE_MUTANT=k, which
 plants one plausible mistake (mutant 20: the paged cache's key and value planes
-swapped): a dropped square in the l2 correction, n_eff =
+swapped; mutant 21: a prefill window one key short): a dropped square in the l2 correction, n_eff =
 l/l2, a flipped gate sign, an off-by-one causal bound, a transposed GQA
 mapping, a sample (not population) std, a log2 temperature, a dropped factor 2
 under the null-floor root, a missing unit-sphere projection, and the wrong
@@ -18,7 +18,7 @@ import pytest
 import oracle
 import oracle_pins as P
 
-MUTANTS = list(range(1, 21))
+MUTANTS = list(range(1, 22))
 
 
 @pytest.fixture(scope="module")
