@@ -41,7 +41,7 @@ class _Cfg(ctypes.Structure):
         ("B", ctypes.c_int), ("T", ctypes.c_int), ("Hq", ctypes.c_int), ("Hkv", ctypes.c_int),
         ("D", ctypes.c_int), ("s", ctypes.c_double), ("alpha", ctypes.c_double),
         ("L", ctypes.c_int), ("beta", ctypes.c_double), ("causal", ctypes.c_int),
-        ("len_mode", ctypes.c_int), ("window", ctypes.c_int),
+        ("window", ctypes.c_int),
     ]
 
 
@@ -58,7 +58,6 @@ class Params:
     L: int = 2048
     beta: float = 1.0
     causal: bool = True
-    len_mode: int = 0  # 0: n = visible keys, 1: n = total T
     window: int = 0    # 0: every causal key; W > 0: the last W of them
 
 
@@ -146,7 +145,7 @@ def polar_fwd(q, k, v, u, p: Params = Params(), rows=None, mode: str = "two_pass
     if k.shape != (B, T, Hkv, D) or v.shape != k.shape:
         raise ValueError("k/v shape mismatch")
     u = np.ascontiguousarray(u, dtype=np.float32)
-    cfg = _Cfg(B, T, Hq, Hkv, D, p.s, p.alpha, p.L, p.beta, int(p.causal), p.len_mode,
+    cfg = _Cfg(B, T, Hq, Hkv, D, p.s, p.alpha, p.L, p.beta, int(p.causal),
                int(p.window))
     if rows is None:
         n = B * Hq * T
@@ -180,7 +179,7 @@ def polar_bwd(q, k, v, u, gout, p: Params = Params(), mutant: int = 0,
     g = np.ascontiguousarray(gout, dtype=np.float64)
     if g.shape != (B, T, Hq, D):
         raise ValueError("gout shape mismatch")
-    cfg = _Cfg(B, T, Hq, Hkv, D, p.s, p.alpha, p.L, p.beta, int(p.causal), p.len_mode,
+    cfg = _Cfg(B, T, Hq, Hkv, D, p.s, p.alpha, p.L, p.beta, int(p.causal),
                int(p.window))
     dq = np.zeros((B, T, Hq, D), np.float64)
     dk = np.zeros((B, T, Hkv, D), np.float64)
@@ -210,7 +209,7 @@ def polar_decode(q, kv_pages, page_table, seqlens, u, p: Params = Params(), rows
     page_table = np.ascontiguousarray(page_table, dtype=np.int32)
     seqlens = np.ascontiguousarray(seqlens, dtype=np.int32)
     u = np.ascontiguousarray(u, dtype=np.float32)
-    cfg = _Cfg(N, 0, Hq, Hkv, D, p.s, p.alpha, p.L, p.beta, 1, 0, int(p.window))
+    cfg = _Cfg(N, 0, Hq, Hkv, D, p.s, p.alpha, p.L, p.beta, 1, int(p.window))
     if rows is None:
         n = N * Hq
         rows_arr = None

@@ -22,7 +22,7 @@
  *   n     = i + 1 (causal prefill)     reading: the length in the length
  *           | T (non-causal)           temperature is the number of keys the
  *           | seqlen (decode)          row can see, so row i never depends on
- *                                      the future (len_mode 1 uses total T).
+ *                                      the future.
  *   window W > 0 (sliding window, the ablation the results section names):
  *                                      the visible keys are the last W of
  *                                      those, j in [i - W + 1, i] (prefill) or
@@ -91,7 +91,6 @@ typedef struct {
     int L;         /* training length L_train */
     double beta;   /* gate slope */
     int causal;    /* prefill: 1 = row i sees keys 0..i */
-    int len_mode;  /* 0: n = visible keys; 1: n = total length T (ablation) */
     int window;    /* 0: all of them; W > 0: only the last W visible keys */
 } oracle_cfg;
 
@@ -321,18 +320,8 @@ static void row_stream(const double *q, const key_src *ks, int64_t n, const orac
 }
 
 static void eval_row(int mode, int block, double theta, const double *q, const key_src *ks,
-                     int64_t n, int64_t n_len, const oracle_cfg *cfg, const float *u_h,
-                     double *zbuf, double *out, double *neff, double *st) {
-    /* n: visible keys; n_len: the length the temperature sees (len_mode). */
-    oracle_cfg c2 = *cfg;
-    (void)c2;
-    if (n_len != n) {
-        /* The temperature uses n_len; everything else uses the visible count n.
-           Fold the ratio into the logit scale so the modes stay unchanged. */
-        double tau_len = length_temperature(n_len, cfg), tau_vis = length_temperature(n, cfg);
-        c2.s = cfg->s * tau_len / tau_vis;
-        cfg = &c2;
-    }
+                     int64_t n, const oracle_cfg *cfg, const float *u_h, double *zbuf,
+                     double *out, double *neff, double *st) {
     if (mode == 1)
         row_brute(q, ks, n, cfg, u_h, zbuf, out, neff, st);
     else if (mode == 2)
@@ -394,7 +383,6 @@ int oracle_polar_fwd(const oracle_cfg *cfg, const void *q, const void *k, const 
         }
         key_src ks = {k, v, dtype, D, cfg->Hkv, g, 0,
                       ((int64_t)b * T * cfg->Hkv + g) * D, (int64_t)cfg->Hkv * D, NULL, lo};
-        int64_t n_len = cfg->len_mode == 1 ? T : n;
         double *zbuf = (double *)malloc(sizeof(double) * (size_t)(n > block ? n : block) + 8);
         if (!zbuf) { bad = 1; continue; }
 #if ORACLE_MUTANT == 10
@@ -402,7 +390,7 @@ int oracle_polar_fwd(const oracle_cfg *cfg, const void *q, const void *k, const 
 #else
         const float *u_h = u + (int64_t)h * D;
 #endif
-        eval_row(mode, block, theta, qrow, &ks, n, n_len, cfg, u_h, zbuf, out + r * D, neff + r,
+        eval_row(mode, block, theta, qrow, &ks, n, cfg, u_h, zbuf, out + r * D, neff + r,
                  stats ? stats + r * 8 : NULL);
         free(zbuf);
     }
@@ -453,7 +441,7 @@ int oracle_polar_decode(const oracle_cfg *cfg, const void *q, const void *kv_pag
         key_src ks = {kv_pages, kv_pages, dtype, D, cfg->Hkv, g, 1, 0, 0, pt, lo};
         double *zbuf = (double *)malloc(sizeof(double) * (size_t)(n > block ? n : block) + 8);
         if (!zbuf) { bad |= 1; continue; }
-        eval_row(mode, block, theta, qrow, &ks, n, n, cfg, u + (int64_t)h * D, zbuf, out + r * D,
+        eval_row(mode, block, theta, qrow, &ks, n, cfg, u + (int64_t)h * D, zbuf, out + r * D,
                  neff + r, stats ? stats + r * 8 : NULL);
         free(zbuf);
     }
@@ -486,7 +474,7 @@ int oracle_polar_bwd(const oracle_cfg *cfg, const void *q, const void *k, const 
                      int dtype, const float *u, const double *gout, double *dq, double *dk,
                      double *dv, double *du) {
     if (!cfg || cfg->D <= 0 || cfg->D > 256 || cfg->Hkv <= 0 || cfg->Hq % cfg->Hkv != 0 ||
-        cfg->L < 2 || cfg->T < 0 || cfg->B < 0 || !cfg->causal || cfg->len_mode != 0)
+        cfg->L < 2 || cfg->T < 0 || cfg->B < 0 || !cfg->causal)
         return -1;
     const int B = cfg->B, T = cfg->T, Hq = cfg->Hq, Hkv = cfg->Hkv, D = cfg->D;
     const int G = Hq / Hkv;
