@@ -2,7 +2,8 @@
 
 One step = one pass of the whole path on one GPU's batch of synthetic input:
   * causal prefill, B=2, Hq=16, Hkv=4, T=16384, d=64, bf16, length temperature
-    active (the extrapolation workload), through polar_attn_fwd; then
+    active (the extrapolation workload), through polar_attn_fwd_ws (the prefill
+    with its key-moment workspace); then
   * paged GQA decode, 32 sequences with 128K-256K tokens of context in 64-token
     pages behind a shuffled page table, Hq=16, Hkv=4, bf16, through
     polar_attn_decode_paged.
@@ -210,6 +211,23 @@ def prefill_rows_flops(rows, w) -> float:
     return float(4.0 * w.D * np.sum(i + 1))
 
 
+def gdelta_mma_flops(B: int, T: int, H: int) -> float:
+    """bf16 tensor-core flops the memory-channel prefill executes per launch:
+    per 64-token chunk and (sequence, head), 256 m16n8k16 products in the chunk
+    kernel (K K^T and Q K^T) and 1056 in the scan (two slices of 32 value rows,
+    each 320 for U = Ut + (-W) S^T with three hi/lo terms and Q S^T with two,
+    80 for P U with two, 128 for the state update with two); 4096 flops each."""
+    chunks = (T + 63) // 64
+    return float(B) * H * chunks * (256 + 1056) * 4096.0
+
+
+def gdelta_io_bytes(w) -> float:
+    """Compulsory HBM bytes of one memory-channel prefill: q, k, v read and out
+    written (bf16), alpha and beta read (fp32), the state read and written."""
+    tok = w.B * w.T * w.H
+    return float(tok * w.D * 2 * 4 + tok * 4 * 2 + w.B * w.H * w.D * w.D * 4 * 2)
+
+
 def cpu_prefill_inputs(seed=0):
     x = W.prefill_inputs(PREFILL, "cpu", seed=seed)
     return {"q": W.to_host_bits(x["q"]), "k": W.to_host_bits(x["k"]), "v": W.to_host_bits(x["v"]),
@@ -238,10 +256,32 @@ def cpu_baseline(budget_s: float, seed=0) -> dict:
     t0 = time.perf_counter()
     _oracle_prefill_rows(x_host, rows, PREFILL)
     dt = time.perf_counter() - t0
-    return {"value": prefill_rows_flops(rows, PREFILL) / dt / 1e12, "unit": "TFLOP/s",
-            "cores": oracle_threads(), "kind": "oracle",
-            "sample": f"{rows.size} seeded random rows of the T=16384 prefill workload "
-                      f"(fp64 two-pass oracle, {dt:.1f} s)"}
+    res = {"value": prefill_rows_flops(rows, PREFILL) / dt / 1e12, "unit": "TFLOP/s",
+           "cores": oracle_threads(), "kind": "oracle",
+           "sample": f"{rows.size} seeded random rows of the T=16384 prefill workload "
+                     f"(fp64 two-pass oracle, {dt:.1f} s)"}
+    res["decode"] = cpu_decode_baseline(seed)
+    return res
+
+
+def cpu_decode_baseline(seed=0, num_seqs=2) -> dict:
+    """The decode oracle on `num_seqs` seeded sequences drawn from the decode
+    workload's length range (every head of each), in algorithmic KV GB/s."""
+    import oracle
+    w = W.small_decode(num_seqs=num_seqs, min_len=DECODE.min_len, max_len=DECODE.max_len,
+                       Hq=DECODE.Hq, Hkv=DECODE.Hkv, seed=seed + 5)
+    x = W.decode_inputs(w, "cpu")
+    q, kv = W.to_host_bits(x["q"]), W.to_host_bits(x["kv_pages"])
+    pt, sl, u = x["page_table"].numpy(), x["seqlens"].numpy(), x["u"].numpy()
+    prm = oracle.Params(s=w.s, alpha=w.alpha, L=w.L, beta=w.beta)
+    t0 = time.perf_counter()
+    oracle.polar_decode(q, kv, pt, sl, u, prm)
+    dt = time.perf_counter() - t0
+    kv_bytes = float(sl.astype(np.int64).sum()) * KV_BYTES_PER_TOKEN
+    return {"value": kv_bytes / dt / 1e9, "unit": "GB/s", "cores": oracle_threads(),
+            "kind": "oracle",
+            "sample": f"{num_seqs} seeded sequences of {int(sl.min())}-{int(sl.max())} tokens, "
+                      f"all {w.Hq} heads (fp64 oracle, {dt:.1f} s)"}
 
 
 # ------------------------------------------------------------------ GPU arm --
@@ -355,6 +395,29 @@ def run_ours(args):
             raise RuntimeError("device status after the windowed prefill")
         t_win = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in ew) / 1e3, world, dev)
         window_res = (wp, t_win)
+
+    # ---- the 8-argument polar_attn_fwd (no workspace) on the same inputs ----
+    plain_res = None
+    if do_pre:
+        def prefill_plain():
+            pa.fwd(xp["q"], xp["k"], xp["v"], xp["u"], out_p, neff_p, stream=stream,
+                   moments=False, **p)
+
+        for _ in range(Wm):
+            prefill_plain()
+        torch.cuda.synchronize(dev)
+        ep = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
+        barrier(world, dev)
+        torch.cuda.synchronize(dev)
+        for i in range(K):
+            ep[i][0].record(stream)
+            prefill_plain()
+            ep[i][1].record(stream)
+        torch.cuda.synchronize(dev)
+        barrier(world, dev)
+        if pa.get_status() != 0:
+            raise RuntimeError("device status after the 8-argument prefill")
+        plain_res = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in ep) / 1e3, world, dev)
 
     # ---- prefill backward on the train-length workload, timed on its own ----
     bwd_res = None
@@ -590,21 +653,31 @@ def run_ours(args):
             # the chunked kernels execute more (the triangular solve, hi/lo
             # splits) to expose parallelism, partly on the tensor cores.
             gp_tf = wg.flops / gp_launch / 1e12
-            alu_peak = 2 * 148 * 128 * 1.965e9 / 1e12
+            mma_fl = gdelta_mma_flops(wg.B, wg.T, wg.H)
+            mma_tf = mma_fl / gp_launch / 1e12
+            traffic_g = profiled_traffic("gdelta", sha_g)
+            io_bytes = gdelta_io_bytes(wg)
             step_bytes = wst.state_bytes + wst.num_seqs * wst.H * wst.D * (4 * 2) + \
                 wst.num_seqs * wst.H * 8 + wst.num_seqs * 4
             gs_gbs = step_bytes / gs_launch / 1e9
             result["gdelta"] = {
                 "workload": wg.describe(), "ms_per_launch": gp_launch * 1e3,
                 "tokens_per_s": aggregate_throughput(tok * Kg, world, t_gp),
+                "recurrence_tflops": gp_tf,
                 "note": "memory channel prefill (polar_gdelta_prefill: chunk kernel + scan kernel; "
                         "bf16 inputs, products on mma.sync with hi/lo-split fp32 operands), timed "
-                        "separately; not part of value"}
+                        "separately; not part of value.  recurrence_tflops counts only the "
+                        "recurrence's own 6 D^2 flops per token and head"}
             result["roofline_gdelta"] = {
-                "bound": "alu", "kernel": "gd_chunk_mma_kernel+gd_scan_mma_kernel",
-                "achieved": gp_tf, "peak": alu_peak, "unit": "TFLOP/s", "frac": gp_tf / alu_peak,
-                "flops_per_launch": wg.flops, "traffic": profiled_traffic("gdelta", sha_g),
-                "peak_source": "fp32 FMA: 148 SMs x 128 lanes x 2 flops x 1965 MHz (max SM clock)"}
+                "bound": "tensor", "kernel": "gd_chunk_mma_kernel+gd_scan_mma_kernel",
+                "achieved": mma_tf, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": mma_tf / peaks["bf16_tflops"], "flops_per_launch": mma_fl,
+                "traffic": traffic_g, "io_bytes_per_launch": io_bytes,
+                "hbm_frac": (None if traffic_g is None else
+                             traffic_g / gp_launch / 1e9 / peaks["hbm_gbs"]),
+                "hbm_frac_of_io": io_bytes / gp_launch / 1e9 / peaks["hbm_gbs"],
+                "peak_source": f"{peak_src} (burst cuBLAS bf16); flops = the bf16 m16n8k16 "
+                               "products the kernels execute, every hi/lo term counted"}
             result["gdelta_step"] = {
                 "workload": wst.describe(), "ms_per_launch": gs_launch * 1e3,
                 "tokens_per_s": aggregate_throughput(wst.num_seqs * Kg, world, t_gs),
@@ -614,6 +687,15 @@ def run_ours(args):
                 "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": gs_gbs / peaks["hbm_gbs"],
                 "bytes_per_launch": step_bytes, "traffic": profiled_traffic("gdelta_step", sha_g),
                 "peak_source": f"{peak_src} (copy bandwidth)"}
+        if plain_res is not None:
+            pl_launch = plain_res / K
+            pl_tf = PREFILL.flops / pl_launch / 1e12
+            result["prefill_no_workspace"] = {
+                "value": pl_tf, "unit": "TFLOP/s", "ms_per_launch": pl_launch * 1e3,
+                "pct_bf16_peak": 100 * pl_tf / peaks["bf16_tflops"],
+                "note": "polar_attn_fwd(q, k, v, u, params, out, neff_out, stream): the same "
+                        "prefill without the key-moment workspace (null-floor sums formed score "
+                        "by score); timed separately after the step loop; not part of value"}
         if window_res is not None:
             wp, t_win = window_res
             w_launch = t_win / K
@@ -651,14 +733,17 @@ def run_ours(args):
 
 def run_reference(args):
     """The fp64 CPU oracle as it stands, on the host cores, on the same metric
-    and unit: each step is a bounded seeded sample of prefill rows."""
+    and unit: each step is a seeded sample of prefill rows, sized (as the
+    cpu_baseline sample is) to keep every host core busy and the whole run
+    within a few minutes."""
     rank, world, _ = dist_env()
     if rank != 0:
         return None
     x_host = cpu_prefill_inputs(0)
     rng = np.random.default_rng(11)
-    rows_per_step = 8
     total = PREFILL.B * PREFILL.Hq * PREFILL.T
+    budget = min(6.0, 150.0 / max(1, args.steps + args.warmup))  # seconds per step
+    rows_per_step = calibrated_rows(x_host, budget, rng, probe_rows=4 * oracle_threads()).size
     for _ in range(args.warmup):
         _oracle_prefill_rows(x_host, rng.integers(0, total, size=rows_per_step), PREFILL)
     flops = 0.0
@@ -669,16 +754,15 @@ def run_reference(args):
         flops += prefill_rows_flops(rows, PREFILL)
     dt = time.perf_counter() - t0
     v = flops / dt / 1e12
+    sample = (f"{rows_per_step} seeded random rows of the T=16384 prefill per step "
+              f"(fp64 two-pass oracle, {oracle_threads()} threads)")
     return {"impl": "reference", "metric": METRIC, "value": v, "unit": "TFLOP/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic",
-            "config": {"workload": PREFILL.describe(),
-                       "sample": f"{rows_per_step} seeded random rows per step"},
+            "config": {"workload": PREFILL.describe(), "sample": sample},
             "cpu_baseline": {"value": v, "unit": "TFLOP/s", "cores": oracle_threads(),
-                             "kind": "oracle",
-                             "sample": f"{rows_per_step} random rows of the T=16384 prefill "
-                                       "per step"},
+                             "kind": "oracle", "sample": sample},
             "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
 

@@ -107,24 +107,41 @@ void polar_attn_default_params(polar_params_t *p, int B, int T, int Hq, int Hkv,
  *  q         [B, T, Hq,  64] dtype, device
  *  k, v      [B, T, Hkv, 64] dtype, device
  *  u         [Hq, 64] float32, device: the per-head count vectors u_h
+ *  params    shape and method constants (read on the host during the call)
  *  out       [B, T, Hq, 64] dtype, device: content + count
  *  neff_out  [B, Hq, T] float32, device: n_eff per row (may be NULL)
- *  workspace device scratch of at least polar_attn_fwd_workspace_size()
- *            bytes, or NULL (then ws_bytes is ignored).  With it, the raw
- *            logit sums of the null floor over the key tiles left of a query
- *            tile come from key moments (sum k, sum k k^T) that a pre-pass
- *            writes here, instead of from every score: the same quantities,
- *            computed faster.  Contents on entry are ignored; calls that
- *            share a workspace must not overlap.  A non-NULL workspace smaller
- *            than required returns POLAR_ERR_WORKSPACE.
+ *  stream    cudaStream_t the work is ordered on
  *
- * Returns POLAR_OK once the work is enqueued.  B = 0 or T = 0 is a no-op.
+ * Needs no scratch memory: the raw logit sums of the null floor are summed
+ * score by score inside the kernel.  Returns POLAR_OK once the work is
+ * enqueued, or an argument error with nothing launched.  B = 0 or T = 0 is a
+ * no-op.
+ */
+polar_status_t polar_attn_fwd(const void *q, const void *k, const void *v, const float *u,
+                              const polar_params_t *params, void *out, float *neff_out,
+                              void *stream);
+
+/*
+ * polar_attn_fwd with a caller-owned workspace, which makes long prefills
+ * faster (the same rows up to rounding).
+ *
+ *  workspace device scratch of at least polar_attn_fwd_workspace_size()
+ *            bytes, or NULL (then ws_bytes is ignored and the call is
+ *            polar_attn_fwd).  With it, the raw logit sums of the null floor
+ *            over the key tiles left of a query tile come from key moments
+ *            (sum k, sum k k^T) that a pre-pass writes here, instead of from
+ *            every score: the same quantities, computed with less work per
+ *            score (used from 32 query tiles on, without a sliding window).
+ *            Contents on entry are ignored; calls that share a workspace must
+ *            not overlap.  A non-NULL workspace smaller than required returns
+ *            POLAR_ERR_WORKSPACE.
+ * Other arguments as polar_attn_fwd.
  */
 size_t polar_attn_fwd_workspace_size(const polar_params_t *params);
 
-polar_status_t polar_attn_fwd(const void *q, const void *k, const void *v, const float *u,
-                              const polar_params_t *params, void *out, float *neff_out,
-                              void *workspace, size_t ws_bytes, void *stream);
+polar_status_t polar_attn_fwd_ws(const void *q, const void *k, const void *v, const float *u,
+                                 const polar_params_t *params, void *out, float *neff_out,
+                                 void *workspace, size_t ws_bytes, void *stream);
 
 /*
  * Backward of the causal prefill: the gradients of a loss L with respect to
@@ -134,7 +151,7 @@ polar_status_t polar_attn_fwd(const void *q, const void *k, const void *v, const
  * tanh-log magnitude, the gate on max logit - null floor, and the floor's mean
  * and spread.  The max contributes through its first index (a subgradient).
  * The window (params->window) is honoured; the key-moment workspace of
- * polar_attn_fwd plays no part.
+ * polar_attn_fwd_ws plays no part.
  *
  *  q, k, v, u  as polar_attn_fwd (dtype bf16 or fp32)
  *  dout       [B, T, Hq, 64] dtype, device
@@ -155,13 +172,14 @@ polar_status_t polar_attn_bwd(const void *q, const void *k, const void *v, const
                               void *stream);
 
 /* Bytes of device staging that polar_attn_fwd_host needs for this shape
- * (inputs, outputs and the workspace). */
+ * (inputs, outputs and the workspace of polar_attn_fwd_ws). */
 size_t polar_attn_fwd_staging_size(const polar_params_t *params);
 
 /*
  * polar_attn_fwd on host buffers: copies q, k, v, u from host memory (pinned
  * memory gives full copy bandwidth) into `staging` (device memory owned by the
- * caller, at least polar_attn_fwd_staging_size bytes), runs the prefill, copies
+ * caller, at least polar_attn_fwd_staging_size bytes), runs the prefill
+ * (polar_attn_fwd_ws with its workspace in the staging buffer), copies
  * out and n_eff back to host memory, and synchronises `stream`.
  */
 polar_status_t polar_attn_fwd_host(const void *q_h, const void *k_h, const void *v_h,
@@ -266,9 +284,17 @@ polar_status_t polar_attn_decode_paged_host(const void *q_h, const void *kv_page
  *  - A shape whose scratch (polar_attn_decode_workspace_size) exceeds
  *    POLAR_NOALLOC_SCRATCH_BYTES is rejected with POLAR_ERR_WORKSPACE and
  *    nothing is launched.
- *  - The first call on a device looks up the array's device address with that
- *    device current (a synchronous runtime query); make that first call before
- *    any stream capture.
+ *  - The first call on a device sets the device up, with that device current:
+ *    it looks up the array's device address (a synchronous runtime query) and
+ *    loads the library's decode kernels and status word onto the device.
+ *    Under CUDA's lazy module loading (the default) that is when the array's
+ *    POLAR_NOALLOC_SCRATCH_BYTES and the kernels' code take device memory, so
+ *    make this first call before handing the remaining free memory to a pool,
+ *    and before any stream capture.  A call with num_seqs = 0 (and otherwise
+ *    valid arguments) does the set-up and nothing else; later calls take no
+ *    device memory.
+ *  - The addresses are kept for the life of the process: do not use the
+ *    library across a device reset (cudaDeviceReset) on that device.
  *  - Every call on a device shares the one array and leaves its contents
  *    behind.  Nothing in it has to start at zero: each split writes its whole
  *    partial state before the merge reads it.  Calls whose work overlaps on the

@@ -129,6 +129,8 @@ FwdLaunch make_fwd(const void *q, const void *k, const void *v, const float *u,
 
 void count_launches(int n) { g_launches.fetch_add(static_cast<uint64_t>(n)); }
 
+int *device_status_word() { return status_ptr(); }
+
 // One bounded wait on a barrier that no thread or copy ever completes.
 __global__ void selftest_timeout_kernel(int *status) {
     __shared__ __align__(8) uint64_t bar;
@@ -182,7 +184,13 @@ size_t polar_attn_fwd_workspace_size(const polar_params_t *p) {
 
 polar_status_t polar_attn_fwd(const void *q, const void *k, const void *v, const float *u,
                               const polar_params_t *params, void *out, float *neff_out,
-                              void *workspace, size_t ws_bytes, void *stream) {
+                              void *stream) {
+    return polar_attn_fwd_ws(q, k, v, u, params, out, neff_out, nullptr, 0, stream);
+}
+
+polar_status_t polar_attn_fwd_ws(const void *q, const void *k, const void *v, const float *u,
+                                 const polar_params_t *params, void *out, float *neff_out,
+                                 void *workspace, size_t ws_bytes, void *stream) {
     polar_status_t st = check_fwd(params);
     if (st != POLAR_OK) return st;
     if (params->B == 0 || params->T == 0) return POLAR_OK;
@@ -286,9 +294,9 @@ polar_status_t polar_attn_fwd_host(const void *q_h, const void *k_h, const void 
         cudaMemcpyAsync(dv, v_h, kb, cudaMemcpyHostToDevice, s) != cudaSuccess ||
         cudaMemcpyAsync(du, u_h, ub, cudaMemcpyHostToDevice, s) != cudaSuccess)
         return POLAR_ERR_CUDA;
-    st = polar_attn_fwd(dq, dk, dv, reinterpret_cast<float *>(du), p, dout,
-                        neff_h ? reinterpret_cast<float *>(dne) : nullptr,
-                        wsb ? dws : nullptr, wsb, stream);
+    st = polar_attn_fwd_ws(dq, dk, dv, reinterpret_cast<float *>(du), p, dout,
+                           neff_h ? reinterpret_cast<float *>(dne) : nullptr,
+                           wsb ? dws : nullptr, wsb, stream);
     if (st != POLAR_OK) return st;
     if (cudaMemcpyAsync(out_h, dout, qb, cudaMemcpyDeviceToHost, s) != cudaSuccess) return POLAR_ERR_CUDA;
     if (neff_h && cudaMemcpyAsync(neff_h, dne, nb, cudaMemcpyDeviceToHost, s) != cudaSuccess)

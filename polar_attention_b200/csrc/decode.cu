@@ -465,6 +465,26 @@ size_t decode_partials_bytes(int num_seqs, int max_pages, int Hq, int Hkv, int c
     return static_cast<size_t>(num_seqs) * chunk * Hq * max_splits * kPartialFloats * sizeof(float);
 }
 
+cudaError_t decode_preload() {
+    // Querying a kernel's attributes loads its code onto the current device
+    // (under lazy module loading that otherwise happens at its first launch).
+    const void *all[] = {reinterpret_cast<const void *>(decode_split_kernel<1, false>),
+                         reinterpret_cast<const void *>(decode_split_kernel<1, true>),
+                         reinterpret_cast<const void *>(decode_split_kernel<2, false>),
+                         reinterpret_cast<const void *>(decode_split_kernel<2, true>),
+                         reinterpret_cast<const void *>(decode_split_kernel<4, false>),
+                         reinterpret_cast<const void *>(decode_split_kernel<4, true>),
+                         reinterpret_cast<const void *>(decode_split_kernel<8, false>),
+                         reinterpret_cast<const void *>(decode_split_kernel<8, true>),
+                         reinterpret_cast<const void *>(decode_merge_kernel)};
+    for (const void *f : all) {
+        cudaFuncAttributes fa;
+        const cudaError_t e = cudaFuncGetAttributes(&fa, f);
+        if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+}
+
 cudaError_t launch_decode(const DecodeLaunch &a) {
     const int G = a.Hq / a.Hkv;
     const int pps = decode_pages_per_split(a.num_seqs, a.max_pages, a.Hkv);

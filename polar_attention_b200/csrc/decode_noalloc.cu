@@ -19,6 +19,10 @@ void *g_scratch_addr[kMaxDevices] = {nullptr};
 
 // In host code g_noalloc_scratch names a host-side stand-in, not device memory,
 // so the device address is looked up once per device, with that device current.
+// The same first call also makes everything the later calls touch resident on
+// the device: looking the address up loads this file's module (the array with
+// it) under lazy module loading, and the status word and the decode kernels are
+// loaded here too, so that later calls allocate no device memory at all.
 polar_status_t scratch_on_current_device(void **addr) {
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return POLAR_ERR_CUDA;
@@ -26,6 +30,8 @@ polar_status_t scratch_on_current_device(void **addr) {
     if (!g_scratch_addr[dev]) {
         void *p = nullptr;
         if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return POLAR_ERR_CUDA;
+        if (!polar::device_status_word() || polar::decode_preload() != cudaSuccess)
+            return POLAR_ERR_CUDA;
         g_scratch_addr[dev] = p;
     }
     *addr = g_scratch_addr[dev];

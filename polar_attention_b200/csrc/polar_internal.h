@@ -101,6 +101,13 @@ size_t fwd_moments_bytes(int B, int T, int Hkv);
 cudaError_t launch_fwd_moments(const void *k, int B, int T, int Hkv, float *rec,
                                cudaStream_t stream);
 
+// Loads the decode kernels' code onto the current device now rather than at
+// their first launch (lazy module loading).
+cudaError_t decode_preload();
+
+// Device address of the per-device status word on the current device, or null.
+int *device_status_word();
+
 // Decode work split: pages per split and the partial-state bytes it needs.
 int decode_pages_per_split(int num_seqs, int max_pages, int Hkv);
 size_t decode_partials_bytes(int num_seqs, int max_pages, int Hq, int Hkv, int chunk);

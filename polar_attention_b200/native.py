@@ -24,6 +24,7 @@ STATUS = {0: "POLAR_OK", 1: "POLAR_ERR_INVALID_ARG", 2: "POLAR_ERR_UNSUPPORTED",
 
 # Every entry point include/polar_attn.h and include/polar_gdelta.h declare.
 EXPORTS = ["polar_attn_default_params", "polar_attn_fwd_workspace_size", "polar_attn_fwd",
+           "polar_attn_fwd_ws",
            "polar_attn_fwd_staging_size",
            "polar_attn_fwd_host", "polar_attn_decode_workspace_size", "polar_attn_decode_paged",
            "polar_attn_decode_staging_size", "polar_attn_decode_paged_host",
@@ -78,7 +79,8 @@ def lib() -> ctypes.CDLL:
             L.polar_attn_default_params.restype = None
             L.polar_attn_fwd_workspace_size.argtypes = [PP]
             L.polar_attn_fwd_workspace_size.restype = Z
-            L.polar_attn_fwd.argtypes = [P, P, P, P, PP, P, P, P, Z, P]
+            L.polar_attn_fwd.argtypes = [P, P, P, P, PP, P, P, P]
+            L.polar_attn_fwd_ws.argtypes = [P, P, P, P, PP, P, P, P, Z, P]
             L.polar_attn_bwd_workspace_size.argtypes = [PP]
             L.polar_attn_bwd_workspace_size.restype = Z
             L.polar_attn_bwd.argtypes = [P, P, P, P, P, PP, P, P, P, P, P, Z, P]
@@ -106,7 +108,7 @@ def lib() -> ctypes.CDLL:
             L.polar_attn_status_string.argtypes = [I]
             L.polar_attn_status_string.restype = ctypes.c_char_p
             L.polar_attn_launch_count.restype = ctypes.c_uint64
-            for name in ("polar_attn_fwd", "polar_attn_fwd_host", "polar_attn_decode_paged",
+            for name in ("polar_attn_fwd", "polar_attn_fwd_ws", "polar_attn_fwd_host", "polar_attn_decode_paged",
                          "polar_attn_decode_paged_host", "polar_attn_get_status",
                          "polar_attn_decode_paged_noalloc", "polar_attn_selftest_exp2",
                          "polar_attn_decode_paged_chunk", "polar_attn_bwd",
@@ -166,8 +168,9 @@ def fwd(q, k, v, u, out=None, neff=None, workspace=None, *, s=8.0, alpha=0.3, L=
         impl="auto", stream=None, want_neff=True, moments=True, window=0):
     """Causal prefill.  q [B,T,Hq,64], k/v [B,T,Hkv,64] (bf16 or fp32, CUDA,
     contiguous), u [Hq,64] fp32.  Returns (out [B,T,Hq,64], neff [B,Hq,T]).
-    moments=True passes a workspace for the key-moment pre-pass (allocated
-    here when `workspace` is None); moments=False passes none."""
+    moments=True calls polar_attn_fwd_ws with a workspace for the key-moment
+    pre-pass (allocated here when `workspace` is None); moments=False calls
+    polar_attn_fwd, which takes none."""
     B, T, Hq, D = q.shape
     Hkv = k.shape[2]
     for t in (q, k, v, u):
@@ -181,18 +184,18 @@ def fwd(q, k, v, u, out=None, neff=None, workspace=None, *, s=8.0, alpha=0.3, L=
         neff = torch.empty((B, Hq, T), device=q.device, dtype=torch.float32)
     p = make_params(B, T, Hq, Hkv, _dt(q), s, alpha, L, beta, impl, window)
     p.head_dim = D
-    ws_bytes = 0
-    if moments:
-        ws_bytes = int(lib().polar_attn_fwd_workspace_size(ctypes.byref(p)))
-        if workspace is None:
-            workspace = torch.empty(max(ws_bytes, 16), device=q.device, dtype=torch.uint8)
-        else:
-            ws_bytes = workspace.numel() * workspace.element_size()
+    if not moments:
+        _check(lib().polar_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(u), ctypes.byref(p),
+                                    _ptr(out), _ptr(neff), _stream(stream)), "polar_attn_fwd")
+        return out, neff
+    ws_bytes = int(lib().polar_attn_fwd_workspace_size(ctypes.byref(p)))
+    if workspace is None:
+        workspace = torch.empty(max(ws_bytes, 16), device=q.device, dtype=torch.uint8)
     else:
-        workspace = None
-    _check(lib().polar_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(u), ctypes.byref(p), _ptr(out),
-                                _ptr(neff), _ptr(workspace), ws_bytes, _stream(stream)),
-           "polar_attn_fwd")
+        ws_bytes = workspace.numel() * workspace.element_size()
+    _check(lib().polar_attn_fwd_ws(_ptr(q), _ptr(k), _ptr(v), _ptr(u), ctypes.byref(p),
+                                   _ptr(out), _ptr(neff), _ptr(workspace), ws_bytes,
+                                   _stream(stream)), "polar_attn_fwd_ws")
     return out, neff
 
 

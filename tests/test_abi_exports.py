@@ -28,6 +28,25 @@ def test_header_declares_the_boundary():
         assert must in names
 
 
+def _declaration(name):
+    src = ""
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        src += re.sub(r"/\*.*?\*/", "", open(h).read(), flags=re.S)
+    m = re.search(r"\b" + name + r"\s*\(([^)]*)\)\s*;", src)
+    assert m, name
+    return [" ".join(a.split()) for a in m.group(1).split(",")]
+
+
+def test_prefill_entry_point_has_the_eight_argument_signature():
+    """polar_attn_fwd(q, k, v, u, params, out, neff_out, stream): the prefill
+    call with no workspace; the workspace form is polar_attn_fwd_ws."""
+    args = _declaration("polar_attn_fwd")
+    names = [a.replace("*", " ").split()[-1] for a in args]
+    assert names == ["q", "k", "v", "u", "params", "out", "neff_out", "stream"], args
+    ws = [a.replace("*", " ").split()[-1] for a in _declaration("polar_attn_fwd_ws")]
+    assert ws == names[:-1] + ["workspace", "ws_bytes", "stream"], ws
+
+
 def test_library_exports_every_declared_symbol():
     from polar_attention_b200 import native
     if not os.path.exists(native.LIB_PATH):

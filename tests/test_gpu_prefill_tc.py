@@ -154,6 +154,23 @@ def test_extrapolation_T16384_sampled(cuda_ok):
     PT.compare(o, n, ref, grp, PT.OUT_TOL_BF16, what="extrapolation_T16384")
 
 
+def test_extrapolation_T16384_eight_argument_call(cuda_ok):
+    """The same full-size workload through polar_attn_fwd(q, k, v, u, params,
+    out, neff_out, stream), which takes no workspace: sampled rows against the
+    oracle, and every row against the workspace call (n_eff does not depend on
+    how the null-floor sums are formed; out moves only by their rounding)."""
+    w = W.EXTRAP
+    x, out, neff = _run(w, moments=False)
+    rows = PT.sample_rows(w.B, w.Hq, w.T, 600, seed=12)
+    ref = PT.oracle_prefill(w, x, rows)
+    o, n, grp = PT.gpu_rows_prefill(out, neff, rows, w.B, w.T, w.Hq)
+    PT.compare(o, n, ref, grp, PT.OUT_TOL_BF16, what="extrapolation_T16384, 8-argument call")
+    _, out_ws, neff_ws = _run(w, x, moments=True)
+    assert ((neff - neff_ws).abs() / neff_ws).amax() < 1e-6
+    err = (out.float() - out_ws.float()).abs().amax() / out_ws.float().abs().amax()
+    assert err < 2e-3, err
+
+
 def test_long_T65536_sampled(cuda_ok):
     """T=65536 with a 16-key needle per kv head matched by the last 64 queries:
     the needle rows and random rows against the oracle, and the needle rows

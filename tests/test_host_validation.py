@@ -33,7 +33,12 @@ def _params(**kw):
 
 
 def _fwd(lib, p, q=A16, out=A16, ws=None, ws_bytes=0):
-    return lib.polar_attn_fwd(q, A16, A16, A16, ctypes.byref(p), out, None, ws, ws_bytes, None)
+    """polar_attn_fwd_ws; without a workspace also polar_attn_fwd, which must
+    refuse exactly the same arguments."""
+    code = lib.polar_attn_fwd_ws(q, A16, A16, A16, ctypes.byref(p), out, None, ws, ws_bytes, None)
+    if ws is None:
+        assert lib.polar_attn_fwd(q, A16, A16, A16, ctypes.byref(p), out, None, None) == code
+    return code
 
 
 @pytest.mark.parametrize("field,value,code", [
