@@ -165,7 +165,7 @@ class ClockSampler:
         return self
 
     def __exit__(self, *exc):
-        if self.proc is not None:
+        if self.proc is not None and self.proc.returncode is None:
             self.proc.terminate()
             try:
                 self.out, _ = self.proc.communicate(timeout=5)
@@ -264,7 +264,7 @@ def cpu_baseline(budget_s: float, seed=0) -> dict:
     return res
 
 
-def cpu_decode_baseline(seed=0, num_seqs=2) -> dict:
+def cpu_decode_baseline(seed=0, num_seqs=4) -> dict:
     """The decode oracle on `num_seqs` seeded sequences drawn from the decode
     workload's length range (every head of each), in algorithmic KV GB/s."""
     import oracle
@@ -347,22 +347,26 @@ def run_ours(args):
     if st != 0:
         raise RuntimeError(f"device status {st} after warm-up")
 
-    with ClockSampler([dev.index]) as clk:
-        time.sleep(0.3)  # let the sampler start before the timed region
-        barrier(world, dev)
-        torch.cuda.synchronize(dev)
-        n0 = pa.launch_count()
-        outer[0].record(stream)
-        for i in range(K):
-            ev[i][0].record(stream)
-            prefill()
-            ev[i][1].record(stream)
-            decode()
-            ev[i][2].record(stream)
-        outer[1].record(stream)
-        torch.cuda.synchronize(dev)
-        launches = pa.launch_count() - n0
-        barrier(world, dev)
+    # The sampler runs through every timed leg below (the step loop alone is
+    # shorter than its sampling interval at small K).
+    clk = ClockSampler([dev.index]).__enter__()
+    import atexit
+    atexit.register(clk.__exit__, None, None, None)  # stop the sampler on any exit path
+    time.sleep(0.3)  # let the sampler start before the timed region
+    barrier(world, dev)
+    torch.cuda.synchronize(dev)
+    n0 = pa.launch_count()
+    outer[0].record(stream)
+    for i in range(K):
+        ev[i][0].record(stream)
+        prefill()
+        ev[i][1].record(stream)
+        decode()
+        ev[i][2].record(stream)
+    outer[1].record(stream)
+    torch.cuda.synchronize(dev)
+    launches = pa.launch_count() - n0
+    barrier(world, dev)
     st = pa.get_status()
     if st != 0:
         raise RuntimeError(f"device status {st} after timing")
@@ -534,6 +538,7 @@ def run_ours(args):
             raise RuntimeError("device status after the multi-token decode")
         t_chunk = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in ec) / 1e3, world, dev)
         chunk_res = (C, t_chunk)
+    clk.__exit__(None, None, None)
     t_all = outer[0].elapsed_time(outer[1]) / 1e3
     t_pre_max = max_over_ranks(t_pre, world, dev)
     t_dec_max = max_over_ranks(t_dec, world, dev)

@@ -156,9 +156,11 @@ def test_extrapolation_T16384_sampled(cuda_ok):
 
 def test_extrapolation_T16384_eight_argument_call(cuda_ok):
     """The same full-size workload through polar_attn_fwd(q, k, v, u, params,
-    out, neff_out, stream), which takes no workspace: sampled rows against the
-    oracle, and every row against the workspace call (n_eff does not depend on
-    how the null-floor sums are formed; out moves only by their rounding)."""
+    out, neff_out, stream), which takes no workspace, and through
+    polar_attn_fwd_ws: both against the oracle on the same sampled rows.  The
+    two calls form the null floor's raw sums in different fp32 orders (score
+    by score, or from key moments), so out may differ by that rounding; n_eff
+    does not depend on those sums and must agree."""
     w = W.EXTRAP
     x, out, neff = _run(w, moments=False)
     rows = PT.sample_rows(w.B, w.Hq, w.T, 600, seed=12)
@@ -166,9 +168,9 @@ def test_extrapolation_T16384_eight_argument_call(cuda_ok):
     o, n, grp = PT.gpu_rows_prefill(out, neff, rows, w.B, w.T, w.Hq)
     PT.compare(o, n, ref, grp, PT.OUT_TOL_BF16, what="extrapolation_T16384, 8-argument call")
     _, out_ws, neff_ws = _run(w, x, moments=True)
+    o, n, grp = PT.gpu_rows_prefill(out_ws, neff_ws, rows, w.B, w.T, w.Hq)
+    PT.compare(o, n, ref, grp, PT.OUT_TOL_BF16, what="extrapolation_T16384, workspace call")
     assert ((neff - neff_ws).abs() / neff_ws).amax() < 1e-6
-    err = (out.float() - out_ws.float()).abs().amax() / out_ws.float().abs().amax()
-    assert err < 2e-3, err
 
 
 def test_long_T65536_sampled(cuda_ok):
