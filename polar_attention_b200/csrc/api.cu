@@ -242,12 +242,14 @@ polar_status_t polar_attn_bwd(const void *q, const void *k, const void *v, const
         !aligned16(dq) || !aligned16(dk) || !aligned16(dv) || !aligned16(workspace))
         return POLAR_ERR_INVALID_ARG;
     if (ws_bytes < bwd_workspace_bytes(p->B, p->T, p->Hq)) return POLAR_ERR_WORKSPACE;
+    int *status = status_ptr();
+    if (!status) return POLAR_ERR_CUDA;
     BwdLaunch a;
     a.q = q; a.k = k; a.v = v; a.dout = dout; a.u = u;
     a.dq = dq; a.dk = dk; a.dv = dv; a.du = du;
     a.B = p->B; a.T = p->T; a.Hq = p->Hq; a.Hkv = p->Hkv; a.dtype = p->dtype;
     a.s = p->logit_scale; a.alpha = p->alpha; a.beta = p->beta; a.L = p->L_train;
-    a.window = p->window; a.workspace = workspace; a.stream = s;
+    a.window = p->window; a.workspace = workspace; a.status = status; a.stream = s;
     return from_cuda(launch_bwd(a));
 }
 

@@ -17,9 +17,10 @@
 //   dS_j    = c dz_j;  dq += dS_j k_j;  dk_j += dS_j q;  dv_j += w_j dA.
 // (w, l, l2 and A may share any reference: content and n_eff are scale-free.)
 //
-// Four launches.  For fp32 inputs they run on the CUDA cores in fp32; for bf16
-// inputs passes 1-3 run their contractions on the tensor cores (mma.sync,
-// below):
+// Four launches.  For fp32 inputs they run on the CUDA cores in fp32 (below);
+// for bf16 inputs pass 1 runs its contractions on mma.sync tensor-core tiles
+// (bwd_rows_mma_kernel) and passes 2-3 are the tcgen05/TMEM kernels of
+// bwd_tc.cu, which read the rows pass's compact coefficient records:
 //  1. rows: one thread per query row recomputes the row's forward state
 //     (streaming, as the CUDA-core prefill does, plus the first argmax) and
 //     writes the row's coefficients: dA, the reference and scales, dl, dl2,
@@ -62,10 +63,11 @@ constexpr int kRecWords = 80;
 
 struct BwdArgs {
     const float *u;
-    float *rec;
+    float *rec;      // fp32 inputs: [B][Hq][T][kRecWords]
     float *du_part;  // [B * row blocks][Hq][64]: per-block sums of gate * T * g
-    __nv_bfloat16 *dab;  // [B][Hq][T][64]: dA rounded to bf16 once (bf16 inputs only)
-    int B, T, Hq, Hkv, window;
+    float *coef;     // bf16 inputs: [B][Hq][Tpad][kBwdCoefWords] (BwdCoef layout)
+    __nv_bfloat16 *dab;  // bf16 inputs: [B][Hq][Tpad][64], dA rounded to bf16
+    int B, T, Tpad, Hq, Hkv, window;
     float s, alpha, L, beta, inv_ln_L;
 };
 
@@ -566,7 +568,8 @@ bwd_rows_mma_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__
 #pragma unroll
     for (int nt = 0; nt < 8; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
     const uint32_t ks_addr = smem_u32(&Ks[0][0]), vs_addr = smem_u32(&Vs[0][0]);
-    const int kend = min(Tlen, row0 + 64);
+    // A block past the end only pads the records to a multiple of 128 rows.
+    const int kend = row0 < Tlen ? min(Tlen, row0 + 64) : 0;
     const int kbeg = a.window > 0 ? max(0, row0 - a.window + 1) / 64 * 64 : 0;
     for (int j0 = kbeg; j0 < kend; j0 += 64) {
         __syncthreads();
@@ -695,22 +698,30 @@ bwd_rows_mma_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__
             dupart[nt][0] = fmaf(gt, gr[nt][0], dupart[nt][0]);
             dupart[nt][1] = fmaf(gt, gr[nt][1], dupart[nt][1]);
         }
-        if (!live) continue;
-        float *rec = a.rec + ((static_cast<size_t>(b) * a.Hq + h) * Tlen + i) * kRecWords;
+        // dA rounded to bf16 and the row's compact coefficient record (rows past
+        // the end: zero dA, and cl2 = c = 0 with nref = -inf, so that their
+        // weights and dS vanish in the later passes without masks).
+        const size_t rrow = (static_cast<size_t>(b) * a.Hq + h) * a.Tpad + i;
 #pragma unroll
         for (int nt = 0; nt < 8; ++nt) {
             const int d = 8 * nt + 2 * tq;
             const float o0 = acc[nt][2 * hr] * inv_an, o1 = acc[nt][2 * hr + 1] * inv_an;
-            const float da0 = (gr[nt][0] - o0 * cg) * inv_an, da1 = (gr[nt][1] - o1 * cg) * inv_an;
-            *reinterpret_cast<float2 *>(rec + kRecDA + d) = make_float2(da0, da1);
-            *reinterpret_cast<uint32_t *>(
-                a.dab + ((static_cast<size_t>(b) * a.Hq + h) * Tlen + i) * kHeadDim + d) = pk2(da0, da1);
+            const float da0 = live ? (gr[nt][0] - o0 * cg) * inv_an : 0.f;
+            const float da1 = live ? (gr[nt][1] - o1 * cg) * inv_an : 0.f;
+            *reinterpret_cast<uint32_t *>(a.dab + rrow * kHeadDim + d) = pk2(da0, da1);
         }
         if (tq == 0) {
-            *reinterpret_cast<float4 *>(rec + 64) = make_float4(m_ref[hr], cl2[hr], c, dl);
-            *reinterpret_cast<float4 *>(rec + 68) = make_float4(dl2, cmu, csS, dm);
-            *reinterpret_cast<float4 *>(rec + kRecJmax) =
-                make_float4(__int_as_float(jmax[hr]), __int_as_float(lo[hr]), gt, 0.0f);
+            float4 *cr = reinterpret_cast<float4 *>(a.coef + rrow * kBwdCoefWords);
+            if (live) {
+                cr[0] = make_float4(cl2[hr], -m_ref[hr], c, c * dl);
+                cr[1] = make_float4(2.0f * c * dl2, c * csS, c * cmu, c * dm);
+                cr[2] = make_float4(__int_as_float(jmax[hr]), __int_as_float(lo[hr]), gt, 0.f);
+            } else {
+                cr[0] = make_float4(0.f, -INFINITY, 0.f, 0.f);
+                cr[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+                cr[2] = make_float4(__int_as_float(-1), __int_as_float(0), 0.f, 0.f);
+            }
+            cr[3] = make_float4(0.f, 0.f, 0.f, 0.f);
         }
     }
     // du: sum over the warp's 16 rows (lanes of equal tq), then over the warps.
@@ -732,172 +743,6 @@ bwd_rows_mma_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__
     }
 }
 
-// dq for bf16 inputs: a warp owns 16 query rows; keys stream in blocks of 64.
-// Three CTAs per SM (a small register spill) measured faster than two.
-__global__ void __launch_bounds__(128, 3)
-bwd_dq_mma_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
-                  const __nv_bfloat16 *__restrict__ v, float *__restrict__ dq, const BwdArgs a) {
-    __shared__ __align__(16) __nv_bfloat16 Ks[64][kPitch];
-    __shared__ __align__(16) __nv_bfloat16 Vs[64][kPitch];
-    const int Tlen = a.T, G = a.Hq / a.Hkv;
-    const int row0 = blockIdx.x * 64, h = blockIdx.y, b = blockIdx.z, g = h / G;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, gq = lane >> 2, tq = lane & 3;
-    const int r0 = row0 + 16 * warp;
-    const size_t qstride = static_cast<size_t>(a.Hq) * kHeadDim;
-    const size_t kstride = static_cast<size_t>(a.Hkv) * kHeadDim;
-    uint32_t qa[4][4], da[4][4];
-    load_a_rows(q + (static_cast<size_t>(b) * Tlen * a.Hq + h) * kHeadDim, qstride, r0, Tlen, qa);
-    // dA rows from the records, rounded to bf16.
-    RowCoef cf[2];
-    int rowi[2];
-#pragma unroll
-    for (int hr = 0; hr < 2; ++hr) {
-        const int r = r0 + gq + 8 * hr;
-        rowi[hr] = r;
-        const float *rp = a.rec + ((static_cast<size_t>(b) * a.Hq + h) * Tlen + (r < Tlen ? r : 0)) * kRecWords;
-#pragma unroll
-        for (int ks = 0; ks < 4; ++ks) {
-            const float2 x0 = *reinterpret_cast<const float2 *>(rp + 16 * ks + 2 * tq);
-            const float2 x1 = *reinterpret_cast<const float2 *>(rp + 16 * ks + 8 + 2 * tq);
-            da[ks][hr] = r < Tlen ? pk2(x0.x, x0.y) : 0u;
-            da[ks][2 + hr] = r < Tlen ? pk2(x1.x, x1.y) : 0u;
-        }
-        cf[hr] = load_coef(rp);
-    }
-    float acc[8][4];
-#pragma unroll
-    for (int nt = 0; nt < 8; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
-    const uint32_t ks_addr = smem_u32(&Ks[0][0]), vs_addr = smem_u32(&Vs[0][0]);
-    const int kend = min(Tlen, row0 + 64);
-    const int kbeg = a.window > 0 ? max(0, row0 - a.window + 1) / 64 * 64 : 0;
-    for (int j0 = kbeg; j0 < kend; j0 += 64) {
-        __syncthreads();
-        stage_rows(Ks, k + ((static_cast<size_t>(b) * Tlen + j0) * a.Hkv + g) * kHeadDim, kstride, Tlen - j0);
-        stage_rows(Vs, v + ((static_cast<size_t>(b) * Tlen + j0) * a.Hkv + g) * kHeadDim, kstride, Tlen - j0);
-        __syncthreads();
-        float sc[8][4], av[8][4];
-        rows_times_tile(qa, ks_addr, sc);
-        rows_times_tile(da, vs_addr, av);
-        uint32_t pa[4][4];
-#pragma unroll
-        for (int nt = 0; nt < 8; ++nt) {
-            float ds[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int hr = e >> 1, i = rowi[hr], j = j0 + 8 * nt + 2 * tq + (e & 1);
-                const bool vis = i < Tlen && j < Tlen && j <= i && j >= cf[hr].lo;
-                float w;
-                const float x = pair_ds(cf[hr], sc[nt][e], av[nt][e], j, w);
-                ds[e] = vis ? x : 0.f;
-            }
-            pa[nt >> 1][(nt & 1) * 2] = pk2(ds[0], ds[1]);
-            pa[nt >> 1][(nt & 1) * 2 + 1] = pk2(ds[2], ds[3]);
-        }
-        frag_times_tile(pa, ks_addr, acc);
-    }
-#pragma unroll
-    for (int hr = 0; hr < 2; ++hr) {
-        const int r = rowi[hr];
-        if (r >= Tlen) continue;
-        float *dst = dq + ((static_cast<size_t>(b) * Tlen + r) * a.Hq + h) * kHeadDim;
-#pragma unroll
-        for (int nt = 0; nt < 8; ++nt)
-            *reinterpret_cast<float2 *>(dst + 8 * nt + 2 * tq) = make_float2(acc[nt][2 * hr], acc[nt][2 * hr + 1]);
-    }
-}
-
-// dk, dv for bf16 inputs: a warp owns 16 keys; the rows that see them stream
-// in blocks of 64, for every query head of the group.  Three CTAs per SM (a
-// small register spill) measured faster than two without one.
-__global__ void __launch_bounds__(128, 3)
-bwd_dkdv_mma_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
-                    const __nv_bfloat16 *__restrict__ v, float *__restrict__ dk,
-                    float *__restrict__ dv, const BwdArgs a) {
-    __shared__ __align__(16) __nv_bfloat16 Qs[64][kPitch];
-    __shared__ __align__(16) __nv_bfloat16 DAs[64][kPitch];
-    __shared__ __align__(16) float Cs[64][12];  // per staged row: ref cl2 c dl dl2 cmu csS dm jmax lo valid
-    const int Tlen = a.T, G = a.Hq / a.Hkv;
-    const int key0 = blockIdx.x * 64, g = blockIdx.y, b = blockIdx.z;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, gq = lane >> 2, tq = lane & 3;
-    const int k0 = key0 + 16 * warp;
-    const size_t kstride = static_cast<size_t>(a.Hkv) * kHeadDim;
-    uint32_t ka[4][4], va[4][4];
-    load_a_rows(k + (static_cast<size_t>(b) * Tlen * a.Hkv + g) * kHeadDim, kstride, k0, Tlen, ka);
-    load_a_rows(v + (static_cast<size_t>(b) * Tlen * a.Hkv + g) * kHeadDim, kstride, k0, Tlen, va);
-    float dka[8][4], dva[8][4];
-#pragma unroll
-    for (int nt = 0; nt < 8; ++nt)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) dka[nt][e] = dva[nt][e] = 0.f;
-    const uint32_t qs_addr = smem_u32(&Qs[0][0]), da_addr = smem_u32(&DAs[0][0]);
-    const int iend = a.window > 0 ? min(Tlen, key0 + 63 + a.window) : Tlen;
-    for (int hh = 0; hh < G; ++hh) {
-        const int h = g * G + hh;
-        const size_t qstride = static_cast<size_t>(a.Hq) * kHeadDim;
-        for (int i0 = key0; i0 < iend; i0 += 64) {
-            __syncthreads();
-            stage_rows(Qs, q + ((static_cast<size_t>(b) * Tlen + i0) * a.Hq + h) * kHeadDim, qstride, Tlen - i0);
-            stage_rows(DAs, a.dab + ((static_cast<size_t>(b) * a.Hq + h) * Tlen + i0) * kHeadDim,
-                       kHeadDim, Tlen - i0);
-            for (int e = threadIdx.x; e < 64 * 11; e += 128) {
-                const int r = e / 11, c = e % 11, i = i0 + r;
-                float val = 0.f;
-                if (i < Tlen) {
-                    const float *rp = a.rec + ((static_cast<size_t>(b) * a.Hq + h) * Tlen + i) * kRecWords;
-                    val = c < 10 ? rp[kRecRef + c] : 1.f;
-                } else if (c == 9) {
-                    val = __int_as_float(0x7fffffff);  // lo past every key: the row sees nothing
-                }
-                Cs[r][c] = val;
-            }
-            __syncthreads();
-            float st[8][4], at[8][4];
-            rows_times_tile(ka, qs_addr, st);  // S^T: keys x rows
-            rows_times_tile(va, da_addr, at);  // <v_j, dA_i>
-            uint32_t ps[4][4], pw[4][4];
-#pragma unroll
-            for (int nt = 0; nt < 8; ++nt) {
-                float ds[4], ws[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int rr = 8 * nt + 2 * tq + (e & 1), i = i0 + rr;
-                    const int j = k0 + gq + 8 * (e >> 1);
-                    const float4 c0 = *reinterpret_cast<const float4 *>(&Cs[rr][0]);
-                    const float4 c1 = *reinterpret_cast<const float4 *>(&Cs[rr][4]);
-                    const float4 c2 = *reinterpret_cast<const float4 *>(&Cs[rr][8]);
-                    RowCoef cf;
-                    cf.ref = c0.x; cf.cl2 = c0.y; cf.c = c0.z; cf.dl = c0.w;
-                    cf.dl2 = c1.x; cf.cmu = c1.y; cf.csS = c1.z; cf.dm = c1.w;
-                    cf.jmax = __float_as_int(c2.x);
-                    cf.lo = __float_as_int(c2.y);
-                    const bool vis = i < Tlen && j < Tlen && j <= i && j >= cf.lo;
-                    float w;
-                    const float x = pair_ds(cf, st[nt][e], at[nt][e], j, w);
-                    ds[e] = vis ? x : 0.f;
-                    ws[e] = vis ? w : 0.f;
-                }
-                ps[nt >> 1][(nt & 1) * 2] = pk2(ds[0], ds[1]);
-                ps[nt >> 1][(nt & 1) * 2 + 1] = pk2(ds[2], ds[3]);
-                pw[nt >> 1][(nt & 1) * 2] = pk2(ws[0], ws[1]);
-                pw[nt >> 1][(nt & 1) * 2 + 1] = pk2(ws[2], ws[3]);
-            }
-            frag_times_tile(ps, qs_addr, dka);  // dK += dS^T Q
-            frag_times_tile(pw, da_addr, dva);  // dV += W^T dA
-        }
-    }
-#pragma unroll
-    for (int hr = 0; hr < 2; ++hr) {
-        const int j = k0 + gq + 8 * hr;
-        if (j >= Tlen) continue;
-        const size_t off = ((static_cast<size_t>(b) * Tlen + j) * a.Hkv + g) * kHeadDim;
-#pragma unroll
-        for (int nt = 0; nt < 8; ++nt) {
-            *reinterpret_cast<float2 *>(dk + off + 8 * nt + 2 * tq) = make_float2(dka[nt][2 * hr], dka[nt][2 * hr + 1]);
-            *reinterpret_cast<float2 *>(dv + off + 8 * nt + 2 * tq) = make_float2(dva[nt][2 * hr], dva[nt][2 * hr + 1]);
-        }
-    }
-}
-
 // -------------------------------------------------------------------- du ---
 // du_h = sum over the row blocks of their partial sums (fixed order).
 __global__ void __launch_bounds__(kHeadDim)
@@ -914,11 +759,15 @@ cudaError_t launch_all(const BwdLaunch &l, const BwdArgs &a) {
             *v = static_cast<const T *>(l.v), *go = static_cast<const T *>(l.dout);
     int nparts;
     if constexpr (std::is_same<T, __nv_bfloat16>::value) {
-        nparts = a.B * ((a.T + 63) / 64);
-        bwd_rows_mma_kernel<<<dim3((a.T + 63) / 64, a.Hq, a.B), 128, 0, l.stream>>>(q, k, v, go, a);
-        bwd_dkdv_mma_kernel<<<dim3((a.T + 63) / 64, a.Hkv, a.B), 128, 0, l.stream>>>(
-            q, k, v, l.dk, l.dv, a);
-        bwd_dq_mma_kernel<<<dim3((a.T + 63) / 64, a.Hq, a.B), 128, 0, l.stream>>>(q, k, v, l.dq, a);
+        nparts = a.B * (a.Tpad / 64);
+        bwd_rows_mma_kernel<<<dim3(a.Tpad / 64, a.Hq, a.B), 128, 0, l.stream>>>(q, k, v, go, a);
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+        e = launch_bwd_tc(l, a.coef, a.dab);
+        if (e != cudaSuccess) return e;
+        bwd_du_kernel<<<a.Hq, kHeadDim, 0, l.stream>>>(l.du, a, nparts);
+        count_launches(2);
+        return cudaGetLastError();
     } else {
         nparts = a.B * ((a.T + kRowsB0 - 1) / kRowsB0);
         bwd_rows_kernel<T><<<dim3((a.T + kRowsB0 - 1) / kRowsB0, a.Hq, a.B), kRowsB0, 0, l.stream>>>(
@@ -935,22 +784,38 @@ cudaError_t launch_all(const BwdLaunch &l, const BwdArgs &a) {
 
 }  // namespace
 
+// fp32 inputs: the 80-word records and the per-128-row du partials.  bf16
+// inputs: the compact records and dA as bf16, both over T rounded up to 128
+// rows, and the per-64-row du partials.  The workspace holds either layout.
 size_t bwd_workspace_bytes(int B, int T, int Hq) {
-    const size_t rec = static_cast<size_t>(B) * Hq * T * kRecWords * sizeof(float);
-    const size_t part =  // per 64-row block (the bf16 rows pass; the fp32 one uses 128-row blocks)
-        static_cast<size_t>(B) * ((T + 63) / 64) * Hq * kHeadDim * sizeof(float);
-    const size_t dab = static_cast<size_t>(B) * Hq * T * kHeadDim * sizeof(__nv_bfloat16);
-    return rec + part + dab;
+    const size_t Tpad = (static_cast<size_t>(T) + 127) / 128 * 128;
+    const size_t fp32 = static_cast<size_t>(B) * Hq * T * kRecWords * sizeof(float) +
+                        static_cast<size_t>(B) * ((T + kRowsB0 - 1) / kRowsB0) * Hq * kHeadDim *
+                            sizeof(float);
+    const size_t bf16 = static_cast<size_t>(B) * Hq * Tpad * kBwdCoefWords * sizeof(float) +
+                        static_cast<size_t>(B) * Hq * Tpad * kHeadDim * sizeof(__nv_bfloat16) +
+                        static_cast<size_t>(B) * (Tpad / 64) * Hq * kHeadDim * sizeof(float);
+    return fp32 > bf16 ? fp32 : bf16;
 }
 
 cudaError_t launch_bwd(const BwdLaunch &l) {
     BwdArgs a;
     a.u = l.u;
-    a.rec = static_cast<float *>(l.workspace);
-    a.du_part = a.rec + static_cast<size_t>(l.B) * l.Hq * l.T * kRecWords;
-    a.dab = reinterpret_cast<__nv_bfloat16 *>(
-        a.du_part + static_cast<size_t>(l.B) * ((l.T + 63) / 64) * l.Hq * kHeadDim);
     a.B = l.B; a.T = l.T; a.Hq = l.Hq; a.Hkv = l.Hkv; a.window = l.window;
+    a.Tpad = (l.T + 127) / 128 * 128;
+    float *ws = static_cast<float *>(l.workspace);
+    if (l.dtype == POLAR_FP32) {
+        a.rec = ws;
+        a.du_part = a.rec + static_cast<size_t>(l.B) * l.Hq * l.T * kRecWords;
+        a.coef = nullptr;
+        a.dab = nullptr;
+    } else {
+        a.rec = nullptr;
+        a.coef = ws;
+        a.dab = reinterpret_cast<__nv_bfloat16 *>(
+            a.coef + static_cast<size_t>(l.B) * l.Hq * a.Tpad * kBwdCoefWords);
+        a.du_part = reinterpret_cast<float *>(a.dab + static_cast<size_t>(l.B) * l.Hq * a.Tpad * kHeadDim);
+    }
     a.s = l.s; a.alpha = l.alpha; a.L = static_cast<float>(l.L); a.beta = l.beta;
     a.inv_ln_L = 1.0f / logf(static_cast<float>(l.L));
     if (l.B == 0 || l.T == 0) return cudaSuccess;

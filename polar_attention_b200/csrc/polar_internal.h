@@ -54,6 +54,7 @@ struct BwdLaunch {
     int L;
     int window;
     void *workspace;               // bwd_workspace_bytes
+    int *status;                   // device status word
     cudaStream_t stream;
 };
 
@@ -81,12 +82,27 @@ struct GdeltaStepLaunch {          // one decode token per sequence, in place
     cudaStream_t stream;
 };
 
+// Per-row coefficient record of the backward's bf16 path (fp32 words), written
+// by the rows pass for every row of the sequence padded to a multiple of 128
+// (rows past the end carry cl2 = c = 0 and nref = -inf, which give zero weights
+// and zero dS without masks), read by the tensor-core dK/dV and dQ passes:
+//   w  = 2^(cl2 S + nref)
+//   dS = w (c <dA, v> + e1 + e2 w) + e3 S + e4   (+ cdm at the row's first argmax)
+enum BwdCoef {
+    kBcCl2 = 0, kBcNref = 1, kBcC = 2, kBcE1 = 3, kBcE2 = 4, kBcE3 = 5, kBcE4 = 6, kBcCdm = 7,
+    kBcJmax = 8, kBcLo = 9, kBcGT = 10, kBwdCoefWords = 16
+};
+
 // Launchers return cudaSuccess or the launch error.
 cudaError_t launch_fwd_simt(const FwdLaunch &a);
 cudaError_t launch_fwd_tc(const FwdLaunch &a);
 cudaError_t launch_decode(const DecodeLaunch &a);
 cudaError_t launch_bwd(const BwdLaunch &a);
 size_t bwd_workspace_bytes(int B, int T, int Hq);
+// The tensor-core dK/dV and dQ passes of the bf16 backward, given the rows
+// pass's coefficient records coef [B][Hq][Tpad][kBwdCoefWords] and dA rounded
+// to bf16, dab [B][Hq][Tpad][64] (Tpad = T rounded up to 128).
+cudaError_t launch_bwd_tc(const BwdLaunch &l, const float *coef, const void *dab);
 cudaError_t launch_gdelta_prefill(const GdeltaLaunch &a);
 cudaError_t launch_gdelta_step(const GdeltaStepLaunch &a);
 size_t gdelta_workspace_bytes(int B, int T, int H);

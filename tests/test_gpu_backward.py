@@ -51,6 +51,7 @@ def _check(name, got, ref, tol, floor):
     for g, r in pairs:
         scale = max(np.max(np.abs(r)), floor)
         worst = max(worst, np.max(np.abs(g - r)) / scale)
+    print(f"{name}: normwise error {worst:.3e} (tol {tol})")
     assert worst <= tol, f"{name}: normwise error {worst:.3e} > {tol}"
     return worst
 
@@ -85,6 +86,27 @@ def test_medium_temperature_active(cuda_ok):
     x = W.prefill_inputs(w, "cpu")
     x["u"] = x["u"] * 25.0
     _compare(w, x, seed=5)
+
+
+def test_multi_tile_gqa4_ragged(cuda_ok):
+    """Twelve query and key tiles with a ragged last one (T = 1500), four query
+    heads per kv head: every (key tile, query tile) pair of the tensor-core
+    passes, the diagonal tiles and the padded rows past the end."""
+    w = W.small_prefill(B=2, T=1500, Hq=8, Hkv=2, dtype="bf16", seed=15, plant="frac",
+                        plant_frac=0.01, L=512)
+    x = W.prefill_inputs(w, "cpu")
+    x["u"] = x["u"] * 25.0
+    _compare(w, x, seed=7)
+
+
+def test_window_multi_tile(cuda_ok):
+    """A sliding window of 200 keys over 900 rows: key tiles whose rows reach
+    past the window's edge, and query tiles that start after it."""
+    w = W.small_prefill(B=1, T=900, Hq=4, Hkv=2, dtype="bf16", seed=16, plant="frac",
+                        plant_frac=0.01, L=64, window=200)
+    x = W.prefill_inputs(w, "cpu")
+    x["u"] = x["u"] * 25.0
+    _compare(w, x, seed=8)
 
 
 def test_deterministic(cuda_ok):
