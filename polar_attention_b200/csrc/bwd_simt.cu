@@ -744,6 +744,21 @@ bwd_rows_mma_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__
 }
 
 // -------------------------------------------------------------------- du ---
+// du partial of one 64-row block per (block, head, batch): the sum over its
+// rows of gate*T (from the coefficient records) times the upstream gradient.
+// Used after the tensor-core rows pass, which writes no du partials.
+__global__ void __launch_bounds__(kHeadDim)
+bwd_du_part_kernel(const __nv_bfloat16 *__restrict__ gout, const BwdArgs a) {
+    const int blk = blockIdx.x, h = blockIdx.y, b = blockIdx.z, d = threadIdx.x;
+    const int r0 = blk * 64, r1 = min(r0 + 64, a.T);
+    float s = 0.0f;
+    for (int r = r0; r < r1; ++r) {
+        const float gt = a.coef[((static_cast<size_t>(b) * a.Hq + h) * a.Tpad + r) * kBwdCoefWords + kBcGT];
+        s = fmaf(gt, __bfloat162float(gout[((static_cast<size_t>(b) * a.T + r) * a.Hq + h) * kHeadDim + d]), s);
+    }
+    a.du_part[((static_cast<size_t>(b) * gridDim.x + blk) * a.Hq + h) * kHeadDim + d] = s;
+}
+
 // du_h = sum over the row blocks of their partial sums (fixed order).
 __global__ void __launch_bounds__(kHeadDim)
 bwd_du_kernel(float *__restrict__ du, const BwdArgs a, int nparts) {
@@ -759,14 +774,26 @@ cudaError_t launch_all(const BwdLaunch &l, const BwdArgs &a) {
             *v = static_cast<const T *>(l.v), *go = static_cast<const T *>(l.dout);
     int nparts;
     if constexpr (std::is_same<T, __nv_bfloat16>::value) {
+        // Rows pass: the forward's tcgen05 sweep where it applies, else the
+        // mma.sync kernel (which also writes the du partials).
         nparts = a.B * (a.Tpad / 64);
-        bwd_rows_mma_kernel<<<dim3(a.Tpad / 64, a.Hq, a.B), 128, 0, l.stream>>>(q, k, v, go, a);
-        cudaError_t e = cudaGetLastError();
+        int launched = 0;
+        cudaError_t e = launch_bwd_rows_tc(l, a.coef, a.dab, a.Tpad);
+        if (e == cudaSuccess) {
+            bwd_du_part_kernel<<<dim3(a.Tpad / 64, a.Hq, a.B), kHeadDim, 0, l.stream>>>(go, a);
+            launched = 1;
+        } else if (e == cudaErrorNotSupported) {
+            bwd_rows_mma_kernel<<<dim3(a.Tpad / 64, a.Hq, a.B), 128, 0, l.stream>>>(q, k, v, go, a);
+            launched = 1;
+        } else {
+            return e;
+        }
+        e = cudaGetLastError();
         if (e != cudaSuccess) return e;
         e = launch_bwd_tc(l, a.coef, a.dab);
         if (e != cudaSuccess) return e;
         bwd_du_kernel<<<a.Hq, kHeadDim, 0, l.stream>>>(l.du, a, nparts);
-        count_launches(2);
+        count_launches(launched + 1);
         return cudaGetLastError();
     } else {
         nparts = a.B * ((a.T + kRowsB0 - 1) / kRowsB0);

@@ -224,11 +224,42 @@ __device__ __forceinline__ void fused_tile(const uint32_t (&sr)[4][32], int thi,
     tl2 = l2a.x + l2a.y;
 }
 
+// Max of the visible raw dots of a half row (keys tlo .. thi of the half when
+// kDiag), and -- when it exceeds `above` -- the first visible key holding it
+// (in *arg; otherwise *arg is left alone).  The backward's rows pass calls this
+// before fused_half<.., kMax = false>, so the search runs while the raw dots
+// are the only tile data in registers.
+template <bool kDiag>
+__device__ __forceinline__ float tile_max_half(const uint32_t (&sr)[2][32], int thi, int tlo,
+                                               float above, int *arg) {
+    float mx[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+    for (int e = 0; e < 64; e += 2) {
+        const float x0 = __uint_as_float(sr[e >> 5][e & 31]), x1 = __uint_as_float(sr[e >> 5][(e & 31) + 1]);
+        if (kDiag)
+            mx[(e >> 1) & 1] = max3(mx[(e >> 1) & 1], (e <= thi && e >= tlo) ? x0 : -INFINITY,
+                                    (e + 1 <= thi && e + 1 >= tlo) ? x1 : -INFINITY);
+        else
+            mx[(e >> 1) & 1] = max3(mx[(e >> 1) & 1], x0, x1);
+    }
+    const float tmax = fmaxf(mx[0], mx[1]);
+    if (tmax > above) {
+        int idx = 64;
+#pragma unroll
+        for (int e = 63; e >= 0; --e) {
+            const bool hit = __uint_as_float(sr[e >> 5][e & 31]) == tmax;
+            idx = (kDiag ? hit && e <= thi && e >= tlo : hit) ? e : idx;
+        }
+        *arg = idx;
+    }
+    return tmax;
+}
+
 // fused_tile for a half row: 64 keys (keys 64*half .. 64*half + 63 of the
 // tile, in sr[0..1][0..31]) of one row, used when two softmax threads share a
 // row.  Key c of this half is visible iff tlo <= c <= thi (both in the half's
 // own coordinates).
-template <bool kDiag, bool kMoments>
+template <bool kDiag, bool kMoments, bool kMax = true>
 __device__ __forceinline__ void fused_half(const uint32_t (&sr)[2][32], int thi, int tlo, float2 sc2,
                                            float neg_m, uint32_t (&pk)[2][16], float &tmax,
                                            float &ts1, float &ts2, float &tl, float &tl2) {
@@ -244,14 +275,14 @@ __device__ __forceinline__ void fused_half(const uint32_t (&sr)[2][32], int thi,
             if (kDiag) {
                 const int col = 32 * cc + 2 * e;
                 const bool v0 = col <= thi && col >= tlo, v1 = col + 1 <= thi && col + 1 >= tlo;
-                mx[e & 1] = max3(mx[e & 1], v0 ? sv.x : -INFINITY, v1 ? sv.y : -INFINITY);
+                if (kMax) mx[e & 1] = max3(mx[e & 1], v0 ? sv.x : -INFINITY, v1 ? sv.y : -INFINITY);
                 x = f2_fma(sv, sc2, nm);
                 x.x = v0 ? x.x : -INFINITY;
                 x.y = v1 ? x.y : -INFINITY;
                 sv.x = v0 ? sv.x : 0.f;
                 sv.y = v1 ? sv.y : 0.f;
             } else {
-                mx[e & 1] = max3(mx[e & 1], sv.x, sv.y);
+                if (kMax) mx[e & 1] = max3(mx[e & 1], sv.x, sv.y);
                 x = f2_fma(sv, sc2, nm);
             }
             if (kDiag || !kMoments) {  // full tiles: from the key moments instead
@@ -288,6 +319,14 @@ struct TcArgs {
     int B, T, Hq, Hkv, nqt, npairs;
     int window;  // 0: all causal keys; W > 0: the last W of each row's
     float s, alpha, L, beta, inv_ln_L;
+    // Backward rows pass (kRows) only: the upstream gradient dL/dout
+    // [B, T, Hq, 64] bf16, and the outputs the backward's tensor-core passes
+    // read: per-row coefficient records [B][Hq][Tpad][kBwdCoefWords] and dA as
+    // bf16 [B][Hq][Tpad][64] (Tpad = T rounded up to the 128-row tile).
+    const __nv_bfloat16 *gout;
+    float *coef;
+    __nv_bfloat16 *dab;
+    int Tpad;
 };
 
 // Epilogue of one row: content = O/|O|, the magnitude channel from the row's
@@ -326,6 +365,102 @@ __device__ __forceinline__ void store_row(const uint32_t (&o)[2][32], float l, f
     if (a.neff) a.neff[(static_cast<size_t>(b) * a.Hq + h) * a.T + row] = ne;
 }
 
+// Epilogue of one row of the backward's rows pass (kRows): with content =
+// O/|O| and g = dL/dout of the row, the chain rule through the magnitude
+// channel (gate, tanh-log of n_eff, null floor) and the direction gives the
+// row's coefficient record (BwdCoef layout, weights relative to the fixed
+// reference cl2) and dA = (g - content <content, g>)/|O|, stored as bf16.  Rows
+// past the end get zero dA and a record whose weights and dS vanish.  All 32
+// lanes of the warp call this (tensor-memory loads are warp-collective).
+__device__ __forceinline__ void store_rec(uint32_t tO, float l, float l2, float m_raw, int jarg,
+                                          float s1, float s2, float c, float cl2, float n, int lo,
+                                          const TcArgs &a, int b, int row, int h) {
+    const bool live = row < a.T;
+    const size_t rrow = (static_cast<size_t>(b) * a.Hq + h) * a.Tpad + row;
+    const uint4 *gp = reinterpret_cast<const uint4 *>(
+        a.gout + ((static_cast<size_t>(b) * a.T + (live ? row : 0)) * a.Hq + h) * kHeadDim);
+    const float4 *u4 = reinterpret_cast<const float4 *>(a.u + static_cast<size_t>(h) * kHeadDim);
+    // Pass 1, 16 dims at a time: |O|^2, <O, g>, <g, u_h>.
+    float nrm = 0.f, og = 0.f, gu = 0.f;
+#pragma unroll
+    for (int ch = 0; ch < 4; ++ch) {
+        uint32_t o[16];
+        tmem_ld16(tO + 16 * ch, o);
+        tmem_wait_ld();
+        const uint4 g0 = live ? __ldg(gp + 2 * ch) : make_uint4(0u, 0u, 0u, 0u);
+        const uint4 g1 = live ? __ldg(gp + 2 * ch + 1) : make_uint4(0u, 0u, 0u, 0u);
+        const uint32_t gw[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const float4 uu = __ldg(u4 + 4 * ch + q);
+            const float ua[4] = {uu.x, uu.y, uu.z, uu.w};
+#pragma unroll
+            for (int x = 0; x < 4; ++x) {
+                const int e = 4 * q + x;
+                const float gv = __uint_as_float(e & 1 ? gw[e >> 1] & 0xFFFF0000u : gw[e >> 1] << 16);
+                const float ov = __uint_as_float(o[e]);
+                nrm = fmaf(ov, ov, nrm);
+                og = fmaf(ov, gv, og);
+                gu = fmaf(gv, ua[x], gu);
+            }
+        }
+    }
+    const float nf = live ? n : 1.0f;
+    const float mean_s = s1 / nf;
+    const float sig_s = sqrtf(fmaxf(s2 / nf - mean_s * mean_s, 0.0f));
+    const float mu = c * mean_s, sigma = c * sig_s;
+    const float kn = sqrtf(2.0f * logf(nf));
+    const float z0 = mu + sigma * kn;
+    const float gate = 1.0f / (1.0f + expf(-a.beta * (c * m_raw - z0)));
+    const float ne_raw = (l * l) / l2;
+    const float ne = fminf(fmaxf(ne_raw, 1.0f), nf);
+    const bool clamped = ne != ne_raw;
+    const float Tm = tanhf(logf(ne) * a.inv_ln_L);
+    const float an = fmaxf(sqrtf(nrm), 1e-30f), inv_an = 1.0f / an;
+    const float cg = og * inv_an;  // <content, g>
+    const float dgate = gu * Tm, dT = gu * gate;
+    const float dneff = clamped ? 0.0f : dT * (1.0f - Tm * Tm) * a.inv_ln_L / ne;
+    const float dl = 2.0f * dneff * l / l2;
+    const float dl2 = -dneff * (l / l2) * (l / l2);
+    const float dm = a.beta * gate * (1.0f - gate) * dgate;
+    const float dsigma = -dm * kn;
+    const float cmu = -dm / nf - (sigma > 0.0f ? dsigma * mu / (nf * sigma) : 0.0f);
+    const float csS = sigma > 0.0f ? dsigma * c / (nf * sigma) : 0.0f;
+    // Pass 2: dA = (g - O cg / |O|) / |O|.
+    uint4 *dst = reinterpret_cast<uint4 *>(a.dab + rrow * kHeadDim);
+    const float sc = inv_an * cg;
+#pragma unroll
+    for (int ch = 0; ch < 4; ++ch) {
+        uint32_t o[16];
+        tmem_ld16(tO + 16 * ch, o);
+        tmem_wait_ld();
+        const uint4 g0 = live ? __ldg(gp + 2 * ch) : make_uint4(0u, 0u, 0u, 0u);
+        const uint4 g1 = live ? __ldg(gp + 2 * ch + 1) : make_uint4(0u, 0u, 0u, 0u);
+        const uint32_t gw[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+        uint32_t d[8];
+#pragma unroll
+        for (int x = 0; x < 8; ++x) {
+            const float g_lo = __uint_as_float(gw[x] << 16), g_hi = __uint_as_float(gw[x] & 0xFFFF0000u);
+            const float d_lo = (g_lo - __uint_as_float(o[2 * x]) * sc) * inv_an;
+            const float d_hi = (g_hi - __uint_as_float(o[2 * x + 1]) * sc) * inv_an;
+            d[x] = live ? pack_bf16(d_lo, d_hi) : 0u;
+        }
+        dst[2 * ch] = make_uint4(d[0], d[1], d[2], d[3]);
+        dst[2 * ch + 1] = make_uint4(d[4], d[5], d[6], d[7]);
+    }
+    float4 *cr = reinterpret_cast<float4 *>(a.coef + rrow * kBwdCoefWords);
+    if (live) {
+        cr[0] = make_float4(cl2, -cl2, c, c * dl);
+        cr[1] = make_float4(2.0f * c * dl2, c * csS, c * cmu, c * dm);
+        cr[2] = make_float4(__int_as_float(jarg), __int_as_float(lo), gate * Tm, 0.f);
+    } else {
+        cr[0] = make_float4(0.f, -INFINITY, 0.f, 0.f);
+        cr[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+        cr[2] = make_float4(__int_as_float(-1), __int_as_float(0), 0.f, 0.f);
+    }
+    cr[3] = make_float4(0.f, 0.f, 0.f, 0.f);
+}
+
 // kFixedRef: the exponentials use the fixed per-row reference m_ref = c*log2e,
 // the largest logit L2-normalised q and k allow (|<q,k>| <= 1); weights then
 // stay <= ~1 and no rescale is needed, so a tile's weights do not wait for
@@ -347,7 +482,10 @@ __device__ __forceinline__ void store_row(const uint32_t (&o)[2][32], float l, f
 // variant from kMomMinTiles query tiles on.
 // kWindow: a sliding window shorter than the sequence (a.window); false
 // compiles every window test away.
-template <bool kFixedRef, int kSplit, bool kMoments, bool kWindow>
+// kRows: the backward's rows pass -- the same forward sweep, which also finds
+// each row's first argmax key, and the store_rec epilogue in place of the
+// output (split rows, fixed reference, no key moments).
+template <bool kFixedRef, int kSplit, bool kMoments, bool kWindow, bool kRows = false>
 __global__ void __launch_bounds__(128 + 256 * kSplit, 1)
 fwd_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
               const __grid_constant__ CUtensorMap tv, const TcArgs a) {
@@ -366,9 +504,10 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CU
     __shared__ uint32_t tmem_base_sh;
     // kSplit == 2: per-row partial statistics of the upper key half
     // (m_raw, S1, S2, l, l2), handed to the lower half for the epilogue.
-    __shared__ float part[kSplit == 2 ? 2 : 1][kSplit == 2 ? kBM : 1][5];
+    __shared__ float part[kSplit == 2 ? 2 : 1][kSplit == 2 ? kBM : 1][6];
     static_assert(kSplit == 1 || kFixedRef, "split rows need the fixed reference");
     static_assert(!kMoments || kSplit == 2, "key moments are used by the split rows only");
+    static_assert(!kRows || (kSplit == 2 && !kMoments), "the rows pass runs the split sweep");
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -600,6 +739,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CU
         const float m_ref = cl2;
         const float2 sc2 = make_float2(cl2, cl2);
         float m_raw = -INFINITY, l = 0.f, l2 = 0.f, s1 = 0.f, s2 = 0.f;
+        int jarg = -1;  // kRows: the first key of the row's max raw dot
         bool ok = true;
         for (int j = 0; j < nkv; ++j) {
             ok = mbar_wait(&s_full[slot], j & 1, a.status);
@@ -613,11 +753,28 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CU
             mbar_arrive(&s_free[slot]);
             uint32_t pk[2][16];
             float tmax, ts1, ts2, tl, tl2;
-            if (masked_tile(j))
-                fused_half<true, kMoments>(sr, vis_hi(j, t) - 64 * half, vis_lo(j, t) - 64 * half,
-                                           sc2, -m_ref, pk, tmax, ts1, ts2, tl, tl2);
-            else
-                fused_half<false, kMoments>(sr, 0, 0, sc2, -m_ref, pk, tmax, ts1, ts2, tl, tl2);
+            if constexpr (kRows) {
+                // A strictly larger tile max moves the argmax to this tile: its
+                // first visible key holding that value (keys in ascending order).
+                int idx = -1;
+                if (masked_tile(j)) {
+                    const int hi = vis_hi(j, t) - 64 * half, lo = vis_lo(j, t) - 64 * half;
+                    tmax = tile_max_half<true>(sr, hi, lo, m_raw, &idx);
+                    float unused;
+                    fused_half<true, false, false>(sr, hi, lo, sc2, -m_ref, pk, unused, ts1, ts2, tl, tl2);
+                } else {
+                    tmax = tile_max_half<false>(sr, 0, 0, m_raw, &idx);
+                    float unused;
+                    fused_half<false, false, false>(sr, 0, 0, sc2, -m_ref, pk, unused, ts1, ts2, tl, tl2);
+                }
+                if (idx >= 0) jarg = (jt0 + j) * kBN + 64 * half + idx;
+            } else {
+                if (masked_tile(j))
+                    fused_half<true, kMoments>(sr, vis_hi(j, t) - 64 * half, vis_lo(j, t) - 64 * half,
+                                               sc2, -m_ref, pk, tmax, ts1, ts2, tl, tl2);
+                else
+                    fused_half<false, kMoments>(sr, 0, 0, sc2, -m_ref, pk, tmax, ts1, ts2, tl, tl2);
+            }
             s1 += ts1;
             s2 += ts2;
             l += tl;
@@ -683,9 +840,17 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CU
             part[slot][t][2] = s2;
             part[slot][t][3] = l;
             part[slot][t][4] = l2;
+            part[slot][t][5] = __int_as_float(jarg);
         }
         named_barrier(1 + slot, 256);
         if (half == 0) {
+            if constexpr (kRows) {
+                // The upper half's keys of a tile follow the lower half's, but tiles
+                // interleave: on a tie the smaller key index is the first argmax.
+                const float om = part[slot][t][0];
+                const int oj = __float_as_int(part[slot][t][5]);
+                if (om > m_raw || (om == m_raw && oj >= 0 && (jarg < 0 || oj < jarg))) jarg = oj;
+            }
             m_raw = fmaxf(m_raw, part[slot][t][0]);
             s1 += part[slot][t][1];
             s2 += part[slot][t][2];
@@ -694,11 +859,16 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CU
             if (ok) ok = mbar_wait(&pv_done[slot], (nkv - 1) & 1, a.status);
             if (__all_sync(0xffffffffu, ok)) {
                 tc_fence_after();
-                uint32_t o[2][32];
-                tmem_ld32(tO, o[0]);
-                tmem_ld32(tO + 32, o[1]);
-                tmem_wait_ld();
-                if (row < a.T) store_row(o, l, l2, m_raw, s1, s2, c, n, a, b, row, h);
+                if constexpr (kRows) {
+                    const int lo = window > 0 ? max(0, row - window + 1) : 0;
+                    store_rec(tO, l, l2, m_raw, jarg, s1, s2, c, cl2, n, lo, a, b, row, h);
+                } else {
+                    uint32_t o[2][32];
+                    tmem_ld32(tO, o[0]);
+                    tmem_ld32(tO + 32, o[1]);
+                    tmem_wait_ld();
+                    if (row < a.T) store_row(o, l, l2, m_raw, s1, s2, c, n, a, b, row, h);
+                }
             }
         }
     } else {
@@ -895,7 +1065,7 @@ cudaError_t launch_fwd_tc(const FwdLaunch &a) {
                          box, CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS)
             return cudaErrorInvalidValue;
     }
-    TcArgs ta;
+    TcArgs ta = {};
     ta.u = a.u;
     ta.out = static_cast<__nv_bfloat16 *>(a.out);
     ta.neff = a.neff;
@@ -934,6 +1104,86 @@ cudaError_t launch_fwd_tc(const FwdLaunch &a) {
     } else {
         fwd_tc_kernel<false, 1, false, false><<<grid, 384, kSmemBytes, a.stream>>>(tq, tk, tv, ta);
     }
+    count_launches(1);
+    return cudaGetLastError();
+}
+
+// The backward's rows pass on the tensor cores: the forward sweep of every
+// (query tile, head pair) with the store_rec epilogue.  Returns
+// cudaErrorNotSupported where this kernel does not apply (fp32 inputs, an odd
+// group size, a logit scale past the fixed reference's range, or a device
+// whose register plan does not hold); the caller then uses its own rows pass.
+cudaError_t launch_bwd_rows_tc(const BwdLaunch &l, float *coef, void *dab, int Tpad) {
+    const int G = l.Hq / l.Hkv;
+    if (l.dtype != POLAR_BF16 || G % 2 != 0) return cudaErrorNotSupported;
+    const bool windowed = l.window > 0 && l.window < l.T;
+    const int n_max = windowed ? l.window : l.T;
+    const float cl2_max = l.s * (n_max > l.L ? 1.0f + l.alpha * logf(static_cast<float>(n_max) / l.L)
+                                             : 1.0f) * 1.4426950408889634f;
+    if (cl2_max > 28.0f) return cudaErrorNotSupported;
+    static std::atomic<uint64_t> configured{0};
+    static std::atomic<uint64_t> plan_ok{0};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const uint64_t bit = 1ull << (dev & 63);
+    const void *fns[] = {reinterpret_cast<const void *>(fwd_tc_kernel<true, 2, false, false, true>),
+                         reinterpret_cast<const void *>(fwd_tc_kernel<true, 2, false, true, true>)};
+    if (!(configured.load() & bit)) {
+        bool fits = true;
+        for (const void *f : fns) {
+            e = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+            if (e != cudaSuccess) return e;
+            cudaFuncAttributes fa;
+            e = cudaFuncGetAttributes(&fa, f);
+            if (e != cudaSuccess) return e;
+            fits = fits && static_cast<long long>(fa.numRegs) * 640 >= 64ll * 128 + 104ll * 512;
+        }
+        if (fits) plan_ok.fetch_or(bit);
+        configured.fetch_or(bit);
+    }
+    if (!(plan_ok.load() & bit)) return cudaErrorNotSupported;
+    CUtensorMap tq, tk, tv;
+    const uint32_t box[4] = {kHeadDim, 1, 128, 1};
+    {
+        const uint64_t dims[4] = {kHeadDim, (uint64_t)l.Hq, (uint64_t)l.T, (uint64_t)l.B};
+        const uint64_t str[3] = {kHeadDim * 2ull, (uint64_t)l.Hq * kHeadDim * 2,
+                                 (uint64_t)l.T * l.Hq * kHeadDim * 2};
+        if (encode_tiled(&tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(l.q), dims, str,
+                         box, CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS)
+            return cudaErrorInvalidValue;
+    }
+    {
+        const uint64_t dims[4] = {kHeadDim, (uint64_t)l.Hkv, (uint64_t)l.T, (uint64_t)l.B};
+        const uint64_t str[3] = {kHeadDim * 2ull, (uint64_t)l.Hkv * kHeadDim * 2,
+                                 (uint64_t)l.T * l.Hkv * kHeadDim * 2};
+        if (encode_tiled(&tk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(l.k), dims, str,
+                         box, CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS ||
+            encode_tiled(&tv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(l.v), dims, str,
+                         box, CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS)
+            return cudaErrorInvalidValue;
+    }
+    TcArgs ta = {};
+    ta.u = l.u;
+    ta.status = l.status;
+    ta.B = l.B; ta.T = l.T; ta.Hq = l.Hq; ta.Hkv = l.Hkv;
+    ta.nqt = Tpad / kBM;
+    ta.npairs = l.Hq / 2;
+    ta.window = windowed ? l.window : 0;
+    ta.s = l.s; ta.alpha = l.alpha; ta.L = static_cast<float>(l.L); ta.beta = l.beta;
+    ta.inv_ln_L = 1.0f / logf(static_cast<float>(l.L));
+    ta.gout = static_cast<const __nv_bfloat16 *>(l.dout);
+    ta.coef = coef;
+    ta.dab = static_cast<__nv_bfloat16 *>(dab);
+    ta.Tpad = Tpad;
+    const long long ctas = static_cast<long long>(ta.nqt) * ta.npairs * l.B;
+    if (ctas <= 0) return cudaSuccess;
+    if (ctas > 0x7fffffffll) return cudaErrorInvalidValue;
+    const unsigned grid = static_cast<unsigned>(ctas);
+    if (windowed)
+        fwd_tc_kernel<true, 2, false, true, true><<<grid, 640, kSmemBytes, l.stream>>>(tq, tk, tv, ta);
+    else
+        fwd_tc_kernel<true, 2, false, false, true><<<grid, 640, kSmemBytes, l.stream>>>(tq, tk, tv, ta);
     count_launches(1);
     return cudaGetLastError();
 }

@@ -103,6 +103,9 @@ size_t bwd_workspace_bytes(int B, int T, int Hq);
 // pass's coefficient records coef [B][Hq][Tpad][kBwdCoefWords] and dA rounded
 // to bf16, dab [B][Hq][Tpad][64] (Tpad = T rounded up to 128).
 cudaError_t launch_bwd_tc(const BwdLaunch &l, const float *coef, const void *dab);
+// The rows pass of the bf16 backward on the tensor cores (fwd_tc.cu): writes
+// coef and dab as above.  cudaErrorNotSupported where it does not apply.
+cudaError_t launch_bwd_rows_tc(const BwdLaunch &l, float *coef, void *dab, int Tpad);
 cudaError_t launch_gdelta_prefill(const GdeltaLaunch &a);
 cudaError_t launch_gdelta_step(const GdeltaStepLaunch &a);
 size_t gdelta_workspace_bytes(int B, int T, int H);

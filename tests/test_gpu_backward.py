@@ -109,6 +109,20 @@ def test_window_multi_tile(cuda_ok):
     _compare(w, x, seed=8)
 
 
+def test_tied_max_takes_the_first_key(cuda_ok):
+    """Every key appears twice in a row (positions 2m and 2m+1, equal bits),
+    so each row's max raw dot is attained by two keys; the max's subgradient
+    goes to the first of them, as in the oracle.  A kernel that split it, or
+    gave it to the later copy, would move dk between the twins."""
+    w = W.small_prefill(B=1, T=600, Hq=4, Hkv=2, dtype="bf16", seed=17, plant="frac",
+                        plant_frac=0.02, L=128)
+    x = W.prefill_inputs(w, "cpu")
+    x["k"][:, 1::2] = x["k"][:, 0::2]
+    x["v"][:, 1::2] = x["v"][:, 0::2]
+    x["u"] = x["u"] * 25.0
+    _compare(w, x, seed=9)
+
+
 def test_deterministic(cuda_ok):
     w = W.small_prefill(B=1, T=700, Hq=4, Hkv=2, dtype="bf16", seed=4, plant="frac",
                         plant_frac=0.02)
