@@ -744,28 +744,52 @@ bwd_rows_mma_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__
 }
 
 // -------------------------------------------------------------------- du ---
-// du partial of one 64-row block per (block, head, batch): the sum over its
-// rows of gate*T (from the coefficient records) times the upstream gradient.
-// Used after the tensor-core rows pass, which writes no du partials.
-__global__ void __launch_bounds__(kHeadDim)
+// du partials of one 64-row block per (block, batch), all heads: the sum over
+// its rows of gate*T (from the coefficient records) times the upstream
+// gradient.  Used after the tensor-core rows pass, which writes no du
+// partials.  Each thread owns 8 consecutive elements of a row's [Hq, 64] slab
+// of dout (one 16-byte load per row).
+__global__ void __launch_bounds__(256)
 bwd_du_part_kernel(const __nv_bfloat16 *__restrict__ gout, const BwdArgs a) {
-    const int blk = blockIdx.x, h = blockIdx.y, b = blockIdx.z, d = threadIdx.x;
+    const int blk = blockIdx.x, b = blockIdx.y;
     const int r0 = blk * 64, r1 = min(r0 + 64, a.T);
-    float s = 0.0f;
-    for (int r = r0; r < r1; ++r) {
-        const float gt = a.coef[((static_cast<size_t>(b) * a.Hq + h) * a.Tpad + r) * kBwdCoefWords + kBcGT];
-        s = fmaf(gt, __bfloat162float(gout[((static_cast<size_t>(b) * a.T + r) * a.Hq + h) * kHeadDim + d]), s);
+    const int chunks = a.Hq * (kHeadDim / 8);
+    for (int c = threadIdx.x; c < chunks; c += blockDim.x) {
+        const int h = c / (kHeadDim / 8), d0 = (c % (kHeadDim / 8)) * 8;
+        float s[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        const float *gtp = a.coef + (static_cast<size_t>(b) * a.Hq + h) * a.Tpad * kBwdCoefWords + kBcGT;
+#pragma unroll 8
+        for (int r = r0; r < r1; ++r) {
+            const float gt = gtp[static_cast<size_t>(r) * kBwdCoefWords];
+            const uint4 g = *reinterpret_cast<const uint4 *>(
+                gout + ((static_cast<size_t>(b) * a.T + r) * a.Hq + h) * kHeadDim + d0);
+            const uint32_t gw[4] = {g.x, g.y, g.z, g.w};
+#pragma unroll
+            for (int x = 0; x < 4; ++x) {
+                s[2 * x] = fmaf(gt, __uint_as_float(gw[x] << 16), s[2 * x]);
+                s[2 * x + 1] = fmaf(gt, __uint_as_float(gw[x] & 0xFFFF0000u), s[2 * x + 1]);
+            }
+        }
+        float4 *dst = reinterpret_cast<float4 *>(
+            a.du_part + ((static_cast<size_t>(b) * gridDim.x + blk) * a.Hq + h) * kHeadDim + d0);
+        dst[0] = make_float4(s[0], s[1], s[2], s[3]);
+        dst[1] = make_float4(s[4], s[5], s[6], s[7]);
     }
-    a.du_part[((static_cast<size_t>(b) * gridDim.x + blk) * a.Hq + h) * kHeadDim + d] = s;
 }
 
-// du_h = sum over the row blocks of their partial sums (fixed order).
-__global__ void __launch_bounds__(kHeadDim)
+// du_h = sum over the row blocks of their partial sums: eight interleaved
+// slices of the partials per head, then the slices, all in a fixed order.
+__global__ void __launch_bounds__(8 * kHeadDim)
 bwd_du_kernel(float *__restrict__ du, const BwdArgs a, int nparts) {
-    const int h = blockIdx.x, d = threadIdx.x;
+    __shared__ float red[8][kHeadDim];
+    const int h = blockIdx.x, d = threadIdx.x & (kHeadDim - 1), sl = threadIdx.x >> 6;
     float s = 0.0f;
-    for (int p = 0; p < nparts; ++p) s += a.du_part[(static_cast<size_t>(p) * a.Hq + h) * kHeadDim + d];
-    du[static_cast<size_t>(h) * kHeadDim + d] = s;
+    for (int p = sl; p < nparts; p += 8) s += a.du_part[(static_cast<size_t>(p) * a.Hq + h) * kHeadDim + d];
+    red[sl][d] = s;
+    __syncthreads();
+    if (sl == 0)
+        du[static_cast<size_t>(h) * kHeadDim + d] = ((red[0][d] + red[1][d]) + (red[2][d] + red[3][d])) +
+                                                     ((red[4][d] + red[5][d]) + (red[6][d] + red[7][d]));
 }
 
 template <typename T>
@@ -780,7 +804,7 @@ cudaError_t launch_all(const BwdLaunch &l, const BwdArgs &a) {
         int launched = 0;
         cudaError_t e = launch_bwd_rows_tc(l, a.coef, a.dab, a.Tpad);
         if (e == cudaSuccess) {
-            bwd_du_part_kernel<<<dim3(a.Tpad / 64, a.Hq, a.B), kHeadDim, 0, l.stream>>>(go, a);
+            bwd_du_part_kernel<<<dim3(a.Tpad / 64, a.B), 256, 0, l.stream>>>(go, a);
             launched = 1;
         } else if (e == cudaErrorNotSupported) {
             bwd_rows_mma_kernel<<<dim3(a.Tpad / 64, a.Hq, a.B), 128, 0, l.stream>>>(q, k, v, go, a);
@@ -792,7 +816,7 @@ cudaError_t launch_all(const BwdLaunch &l, const BwdArgs &a) {
         if (e != cudaSuccess) return e;
         e = launch_bwd_tc(l, a.coef, a.dab);
         if (e != cudaSuccess) return e;
-        bwd_du_kernel<<<a.Hq, kHeadDim, 0, l.stream>>>(l.du, a, nparts);
+        bwd_du_kernel<<<a.Hq, 8 * kHeadDim, 0, l.stream>>>(l.du, a, nparts);
         count_launches(launched + 1);
         return cudaGetLastError();
     } else {
@@ -804,7 +828,7 @@ cudaError_t launch_all(const BwdLaunch &l, const BwdArgs &a) {
         bwd_dq_kernel<T><<<dim3((a.T + kKeyTile - 1) / kKeyTile, a.Hq, a.B), 128, 0, l.stream>>>(
             q, k, v, l.dq, a);
     }
-    bwd_du_kernel<<<a.Hq, kHeadDim, 0, l.stream>>>(l.du, a, nparts);
+    bwd_du_kernel<<<a.Hq, 8 * kHeadDim, 0, l.stream>>>(l.du, a, nparts);
     count_launches(4);
     return cudaGetLastError();
 }

@@ -15,7 +15,7 @@
 // registers.
 //
 // dK/dV pass: one CTA per (128-key tile, kv head, batch).  Q, dA and the rows'
-// coefficient records stream through a two-stage ring for every query tile at
+// coefficient records stream through a three-stage ring for every query tile at
 // or after the key tile and every query head of the group.  The coefficient
 // threads write W and dS as one bf16 tile each in shared memory, row by row
 // (a row's 128 keys contiguous, 128B-swizzled), which the tensor core reads as
@@ -23,8 +23,9 @@
 // dV accumulate in tensor memory (keys as lanes) over the whole loop.
 //
 // dQ pass: one CTA per (128-row query tile, query head, batch), the forward's
-// layout: K and V tiles stream through a three-stage ring; dS goes to tensor
-// memory as bf16 and is the A operand of dQ += dS K.  The argmax term
+// layout: K and V tiles stream through a four-stage ring; dS goes to tensor
+// memory as bf16 (two buffers, so that the coefficient threads never wait for
+// the previous tile's dQ product) and is the A operand of dQ += dS K.  The argmax term
 // c dm k_{jmax} is added in fp32 in the epilogue.
 //
 // Warp roles (384 threads): warp 0 the TMA producer, warp 1 the tensor-memory
@@ -45,18 +46,19 @@ constexpr int kTl = 128;                       // rows per query tile = keys per
 constexpr int kTileB = kTl * 128;              // bytes of a 128 x 64 bf16 tile
 constexpr int kCoefTileB = kTl * kBwdCoefWords * 4;  // 8 KB
 
-// dK/dV pass shared memory: K, V | 2 stages x (Q, dA, coefficients) | W, dS.
-constexpr int kKvStages = 2;
+// dK/dV pass shared memory: K, V | 3 stages x (Q, dA, coefficients) | W, dS
+// (217 KB).
+constexpr int kKvStages = 3;
 constexpr int kKvStageB = 2 * kTileB + kCoefTileB;
 constexpr int kDkdvSmem = 2 * kTileB + kKvStages * kKvStageB + 4 * kTileB + 1024;
-// dQ pass shared memory: Q, dA | 3 stages x (K, V).
-constexpr int kDqStages = 3;
+// dQ pass shared memory: Q, dA | 4 stages x (K, V) (161 KB).
+constexpr int kDqStages = 4;
 constexpr int kDqSmem = 2 * kTileB + kDqStages * 2 * kTileB + 1024;
 
 // Tensor-memory columns (512 allocated).  Both passes: S 0-127, <dA, v> 128-255.
 constexpr uint32_t kColS = 0, kColAV = 128;
 constexpr uint32_t kColDK = 256, kColDV = 320;  // dK/dV pass (fp32, keys as lanes)
-constexpr uint32_t kColDS = 256, kColDQ = 320;  // dQ pass: dS (bf16 pairs), dQ (fp32)
+constexpr uint32_t kColDS = 256, kColDQ = 384;  // dQ pass: dS (bf16 pairs, two buffers), dQ (fp32)
 
 struct BwdTcArgs {
     const float *coef;            // [B][Hq][Tpad][kBwdCoefWords]
@@ -136,8 +138,8 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant
     if (warp == 0 && lane == 0) {
         mbar_init(&kv_full, 1);
         mbar_init(&st_full, 1);
-        mbar_init(&st_free, 256);
-        mbar_init(&wd_full, 256);
+        mbar_init(&st_free, 8);   // one arrival per coefficient warp
+        mbar_init(&wd_full, 8);
         mbar_init(&wd_free, 1);
         mbar_init(&acc_done, 1);
         mbar_init(&mma_idle, 1);
@@ -264,7 +266,8 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant
             tmem_ld32(lane_base + kColAV + 64 * wg + 32, ar[1]);
             tmem_wait_ld();
             tc_fence_before();
-            mbar_arrive(&st_free);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&st_free);  // the warp's loads are complete
             // Keys of this half visible to row i: lo_i .. i (causal, window).
             const bool masked = qt == kt || (a.window > 0 && qt * kTl + kTl - a.window > key0);
             const int e_hi = i - kbase, e_lo = __float_as_int(c2.y) - kbase;
@@ -296,7 +299,8 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant
                 *p = __float2bfloat16_rn(__bfloat162float(*p) + c1.w);
             }
             fence_proxy_async_smem();  // the tensor core reads W and dS through the async proxy
-            mbar_arrive(&wd_full);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&wd_full);  // after every lane's stores and fence
         }
         // Epilogue: dK (first warpgroup) and dV (second) of key key0 + t.
         if (ok) ok = mbar_wait(&acc_done, 0, a.status);
@@ -341,8 +345,8 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__
     uint8_t *sQ = smem, *sDA = smem + kTileB;
     uint8_t *sKV = smem + 2 * kTileB;  // stage s: K at s * 2 tiles, V after it
 
-    __shared__ __align__(8) uint64_t q_full, st_full, st_free, ds_full, ds_free, acc_done, mma_idle;
-    __shared__ __align__(8) uint64_t kv_full[kDqStages], kv_empty[kDqStages];
+    __shared__ __align__(8) uint64_t q_full, st_full, st_free, ds_full, acc_done, mma_idle;
+    __shared__ __align__(8) uint64_t ds_free[2], kv_full[kDqStages], kv_empty[kDqStages];
     __shared__ uint32_t tmem_base_sh;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -358,9 +362,10 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__
     if (warp == 0 && lane == 0) {
         mbar_init(&q_full, 1);
         mbar_init(&st_full, 1);
-        mbar_init(&st_free, 256);
-        mbar_init(&ds_full, 256);
-        mbar_init(&ds_free, 1);
+        mbar_init(&st_free, 8);   // one arrival per coefficient warp
+        mbar_init(&ds_full, 8);
+        mbar_init(&ds_free[0], 1);
+        mbar_init(&ds_free[1], 1);
         mbar_init(&acc_done, 1);
         mbar_init(&mma_idle, 1);
         for (int s = 0; s < kDqStages; ++s) {
@@ -419,9 +424,9 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__
                 const uint32_t k_mn = kv_lo(s, 0, 8192);
 #pragma unroll
                 for (int kk = 0; kk < kTl / 16; ++kk)
-                    mma_ts2(tmem + kColDQ, tmem + kColDS + 8 * kk, k_mn + 128 * kk, hi, idesc_dq,
-                            (m > 0 || kk > 0) ? 1u : 0u);
-                tc_commit(&ds_free);
+                    mma_ts2(tmem + kColDQ, tmem + kColDS + 64 * (m & 1) + 8 * kk, k_mn + 128 * kk, hi,
+                            idesc_dq, (m > 0 || kk > 0) ? 1u : 0u);
+                tc_commit(&ds_free[m & 1]);
                 tc_commit(&kv_empty[s]);
             };
             for (int n = 0; n < nk && ok; ++n) {
@@ -470,7 +475,8 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__
             tmem_ld32(lane_base + kColAV + 64 * wg + 32, ar[1]);
             tmem_wait_ld();
             tc_fence_before();
-            mbar_arrive(&st_free);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&st_free);
             const bool masked = jt == qt || (a.window > 0 && jt * kTl < min(q0 + kTl, a.T) - a.window);
             const int kbase = jt * kTl + 64 * wg;
             uint32_t dp[32], unused[32];
@@ -479,8 +485,9 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__
                                         unused, dp);
             else
                 pair_grads<false, false>(sr, ar, c0, c1, 0, 0, unused, dp);
-            if (n > 0) {
-                ok = mbar_wait(&ds_free, (n - 1) & 1, a.status);
+            // dS(n) goes to buffer n % 2: free once dQ(n-2) has read it.
+            if (n > 1) {
+                ok = mbar_wait(&ds_free[n & 1], ((n - 2) >> 1) & 1, a.status);
                 if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
                 tc_fence_after();
             }
@@ -490,11 +497,13 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__
                 d0[e] = dp[e];
                 d1[e] = dp[16 + e];
             }
-            tmem_st16(lane_base + kColDS + 32 * wg, d0);
-            tmem_st16(lane_base + kColDS + 32 * wg + 16, d1);
+            const uint32_t tds = lane_base + kColDS + 64 * (n & 1) + 32 * wg;
+            tmem_st16(tds, d0);
+            tmem_st16(tds + 16, d1);
             tmem_wait_st();
             tc_fence_before();
-            mbar_arrive(&ds_full);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&ds_full);
         }
         // Epilogue: 32 of the 64 dims of dQ per warpgroup, plus the argmax term
         // c dm k_{jmax} in fp32.
