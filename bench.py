@@ -71,6 +71,9 @@ def parse_args(argv=None):
                     help="timed launches of the memory channel (prefill and decode step); 0 skips")
     ap.add_argument("--window", type=int, default=4096,
                     help="sliding window of the separately timed windowed prefill (0 skips it)")
+    ap.add_argument("--per-head-steps", type=int, default=5,
+                    help="timed launches of the test-only per-head decode (each page read once "
+                         "per query head), for the grouped kernel's traffic saving; 0 skips it")
     ap.add_argument("--chunk", type=int, default=4,
                     help="query tokens per sequence of the separately timed multi-token decode "
                          "(0 skips it)")
@@ -539,6 +542,32 @@ def run_ours(args):
         t_chunk = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in ec) / 1e3, world, dev)
         chunk_res = (C, t_chunk)
     clk.__exit__(None, None, None)
+    # ---- test-only per-head decode on the same cache, timed on its own ----
+    per_head_res = None
+    if do_dec and args.per_head_steps > 0:
+        from polar_attention_b200 import native as N
+
+        def per_head_decode():
+            N.selftest_decode_per_head(xd["q"], xd["kv_pages"], xd["page_table"], xd["seqlens"],
+                                       xd["u"], out_d, neff_d, ws, stream=stream, **p)
+
+        for _ in range(min(Wm, 3)):
+            per_head_decode()
+        torch.cuda.synchronize(dev)
+        Kh = args.per_head_steps
+        eh = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(Kh)]
+        barrier(world, dev)
+        torch.cuda.synchronize(dev)
+        for i in range(Kh):
+            eh[i][0].record(stream)
+            per_head_decode()
+            eh[i][1].record(stream)
+        torch.cuda.synchronize(dev)
+        barrier(world, dev)
+        if pa.get_status() != 0:
+            raise RuntimeError("device status after the per-head decode")
+        per_head_res = (Kh, max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in eh) / 1e3, world,
+                                           dev))
     t_all = outer[0].elapsed_time(outer[1]) / 1e3
     t_pre_max = max_over_ranks(t_pre, world, dev)
     t_dec_max = max_over_ranks(t_dec, world, dev)
@@ -593,7 +622,7 @@ def run_ours(args):
         dec_launch_s = t_dec / K
         tf = PREFILL.flops / pre_launch_s / 1e12 if do_pre else 0.0
         gbs = kv_bytes / dec_launch_s / 1e9 if do_dec else 0.0
-        sha_p = source_sha("fwd_tc.cu", "fwd_moments.cu", "polar_common.cuh")
+        sha_p = source_sha("fwd_tc.cu", "fwd_moments.cu", "polar_common.cuh", "tc_common.cuh")
         sha_d = source_sha("decode.cu", "polar_common.cuh")
         value = aggregate_throughput(PREFILL.flops * K, world, t_pre_max) / 1e12 if do_pre else 0.0
         dec_value = aggregate_throughput(kv_bytes * K, world, t_dec_max) / 1e9 if do_dec else 0.0
@@ -698,6 +727,7 @@ def run_ours(args):
             result["prefill_no_workspace"] = {
                 "value": pl_tf, "unit": "TFLOP/s", "ms_per_launch": pl_launch * 1e3,
                 "pct_bf16_peak": 100 * pl_tf / peaks["bf16_tflops"],
+                "traffic": profiled_traffic("prefill_no_workspace", sha_p),
                 "note": "polar_attn_fwd(q, k, v, u, params, out, neff_out, stream): the same "
                         "prefill without the key-moment workspace (null-floor sums formed score "
                         "by score); timed separately after the step loop; not part of value"}
@@ -712,6 +742,18 @@ def run_ours(args):
                 "note": "sliding-window prefill on the same T=16384 inputs, flops of the visible "
                         "(query, key) pairs; timed separately after the step loop, L2 warm from "
                         "the previous launch; not part of value"}
+        if per_head_res is not None:
+            Kh, t_h = per_head_res
+            h_launch = t_h / Kh
+            result["decode_per_head"] = {
+                "ms_per_launch": h_launch * 1e3,
+                "time_vs_grouped": h_launch / dec_launch_s,
+                "kv_bytes_requested_per_launch": kv_bytes * DECODE.Hq / DECODE.Hkv,
+                "note": "test-only polar_attn_selftest_decode_per_head: the same decode with one "
+                        "query head per CTA, so each KV page is requested once per query head "
+                        "(Hq/Hkv = 4 times per group); timed separately.  Concurrent CTAs of a "
+                        "group share the re-reads in L2, so its DRAM bytes grow far less than 4x "
+                        "(measured with ncu)"}
         if chunk_res is not None:
             C, t_chunk = chunk_res
             c_launch = t_chunk / K

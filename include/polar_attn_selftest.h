@@ -31,6 +31,24 @@ polar_status_t polar_attn_selftest_exp2(const float *x, float *poly, float *mufu
  */
 polar_status_t polar_attn_selftest_timeout(void *stream);
 
+/*
+ * The paged decode with one query head per CTA: the same kernels, arguments,
+ * layouts, results and errors as polar_attn_decode_paged, except that each
+ * CTA reads the key/value pages of its query head's kv head for that head
+ * alone, so that every page is read once per query head rather than once per
+ * group.  It exists to measure the DRAM traffic the grouped kernel saves
+ * ("GQA-Grouped Paged Decode Kernel", section 2.2: a group of Hq/Hkv query
+ * heads shares each page read, cutting decode traffic by that factor).
+ * Single-token decode only; workspace as polar_attn_decode_workspace_size.
+ */
+polar_status_t polar_attn_selftest_decode_per_head(const void *q, const void *kv_pages,
+                                                   int num_pages, const int32_t *page_table,
+                                                   int max_pages, const int32_t *seqlens,
+                                                   int num_seqs, const float *u,
+                                                   const polar_params_t *params, void *out,
+                                                   float *neff_out, void *workspace,
+                                                   size_t ws_bytes, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -351,6 +351,7 @@ polar_status_t polar_attn_decode_paged_chunk(const void *q, const void *kv_pages
     if (!status) return POLAR_ERR_CUDA;
     DecodeLaunch a;
     a.chunk = chunk;
+    a.per_head = 0;
     a.q = q; a.kv_pages = kv_pages; a.num_pages = num_pages; a.page_table = page_table;
     a.max_pages = max_pages; a.seqlens = seqlens; a.num_seqs = num_seqs; a.u = u; a.out = out;
     a.neff = neff_out; a.Hq = p->Hq; a.Hkv = p->Hkv; a.s = p->logit_scale; a.alpha = p->alpha;
@@ -455,6 +456,40 @@ polar_status_t polar_attn_selftest_timeout(void *stream) {
     selftest_timeout_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(status);
     count_launches(1);
     return from_cuda(cudaGetLastError());
+}
+
+polar_status_t polar_attn_selftest_decode_per_head(const void *q, const void *kv_pages,
+                                                   int num_pages, const int32_t *page_table,
+                                                   int max_pages, const int32_t *seqlens,
+                                                   int num_seqs, const float *u,
+                                                   const polar_params_t *p, void *out,
+                                                   float *neff_out, void *workspace,
+                                                   size_t ws_bytes, void *stream) {
+    polar_status_t st = check_decode(p, num_seqs, max_pages);
+    if (st != POLAR_OK) return st;
+    if (num_seqs == 0) return POLAR_OK;
+    if (num_pages < 1 || static_cast<long long>(num_pages) * 2 * p->Hkv * kPage > (1ll << 31) - 1)
+        return POLAR_ERR_INVALID_ARG;
+    if (!q || !kv_pages || !page_table || !seqlens || !u || !out || !workspace)
+        return POLAR_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(kv_pages) || !aligned16(u) || !aligned16(out) ||
+        !aligned16(workspace) || !aligned4(page_table) || !aligned4(seqlens) ||
+        (neff_out && !aligned4(neff_out)))
+        return POLAR_ERR_INVALID_ARG;
+    if (ws_bytes < decode_partials_bytes(num_seqs, max_pages, p->Hq, p->Hkv, 1))
+        return POLAR_ERR_WORKSPACE;
+    int *status = status_ptr();
+    if (!status) return POLAR_ERR_CUDA;
+    DecodeLaunch a;
+    a.chunk = 1;
+    a.per_head = 1;
+    a.q = q; a.kv_pages = kv_pages; a.num_pages = num_pages; a.page_table = page_table;
+    a.max_pages = max_pages; a.seqlens = seqlens; a.num_seqs = num_seqs; a.u = u; a.out = out;
+    a.neff = neff_out; a.Hq = p->Hq; a.Hkv = p->Hkv; a.s = p->logit_scale; a.alpha = p->alpha;
+    a.beta = p->beta; a.L = p->L_train; a.window = p->window; a.workspace = workspace;
+    a.status = status;
+    a.stream = static_cast<cudaStream_t>(stream);
+    return from_cuda(launch_decode(a));
 }
 
 size_t polar_gdelta_prefill_workspace_size(const polar_gdelta_params_t *p) {

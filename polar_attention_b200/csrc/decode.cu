@@ -45,6 +45,8 @@ struct SplitArgs {
     int chunk;  // query tokens per sequence (the last `chunk` cache positions)
     int window; // 0: every cached position; W > 0: each row's last W
     float s, alpha, L;
+    int kv_div; // grid heads per kv head whose pages a CTA reads: 1, except in the
+                // per-head self-test (one query head per CTA, so kv head = h / G)
 };
 
 // Page of the earliest cache position any query row of a sequence sees.
@@ -154,7 +156,7 @@ decode_split_kernel(const __grid_constant__ CUtensorMap kv_map, const SplitArgs 
         const int phys = pt[kk];
         if (phys >= 0 && phys < a.num_pages) {
             mbar_arrive_expect_tx(&full_bar[st], kStageBytes);
-            const int row = (phys * 2 * a.Hkv + g) * kPage;  // K block of head g
+            const int row = (phys * 2 * a.Hkv + g / a.kv_div) * kPage;  // K block of the kv head
             tma_load_2d(smem + st * kStageBytes, &kv_map, 0, row, &full_bar[st]);
             tma_load_2d(smem + st * kStageBytes + kChunkBytes, &kv_map, 0, row + a.Hkv * kPage,
                         &full_bar[st]);
@@ -486,7 +488,7 @@ cudaError_t decode_preload() {
 }
 
 cudaError_t launch_decode(const DecodeLaunch &a) {
-    const int G = a.Hq / a.Hkv;
+    const int G = a.per_head ? 1 : a.Hq / a.Hkv;
     const int pps = decode_pages_per_split(a.num_seqs, a.max_pages, a.Hkv);
     const int max_splits = (a.max_pages + pps - 1) / pps;
 
@@ -501,8 +503,38 @@ cudaError_t launch_decode(const DecodeLaunch &a) {
 
     SplitArgs sa{a.page_table, a.seqlens, static_cast<const __nv_bfloat16 *>(a.q),
                  static_cast<float *>(a.workspace), a.status, a.num_pages, a.max_pages, a.Hq, a.Hkv,
-                 pps, max_splits, a.chunk, a.window, a.s, a.alpha, static_cast<float>(a.L)};
+                 pps, max_splits, a.chunk, a.window, a.s, a.alpha, static_cast<float>(a.L), 1};
     if (a.chunk < 1 || G * a.chunk > 16) return cudaErrorInvalidValue;
+    if (a.per_head) {
+        // Test-only: one query head per CTA (grid y over the query heads), each
+        // reading its kv head's pages on its own, so that every page is read
+        // once per query head instead of once per group.
+        if (a.chunk != 1) return cudaErrorInvalidValue;
+        sa.kv_div = a.Hq / a.Hkv;
+        static std::atomic<uint64_t> configured{0};
+        int dev = 0;
+        cudaError_t e = cudaGetDevice(&dev);
+        if (e != cudaSuccess) return e;
+        const uint64_t bit = 1ull << (dev & 63);
+        if (!(configured.load() & bit)) {
+            e = cudaFuncSetAttribute(decode_split_kernel<1, false>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, kSplitSmem);
+            if (e != cudaSuccess) return e;
+            configured.fetch_or(bit);
+        }
+        decode_split_kernel<1, false><<<dim3(max_splits, a.Hq, a.num_seqs), 128, kSplitSmem,
+                                        a.stream>>>(map, sa);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+        dim3 mgrid(a.Hq, a.num_seqs);
+        decode_merge_kernel<<<mgrid, 32, 0, a.stream>>>(
+            static_cast<const float *>(a.workspace), a.seqlens, a.u,
+            static_cast<__nv_bfloat16 *>(a.out), a.neff, a.Hq, 1, a.window, a.max_pages, pps,
+            max_splits, a.s, a.alpha, static_cast<float>(a.L), a.beta,
+            1.0f / logf(static_cast<float>(a.L)));
+        count_launches(2);
+        return cudaGetLastError();
+    }
     cudaError_t e;
     switch (G) {
         case 1: e = launch_split_rows<1>(map, sa, a.num_seqs, a.stream); break;

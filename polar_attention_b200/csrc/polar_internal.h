@@ -40,6 +40,7 @@ struct DecodeLaunch {
     int window;  // 0: all cached positions; W > 0: the last W of each row's
     void *workspace;
     int chunk;  // query tokens per sequence (1 for plain decode)
+    int per_head;  // test-only: one query head per CTA (pages read once per query head)
     int *status;
     cudaStream_t stream;
 };

@@ -33,7 +33,7 @@ EXPORTS = ["polar_attn_default_params", "polar_attn_fwd_workspace_size", "polar_
            "polar_attn_decode_chunk_workspace_size", "polar_attn_decode_paged_chunk",
            "polar_attn_bwd_workspace_size", "polar_attn_bwd",
            "polar_gdelta_prefill_workspace_size", "polar_gdelta_prefill", "polar_gdelta_step",
-           "polar_attn_selftest_timeout"]
+           "polar_attn_selftest_timeout", "polar_attn_selftest_decode_per_head"]
 
 
 class PolarError(RuntimeError):
@@ -99,6 +99,8 @@ def lib() -> ctypes.CDLL:
             L.polar_attn_decode_paged_noalloc.argtypes = [P, P, I, P, I, P, I, P, PP, P, P, P]
             L.polar_attn_selftest_exp2.argtypes = [P, P, P, I, P]
             L.polar_attn_selftest_timeout.argtypes = [P]
+            L.polar_attn_selftest_decode_per_head.argtypes = [P, P, I, P, I, P, I, P, PP, P, P, P,
+                                                              Z, P]
             GP = ctypes.POINTER(GdeltaParams)
             L.polar_gdelta_prefill_workspace_size.argtypes = [GP]
             L.polar_gdelta_prefill_workspace_size.restype = Z
@@ -113,7 +115,7 @@ def lib() -> ctypes.CDLL:
                          "polar_attn_decode_paged_noalloc", "polar_attn_selftest_exp2",
                          "polar_attn_decode_paged_chunk", "polar_attn_bwd",
                          "polar_gdelta_prefill", "polar_gdelta_step",
-                         "polar_attn_selftest_timeout"):
+                         "polar_attn_selftest_timeout", "polar_attn_selftest_decode_per_head"):
                 getattr(L, name).restype = I
             _lib = L
     return _lib
@@ -423,6 +425,30 @@ def gdelta_step(q, k, v, alpha, beta, state_pool, slots, out=None, *, accumulate
                                    ctypes.byref(p), _ptr(out), _stream(stream)),
            "polar_gdelta_step")
     return out
+
+
+def selftest_decode_per_head(q, kv_pages, page_table, seqlens, u, out=None, neff=None,
+                             workspace=None, *, s=8.0, alpha=0.3, L=2048, beta=1.0, stream=None,
+                             window=0):
+    """polar_attn_selftest_decode_per_head: decode_paged with one query head per
+    CTA (pages read once per query head).  Returns (out, neff)."""
+    N, Hq, D = q.shape
+    P_, _, Hkv, _, _ = kv_pages.shape
+    max_pages = page_table.shape[1]
+    p = make_params(0, 0, Hq, Hkv, _dt(q), s, alpha, L, beta, window=window)
+    p.head_dim = D
+    ws_need = int(lib().polar_attn_decode_workspace_size(N, max_pages, ctypes.byref(p)))
+    if workspace is None:
+        workspace = torch.empty(max(ws_need, 16), device=q.device, dtype=torch.uint8)
+    if out is None:
+        out = torch.empty_like(q)
+    if neff is None:
+        neff = torch.empty((N, Hq), device=q.device, dtype=torch.float32)
+    _check(lib().polar_attn_selftest_decode_per_head(
+        _ptr(q), _ptr(kv_pages), P_, _ptr(page_table), max_pages, _ptr(seqlens), N, _ptr(u),
+        ctypes.byref(p), _ptr(out), _ptr(neff), _ptr(workspace), workspace.numel(),
+        _stream(stream)), "polar_attn_selftest_decode_per_head")
+    return out, neff
 
 
 def selftest_timeout(stream=None):

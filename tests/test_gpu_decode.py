@@ -152,3 +152,19 @@ def test_full_workload_sampled(cuda_ok):
     o = out[seqs].float().cpu().numpy().reshape(len(seqs) * w.Hq, -1).astype(np.float64)
     n = neff[seqs].cpu().numpy().reshape(-1).astype(np.float64)
     PT.compare(o, n, ref, np.arange(len(seqs) * w.Hq), PT.OUT_TOL_BF16, what="decode full")
+
+
+def test_per_head_variant_reads_the_same_pages(cuda_ok):
+    """The test-only per-head decode (one query head per CTA, each page read
+    once per query head) gives the grouped decode's rows bit for bit: the mma
+    rows of a group are independent, and the merge is the same."""
+    from polar_attention_b200 import native
+    w = W.small_decode(num_seqs=5, min_len=1, max_len=40000, Hq=16, Hkv=4, seed=33, plant=2)
+    x = PT.to_device(W.decode_inputs(w, "cpu"))
+    p = dict(s=w.s, alpha=w.alpha, L=w.L, beta=w.beta)
+    a, na = pa.decode_paged(x["q"], x["kv_pages"], x["page_table"], x["seqlens"], x["u"], **p)
+    b, nb = native.selftest_decode_per_head(x["q"], x["kv_pages"], x["page_table"],
+                                            x["seqlens"], x["u"], **p)
+    torch.cuda.synchronize()
+    assert pa.get_status() == 0
+    assert torch.equal(a, b) and torch.equal(na, nb)
