@@ -43,6 +43,7 @@
 #include "polar_common.cuh"
 #include "polar_gdelta.h"
 #include "polar_internal.h"
+#include "tc_common.cuh"
 
 namespace polar {
 namespace {
@@ -892,72 +893,152 @@ __device__ __forceinline__ void load16<__nv_bfloat16>(const __nv_bfloat16 *src, 
     }
 }
 
-// Decode step: one CTA per (sequence, head); thread owns S[tid/4][16 (tid%4) .. +16).
-// Every warp takes the query and key norms itself (two elements a lane and a
-// warp sum) and each thread reads its own 16 columns of q and k, so the warps
-// never wait for one another.
-template <typename Tin>
-__global__ void __launch_bounds__(256, sizeof(Tin) == 2 ? 4 : 3)
-gd_step_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
-                                                      const Tin *__restrict__ v,
-                                                      const float *__restrict__ alpha,
-                                                      const float *__restrict__ beta, float *pool,
-                                                      int num_slots, const int32_t *__restrict__ slots,
-                                                      int H, Tin *out, int accumulate, int *status) {
-    const int seq = blockIdx.x / H, h = blockIdx.x % H;
-    const int slot = slots[seq];
-    if (slot < 0) return;
-    if (slot >= num_slots) {
-        if (threadIdx.x == 0) record_error(status, POLAR_ERR_BAD_SLOT);
-        return;
-    }
-    const int tid = threadIdx.x, lane = tid & 31;
-    const int r = tid >> 2, c0 = 16 * (tid & 3);
-    float *S = pool + ((static_cast<size_t>(slot) * H + h) * 64 + r) * 64 + c0;
-    float4 s[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) s[i] = reinterpret_cast<const float4 *>(S)[i];
-    const size_t row = static_cast<size_t>(seq) * H + h;
-    const Tin *qr = q + row * kHeadDim, *kr = k + row * kHeadDim;
-    const float q0 = to_f<Tin>(qr[lane]), q1 = to_f<Tin>(qr[lane + 32]);
-    const float k0 = to_f<Tin>(kr[lane]), k1 = to_f<Tin>(kr[lane + 32]);
-    float qc[16], kc[16];
-    load16<Tin>(qr + c0, qc);
-    load16<Tin>(kr + c0, kc);
-    const float vr = to_f<Tin>(v[row * kHeadDim + r]);
-    const float al = alpha[row], be = beta[row];
-    const float sq = warp_sum(fmaf(q0, q0, q1 * q1)), sk2 = warp_sum(fmaf(k0, k0, k1 * k1));
-    const float iq = sq > 0.0f ? 1.0f / sqrtf(sq) : 0.0f;
-    const float ik = sk2 > 0.0f ? 1.0f / sqrtf(sk2) : 0.0f;
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-        qc[i] *= iq;
-        kc[i] *= ik;
-    }
+// Decode step, persistent: a grid of three CTAs per SM walks the (sequence,
+// head) items.  Thread 0 of each CTA streams items through a ring of
+// kStepStages shared-memory stages with bulk copies (the item's 16 KB state,
+// and its q, k and v rows), kStepStages items ahead of the update, so that an
+// SM keeps up to 3 x 4 states moving.  The update reads the stage, and each
+// thread writes its part of the new state straight back to the pool.  Thread t
+// owns the float4 slots t, t + 256, t + 512, t + 768 of the 64 x 64 state:
+// rows t/16 + 16 i (i = 0..3), columns 4 (t % 16) .. + 3, so the shared-memory
+// reads and the global writes are consecutive 16-byte pieces across a warp;
+// the sixteen threads of a row hold all its 64 columns and sum among
+// themselves with shuffles.
+constexpr int kStepStages = 4;
+constexpr int kStepStateB = 64 * 64 * 4;
 
-    float sk = 0.0f;
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-        sk = dot4(s[i], make_float4(kc[4 * i], kc[4 * i + 1], kc[4 * i + 2], kc[4 * i + 3]), sk);
-    sk += __shfl_xor_sync(0xffffffffu, sk, 1);
-    sk += __shfl_xor_sync(0xffffffffu, sk, 2);
-    const float w = be * (vr - al * sk);
-    float o = 0.0f;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        s[i].x = fmaf(al, s[i].x, w * kc[4 * i]);
-        s[i].y = fmaf(al, s[i].y, w * kc[4 * i + 1]);
-        s[i].z = fmaf(al, s[i].z, w * kc[4 * i + 2]);
-        s[i].w = fmaf(al, s[i].w, w * kc[4 * i + 3]);
-        o = dot4(s[i], make_float4(qc[4 * i], qc[4 * i + 1], qc[4 * i + 2], qc[4 * i + 3]), o);
-        reinterpret_cast<float4 *>(S)[i] = s[i];
+template <typename Tin>
+struct StepSmem {
+    float st[kStepStages][64 * 64];
+    Tin rows[kStepStages][3][kHeadDim];  // q, k, v
+    int item[kStepStages];               // item index, or -1: nothing to update
+    int slot[kStepStages];               // its state's slot in the pool
+    uint64_t full[kStepStages];
+};
+
+template <typename Tin>
+__global__ void __launch_bounds__(256, 3)
+gd_step_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *__restrict__ v,
+               const float *__restrict__ alpha, const float *__restrict__ beta, float *pool,
+               int num_slots, const int32_t *__restrict__ slots, int H, int nitems, Tin *out,
+               int accumulate, int *status) {
+    extern __shared__ __align__(128) uint8_t step_raw[];
+    StepSmem<Tin> &sm = *reinterpret_cast<StepSmem<Tin> *>(step_raw);
+    const int tid = threadIdx.x, lane = tid & 31;
+    const int G = gridDim.x;
+    const int mine = nitems > static_cast<int>(blockIdx.x)
+                         ? (nitems - static_cast<int>(blockIdx.x) + G - 1) / G : 0;
+    if (tid == 0) {
+        for (int s = 0; s < kStepStages; ++s) mbar_init(&sm.full[s], 1);
+        fence_barrier_init();
     }
-    o += __shfl_xor_sync(0xffffffffu, o, 1);
-    o += __shfl_xor_sync(0xffffffffu, o, 2);
-    if ((tid & 3) == 0) {
-        Tin *dst = out + row * kHeadDim + r;
-        *dst = from_f<Tin>(accumulate ? to_f<Tin>(*dst) + o : o);
+    __syncthreads();
+    // Thread 0: stage n of this CTA's item list (item blockIdx.x + n G).
+    auto issue = [&](int n) {
+        const int s = n % kStepStages;
+        const int item = static_cast<int>(blockIdx.x) + n * G;
+        const int seq = item / H, h = item % H;
+        const int slot = slots[seq];
+        if (slot < 0 || slot >= num_slots) {
+            if (slot >= num_slots) record_error(status, POLAR_ERR_BAD_SLOT);
+            sm.item[s] = -1;
+            mbar_arrive(&sm.full[s]);
+            return;
+        }
+        sm.item[s] = item;
+        sm.slot[s] = slot;
+        const size_t row = static_cast<size_t>(item);  // (seq, h) row of q, k, v, out
+        constexpr uint32_t rb = kHeadDim * sizeof(Tin);
+        mbar_arrive_expect_tx(&sm.full[s], kStepStateB + 3 * rb);
+        bulk_load(sm.st[s], pool + (static_cast<size_t>(slot) * H + h) * 64 * 64, kStepStateB,
+                  &sm.full[s]);
+        bulk_load(sm.rows[s][0], q + row * kHeadDim, rb, &sm.full[s]);
+        bulk_load(sm.rows[s][1], k + row * kHeadDim, rb, &sm.full[s]);
+        bulk_load(sm.rows[s][2], v + row * kHeadDim, rb, &sm.full[s]);
+    };
+    int issued = 0;
+    if (tid == 0)
+        for (; issued < min(mine, kStepStages); ++issued) issue(issued);
+    const int c4 = 4 * (tid & 15);  // first of this thread's four columns
+    const int r0 = tid >> 4;        // first of its rows r0 + 16 i
+    bool ok = true;
+    int n = 0;
+#pragma unroll 1
+    for (; n < mine; ++n) {
+        const int s = n % kStepStages;
+        ok = mbar_wait(&sm.full[s], (n / kStepStages) & 1, status);
+        if (!__syncthreads_and(ok)) break;
+        const int item = sm.item[s], slot = sm.slot[s];
+        float4 x[4];
+        float kc[4], qc[4], vr[4], sq = 0.0f, sk2 = 0.0f, al = 0.0f, be = 0.0f;
+        if (item >= 0) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                x[i] = reinterpret_cast<const float4 *>(sm.st[s])[tid + 256 * i];
+                kc[i] = to_f<Tin>(sm.rows[s][1][c4 + i]);
+                qc[i] = to_f<Tin>(sm.rows[s][0][c4 + i]);
+                vr[i] = to_f<Tin>(sm.rows[s][2][r0 + 16 * i]);
+            }
+            // Norms: the q and k rows are also in every 16-lane group.
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                sq = fmaf(qc[i], qc[i], sq);
+                sk2 = fmaf(kc[i], kc[i], sk2);
+            }
+            al = __ldg(alpha + item);
+            be = __ldg(beta + item);
+        }
+        // The stage is read: thread 0 refills it with the item kStepStages ahead.
+        __syncthreads();
+        if (tid == 0 && issued < mine) {
+            fence_proxy_async_smem();  // the reads above come before the copy's writes
+            issue(issued++);
+        }
+        if (item < 0) continue;
+#pragma unroll
+        for (int o = 1; o < 16; o <<= 1) {
+            sq += __shfl_xor_sync(0xffffffffu, sq, o);
+            sk2 += __shfl_xor_sync(0xffffffffu, sk2, o);
+        }
+        const float iq = sq > 0.0f ? 1.0f / sqrtf(sq) : 0.0f;
+        const float ik = sk2 > 0.0f ? 1.0f / sqrtf(sk2) : 0.0f;
+        float sk[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            sk[i] = dot4(x[i], make_float4(kc[0] * ik, kc[1] * ik, kc[2] * ik, kc[3] * ik), 0.0f);
+#pragma unroll
+        for (int o = 1; o < 16; o <<= 1)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) sk[i] += __shfl_xor_sync(0xffffffffu, sk[i], o);
+        float *S = pool + (static_cast<size_t>(slot) * H + item % H) * 64 * 64;
+        float ov[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float wk = be * (vr[i] - al * sk[i]) * ik;
+            x[i].x = fmaf(al, x[i].x, wk * kc[0]);
+            x[i].y = fmaf(al, x[i].y, wk * kc[1]);
+            x[i].z = fmaf(al, x[i].z, wk * kc[2]);
+            x[i].w = fmaf(al, x[i].w, wk * kc[3]);
+            reinterpret_cast<float4 *>(S)[tid + 256 * i] = x[i];
+            ov[i] = dot4(x[i], make_float4(qc[0], qc[1], qc[2], qc[3]), 0.0f);
+        }
+#pragma unroll
+        for (int o = 1; o < 16; o <<= 1)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) ov[i] += __shfl_xor_sync(0xffffffffu, ov[i], o);
+        if ((lane & 15) == 0) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                Tin *dst = out + static_cast<size_t>(item) * kHeadDim + r0 + 16 * i;
+                const float o = ov[i] * iq;
+                *dst = from_f<Tin>(accumulate ? to_f<Tin>(*dst) + o : o);
+            }
+        }
     }
+    // After a timed-out wait: every copy thread 0 started lands (or its wait
+    // runs out) before shared memory is released.
+    if (tid == 0)
+        for (; n < issued; ++n) mbar_wait(&sm.full[n % kStepStages], (n / kStepStages) & 1, status);
 }
 
 constexpr size_t kChunkSmem = (4 * kC * kPitch + 5 * kC) * sizeof(float);
@@ -1025,17 +1106,43 @@ cudaError_t launch_gdelta_prefill(const GdeltaLaunch &l) {
 
 cudaError_t launch_gdelta_step(const GdeltaStepLaunch &l) {
     if (l.num_seqs == 0) return cudaSuccess;
-    const unsigned grid = static_cast<unsigned>(l.num_seqs) * static_cast<unsigned>(l.H);
+    static std::atomic<uint64_t> sm_known{0};
+    static int sm_count[64] = {0};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev >= 64) return cudaErrorInvalidDevice;
+    if (!(sm_known.load() & (1ull << dev))) {
+        int n = 0;
+        e = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        if (e != cudaSuccess) return e;
+        sm_count[dev] = n;
+        sm_known.fetch_or(1ull << dev);
+    }
+    const long long items = static_cast<long long>(l.num_seqs) * l.H;
+    const unsigned grid = static_cast<unsigned>(std::min<long long>(items, 3ll * sm_count[dev]));
+    static std::atomic<uint64_t> configured{0};
+    if (!(configured.load() & (1ull << dev))) {
+        e = cudaFuncSetAttribute(gd_step_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(sizeof(StepSmem<float>)));
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(gd_step_kernel<__nv_bfloat16>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     static_cast<int>(sizeof(StepSmem<__nv_bfloat16>)));
+        if (e != cudaSuccess) return e;
+        configured.fetch_or(1ull << dev);
+    }
     if (l.dtype == POLAR_FP32) {
-        gd_step_kernel<float><<<grid, 256, 0, l.stream>>>(
+        gd_step_kernel<float><<<grid, 256, sizeof(StepSmem<float>), l.stream>>>(
             static_cast<const float *>(l.q), static_cast<const float *>(l.k),
             static_cast<const float *>(l.v), l.alpha, l.beta, l.pool, l.num_slots, l.slots, l.H,
-            static_cast<float *>(l.out), l.accumulate, l.status);
+            static_cast<int>(items), static_cast<float *>(l.out), l.accumulate, l.status);
     } else {
-        gd_step_kernel<__nv_bfloat16><<<grid, 256, 0, l.stream>>>(
+        gd_step_kernel<__nv_bfloat16><<<grid, 256, sizeof(StepSmem<__nv_bfloat16>), l.stream>>>(
             static_cast<const __nv_bfloat16 *>(l.q), static_cast<const __nv_bfloat16 *>(l.k),
             static_cast<const __nv_bfloat16 *>(l.v), l.alpha, l.beta, l.pool, l.num_slots,
-            l.slots, l.H, static_cast<__nv_bfloat16 *>(l.out), l.accumulate, l.status);
+            l.slots, l.H, static_cast<int>(items), static_cast<__nv_bfloat16 *>(l.out),
+            l.accumulate, l.status);
     }
     count_launches(1);
     return cudaGetLastError();
