@@ -679,7 +679,7 @@ def run_ours(args):
                         "part of value"}
         if gd_res is not None:
             wg, wst, Kg, t_gp, t_gs = gd_res
-            sha_g = source_sha("gdelta.cu", "polar_common.cuh")
+            sha_g = source_sha("gdelta.cu", "polar_common.cuh", "tc_common.cuh")
             gp_launch, gs_launch = t_gp / Kg, t_gs / Kg
             tok = wg.B * wg.T
             # The recurrence's own arithmetic (S k, the rank-one write, S q:

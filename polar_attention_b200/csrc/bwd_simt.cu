@@ -744,25 +744,28 @@ bwd_rows_mma_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__
 }
 
 // -------------------------------------------------------------------- du ---
-// du partials of one 64-row block per (block, batch), all heads: the sum over
+// du partials of one 16-row block per (block, batch), all heads: the sum over
 // its rows of gate*T (from the coefficient records) times the upstream
 // gradient.  Used after the tensor-core rows pass, which writes no du
 // partials.  Each thread owns 8 consecutive elements of a row's [Hq, 64] slab
-// of dout (one 16-byte load per row).
-__global__ void __launch_bounds__(256)
+// of dout and issues its 16 rows' 16-byte loads together.
+constexpr int kDuRows = 16;
+__global__ void __launch_bounds__(128)
 bwd_du_part_kernel(const __nv_bfloat16 *__restrict__ gout, const BwdArgs a) {
     const int blk = blockIdx.x, b = blockIdx.y;
-    const int r0 = blk * 64, r1 = min(r0 + 64, a.T);
+    const int r0 = blk * kDuRows;
     const int chunks = a.Hq * (kHeadDim / 8);
     for (int c = threadIdx.x; c < chunks; c += blockDim.x) {
         const int h = c / (kHeadDim / 8), d0 = (c % (kHeadDim / 8)) * 8;
         float s[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        const float *gtp = a.coef + (static_cast<size_t>(b) * a.Hq + h) * a.Tpad * kBwdCoefWords + kBcGT;
-#pragma unroll 8
-        for (int r = r0; r < r1; ++r) {
+        const float *gtp = a.coef + ((static_cast<size_t>(b) * a.Hq + h) * a.Tpad + r0) * kBwdCoefWords + kBcGT;
+        const __nv_bfloat16 *gp = gout + ((static_cast<size_t>(b) * a.T + r0) * a.Hq + h) * kHeadDim + d0;
+        const size_t rstride = static_cast<size_t>(a.Hq) * kHeadDim;
+#pragma unroll
+        for (int r = 0; r < kDuRows; ++r) {
+            if (r0 + r >= a.T) break;
             const float gt = gtp[static_cast<size_t>(r) * kBwdCoefWords];
-            const uint4 g = *reinterpret_cast<const uint4 *>(
-                gout + ((static_cast<size_t>(b) * a.T + r) * a.Hq + h) * kHeadDim + d0);
+            const uint4 g = *reinterpret_cast<const uint4 *>(gp + r * rstride);
             const uint32_t gw[4] = {g.x, g.y, g.z, g.w};
 #pragma unroll
             for (int x = 0; x < 4; ++x) {
@@ -777,19 +780,25 @@ bwd_du_part_kernel(const __nv_bfloat16 *__restrict__ gout, const BwdArgs a) {
     }
 }
 
-// du_h = sum over the row blocks of their partial sums: eight interleaved
+// du_h = sum over the row blocks of their partial sums: sixteen interleaved
 // slices of the partials per head, then the slices, all in a fixed order.
-__global__ void __launch_bounds__(8 * kHeadDim)
+constexpr int kDuSlices = 16;
+__global__ void __launch_bounds__(kDuSlices * kHeadDim)
 bwd_du_kernel(float *__restrict__ du, const BwdArgs a, int nparts) {
-    __shared__ float red[8][kHeadDim];
+    __shared__ float red[kDuSlices][kHeadDim];
     const int h = blockIdx.x, d = threadIdx.x & (kHeadDim - 1), sl = threadIdx.x >> 6;
     float s = 0.0f;
-    for (int p = sl; p < nparts; p += 8) s += a.du_part[(static_cast<size_t>(p) * a.Hq + h) * kHeadDim + d];
+#pragma unroll 8
+    for (int p = sl; p < nparts; p += kDuSlices)
+        s += a.du_part[(static_cast<size_t>(p) * a.Hq + h) * kHeadDim + d];
     red[sl][d] = s;
     __syncthreads();
-    if (sl == 0)
-        du[static_cast<size_t>(h) * kHeadDim + d] = ((red[0][d] + red[1][d]) + (red[2][d] + red[3][d])) +
-                                                     ((red[4][d] + red[5][d]) + (red[6][d] + red[7][d]));
+    if (sl == 0) {
+        float t = 0.0f;
+#pragma unroll
+        for (int i = 0; i < kDuSlices; ++i) t += red[i][d];
+        du[static_cast<size_t>(h) * kHeadDim + d] = t;
+    }
 }
 
 template <typename T>
@@ -800,13 +809,14 @@ cudaError_t launch_all(const BwdLaunch &l, const BwdArgs &a) {
     if constexpr (std::is_same<T, __nv_bfloat16>::value) {
         // Rows pass: the forward's tcgen05 sweep where it applies, else the
         // mma.sync kernel (which also writes the du partials).
-        nparts = a.B * (a.Tpad / 64);
         int launched = 0;
         cudaError_t e = launch_bwd_rows_tc(l, a.coef, a.dab, a.Tpad);
         if (e == cudaSuccess) {
-            bwd_du_part_kernel<<<dim3(a.Tpad / 64, a.B), 256, 0, l.stream>>>(go, a);
+            nparts = a.B * (a.Tpad / kDuRows);
+            bwd_du_part_kernel<<<dim3(a.Tpad / kDuRows, a.B), 128, 0, l.stream>>>(go, a);
             launched = 1;
         } else if (e == cudaErrorNotSupported) {
+            nparts = a.B * (a.Tpad / 64);
             bwd_rows_mma_kernel<<<dim3(a.Tpad / 64, a.Hq, a.B), 128, 0, l.stream>>>(q, k, v, go, a);
             launched = 1;
         } else {
@@ -816,7 +826,7 @@ cudaError_t launch_all(const BwdLaunch &l, const BwdArgs &a) {
         if (e != cudaSuccess) return e;
         e = launch_bwd_tc(l, a.coef, a.dab);
         if (e != cudaSuccess) return e;
-        bwd_du_kernel<<<a.Hq, 8 * kHeadDim, 0, l.stream>>>(l.du, a, nparts);
+        bwd_du_kernel<<<a.Hq, kDuSlices * kHeadDim, 0, l.stream>>>(l.du, a, nparts);
         count_launches(launched + 1);
         return cudaGetLastError();
     } else {
@@ -828,7 +838,7 @@ cudaError_t launch_all(const BwdLaunch &l, const BwdArgs &a) {
         bwd_dq_kernel<T><<<dim3((a.T + kKeyTile - 1) / kKeyTile, a.Hq, a.B), 128, 0, l.stream>>>(
             q, k, v, l.dq, a);
     }
-    bwd_du_kernel<<<a.Hq, 8 * kHeadDim, 0, l.stream>>>(l.du, a, nparts);
+    bwd_du_kernel<<<a.Hq, kDuSlices * kHeadDim, 0, l.stream>>>(l.du, a, nparts);
     count_launches(4);
     return cudaGetLastError();
 }
@@ -837,7 +847,8 @@ cudaError_t launch_all(const BwdLaunch &l, const BwdArgs &a) {
 
 // fp32 inputs: the 80-word records and the per-128-row du partials.  bf16
 // inputs: the compact records and dA as bf16, both over T rounded up to 128
-// rows, and the per-64-row du partials.  The workspace holds either layout.
+// rows, and du partials per 16-row block (per 64-row block after the mma.sync
+// rows pass).  The workspace holds either layout.
 size_t bwd_workspace_bytes(int B, int T, int Hq) {
     const size_t Tpad = (static_cast<size_t>(T) + 127) / 128 * 128;
     const size_t fp32 = static_cast<size_t>(B) * Hq * T * kRecWords * sizeof(float) +
@@ -845,7 +856,7 @@ size_t bwd_workspace_bytes(int B, int T, int Hq) {
                             sizeof(float);
     const size_t bf16 = static_cast<size_t>(B) * Hq * Tpad * kBwdCoefWords * sizeof(float) +
                         static_cast<size_t>(B) * Hq * Tpad * kHeadDim * sizeof(__nv_bfloat16) +
-                        static_cast<size_t>(B) * (Tpad / 64) * Hq * kHeadDim * sizeof(float);
+                        static_cast<size_t>(B) * (Tpad / kDuRows) * Hq * kHeadDim * sizeof(float);
     return fp32 > bf16 ? fp32 : bf16;
 }
 
