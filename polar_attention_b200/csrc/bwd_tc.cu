@@ -551,6 +551,265 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__
     }
 }
 
+
+// -------------------------------------------------------- dQ pass, head pair ---
+// The dQ pass for an even group size, in the forward's layout: one CTA per
+// (128-row query tile, pair of query heads of one kv group, batch), both heads
+// sharing every K/V tile.  Each key tile is taken in two 64-key halves: for
+// each head, S and <dA, v> of one half at a time (N = 64) sit in tensor memory
+// next to the head's dS (the whole tile, bf16) and its dQ accumulator, 256
+// columns per head.  Each head has its own coefficient warpgroup, so one
+// head's arithmetic overlaps the other head's products; one thread issues the
+// score products (both heads, both halves) and another the dQ products.
+constexpr int kDq2Stages = 4;
+constexpr int kDq2Smem = 4 * kTileB + kDq2Stages * 2 * kTileB + 1024;  // 193 KB
+constexpr uint32_t kC2S = 0, kC2AV = 64, kC2DS = 128, kC2DQ = 192;  // per head: + 256 * slot
+
+__global__ void __launch_bounds__(384, 1)
+bwd_dq2_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
+                  const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tda,
+                  const BwdTcArgs a) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = align1024(smem_raw);
+    uint8_t *sQ = smem;                    // Q of head slot 0, then slot 1
+    uint8_t *sDA = smem + 2 * kTileB;      // dA of slot 0, then slot 1
+    uint8_t *sKV = smem + 4 * kTileB;      // stage s: K at s * 2 tiles, V after it
+
+    __shared__ __align__(8) uint64_t q_full, acc_done, mma_idle[2];
+    __shared__ __align__(8) uint64_t st_full[2], st_free[2], ds_full[2], ds_free[2];
+    __shared__ __align__(8) uint64_t kv_full[kDq2Stages], kv_empty[kDq2Stages];
+    __shared__ uint32_t tmem_base_sh;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int npairs = a.Hq / 2;
+    const int per_qt = npairs * a.B;
+    const int qt = a.nt - 1 - static_cast<int>(blockIdx.x) / per_qt;  // longest rows first
+    const int rem = static_cast<int>(blockIdx.x) % per_qt;
+    const int h0 = 2 * (rem % npairs), b = rem / npairs;
+    const int g = h0 / a.G;
+    const int q0 = qt * kTl;
+    const int jt0 = a.window > 0 ? max(0, q0 - a.window + 1) / kTl : 0;
+    const int nk = qt - jt0 + 1;
+
+    if (warp == 0 && lane == 0) {
+        mbar_init(&q_full, 1);
+        mbar_init(&acc_done, 1);
+        mbar_init(&mma_idle[0], 1);
+        mbar_init(&mma_idle[1], 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&st_full[i], 1);
+            mbar_init(&st_free[i], 4);  // one arrival per warp of the head's warpgroup
+            mbar_init(&ds_full[i], 4);
+            mbar_init(&ds_free[i], 1);
+        }
+        for (int s = 0; s < kDq2Stages; ++s) {
+            mbar_init(&kv_full[s], 1);
+            mbar_init(&kv_empty[s], 2);  // one commit from each issuer
+        }
+        fence_barrier_init();
+    }
+    if (warp == 1) tmem_alloc_512(&tmem_base_sh);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = tmem_base_sh;
+
+    if (warp < 4) {
+        reg_dealloc<64>();
+        if (warp == 0 && lane == 0) {
+            // --------------------------------------------------- TMA producer
+            tma_prefetch_desc(&tq);
+            tma_prefetch_desc(&tk);
+            tma_prefetch_desc(&tv);
+            tma_prefetch_desc(&tda);
+            mbar_arrive_expect_tx(&q_full, 4 * kTileB);
+            for (int i = 0; i < 2; ++i) {
+                tma_load_4d(sQ + i * kTileB, &tq, 0, h0 + i, q0, b, &q_full);
+                tma_load_3d(sDA + i * kTileB, &tda, 0, q0, b * a.Hq + h0 + i, &q_full);
+            }
+            int issued = 0;
+            bool ok = true;
+            for (int n = 0; n < nk && ok; ++n) {
+                const int s = n % kDq2Stages;
+                if (n >= kDq2Stages &&
+                    !(ok = mbar_wait(&kv_empty[s], ((n / kDq2Stages) - 1) & 1, a.status)))
+                    break;
+                uint8_t *st = sKV + s * 2 * kTileB;
+                mbar_arrive_expect_tx(&kv_full[s], 2 * kTileB);
+                tma_load_4d(st, &tk, 0, g, (jt0 + n) * kTl, b, &kv_full[s]);
+                tma_load_4d(st + kTileB, &tv, 0, g, (jt0 + n) * kTl, b, &kv_full[s]);
+                ++issued;
+            }
+            mbar_wait(&q_full, 0, a.status);
+            for (int n = (issued > kDq2Stages ? issued - kDq2Stages : 0); n < issued; ++n)
+                mbar_wait(&kv_full[n % kDq2Stages], (n / kDq2Stages) & 1, a.status);
+        } else if ((warp == 1 || warp == 2) && lane == 0) {
+            const uint32_t hi = kSdescHi128B;
+            auto kv_lo = [&](int s, int which, uint32_t lbo) {
+                return sdesc_lo(smem_u32(sKV + s * 2 * kTileB + which * kTileB), lbo);
+            };
+            bool ok = true;
+            if (warp == 1) {
+                // ------------------- score issuer: S and <dA, v> per head and half
+                constexpr uint32_t idesc_h = idesc_bf16(kTl, 64, false);  // N = 64 keys
+                ok = mbar_wait(&q_full, 0, a.status);
+                for (int n = 0; n < nk && ok; ++n) {
+                    const int s = n % kDq2Stages;
+                    if (!(ok = mbar_wait(&kv_full[s], (n / kDq2Stages) & 1, a.status))) break;
+                    for (int half = 0; half < 2 && ok; ++half) {
+                        for (int i = 0; i < 2 && ok; ++i) {
+                            const int step = 2 * n + half;
+                            if (step > 0 && !(ok = mbar_wait(&st_free[i], (step - 1) & 1, a.status)))
+                                break;
+                            tc_fence_after();
+                            // keys 64 half .. + 63: 64 rows of 128 B further into the tile
+                            const uint32_t k_k = kv_lo(s, 0, 16) + 512 * half;
+                            const uint32_t v_k = kv_lo(s, 1, 16) + 512 * half;
+                            const uint32_t q_k = sdesc_lo(smem_u32(sQ + i * kTileB), 16);
+                            const uint32_t a_k = sdesc_lo(smem_u32(sDA + i * kTileB), 16);
+                            const uint32_t col = tmem + 256 * i;
+                            mma_ss2<0>(col + kC2S, q_k, hi, k_k, hi, idesc_h);
+#pragma unroll
+                            for (int kk = 1; kk < 4; ++kk)
+                                mma_ss2<1>(col + kC2S, q_k + 2 * kk, hi, k_k + 2 * kk, hi, idesc_h);
+                            mma_ss2<0>(col + kC2AV, a_k, hi, v_k, hi, idesc_h);
+#pragma unroll
+                            for (int kk = 1; kk < 4; ++kk)
+                                mma_ss2<1>(col + kC2AV, a_k + 2 * kk, hi, v_k + 2 * kk, hi, idesc_h);
+                            tc_commit(&st_full[i]);
+                        }
+                    }
+                    if (ok) tc_commit(&kv_empty[s]);
+                }
+            } else {
+                // ------------------------------------ dQ issuer: dQ += dS K per head
+                constexpr uint32_t idesc_dq = idesc_bf16(kTl, 64, true);  // K as MN-major B
+                for (int n = 0; n < nk && ok; ++n) {
+                    const int s = n % kDq2Stages;
+                    if (!(ok = mbar_wait(&kv_full[s], (n / kDq2Stages) & 1, a.status))) break;
+                    const uint32_t k_mn = kv_lo(s, 0, 8192);
+                    for (int i = 0; i < 2 && ok; ++i) {
+                        if (!(ok = mbar_wait(&ds_full[i], n & 1, a.status))) break;
+                        tc_fence_after();
+                        const uint32_t col = tmem + 256 * i;
+#pragma unroll
+                        for (int kk = 0; kk < kTl / 16; ++kk)
+                            mma_ts2(col + kC2DQ, col + kC2DS + 8 * kk, k_mn + 128 * kk, hi, idesc_dq,
+                                    (n > 0 || kk > 0) ? 1u : 0u);
+                        tc_commit(&ds_free[i]);
+                    }
+                    if (ok) tc_commit(&kv_empty[s]);
+                }
+                tc_commit(&acc_done);
+            }
+            // Every MMA this thread issued completes before tensor memory is freed.
+            tc_commit(&mma_idle[warp - 1]);
+            mbar_wait(&mma_idle[warp - 1], 0, a.status);
+        }
+    } else {
+        reg_alloc<208>();
+        // ------------------------------- coefficient warpgroups, one per head
+        const int slot = (warp - 4) >> 2;
+        const int wq = warp & 3;
+        const int t = 32 * wq + lane;     // row within the tile = TMEM lane
+        const int h = h0 + slot, i = q0 + t;
+        const uint32_t lane_base = tmem + (static_cast<uint32_t>(32 * wq) << 16) + 256 * slot;
+        const float4 *cr = reinterpret_cast<const float4 *>(
+            a.coef + ((static_cast<size_t>(b) * a.Hq + h) * a.Tpad + i) * kBwdCoefWords);
+        const float4 c0 = __ldg(cr), c1 = __ldg(cr + 1), c2 = __ldg(cr + 2);
+        bool ok = true;
+        for (int n = 0; n < nk && ok; ++n) {
+            const int jt = jt0 + n;
+            const bool masked = jt == qt || (a.window > 0 && jt * kTl < min(q0 + kTl, a.T) - a.window);
+            for (int half = 0; half < 2; ++half) {
+                const int step = 2 * n + half;
+                ok = mbar_wait(&st_full[slot], step & 1, a.status);
+                if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+                tc_fence_after();
+                uint32_t sr[2][32], ar[2][32];
+                tmem_ld32(lane_base + kC2S, sr[0]);
+                tmem_ld32(lane_base + kC2S + 32, sr[1]);
+                tmem_ld32(lane_base + kC2AV, ar[0]);
+                tmem_ld32(lane_base + kC2AV + 32, ar[1]);
+                tmem_wait_ld();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&st_free[slot]);
+                const int kbase = jt * kTl + 64 * half;
+                uint32_t dp[32], unused[32];
+                if (masked)
+                    pair_grads<true, false>(sr, ar, c0, c1, __float_as_int(c2.y) - kbase, i - kbase,
+                                            unused, dp);
+                else
+                    pair_grads<false, false>(sr, ar, c0, c1, 0, 0, unused, dp);
+                // dS of the previous tile consumed by its dQ product before the first half.
+                if (half == 0 && n > 0) {
+                    ok = mbar_wait(&ds_free[slot], (n - 1) & 1, a.status);
+                    if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+                    tc_fence_after();
+                }
+                uint32_t d0[16], d1[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                    d0[e] = dp[e];
+                    d1[e] = dp[16 + e];
+                }
+                tmem_st16(lane_base + kC2DS + 32 * half, d0);
+                tmem_st16(lane_base + kC2DS + 32 * half + 16, d1);
+                tmem_wait_st();
+                tc_fence_before();
+                if (half == 1) {
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&ds_full[slot]);
+                }
+            }
+        }
+        // Epilogue: dQ of row i and head h, plus the argmax term c dm k_{jmax} in fp32.
+        if (ok) ok = mbar_wait(&acc_done, 0, a.status);
+        if (__all_sync(0xffffffffu, ok) && nk > 0) {
+            tc_fence_after();
+            uint32_t o[2][32];
+            tmem_ld32(lane_base + kC2DQ, o[0]);
+            tmem_ld32(lane_base + kC2DQ + 32, o[1]);
+            tmem_wait_ld();
+            const int jm = __float_as_int(c2.x);
+            if (i < a.T) {
+                float v[64];
+#pragma unroll
+                for (int e = 0; e < 64; ++e) v[e] = __uint_as_float(o[e >> 5][e & 31]);
+                if (jm >= 0 && jm < a.T) {
+                    const uint4 *kr = reinterpret_cast<const uint4 *>(
+                        a.k + ((static_cast<size_t>(b) * a.T + jm) * a.Hkv + g) * kHeadDim);
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) {
+                        const uint4 kk = __ldg(kr + c);
+                        const uint32_t kw[4] = {kk.x, kk.y, kk.z, kk.w};
+#pragma unroll
+                        for (int x = 0; x < 4; ++x) {
+                            v[8 * c + 2 * x] = fmaf(c1.w, __uint_as_float(kw[x] << 16), v[8 * c + 2 * x]);
+                            v[8 * c + 2 * x + 1] =
+                                fmaf(c1.w, __uint_as_float(kw[x] & 0xFFFF0000u), v[8 * c + 2 * x + 1]);
+                        }
+                    }
+                }
+                float4 *dst = reinterpret_cast<float4 *>(
+                    a.dq + ((static_cast<size_t>(b) * a.T + i) * a.Hq + h) * kHeadDim);
+#pragma unroll
+                for (int c = 0; c < 16; ++c)
+                    dst[c] = make_float4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc_512(tmem);
+    }
+}
+
 }  // namespace
 
 cudaError_t launch_bwd_tc(const BwdLaunch &l, const float *coef, const void *dab) {
@@ -566,10 +825,14 @@ cudaError_t launch_bwd_tc(const BwdLaunch &l, const float *coef, const void *dab
         e = cudaFuncSetAttribute(bwd_dq_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  kDqSmem);
         if (e != cudaSuccess) return e;
+        e = cudaFuncSetAttribute(bwd_dq2_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 kDq2Smem);
+        if (e != cudaSuccess) return e;
         // setmaxnreg hands out only the registers the block was launched with:
         // 64 x 128 (producer, issuer) + 208 x 256 (coefficient threads) must fit.
         const void *fns[] = {reinterpret_cast<const void *>(bwd_dkdv_tc_kernel),
-                             reinterpret_cast<const void *>(bwd_dq_tc_kernel)};
+                             reinterpret_cast<const void *>(bwd_dq_tc_kernel),
+                             reinterpret_cast<const void *>(bwd_dq2_tc_kernel)};
         for (const void *f : fns) {
             cudaFuncAttributes fa;
             e = cudaFuncGetAttributes(&fa, f);
@@ -622,7 +885,12 @@ cudaError_t launch_bwd_tc(const BwdLaunch &l, const float *coef, const void *dab
     if (kv_ctas > 0x7fffffffll || q_ctas > 0x7fffffffll) return cudaErrorInvalidValue;
     bwd_dkdv_tc_kernel<<<static_cast<unsigned>(kv_ctas), 384, kDkdvSmem, l.stream>>>(tq, tk, tv,
                                                                                      tda, a);
-    bwd_dq_tc_kernel<<<static_cast<unsigned>(q_ctas), 384, kDqSmem, l.stream>>>(tq, tk, tv, tda, a);
+    if (a.G % 2 == 0)  // head pairs share each K/V tile
+        bwd_dq2_tc_kernel<<<static_cast<unsigned>(q_ctas / 2), 384, kDq2Smem, l.stream>>>(tq, tk,
+                                                                                           tv, tda, a);
+    else
+        bwd_dq_tc_kernel<<<static_cast<unsigned>(q_ctas), 384, kDqSmem, l.stream>>>(tq, tk, tv,
+                                                                                     tda, a);
     count_launches(2);
     return cudaGetLastError();
 }
