@@ -180,7 +180,11 @@ size_t polar_attn_fwd_staging_size(const polar_params_t *params);
  * memory gives full copy bandwidth) into `staging` (device memory owned by the
  * caller, at least polar_attn_fwd_staging_size bytes), runs the prefill
  * (polar_attn_fwd_ws with its workspace in the staging buffer), copies
- * out and n_eff back to host memory, and synchronises `stream`.
+ * out and n_eff back to host memory, and synchronises `stream`.  The work
+ * goes batch by batch: batch b runs on `stream` while batch b+1's inputs are
+ * copied in and batch b-1's outputs copied out, on two copy streams the
+ * library creates once per device and joins to `stream` through events.
+ * Host-buffer calls on one device are serialised.
  */
 polar_status_t polar_attn_fwd_host(const void *q_h, const void *k_h, const void *v_h,
                                    const float *u_h, const polar_params_t *params, void *out_h,

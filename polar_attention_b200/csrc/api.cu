@@ -37,6 +37,39 @@ int *status_ptr() {
     return g_status_addr[dev];
 }
 
+// Copy streams and events of the host-buffer prefill, created once per device:
+// inputs go in on `in`, outputs come back on `out` (two copy engines), joined to
+// the caller's stream through events.  `mu` serialises host-buffer calls on a
+// device, which share these.
+struct HostPipe {
+    std::mutex mu;
+    bool ready = false;
+    cudaStream_t in = nullptr, out = nullptr;
+    cudaEvent_t start = nullptr, out_done = nullptr, in_done[2] = {}, comp_done[2] = {};
+};
+HostPipe g_pipe[kMaxDevices];
+
+HostPipe *host_pipe() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    HostPipe &hp = g_pipe[dev];
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!hp.ready) {
+        const unsigned ef = cudaEventDisableTiming;
+        if (cudaStreamCreateWithFlags(&hp.in, cudaStreamNonBlocking) != cudaSuccess ||
+            cudaStreamCreateWithFlags(&hp.out, cudaStreamNonBlocking) != cudaSuccess ||
+            cudaEventCreateWithFlags(&hp.start, ef) != cudaSuccess ||
+            cudaEventCreateWithFlags(&hp.out_done, ef) != cudaSuccess)
+            return nullptr;
+        for (int i = 0; i < 2; ++i)
+            if (cudaEventCreateWithFlags(&hp.in_done[i], ef) != cudaSuccess ||
+                cudaEventCreateWithFlags(&hp.comp_done[i], ef) != cudaSuccess)
+                return nullptr;
+        hp.ready = true;
+    }
+    return &hp;
+}
+
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -290,18 +323,47 @@ polar_status_t polar_attn_fwd_host(const void *q_h, const void *k_h, const void 
     char *dout = du + round_up(ub, 256);
     char *dne = dout + round_up(qb, 256);
     char *dws = dne + round_up(nb, 256);
-    const size_t wsb = fwd_moments_bytes(p->B, p->T, p->Hkv);
-    if (cudaMemcpyAsync(dq, q_h, qb, cudaMemcpyHostToDevice, s) != cudaSuccess ||
-        cudaMemcpyAsync(dk, k_h, kb, cudaMemcpyHostToDevice, s) != cudaSuccess ||
-        cudaMemcpyAsync(dv, v_h, kb, cudaMemcpyHostToDevice, s) != cudaSuccess ||
-        cudaMemcpyAsync(du, u_h, ub, cudaMemcpyHostToDevice, s) != cudaSuccess)
+    // Batch by batch: the inputs of batch b+1 go in and the outputs of batch b-1
+    // come back while batch b runs on `stream`.
+    HostPipe *hp = host_pipe();
+    if (!hp) return POLAR_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(hp->mu);
+    const size_t qbb = qb / p->B, kbb = kb / p->B, nbb = nb / p->B;  // one batch
+    polar_params_t p1 = *p;
+    p1.B = 1;
+    const size_t wsb = fwd_moments_bytes(1, p->T, p->Hkv);
+    const char *qh = static_cast<const char *>(q_h), *kh = static_cast<const char *>(k_h),
+               *vh = static_cast<const char *>(v_h);
+    char *oh = static_cast<char *>(out_h), *nh = reinterpret_cast<char *>(neff_h);
+    // The copies start after earlier work on `stream` (which may still use the staging).
+    if (cudaEventRecord(hp->start, s) != cudaSuccess ||
+        cudaStreamWaitEvent(hp->in, hp->start, 0) != cudaSuccess ||
+        cudaStreamWaitEvent(hp->out, hp->start, 0) != cudaSuccess ||
+        cudaMemcpyAsync(du, u_h, ub, cudaMemcpyHostToDevice, hp->in) != cudaSuccess)
         return POLAR_ERR_CUDA;
-    st = polar_attn_fwd_ws(dq, dk, dv, reinterpret_cast<float *>(du), p, dout,
-                           neff_h ? reinterpret_cast<float *>(dne) : nullptr,
-                           wsb ? dws : nullptr, wsb, stream);
-    if (st != POLAR_OK) return st;
-    if (cudaMemcpyAsync(out_h, dout, qb, cudaMemcpyDeviceToHost, s) != cudaSuccess) return POLAR_ERR_CUDA;
-    if (neff_h && cudaMemcpyAsync(neff_h, dne, nb, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    for (int b = 0; b < p->B; ++b) {
+        const int e2 = b & 1;
+        if (cudaMemcpyAsync(dq + b * qbb, qh + b * qbb, qbb, cudaMemcpyHostToDevice, hp->in) != cudaSuccess ||
+            cudaMemcpyAsync(dk + b * kbb, kh + b * kbb, kbb, cudaMemcpyHostToDevice, hp->in) != cudaSuccess ||
+            cudaMemcpyAsync(dv + b * kbb, vh + b * kbb, kbb, cudaMemcpyHostToDevice, hp->in) != cudaSuccess ||
+            cudaEventRecord(hp->in_done[e2], hp->in) != cudaSuccess ||
+            cudaStreamWaitEvent(s, hp->in_done[e2], 0) != cudaSuccess)
+            return POLAR_ERR_CUDA;
+        st = polar_attn_fwd_ws(dq + b * qbb, dk + b * kbb, dv + b * kbb, reinterpret_cast<float *>(du),
+                               &p1, dout + b * qbb,
+                               neff_h ? reinterpret_cast<float *>(dne + b * nbb) : nullptr,
+                               wsb ? dws : nullptr, wsb, stream);
+        if (st != POLAR_OK) return st;
+        if (cudaEventRecord(hp->comp_done[e2], s) != cudaSuccess ||
+            cudaStreamWaitEvent(hp->out, hp->comp_done[e2], 0) != cudaSuccess ||
+            cudaMemcpyAsync(oh + b * qbb, dout + b * qbb, qbb, cudaMemcpyDeviceToHost, hp->out) != cudaSuccess)
+            return POLAR_ERR_CUDA;
+        if (neff_h && cudaMemcpyAsync(nh + b * nbb, dne + b * nbb, nbb, cudaMemcpyDeviceToHost,
+                                      hp->out) != cudaSuccess)
+            return POLAR_ERR_CUDA;
+    }
+    if (cudaEventRecord(hp->out_done, hp->out) != cudaSuccess ||
+        cudaStreamWaitEvent(s, hp->out_done, 0) != cudaSuccess)
         return POLAR_ERR_CUDA;
     return from_cuda(cudaStreamSynchronize(s));
 }

@@ -123,6 +123,24 @@ def test_tied_max_takes_the_first_key(cuda_ok):
     _compare(w, x, seed=9)
 
 
+def test_train_length_full_size_batch0(cuda_ok):
+    """The bench's backward launch (B=8, T=2048, Hq=16, Hkv=4, bf16, 1% planted
+    keys): the whole call runs on the GPU, and batch 0's gradients (every row,
+    key and dimension of it; batches are independent) are checked against the
+    oracle run on batch 0 alone.  du sums over every batch, so it is left to
+    the smaller tests, which compare it with the oracle directly."""
+    w = W.TRAIN
+    x = W.prefill_inputs(w, "cpu")
+    gout = _gout(w, seed=21)
+    dq, dk, dv, _ = _run(w, x, gout)
+    x0 = {k: (v[:1] if k in ("q", "k", "v") else v) for k, v in x.items()}
+    import dataclasses
+    w0 = dataclasses.replace(w, B=1)
+    ref = PT.oracle_bwd(w0, x0, gout[:1])
+    for name, g, r in zip(("dq", "dk", "dv"), (dq[:1], dk[:1], dv[:1]), ref[:3]):
+        _check(f"{name} full-size batch 0", g, r, GRAD_TOL["bf16"], GRAD_FLOOR["bf16"])
+
+
 def test_deterministic(cuda_ok):
     w = W.small_prefill(B=1, T=700, Hq=4, Hkv=2, dtype="bf16", seed=4, plant="frac",
                         plant_frac=0.02)

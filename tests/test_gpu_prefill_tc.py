@@ -214,3 +214,24 @@ def test_unnormalised_inputs_are_reported(cuda_ok):
     torch.cuda.synchronize()
     assert pa.get_status() == 1  # POLAR_ERR_INVALID_ARG
     assert pa.get_status() == 0
+
+
+@pytest.mark.parametrize("T", [300, 4500])
+def test_host_buffers_match_device_buffers(cuda_ok, T):
+    """polar_attn_fwd_host runs the prefill batch by batch, overlapping each
+    batch's copies with its neighbours' compute: with three batches, on the key
+    moments path (T=4500) and below it, its rows equal the device-buffer call's
+    bit for bit (a row does not depend on the other batches)."""
+    w = W.small_prefill(B=3, T=T, Hq=8, Hkv=2, dtype="bf16", seed=T, plant="frac",
+                        plant_frac=0.01, L=512)
+    x = W.prefill_inputs(w, "cpu")
+    xd = PT.to_device(x)
+    p = dict(s=w.s, alpha=w.alpha, L=w.L, beta=w.beta)
+    ref, nref = pa.fwd(xd["q"], xd["k"], xd["v"], xd["u"], **p)
+    pin = lambda t: t.contiguous().pin_memory()  # noqa: E731
+    ho = torch.empty_like(x["q"]).pin_memory()
+    hn = torch.empty((w.B, w.Hq, w.T)).pin_memory()
+    stg = torch.empty(pa.fwd_staging_size(w.B, w.T, w.Hq, w.Hkv), device="cuda", dtype=torch.uint8)
+    pa.fwd_host(pin(x["q"]), pin(x["k"]), pin(x["v"]), pin(x["u"]), ho, hn, stg, **p)
+    assert pa.get_status() == 0
+    assert torch.equal(ho, ref.cpu()) and torch.equal(hn, nref.cpu())
