@@ -459,8 +459,41 @@ def run_ours(args):
         if pa.get_status() != 0:
             raise RuntimeError("device status after the backward")
         t_b = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in eb) / 1e3, world, dev)
-        bwd_res = (wb, Kb, t_b)
-        del xb, gb, gq, gk, gv, gu, wsb
+
+        # The training pair: the forward that saves each row's state, then the
+        # backward from that state (no forward sweep in the backward).
+        ob = torch.empty_like(xb["q"])
+        nb = torch.empty((wb.B, wb.Hq, wb.T), device=dev, dtype=torch.float32)
+        sb = torch.empty((wb.B, wb.Hq, wb.T, 8), device=dev, dtype=torch.float32)
+
+        def forward_train():
+            pa.fwd_train(xb["q"], xb["k"], xb["v"], xb["u"], ob, nb, sb, stream=stream,
+                         s=wb.s, alpha=wb.alpha, L=wb.L, beta=wb.beta)
+
+        def backward_state():
+            pa.bwd_from_state(xb["q"], xb["k"], xb["v"], xb["u"], ob, sb, gb, gq, gk, gv, gu, wsb,
+                              stream=stream, s=wb.s, alpha=wb.alpha, L=wb.L, beta=wb.beta)
+
+        def timed(fn):
+            for _ in range(min(Wm, 3)):
+                fn()
+            ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(Kb)]
+            barrier(world, dev)
+            torch.cuda.synchronize(dev)
+            for i in range(Kb):
+                ev[i][0].record(stream)
+                fn()
+                ev[i][1].record(stream)
+            torch.cuda.synchronize(dev)
+            barrier(world, dev)
+            if pa.get_status() != 0:
+                raise RuntimeError("device status after the training pair")
+            return max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in ev) / 1e3, world, dev)
+
+        t_ft = timed(forward_train)
+        t_bs = timed(backward_state)
+        bwd_res = (wb, Kb, t_b, t_ft, t_bs)
+        del xb, gb, gq, gk, gv, gu, wsb, ob, nb, sb
 
     # ---- memory channel: chunked prefill and in-place decode step, timed on their own ----
     gd_res = None
@@ -622,7 +655,8 @@ def run_ours(args):
         dec_launch_s = t_dec / K
         tf = PREFILL.flops / pre_launch_s / 1e12 if do_pre else 0.0
         gbs = kv_bytes / dec_launch_s / 1e9 if do_dec else 0.0
-        sha_p = source_sha("fwd_tc.cu", "fwd_moments.cu", "polar_common.cuh", "tc_common.cuh")
+        sha_p = source_sha("fwd_tc.cu", "fwd_moments.cu", "polar_common.cuh", "tc_common.cuh",
+                           "bwd_coef.cuh")
         sha_d = source_sha("decode.cu", "polar_common.cuh")
         value = aggregate_throughput(PREFILL.flops * K, world, t_pre_max) / 1e12 if do_pre else 0.0
         dec_value = aggregate_throughput(kv_bytes * K, world, t_dec_max) / 1e9 if do_dec else 0.0
@@ -667,16 +701,31 @@ def run_ours(args):
             "e2e": e2e,
         }
         if bwd_res is not None:
-            wb, Kb, t_b = bwd_res
+            wb, Kb, t_b, t_ft, t_bs = bwd_res
             b_launch = t_b / Kb
             b_fl = 2.5 * wb.flops
             result["backward"] = {
                 "workload": wb.describe(), "value": b_fl / b_launch / 1e12, "unit": "TFLOP/s",
                 "ms_per_launch": b_launch * 1e3, "flops_per_launch": b_fl, "launches": Kb,
-                "note": "prefill backward (polar_attn_bwd: dq, dk, dv, du; mma.sync tensor cores for "
-                        "bf16 inputs), flops "
-                        "counted as 2.5x the forward's visible-pair flops; timed separately; not "
-                        "part of value"}
+                "note": "prefill backward that recomputes each row's forward state (polar_attn_bwd: "
+                        "dq, dk, dv, du; tcgen05 tensor cores for bf16 inputs), flops counted as "
+                        "2.5x the forward's visible-pair flops; timed separately; not part of value"}
+            ft_launch, bs_launch = t_ft / Kb, t_bs / Kb
+            result["training_pair"] = {
+                "workload": wb.describe(), "launches": Kb,
+                "forward_train": {"ms_per_launch": ft_launch * 1e3,
+                                  "value": wb.flops / ft_launch / 1e12, "unit": "TFLOP/s",
+                                  "flops_per_launch": wb.flops},
+                "backward_from_state": {"ms_per_launch": bs_launch * 1e3,
+                                        "value": b_fl / bs_launch / 1e12, "unit": "TFLOP/s",
+                                        "flops_per_launch": b_fl},
+                "step": {"ms_per_launch": (ft_launch + bs_launch) * 1e3,
+                         "value": 3.5 * wb.flops / (ft_launch + bs_launch) / 1e12,
+                         "unit": "TFLOP/s"},
+                "note": "polar_attn_fwd_train (forward that also saves each row's streaming state) "
+                        "then polar_attn_bwd_from_state (backward from out and that state, no "
+                        "forward sweep); flops: 1x and 2.5x the forward's visible-pair flops; "
+                        "timed separately; not part of value"}
         if gd_res is not None:
             wg, wst, Kg, t_gp, t_gs = gd_res
             sha_g = source_sha("gdelta.cu", "polar_common.cuh", "tc_common.cuh")

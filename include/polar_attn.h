@@ -161,8 +161,10 @@ polar_status_t polar_attn_fwd_ws(const void *q, const void *k, const void *v, co
  *  workspace  device scratch of at least polar_attn_bwd_workspace_size() bytes
  *             (per-row coefficients); contents on entry are ignored
  *
- * Computed on the CUDA cores in fp32; deterministic.  B = 0 or T = 0 writes
- * du = 0 and nothing else.
+ * bf16 inputs: the contractions run on the tensor cores (tcgen05, bf16
+ * operands, fp32 accumulation), with the weights, dS and dA rounded to bf16 as
+ * operands; fp32 inputs: the CUDA cores in fp32.  Deterministic: no atomics,
+ * fixed summation orders.  B = 0 or T = 0 writes du = 0 and nothing else.
  */
 size_t polar_attn_bwd_workspace_size(const polar_params_t *params);
 
@@ -170,6 +172,48 @@ polar_status_t polar_attn_bwd(const void *q, const void *k, const void *v, const
                               const void *dout, const polar_params_t *params, float *dq,
                               float *dk, float *dv, float *du, void *workspace, size_t ws_bytes,
                               void *stream);
+
+/*
+ * Training pair: a forward that also saves each row's streaming state, and a
+ * backward that starts from that state instead of recomputing the forward
+ * sweep.  The state is what the fused kernel already carries per row ("Fused
+ * Polar Attention Kernel", section 2.2 of the technical summary: the streaming
+ * sums l and l2, the max logit, the null floor's raw sums) plus |acc| and the
+ * first argmax key; the backward of section 3's training use needs nothing
+ * else besides out and dL/dout.
+ *
+ *  state  [B, Hq, T, 8] float32, device, 16-byte aligned, owned by the caller
+ *         (polar_attn_fwd_state_size bytes): per row l, l2 (weights relative
+ *         to the fixed reference c log2 e), max_j <q, k_j>, S1, S2, |acc|,
+ *         the first argmax key (int32 bits), 0.
+ *
+ * polar_attn_fwd_train writes out and neff_out as polar_attn_fwd does (equal up
+ * to rounding: it never uses the key moments) and the state.  Where the state
+ * path does not apply -- fp32 inputs, an odd group size Hq/Hkv, a logit scale
+ * times length temperature above 28/log2(e) (the fixed reference's range),
+ * params->impl = POLAR_IMPL_SIMT -- it is exactly polar_attn_fwd and leaves
+ * `state` untouched; polar_attn_bwd_from_state, given the same params, then
+ * recomputes the rows as polar_attn_bwd does.  So the pair is valid for every
+ * shape polar_attn_fwd accepts.
+ *
+ * polar_attn_bwd_from_state: arguments, outputs, workspace and errors as
+ * polar_attn_bwd, plus out (the training forward's output, [B, T, Hq, 64]
+ * dtype) and its state, both unchanged since that call with the same params
+ * and inputs.  With the state it runs a rows kernel over (row, head) in place
+ * of the forward sweep; the direction comes from out - count * u_h, so dA
+ * carries out's bf16 rounding.  Asynchronous on `stream`.
+ */
+size_t polar_attn_fwd_state_size(const polar_params_t *params);
+
+polar_status_t polar_attn_fwd_train(const void *q, const void *k, const void *v, const float *u,
+                                    const polar_params_t *params, void *out, float *neff_out,
+                                    float *state, void *stream);
+
+polar_status_t polar_attn_bwd_from_state(const void *q, const void *k, const void *v,
+                                         const float *u, const void *out, const float *state,
+                                         const void *dout, const polar_params_t *params,
+                                         float *dq, float *dk, float *dv, float *du,
+                                         void *workspace, size_t ws_bytes, void *stream);
 
 /* Bytes of device staging that polar_attn_fwd_host needs for this shape
  * (inputs, outputs and the workspace of polar_attn_fwd_ws). */

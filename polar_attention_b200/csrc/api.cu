@@ -154,7 +154,7 @@ FwdLaunch make_fwd(const void *q, const void *k, const void *v, const float *u,
     a.B = p->B; a.T = p->T; a.Hq = p->Hq; a.Hkv = p->Hkv; a.dtype = p->dtype;
     a.s = p->logit_scale; a.alpha = p->alpha; a.beta = p->beta; a.L = p->L_train;
     a.window = p->window;
-    a.status = status; a.moments = nullptr; a.stream = stream;
+    a.status = status; a.moments = nullptr; a.state = nullptr; a.stream = stream;
     return a;
 }
 
@@ -284,6 +284,68 @@ polar_status_t polar_attn_bwd(const void *q, const void *k, const void *v, const
     a.s = p->logit_scale; a.alpha = p->alpha; a.beta = p->beta; a.L = p->L_train;
     a.window = p->window; a.workspace = workspace; a.status = status; a.stream = s;
     return from_cuda(launch_bwd(a));
+}
+
+size_t polar_attn_fwd_state_size(const polar_params_t *p) {
+    if (check_fwd(p) != POLAR_OK) return 0;
+    return static_cast<size_t>(p->B) * p->Hq * p->T * kFwdStateWords * sizeof(float);
+}
+
+polar_status_t polar_attn_fwd_train(const void *q, const void *k, const void *v, const float *u,
+                                    const polar_params_t *params, void *out, float *neff_out,
+                                    float *state, void *stream) {
+    polar_status_t st = check_fwd(params);
+    if (st != POLAR_OK) return st;
+    if (params->B == 0 || params->T == 0) return POLAR_OK;
+    if (!state || !aligned16(state)) return POLAR_ERR_INVALID_ARG;
+    const int sup = fwd_state_supported(params->dtype, params->T, params->Hq, params->Hkv,
+                                        params->logit_scale, params->alpha, params->L_train,
+                                        params->window);
+    if (sup < 0) return POLAR_ERR_CUDA;
+    // No saved state for this shape: the plain forward (the backward then
+    // recomputes the rows).
+    if (sup == 0 || params->impl == POLAR_IMPL_SIMT)
+        return polar_attn_fwd_ws(q, k, v, u, params, out, neff_out, nullptr, 0, stream);
+    if (!q || !k || !v || !u || !out) return POLAR_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(u) || !aligned16(out) ||
+        (neff_out && (reinterpret_cast<uintptr_t>(neff_out) & 3u)))
+        return POLAR_ERR_INVALID_ARG;
+    int *status = status_ptr();
+    if (!status) return POLAR_ERR_CUDA;
+    FwdLaunch a = make_fwd(q, k, v, u, params, out, neff_out, status,
+                           static_cast<cudaStream_t>(stream));
+    a.state = state;
+    return from_cuda(launch_fwd_train_tc(a));
+}
+
+polar_status_t polar_attn_bwd_from_state(const void *q, const void *k, const void *v,
+                                         const float *u, const void *out, const float *state,
+                                         const void *dout, const polar_params_t *p, float *dq,
+                                         float *dk, float *dv, float *du, void *workspace,
+                                         size_t ws_bytes, void *stream) {
+    polar_status_t st = check_fwd(p);
+    if (st != POLAR_OK) return st;
+    if (!du || !aligned16(du)) return POLAR_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (p->B == 0 || p->T == 0)
+        return from_cuda(cudaMemsetAsync(du, 0, static_cast<size_t>(p->Hq) * kHeadDim * 4, s));
+    if (!q || !k || !v || !u || !out || !state || !dout || !dq || !dk || !dv || !workspace)
+        return POLAR_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(u) || !aligned16(out) ||
+        !aligned16(state) || !aligned16(dout) || !aligned16(dq) || !aligned16(dk) ||
+        !aligned16(dv) || !aligned16(workspace))
+        return POLAR_ERR_INVALID_ARG;
+    if (ws_bytes < bwd_workspace_bytes(p->B, p->T, p->Hq)) return POLAR_ERR_WORKSPACE;
+    int *status = status_ptr();
+    if (!status) return POLAR_ERR_CUDA;
+    BwdLaunch a;
+    a.q = q; a.k = k; a.v = v; a.dout = dout; a.u = u;
+    a.dq = dq; a.dk = dk; a.dv = dv; a.du = du;
+    a.B = p->B; a.T = p->T; a.Hq = p->Hq; a.Hkv = p->Hkv; a.dtype = p->dtype;
+    a.s = p->logit_scale; a.alpha = p->alpha; a.beta = p->beta; a.L = p->L_train;
+    a.window = p->window; a.workspace = workspace; a.status = status; a.stream = s;
+    if (p->impl == POLAR_IMPL_SIMT) return from_cuda(launch_bwd(a));
+    return from_cuda(launch_bwd_from_state(a, out, state));
 }
 
 size_t polar_attn_fwd_staging_size(const polar_params_t *p) {

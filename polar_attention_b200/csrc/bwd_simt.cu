@@ -36,6 +36,7 @@
 // test is an index comparison.
 #include <type_traits>
 
+#include "bwd_coef.cuh"
 #include "polar_common.cuh"
 #include "polar_internal.h"
 
@@ -780,6 +781,162 @@ bwd_du_part_kernel(const __nv_bfloat16 *__restrict__ gout, const BwdArgs a) {
     }
 }
 
+// Rows kernel of the backward from a training forward's saved state (bf16):
+// per (row, head), the coefficient record and dA from the row's saved
+// streaming state, out and g = dL/dout, without the forward sweep.  With
+// count = gate * T from the state, content = out - count * u_h (out rounded to
+// bf16, as the forward stored it), <content, g> = <out, g> - count <g, u_h>
+// and dA = (g - content <content, g>) / |acc|.
+// A block takes 16 rows of one batch and up to 8 heads (blockIdx.z: head
+// group), in three phases:
+//  A. eight threads per (row, head), each with 8 of the 64 components, load
+//     g and out (all of a thread's rows at once) and reduce <out, g> and
+//     <g, u_h> among themselves;
+//  B. one thread per (row, head) turns the saved state into the magnitude
+//     channel's scalars and writes the record;
+//  C. the eight threads write dA and sum count * g into the du partials (the
+//     16-row blocks of bwd_du_part_kernel).
+// Rows T .. Tpad - 1 get the null record and dA = 0.
+constexpr int kStHeads = 8;                           // heads per block
+constexpr int kStChunks = kStHeads * (kHeadDim / 8);  // 64 (head, 8-component) chunks
+constexpr int kStGroups = 256 / kStChunks;            // 4 row groups of 64 threads
+constexpr int kStRowsPerThread = kDuRows / kStGroups; // rows rg, rg + 4, rg + 8, rg + 12
+__global__ void __launch_bounds__(256, 2)
+bwd_state_rows_kernel(const __nv_bfloat16 *__restrict__ out, const __nv_bfloat16 *__restrict__ gout,
+                      const float *__restrict__ state, const BwdArgs a) {
+    __shared__ float s_og[kDuRows][kStHeads], s_gu[kDuRows][kStHeads];
+    __shared__ float s_gt[kDuRows][kStHeads], s_cg[kDuRows][kStHeads], s_ia[kDuRows][kStHeads];
+    __shared__ __align__(16) float s_du[kStGroups - 1][kStChunks][8];
+    const int blk = blockIdx.x, b = blockIdx.y, h0 = blockIdx.z * kStHeads;
+    const int nh = min(kStHeads, a.Hq - h0);
+    const int r0 = blk * kDuRows;
+    const int t = threadIdx.x, c = t % kStChunks, rg = t / kStChunks;
+    const int hl = c >> 3, h = h0 + hl, d0 = (c & 7) * 8;
+    const bool act = hl < nh;
+    const size_t rstride = static_cast<size_t>(a.Hq) * kHeadDim;
+    float uu[8];
+    {
+        const float *up = a.u + static_cast<size_t>(act ? h : h0) * kHeadDim + d0;
+        const float4 u0 = *reinterpret_cast<const float4 *>(up);
+        const float4 u1 = *reinterpret_cast<const float4 *>(up + 4);
+        uu[0] = u0.x; uu[1] = u0.y; uu[2] = u0.z; uu[3] = u0.w;
+        uu[4] = u1.x; uu[5] = u1.y; uu[6] = u1.z; uu[7] = u1.w;
+    }
+    // The saved state of this thread's (row, head) of phase B, loaded with
+    // phase A's loads.
+    const int brl = t / kStHeads, bhb = t % kStHeads, brow = r0 + brl, bh = h0 + bhb;
+    const bool bact = t < kDuRows * kStHeads && bhb < nh && brow < a.Tpad;
+    float4 st0 = make_float4(0.f, 0.f, 0.f, 0.f), st1 = st0;
+    if (bact && brow < a.T) {
+        const float4 *sp = reinterpret_cast<const float4 *>(
+            state + ((static_cast<size_t>(b) * a.Hq + bh) * a.T + brow) * kFwdStateWords);
+        st0 = sp[0];
+        st1 = sp[1];
+    }
+    // A: every load first, then the 8-lane reductions.
+    uint4 gw[kStRowsPerThread], ow[kStRowsPerThread];
+#pragma unroll
+    for (int i = 0; i < kStRowsPerThread; ++i) {
+        const int row = r0 + rg + kStGroups * i;
+        const bool live = act && row < a.T;
+        const size_t off = (static_cast<size_t>(b) * a.T + (live ? row : 0)) * rstride +
+                           static_cast<size_t>(live ? h : 0) * kHeadDim + d0;
+        gw[i] = live ? *reinterpret_cast<const uint4 *>(gout + off) : make_uint4(0u, 0u, 0u, 0u);
+        ow[i] = live ? *reinterpret_cast<const uint4 *>(out + off) : make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int i = 0; i < kStRowsPerThread; ++i) {
+        const uint32_t g4[4] = {gw[i].x, gw[i].y, gw[i].z, gw[i].w};
+        const uint32_t o4[4] = {ow[i].x, ow[i].y, ow[i].z, ow[i].w};
+        float og = 0.f, gu = 0.f;
+#pragma unroll
+        for (int x = 0; x < 4; ++x) {
+            const float g0 = __uint_as_float(g4[x] << 16), g1 = __uint_as_float(g4[x] & 0xFFFF0000u);
+            og = fmaf(__uint_as_float(o4[x] << 16), g0, og);
+            og = fmaf(__uint_as_float(o4[x] & 0xFFFF0000u), g1, og);
+            gu = fmaf(g0, uu[2 * x], gu);
+            gu = fmaf(g1, uu[2 * x + 1], gu);
+        }
+#pragma unroll
+        for (int o = 1; o < 8; o <<= 1) {
+            og += __shfl_xor_sync(0xffffffffu, og, o);
+            gu += __shfl_xor_sync(0xffffffffu, gu, o);
+        }
+        if ((c & 7) == 0) {
+            s_og[rg + kStGroups * i][hl] = og;
+            s_gu[rg + kStGroups * i][hl] = gu;
+        }
+    }
+    __syncthreads();
+    // B: one (row, head) per thread.
+    if (bact) {
+        const size_t rrow = (static_cast<size_t>(b) * a.Hq + bh) * a.Tpad + brow;
+        float gt = 0.f, cg = 0.f, ia = 0.f;
+        if (brow < a.T) {
+            const float l = st0.x, l2 = st0.y;
+            const float n = static_cast<float>(a.window > 0 ? min(brow + 1, a.window) : brow + 1);
+            const float cc = a.s * length_temperature(n, a.alpha, a.L);
+            const RowMag m = row_mag(l, l2, st0.z, st0.w, st1.x, cc, n, a.beta, a.inv_ln_L);
+            const float gu = s_gu[brl][bhb];
+            gt = m.gate * m.Tm;
+            cg = s_og[brl][bhb] - gt * gu;  // <content, g>
+            ia = 1.0f / st1.y;
+            const int lo = a.window > 0 ? max(0, brow - a.window + 1) : 0;
+            store_coef_record(a.coef + rrow * kBwdCoefWords, true, m, gu, l, l2, cc, cc * kLog2e, n,
+                              a.beta, a.inv_ln_L, __float_as_int(st1.z), lo);
+        } else {
+            store_coef_record(a.coef + rrow * kBwdCoefWords, false, RowMag{}, 0.f, 0.f, 0.f, 0.f, 0.f,
+                              1.f, a.beta, a.inv_ln_L, -1, 0);
+        }
+        s_gt[brl][bhb] = gt;
+        s_cg[brl][bhb] = cg;
+        s_ia[brl][bhb] = ia;
+    }
+    __syncthreads();
+    // C: dA and the du partials.
+    float du[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int i = 0; i < kStRowsPerThread; ++i) {
+        const int rl = rg + kStGroups * i, row = r0 + rl;
+        if (!act || row >= a.Tpad) continue;
+        const size_t rrow = (static_cast<size_t>(b) * a.Hq + h) * a.Tpad + row;
+        uint4 *dst = reinterpret_cast<uint4 *>(a.dab + rrow * kHeadDim + d0);
+        if (row >= a.T) {
+            *dst = make_uint4(0u, 0u, 0u, 0u);
+            continue;
+        }
+        const float gt = s_gt[rl][hl], cg = s_cg[rl][hl], ia = s_ia[rl][hl];
+        const uint32_t g4[4] = {gw[i].x, gw[i].y, gw[i].z, gw[i].w};
+        const uint32_t o4[4] = {ow[i].x, ow[i].y, ow[i].z, ow[i].w};
+        uint32_t d[4];
+#pragma unroll
+        for (int x = 0; x < 4; ++x) {
+            const float g0 = __uint_as_float(g4[x] << 16), g1 = __uint_as_float(g4[x] & 0xFFFF0000u);
+            const float c0v = fmaf(-gt, uu[2 * x], __uint_as_float(o4[x] << 16));
+            const float c1v = fmaf(-gt, uu[2 * x + 1], __uint_as_float(o4[x] & 0xFFFF0000u));
+            d[x] = pk2((g0 - c0v * cg) * ia, (g1 - c1v * cg) * ia);
+            du[2 * x] = fmaf(gt, g0, du[2 * x]);
+            du[2 * x + 1] = fmaf(gt, g1, du[2 * x + 1]);
+        }
+        *dst = make_uint4(d[0], d[1], d[2], d[3]);
+    }
+    if (rg > 0) {
+        *reinterpret_cast<float4 *>(&s_du[rg - 1][c][0]) = make_float4(du[0], du[1], du[2], du[3]);
+        *reinterpret_cast<float4 *>(&s_du[rg - 1][c][4]) = make_float4(du[4], du[5], du[6], du[7]);
+    }
+    __syncthreads();
+    if (rg == 0 && act) {
+#pragma unroll
+        for (int g = 0; g < kStGroups - 1; ++g)
+#pragma unroll
+            for (int x = 0; x < 8; ++x) du[x] += s_du[g][c][x];
+        float4 *dp = reinterpret_cast<float4 *>(
+            a.du_part + ((static_cast<size_t>(b) * gridDim.x + blk) * a.Hq + h) * kHeadDim + d0);
+        dp[0] = make_float4(du[0], du[1], du[2], du[3]);
+        dp[1] = make_float4(du[4], du[5], du[6], du[7]);
+    }
+}
+
 // du_h = sum over the row blocks of their partial sums: sixteen interleaved
 // slices of the partials per head, then the slices, all in a fixed order.
 constexpr int kDuSlices = 16;
@@ -860,7 +1017,9 @@ size_t bwd_workspace_bytes(int B, int T, int Hq) {
     return fp32 > bf16 ? fp32 : bf16;
 }
 
-cudaError_t launch_bwd(const BwdLaunch &l) {
+namespace {
+
+BwdArgs make_args(const BwdLaunch &l) {
     BwdArgs a;
     a.u = l.u;
     a.B = l.B; a.T = l.T; a.Hq = l.Hq; a.Hkv = l.Hkv; a.window = l.window;
@@ -880,8 +1039,37 @@ cudaError_t launch_bwd(const BwdLaunch &l) {
     }
     a.s = l.s; a.alpha = l.alpha; a.L = static_cast<float>(l.L); a.beta = l.beta;
     a.inv_ln_L = 1.0f / logf(static_cast<float>(l.L));
+    return a;
+}
+
+}  // namespace
+
+cudaError_t launch_bwd(const BwdLaunch &l) {
+    const BwdArgs a = make_args(l);
     if (l.B == 0 || l.T == 0) return cudaSuccess;
     return l.dtype == POLAR_FP32 ? launch_all<float>(l, a) : launch_all<__nv_bfloat16>(l, a);
+}
+
+// From a training forward's saved state: the state rows kernel (record, dA and
+// du partials), the tensor-core dK/dV and dQ passes, du.  Where the training
+// forward saved no state (fwd_state_supported false for this shape), the rows
+// are recomputed as in launch_bwd.
+cudaError_t launch_bwd_from_state(const BwdLaunch &l, const void *out, const float *state) {
+    const int sup = fwd_state_supported(l.dtype, l.T, l.Hq, l.Hkv, l.s, l.alpha, l.L, l.window);
+    if (sup < 0) return cudaErrorUnknown;
+    if (sup == 0) return launch_bwd(l);
+    const BwdArgs a = make_args(l);
+    if (l.B == 0 || l.T == 0) return cudaSuccess;
+    bwd_state_rows_kernel<<<dim3(a.Tpad / kDuRows, a.B, (a.Hq + kStHeads - 1) / kStHeads), 256, 0,
+                            l.stream>>>(
+        static_cast<const __nv_bfloat16 *>(out), static_cast<const __nv_bfloat16 *>(l.dout), state, a);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    e = launch_bwd_tc(l, a.coef, a.dab);
+    if (e != cudaSuccess) return e;
+    bwd_du_kernel<<<a.Hq, kDuSlices * kHeadDim, 0, l.stream>>>(l.du, a, a.B * (a.Tpad / kDuRows));
+    count_launches(2);
+    return cudaGetLastError();
 }
 
 }  // namespace polar

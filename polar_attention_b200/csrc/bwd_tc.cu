@@ -34,6 +34,7 @@
 // bounded (mbar_wait): on a timeout the kernel records POLAR_ERR_TIMEOUT and
 // leaves its loop.
 #include <atomic>
+#include <mutex>
 
 #include "polar_common.cuh"
 #include "polar_internal.h"
@@ -810,6 +811,33 @@ bwd_dq2_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
     }
 }
 
+// A second stream per device for the dQ pass, which depends on the dK/dV
+// pass for nothing: the two run side by side, so the dQ CTAs fill the SMs
+// that the dK/dV pass's last wave leaves idle.  The mutex keeps one caller's
+// fork (record, wait) and join from interleaving with another's.
+struct SideStream {
+    cudaStream_t s = nullptr;
+    cudaEvent_t fork = nullptr, join = nullptr;
+    std::mutex mu;
+    bool ready = false;
+};
+
+SideStream *side_stream(int dev) {
+    static SideStream ss[64];
+    static std::mutex init_mu;
+    if (dev < 0 || dev >= 64) return nullptr;
+    SideStream &x = ss[dev];
+    std::lock_guard<std::mutex> lk(init_mu);
+    if (!x.ready) {
+        if (cudaStreamCreateWithFlags(&x.s, cudaStreamNonBlocking) != cudaSuccess ||
+            cudaEventCreateWithFlags(&x.fork, cudaEventDisableTiming) != cudaSuccess ||
+            cudaEventCreateWithFlags(&x.join, cudaEventDisableTiming) != cudaSuccess)
+            return nullptr;
+        x.ready = true;
+    }
+    return &x;
+}
+
 }  // namespace
 
 cudaError_t launch_bwd_tc(const BwdLaunch &l, const float *coef, const void *dab) {
@@ -883,16 +911,26 @@ cudaError_t launch_bwd_tc(const BwdLaunch &l, const float *coef, const void *dab
     const long long kv_ctas = static_cast<long long>(a.nt) * l.Hkv * l.B;
     const long long q_ctas = static_cast<long long>(a.nt) * l.Hq * l.B;
     if (kv_ctas > 0x7fffffffll || q_ctas > 0x7fffffffll) return cudaErrorInvalidValue;
+    SideStream *ss = side_stream(dev);
+    if (!ss) return cudaErrorUnknown;
+    std::lock_guard<std::mutex> lk(ss->mu);
+    e = cudaEventRecord(ss->fork, l.stream);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(ss->s, ss->fork, 0);
+    if (e != cudaSuccess) return e;
     bwd_dkdv_tc_kernel<<<static_cast<unsigned>(kv_ctas), 384, kDkdvSmem, l.stream>>>(tq, tk, tv,
                                                                                      tda, a);
     if (a.G % 2 == 0)  // head pairs share each K/V tile
-        bwd_dq2_tc_kernel<<<static_cast<unsigned>(q_ctas / 2), 384, kDq2Smem, l.stream>>>(tq, tk,
-                                                                                           tv, tda, a);
+        bwd_dq2_tc_kernel<<<static_cast<unsigned>(q_ctas / 2), 384, kDq2Smem, ss->s>>>(tq, tk, tv,
+                                                                                        tda, a);
     else
-        bwd_dq_tc_kernel<<<static_cast<unsigned>(q_ctas), 384, kDqSmem, l.stream>>>(tq, tk, tv,
-                                                                                     tda, a);
+        bwd_dq_tc_kernel<<<static_cast<unsigned>(q_ctas), 384, kDqSmem, ss->s>>>(tq, tk, tv, tda, a);
+    e = cudaGetLastError();
+    // Join even after a failed launch, so that the caller's stream never runs
+    // ahead of work already queued on the side stream.
+    const cudaError_t ej = cudaEventRecord(ss->join, ss->s);
+    const cudaError_t ew = ej == cudaSuccess ? cudaStreamWaitEvent(l.stream, ss->join, 0) : ej;
     count_launches(2);
-    return cudaGetLastError();
+    return e != cudaSuccess ? e : ew;
 }
 
 }  // namespace polar

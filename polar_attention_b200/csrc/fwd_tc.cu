@@ -31,6 +31,7 @@
 #include <algorithm>
 #include <atomic>
 
+#include "bwd_coef.cuh"
 #include "polar_attn_selftest.h"
 #include "polar_common.cuh"
 #include "polar_internal.h"
@@ -327,11 +328,14 @@ struct TcArgs {
     float *coef;
     __nv_bfloat16 *dab;
     int Tpad;
+    // Training forward (kSave) only: the saved row state [B][Hq][T][kFwdStateWords].
+    float *state;
 };
 
 // Epilogue of one row: content = O/|O|, the magnitude channel from the row's
 // streaming state, out = content + count (bf16, 128-bit stores) and n_eff.
-__device__ __forceinline__ void store_row(const uint32_t (&o)[2][32], float l, float l2,
+// Returns |O| (floored at 1e-30).
+__device__ __forceinline__ float store_row(const uint32_t (&o)[2][32], float l, float l2,
                                           float m_raw, float s1, float s2, float c, float n,
                                           const TcArgs &a, int b, int row, int h) {
     float ne;
@@ -344,7 +348,7 @@ __device__ __forceinline__ void store_row(const uint32_t (&o)[2][32], float l, f
             const float x = __uint_as_float(o[hh][e]);
             nrm = fmaf(x, x, nrm);
         }
-    const float inv = 1.0f / fmaxf(sqrtf(nrm), 1e-30f);
+    const float an = fmaxf(sqrtf(nrm), 1e-30f), inv = 1.0f / an;
     const float4 *u4 = reinterpret_cast<const float4 *>(a.u + static_cast<size_t>(h) * kHeadDim);
     uint4 *dst = reinterpret_cast<uint4 *>(a.out + ((static_cast<size_t>(b) * a.T + row) * a.Hq + h) *
                                                        kHeadDim);
@@ -363,6 +367,7 @@ __device__ __forceinline__ void store_row(const uint32_t (&o)[2][32], float l, f
         dst[ch] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
     }
     if (a.neff) a.neff[(static_cast<size_t>(b) * a.Hq + h) * a.T + row] = ne;
+    return an;
 }
 
 // Epilogue of one row of the backward's rows pass (kRows): with content =
@@ -406,26 +411,9 @@ __device__ __forceinline__ void store_rec(uint32_t tO, float l, float l2, float 
         }
     }
     const float nf = live ? n : 1.0f;
-    const float mean_s = s1 / nf;
-    const float sig_s = sqrtf(fmaxf(s2 / nf - mean_s * mean_s, 0.0f));
-    const float mu = c * mean_s, sigma = c * sig_s;
-    const float kn = sqrtf(2.0f * logf(nf));
-    const float z0 = mu + sigma * kn;
-    const float gate = 1.0f / (1.0f + expf(-a.beta * (c * m_raw - z0)));
-    const float ne_raw = (l * l) / l2;
-    const float ne = fminf(fmaxf(ne_raw, 1.0f), nf);
-    const bool clamped = ne != ne_raw;
-    const float Tm = tanhf(logf(ne) * a.inv_ln_L);
+    const RowMag m = row_mag(l, l2, m_raw, s1, s2, c, nf, a.beta, a.inv_ln_L);
     const float an = fmaxf(sqrtf(nrm), 1e-30f), inv_an = 1.0f / an;
     const float cg = og * inv_an;  // <content, g>
-    const float dgate = gu * Tm, dT = gu * gate;
-    const float dneff = clamped ? 0.0f : dT * (1.0f - Tm * Tm) * a.inv_ln_L / ne;
-    const float dl = 2.0f * dneff * l / l2;
-    const float dl2 = -dneff * (l / l2) * (l / l2);
-    const float dm = a.beta * gate * (1.0f - gate) * dgate;
-    const float dsigma = -dm * kn;
-    const float cmu = -dm / nf - (sigma > 0.0f ? dsigma * mu / (nf * sigma) : 0.0f);
-    const float csS = sigma > 0.0f ? dsigma * c / (nf * sigma) : 0.0f;
     // Pass 2: dA = (g - O cg / |O|) / |O|.
     uint4 *dst = reinterpret_cast<uint4 *>(a.dab + rrow * kHeadDim);
     const float sc = inv_an * cg;
@@ -448,17 +436,8 @@ __device__ __forceinline__ void store_rec(uint32_t tO, float l, float l2, float 
         dst[2 * ch] = make_uint4(d[0], d[1], d[2], d[3]);
         dst[2 * ch + 1] = make_uint4(d[4], d[5], d[6], d[7]);
     }
-    float4 *cr = reinterpret_cast<float4 *>(a.coef + rrow * kBwdCoefWords);
-    if (live) {
-        cr[0] = make_float4(cl2, -cl2, c, c * dl);
-        cr[1] = make_float4(2.0f * c * dl2, c * csS, c * cmu, c * dm);
-        cr[2] = make_float4(__int_as_float(jarg), __int_as_float(lo), gate * Tm, 0.f);
-    } else {
-        cr[0] = make_float4(0.f, -INFINITY, 0.f, 0.f);
-        cr[1] = make_float4(0.f, 0.f, 0.f, 0.f);
-        cr[2] = make_float4(__int_as_float(-1), __int_as_float(0), 0.f, 0.f);
-    }
-    cr[3] = make_float4(0.f, 0.f, 0.f, 0.f);
+    store_coef_record(a.coef + rrow * kBwdCoefWords, live, m, gu, l, l2, c, cl2, nf, a.beta,
+                      a.inv_ln_L, jarg, lo);
 }
 
 // kFixedRef: the exponentials use the fixed per-row reference m_ref = c*log2e,
@@ -485,7 +464,11 @@ __device__ __forceinline__ void store_rec(uint32_t tO, float l, float l2, float 
 // kRows: the backward's rows pass -- the same forward sweep, which also finds
 // each row's first argmax key, and the store_rec epilogue in place of the
 // output (split rows, fixed reference, no key moments).
-template <bool kFixedRef, int kSplit, bool kMoments, bool kWindow, bool kRows = false>
+// kSave: the training forward -- the rows pass's sweep (with the argmax) and
+// the forward's output, plus each row's streaming state (FwdState layout) for
+// the backward.
+template <bool kFixedRef, int kSplit, bool kMoments, bool kWindow, bool kRows = false,
+          bool kSave = false>
 __global__ void __launch_bounds__(128 + 256 * kSplit, 1)
 fwd_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
               const __grid_constant__ CUtensorMap tv, const TcArgs a) {
@@ -508,6 +491,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CU
     static_assert(kSplit == 1 || kFixedRef, "split rows need the fixed reference");
     static_assert(!kMoments || kSplit == 2, "key moments are used by the split rows only");
     static_assert(!kRows || (kSplit == 2 && !kMoments), "the rows pass runs the split sweep");
+    static_assert(!kSave || (kSplit == 2 && !kMoments && !kRows), "the training forward runs the split sweep");
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -739,7 +723,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CU
         const float m_ref = cl2;
         const float2 sc2 = make_float2(cl2, cl2);
         float m_raw = -INFINITY, l = 0.f, l2 = 0.f, s1 = 0.f, s2 = 0.f;
-        int jarg = -1;  // kRows: the first key of the row's max raw dot
+        int jarg = -1;  // kRows, kSave: the first key of the row's max raw dot
         bool ok = true;
         for (int j = 0; j < nkv; ++j) {
             ok = mbar_wait(&s_full[slot], j & 1, a.status);
@@ -753,7 +737,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CU
             mbar_arrive(&s_free[slot]);
             uint32_t pk[2][16];
             float tmax, ts1, ts2, tl, tl2;
-            if constexpr (kRows) {
+            if constexpr (kRows || kSave) {
                 // A strictly larger tile max moves the argmax to this tile: its
                 // first visible key holding that value (keys in ascending order).
                 int idx = -1;
@@ -844,7 +828,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CU
         }
         named_barrier(1 + slot, 256);
         if (half == 0) {
-            if constexpr (kRows) {
+            if constexpr (kRows || kSave) {
                 // The upper half's keys of a tile follow the lower half's, but tiles
                 // interleave: on a tie the smaller key index is the first argmax.
                 const float om = part[slot][t][0];
@@ -867,7 +851,15 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CU
                     tmem_ld32(tO, o[0]);
                     tmem_ld32(tO + 32, o[1]);
                     tmem_wait_ld();
-                    if (row < a.T) store_row(o, l, l2, m_raw, s1, s2, c, n, a, b, row, h);
+                    if (row < a.T) {
+                        const float an = store_row(o, l, l2, m_raw, s1, s2, c, n, a, b, row, h);
+                        if constexpr (kSave) {
+                            float4 *st = reinterpret_cast<float4 *>(
+                                a.state + ((static_cast<size_t>(b) * a.Hq + h) * a.T + row) * kFwdStateWords);
+                            st[0] = make_float4(l, l2, m_raw, s1);
+                            st[1] = make_float4(s2, an, __int_as_float(jarg), 0.f);
+                        }
+                    }
                 }
             }
         }
@@ -1008,6 +1000,24 @@ __global__ void selftest_exp2_kernel(const float2 *x, float2 *poly, float2 *mufu
     mufu[i] = make_float2(ex2(v.x), ex2(v.y));
 }
 
+// Tensor maps of q [B, T, Hq, 64] and k, v [B, T, Hkv, 64] bf16 as 4-D tensors
+// (d, head, t, b): tiles of 128 rows x 64 with the 128-byte swizzle.
+bool make_qkv_maps(const void *q, const void *k, const void *v, int B, int T, int Hq, int Hkv,
+                   CUtensorMap *tq, CUtensorMap *tk, CUtensorMap *tv) {
+    const uint32_t box[4] = {kHeadDim, 1, 128, 1};
+    const uint64_t qdims[4] = {kHeadDim, (uint64_t)Hq, (uint64_t)T, (uint64_t)B};
+    const uint64_t qstr[3] = {kHeadDim * 2ull, (uint64_t)Hq * kHeadDim * 2, (uint64_t)T * Hq * kHeadDim * 2};
+    const uint64_t kdims[4] = {kHeadDim, (uint64_t)Hkv, (uint64_t)T, (uint64_t)B};
+    const uint64_t kstr[3] = {kHeadDim * 2ull, (uint64_t)Hkv * kHeadDim * 2,
+                              (uint64_t)T * Hkv * kHeadDim * 2};
+    return encode_tiled(tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(q), qdims, qstr, box,
+                        CU_TENSOR_MAP_SWIZZLE_128B) == CUDA_SUCCESS &&
+           encode_tiled(tk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(k), kdims, kstr, box,
+                        CU_TENSOR_MAP_SWIZZLE_128B) == CUDA_SUCCESS &&
+           encode_tiled(tv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(v), kdims, kstr, box,
+                        CU_TENSOR_MAP_SWIZZLE_128B) == CUDA_SUCCESS;
+}
+
 }  // namespace
 
 cudaError_t launch_fwd_tc(const FwdLaunch &a) {
@@ -1046,25 +1056,7 @@ cudaError_t launch_fwd_tc(const FwdLaunch &a) {
     }
     // [B, T, H, 64] bf16 as a 4-D tensor (d, head, t, b); tiles of 128 rows x 64.
     CUtensorMap tq, tk, tv;
-    const uint32_t box[4] = {kHeadDim, 1, 128, 1};
-    {
-        const uint64_t dims[4] = {kHeadDim, (uint64_t)a.Hq, (uint64_t)a.T, (uint64_t)a.B};
-        const uint64_t str[3] = {kHeadDim * 2ull, (uint64_t)a.Hq * kHeadDim * 2,
-                                 (uint64_t)a.T * a.Hq * kHeadDim * 2};
-        if (encode_tiled(&tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(a.q), dims, str,
-                         box, CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS)
-            return cudaErrorInvalidValue;
-    }
-    {
-        const uint64_t dims[4] = {kHeadDim, (uint64_t)a.Hkv, (uint64_t)a.T, (uint64_t)a.B};
-        const uint64_t str[3] = {kHeadDim * 2ull, (uint64_t)a.Hkv * kHeadDim * 2,
-                                 (uint64_t)a.T * a.Hkv * kHeadDim * 2};
-        if (encode_tiled(&tk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(a.k), dims, str,
-                         box, CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS ||
-            encode_tiled(&tv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(a.v), dims, str,
-                         box, CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS)
-            return cudaErrorInvalidValue;
-    }
+    if (!make_qkv_maps(a.q, a.k, a.v, a.B, a.T, a.Hq, a.Hkv, &tq, &tk, &tv)) return cudaErrorInvalidValue;
     TcArgs ta = {};
     ta.u = a.u;
     ta.out = static_cast<__nv_bfloat16 *>(a.out);
@@ -1144,25 +1136,7 @@ cudaError_t launch_bwd_rows_tc(const BwdLaunch &l, float *coef, void *dab, int T
     }
     if (!(plan_ok.load() & bit)) return cudaErrorNotSupported;
     CUtensorMap tq, tk, tv;
-    const uint32_t box[4] = {kHeadDim, 1, 128, 1};
-    {
-        const uint64_t dims[4] = {kHeadDim, (uint64_t)l.Hq, (uint64_t)l.T, (uint64_t)l.B};
-        const uint64_t str[3] = {kHeadDim * 2ull, (uint64_t)l.Hq * kHeadDim * 2,
-                                 (uint64_t)l.T * l.Hq * kHeadDim * 2};
-        if (encode_tiled(&tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(l.q), dims, str,
-                         box, CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS)
-            return cudaErrorInvalidValue;
-    }
-    {
-        const uint64_t dims[4] = {kHeadDim, (uint64_t)l.Hkv, (uint64_t)l.T, (uint64_t)l.B};
-        const uint64_t str[3] = {kHeadDim * 2ull, (uint64_t)l.Hkv * kHeadDim * 2,
-                                 (uint64_t)l.T * l.Hkv * kHeadDim * 2};
-        if (encode_tiled(&tk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(l.k), dims, str,
-                         box, CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS ||
-            encode_tiled(&tv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(l.v), dims, str,
-                         box, CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS)
-            return cudaErrorInvalidValue;
-    }
+    if (!make_qkv_maps(l.q, l.k, l.v, l.B, l.T, l.Hq, l.Hkv, &tq, &tk, &tv)) return cudaErrorInvalidValue;
     TcArgs ta = {};
     ta.u = l.u;
     ta.status = l.status;
@@ -1184,6 +1158,81 @@ cudaError_t launch_bwd_rows_tc(const BwdLaunch &l, float *coef, void *dab, int T
         fwd_tc_kernel<true, 2, false, true, true><<<grid, 640, kSmemBytes, l.stream>>>(tq, tk, tv, ta);
     else
         fwd_tc_kernel<true, 2, false, false, true><<<grid, 640, kSmemBytes, l.stream>>>(tq, tk, tv, ta);
+    count_launches(1);
+    return cudaGetLastError();
+}
+
+// Per device: the training forward's register plan holds (bit set) and has
+// been checked (bit set in state_checked).
+static std::atomic<uint64_t> state_checked{0};
+static std::atomic<uint64_t> state_plan_ok{0};
+
+static cudaError_t check_state_plan(int dev, bool *ok) {
+    const uint64_t bit = 1ull << (dev & 63);
+    if (!(state_checked.load() & bit)) {
+        const void *fns[] = {
+            reinterpret_cast<const void *>(fwd_tc_kernel<true, 2, false, false, false, true>),
+            reinterpret_cast<const void *>(fwd_tc_kernel<true, 2, false, true, false, true>)};
+        bool fits = true;
+        for (const void *f : fns) {
+            cudaError_t e = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+            if (e != cudaSuccess) return e;
+            cudaFuncAttributes fa;
+            e = cudaFuncGetAttributes(&fa, f);
+            if (e != cudaSuccess) return e;
+            fits = fits && static_cast<long long>(fa.numRegs) * 640 >= 64ll * 128 + 104ll * 512;
+        }
+        if (fits) state_plan_ok.fetch_or(bit);
+        state_checked.fetch_or(bit);
+    }
+    *ok = (state_plan_ok.load() & bit) != 0;
+    return cudaSuccess;
+}
+
+int fwd_state_supported(int dtype, int T, int Hq, int Hkv, float s, float alpha, int L, int window) {
+    if (dtype != POLAR_BF16 || Hkv <= 0 || (Hq / Hkv) % 2 != 0) return 0;
+    const bool windowed = window > 0 && window < T;
+    const int n_max = windowed ? window : T;
+    const float cl2_max = s * (n_max > L ? 1.0f + alpha * logf(static_cast<float>(n_max) / L) : 1.0f) *
+                          1.4426950408889634f;
+    if (cl2_max > 28.0f) return 0;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+    bool ok = false;
+    if (check_state_plan(dev, &ok) != cudaSuccess) return -1;
+    return ok ? 1 : 0;
+}
+
+// The training forward: the split kernel's sweep with the first-argmax search,
+// the forward's output and n_eff, and each row's streaming state.
+cudaError_t launch_fwd_train_tc(const FwdLaunch &a) {
+    if (!a.state) return cudaErrorInvalidValue;
+    const int sup = fwd_state_supported(a.dtype, a.T, a.Hq, a.Hkv, a.s, a.alpha, a.L, a.window);
+    if (sup < 0) return cudaErrorUnknown;
+    if (sup == 0) return cudaErrorNotSupported;
+    CUtensorMap tq, tk, tv;
+    if (!make_qkv_maps(a.q, a.k, a.v, a.B, a.T, a.Hq, a.Hkv, &tq, &tk, &tv)) return cudaErrorInvalidValue;
+    TcArgs ta = {};
+    ta.u = a.u;
+    ta.out = static_cast<__nv_bfloat16 *>(a.out);
+    ta.neff = a.neff;
+    ta.status = a.status;
+    ta.state = a.state;
+    ta.B = a.B; ta.T = a.T; ta.Hq = a.Hq; ta.Hkv = a.Hkv;
+    ta.nqt = (a.T + kBM - 1) / kBM;
+    const bool windowed = a.window > 0 && a.window < a.T;
+    ta.window = windowed ? a.window : 0;
+    ta.npairs = a.Hq / 2;
+    ta.s = a.s; ta.alpha = a.alpha; ta.L = static_cast<float>(a.L); ta.beta = a.beta;
+    ta.inv_ln_L = 1.0f / logf(static_cast<float>(a.L));
+    const long long ctas = static_cast<long long>(ta.nqt) * ta.npairs * a.B;
+    if (ctas <= 0) return cudaSuccess;
+    if (ctas > 0x7fffffffll) return cudaErrorInvalidValue;
+    const unsigned grid = static_cast<unsigned>(ctas);
+    if (windowed)
+        fwd_tc_kernel<true, 2, false, true, false, true><<<grid, 640, kSmemBytes, a.stream>>>(tq, tk, tv, ta);
+    else
+        fwd_tc_kernel<true, 2, false, false, false, true><<<grid, 640, kSmemBytes, a.stream>>>(tq, tk, tv, ta);
     count_launches(1);
     return cudaGetLastError();
 }

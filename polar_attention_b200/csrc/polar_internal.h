@@ -21,6 +21,7 @@ struct FwdLaunch {
     int window;   // 0: all causal keys; W > 0: the last W
     int *status;  // device status word
     float *moments;  // key-moment records (fwd_moments_bytes), or null
+    float *state;    // training forward: saved row state (FwdState layout), or null
     cudaStream_t stream;
 };
 
@@ -94,6 +95,16 @@ enum BwdCoef {
     kBcJmax = 8, kBcLo = 9, kBcGT = 10, kBwdCoefWords = 16
 };
 
+// Saved row state of a training forward (fp32 words per (batch, head, row),
+// [B][Hq][T][kFwdStateWords]): the streaming sums l, l2 of the weights
+// 2^(cl2 S - cl2) (the fixed reference), the max raw dot, the raw sums S1, S2,
+// |acc| and the first argmax key (int32 bits).  The backward rebuilds each
+// row's coefficient record and dA from it, out and dL/dout.
+enum FwdState {
+    kFsL = 0, kFsL2 = 1, kFsMax = 2, kFsS1 = 3, kFsS2 = 4, kFsNorm = 5, kFsArg = 6,
+    kFwdStateWords = 8
+};
+
 // Launchers return cudaSuccess or the launch error.
 cudaError_t launch_fwd_simt(const FwdLaunch &a);
 cudaError_t launch_fwd_tc(const FwdLaunch &a);
@@ -107,6 +118,18 @@ cudaError_t launch_bwd_tc(const BwdLaunch &l, const float *coef, const void *dab
 // The rows pass of the bf16 backward on the tensor cores (fwd_tc.cu): writes
 // coef and dab as above.  cudaErrorNotSupported where it does not apply.
 cudaError_t launch_bwd_rows_tc(const BwdLaunch &l, float *coef, void *dab, int Tpad);
+// Whether the training forward saves its row state for this shape on the
+// current device (bf16, an even group size, the fixed exponential reference,
+// the kernel's register plan); where it does not, the training forward is the
+// plain forward and the backward recomputes the rows.  Negative: CUDA error.
+int fwd_state_supported(int dtype, int T, int Hq, int Hkv, float s, float alpha, int L,
+                        int window);
+// The training forward with the saved row state (a.state non-null); only
+// where fwd_state_supported holds.
+cudaError_t launch_fwd_train_tc(const FwdLaunch &a);
+// The bf16 backward from a training forward's saved state: rows kernel (record,
+// dA, du partials), the tensor-core dK/dV and dQ passes, du.
+cudaError_t launch_bwd_from_state(const BwdLaunch &l, const void *out, const float *state);
 cudaError_t launch_gdelta_prefill(const GdeltaLaunch &a);
 cudaError_t launch_gdelta_step(const GdeltaStepLaunch &a);
 size_t gdelta_workspace_bytes(int B, int T, int H);

@@ -33,7 +33,8 @@ EXPORTS = ["polar_attn_default_params", "polar_attn_fwd_workspace_size", "polar_
            "polar_attn_decode_chunk_workspace_size", "polar_attn_decode_paged_chunk",
            "polar_attn_bwd_workspace_size", "polar_attn_bwd",
            "polar_gdelta_prefill_workspace_size", "polar_gdelta_prefill", "polar_gdelta_step",
-           "polar_attn_selftest_timeout", "polar_attn_selftest_decode_per_head"]
+           "polar_attn_selftest_timeout", "polar_attn_selftest_decode_per_head",
+           "polar_attn_fwd_state_size", "polar_attn_fwd_train", "polar_attn_bwd_from_state"]
 
 
 class PolarError(RuntimeError):
@@ -84,6 +85,10 @@ def lib() -> ctypes.CDLL:
             L.polar_attn_bwd_workspace_size.argtypes = [PP]
             L.polar_attn_bwd_workspace_size.restype = Z
             L.polar_attn_bwd.argtypes = [P, P, P, P, P, PP, P, P, P, P, P, Z, P]
+            L.polar_attn_fwd_state_size.argtypes = [PP]
+            L.polar_attn_fwd_state_size.restype = Z
+            L.polar_attn_fwd_train.argtypes = [P, P, P, P, PP, P, P, P, P]
+            L.polar_attn_bwd_from_state.argtypes = [P, P, P, P, P, P, P, PP, P, P, P, P, P, Z, P]
             L.polar_attn_fwd_staging_size.argtypes = [PP]
             L.polar_attn_fwd_staging_size.restype = Z
             L.polar_attn_fwd_host.argtypes = [P, P, P, P, PP, P, P, P, Z, P]
@@ -115,7 +120,8 @@ def lib() -> ctypes.CDLL:
                          "polar_attn_decode_paged_noalloc", "polar_attn_selftest_exp2",
                          "polar_attn_decode_paged_chunk", "polar_attn_bwd",
                          "polar_gdelta_prefill", "polar_gdelta_step",
-                         "polar_attn_selftest_timeout", "polar_attn_selftest_decode_per_head"):
+                         "polar_attn_selftest_timeout", "polar_attn_selftest_decode_per_head",
+                         "polar_attn_fwd_train", "polar_attn_bwd_from_state"):
                 getattr(L, name).restype = I
             _lib = L
     return _lib
@@ -231,6 +237,68 @@ def bwd(q, k, v, u, dout, dq=None, dk=None, dv=None, du=None, workspace=None, *,
     _check(lib().polar_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(u), _ptr(dout), ctypes.byref(p),
                                 _ptr(dq), _ptr(dk), _ptr(dv), _ptr(du), _ptr(workspace),
                                 workspace.numel(), _stream(stream)), "polar_attn_bwd")
+    return dq, dk, dv, du
+
+
+def fwd_state_size(B: int, T: int, Hq: int, Hkv: int) -> int:
+    p = make_params(B, T, Hq, Hkv, POLAR_BF16)
+    return int(lib().polar_attn_fwd_state_size(ctypes.byref(p)))
+
+
+def fwd_train(q, k, v, u, out=None, neff=None, state=None, *, s=8.0, alpha=0.3, L=2048, beta=1.0,
+              impl="auto", window=0, stream=None, want_neff=True):
+    """Training forward: as fwd, plus each row's saved state for
+    bwd_from_state.  Returns (out, neff, state); state is a float32
+    [B, Hq, T, 8] tensor (left untouched where the state path does not
+    apply)."""
+    B, T, Hq, D = q.shape
+    Hkv = k.shape[2]
+    for t in (q, k, v, u):
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError("inputs must be contiguous CUDA tensors")
+    if u.dtype != torch.float32:
+        raise TypeError("u must be float32")
+    if out is None:
+        out = torch.empty_like(q)
+    if neff is None and want_neff:
+        neff = torch.empty((B, Hq, T), device=q.device, dtype=torch.float32)
+    if state is None:
+        state = torch.empty((B, Hq, T, 8), device=q.device, dtype=torch.float32)
+    p = make_params(B, T, Hq, Hkv, _dt(q), s, alpha, L, beta, impl, window)
+    p.head_dim = D
+    _check(lib().polar_attn_fwd_train(_ptr(q), _ptr(k), _ptr(v), _ptr(u), ctypes.byref(p),
+                                      _ptr(out), _ptr(neff), _ptr(state), _stream(stream)),
+           "polar_attn_fwd_train")
+    return out, neff, state
+
+
+def bwd_from_state(q, k, v, u, out, state, dout, dq=None, dk=None, dv=None, du=None,
+                   workspace=None, *, s=8.0, alpha=0.3, L=2048, beta=1.0, impl="auto", window=0,
+                   stream=None):
+    """Backward from a training forward's out and saved state (fwd_train with
+    the same arguments).  Returns fp32 (dq, dk, dv, du) as bwd."""
+    B, T, Hq, D = q.shape
+    Hkv = k.shape[2]
+    for t in (q, k, v, u, out, state, dout):
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError("inputs must be contiguous CUDA tensors")
+    if dout.dtype != q.dtype or out.dtype != q.dtype:
+        raise TypeError("out and dout must have the dtype of q")
+    p = make_params(B, T, Hq, Hkv, _dt(q), s, alpha, L, beta, impl, window)
+    p.head_dim = D
+    f32 = torch.float32
+    dq = torch.empty(q.shape, device=q.device, dtype=f32) if dq is None else dq
+    dk = torch.empty(k.shape, device=q.device, dtype=f32) if dk is None else dk
+    dv = torch.empty(v.shape, device=q.device, dtype=f32) if dv is None else dv
+    du = torch.empty(u.shape, device=q.device, dtype=f32) if du is None else du
+    need = int(lib().polar_attn_bwd_workspace_size(ctypes.byref(p)))
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), device=q.device, dtype=torch.uint8)
+    _check(lib().polar_attn_bwd_from_state(_ptr(q), _ptr(k), _ptr(v), _ptr(u), _ptr(out),
+                                           _ptr(state), _ptr(dout), ctypes.byref(p), _ptr(dq),
+                                           _ptr(dk), _ptr(dv), _ptr(du), _ptr(workspace),
+                                           workspace.numel(), _stream(stream)),
+           "polar_attn_bwd_from_state")
     return dq, dk, dv, du
 
 

@@ -59,8 +59,36 @@ def _fwd(lib, p, q=A16, out=A16, ws=None, ws_bytes=0):
 def test_prefill_refuses_bad_params(lib, field, value, code):
     p = _params(**{field: value})
     assert _fwd(lib, p) == code
+    assert lib.polar_attn_fwd_train(A16, A16, A16, A16, ctypes.byref(p), A16, None, A16, None) == code
+    assert _bwd_state(lib, p) == code
     assert lib.polar_attn_fwd_workspace_size(ctypes.byref(p)) == 0
     assert lib.polar_attn_bwd_workspace_size(ctypes.byref(p)) == 0
+    assert lib.polar_attn_fwd_state_size(ctypes.byref(p)) == 0
+
+
+def _bwd_state(lib, p, out=A16, state=A16, ws_bytes=1 << 30):
+    return lib.polar_attn_bwd_from_state(A16, A16, A16, A16, out, state, A16, ctypes.byref(p), A16,
+                                         A16, A16, A16, A16, ws_bytes, None)
+
+
+def test_training_pair_checks(lib):
+    """polar_attn_fwd_train needs an aligned state buffer; polar_attn_bwd_from_state
+    needs out, the state and the backward's workspace; the state is B*Hq*T rows
+    of 8 fp32 words."""
+    p = _params(B=2, T=300, Hq=4, Hkv=2)
+    assert lib.polar_attn_fwd_state_size(ctypes.byref(p)) == 2 * 4 * 300 * 8 * 4
+    assert lib.polar_attn_fwd_train(A16, A16, A16, A16, ctypes.byref(p), A16, None, None, None) == INVALID
+    assert lib.polar_attn_fwd_train(A16, A16, A16, A16, ctypes.byref(p), A16, None, MIS, None) == INVALID
+    assert _bwd_state(lib, p, out=None) == INVALID
+    assert _bwd_state(lib, p, out=MIS) == INVALID
+    assert _bwd_state(lib, p, state=None) == INVALID
+    assert _bwd_state(lib, p, state=MIS) == INVALID
+    need = lib.polar_attn_bwd_workspace_size(ctypes.byref(p))
+    assert _bwd_state(lib, p, ws_bytes=need - 1) == WORKSPACE
+    for shape in ({"B": 0}, {"T": 0}):
+        e = _params(**shape)
+        assert lib.polar_attn_fwd_train(None, None, None, None, ctypes.byref(e), None, None, None,
+                                        None) == OK
 
 
 def test_prefill_pointer_and_workspace_checks(lib):
