@@ -225,10 +225,14 @@ size_t polar_attn_fwd_staging_size(const polar_params_t *params);
  * caller, at least polar_attn_fwd_staging_size bytes), runs the prefill
  * (polar_attn_fwd_ws with its workspace in the staging buffer), copies
  * out and n_eff back to host memory, and synchronises `stream`.  The work
- * goes batch by batch: batch b runs on `stream` while batch b+1's inputs are
- * copied in and batch b-1's outputs copied out, on two copy streams the
- * library creates once per device and joins to `stream` through events.
- * Host-buffer calls on one device are serialised.
+ * goes batch by batch and, for the tensor-core prefill from T = 2048 on, in
+ * row segments of whole 1024-row key chunks (about T/4 rows): the query tiles
+ * of rows r0 .. r1 - 1 run on `stream` as soon as the rows 0 .. r1 - 1 of q,
+ * k and v are in, while the next segment's inputs are copied in and the
+ * previous segment's outputs copied out, on two copy streams the library
+ * creates once per device and joins to `stream` through events.  The results
+ * are those of polar_attn_fwd_ws, bit for bit.  Host-buffer calls on one
+ * device are serialised.
  */
 polar_status_t polar_attn_fwd_host(const void *q_h, const void *k_h, const void *v_h,
                                    const float *u_h, const polar_params_t *params, void *out_h,

@@ -155,6 +155,7 @@ FwdLaunch make_fwd(const void *q, const void *k, const void *v, const float *u,
     a.s = p->logit_scale; a.alpha = p->alpha; a.beta = p->beta; a.L = p->L_train;
     a.window = p->window;
     a.status = status; a.moments = nullptr; a.state = nullptr; a.stream = stream;
+    a.qt_lo = 0; a.qt_cnt = 0;
     return a;
 }
 
@@ -403,26 +404,55 @@ polar_status_t polar_attn_fwd_host(const void *q_h, const void *k_h, const void 
         cudaStreamWaitEvent(hp->out, hp->start, 0) != cudaSuccess ||
         cudaMemcpyAsync(du, u_h, ub, cudaMemcpyHostToDevice, hp->in) != cudaSuccess)
         return POLAR_ERR_CUDA;
+    // Each batch goes in row segments of whole 1024-row key chunks, so that a
+    // segment's copies in and out overlap the prefill of its neighbours: the
+    // query tiles of rows r0 .. r1 - 1 need the keys of rows 0 .. r1 - 1 only,
+    // and the key-moment records of those keys.  The tensor-core prefill takes
+    // a query-tile range; the CUDA-core one runs whole batches.
+    const bool tc = p->dtype == POLAR_BF16 && (p->Hq / p->Hkv) % 2 == 0 && p->impl != POLAR_IMPL_SIMT;
+    const size_t qrow = static_cast<size_t>(p->Hq) * kHeadDim * e, krow = static_cast<size_t>(p->Hkv) * kHeadDim * e;
+    const int seg_rows = tc && p->T >= 2048 ? static_cast<int>(round_up((p->T + 3) / 4, 1024)) : p->T;
+    int *status = status_ptr();
+    if (!status) return POLAR_ERR_CUDA;
+    int ev = 0;
     for (int b = 0; b < p->B; ++b) {
-        const int e2 = b & 1;
-        if (cudaMemcpyAsync(dq + b * qbb, qh + b * qbb, qbb, cudaMemcpyHostToDevice, hp->in) != cudaSuccess ||
-            cudaMemcpyAsync(dk + b * kbb, kh + b * kbb, kbb, cudaMemcpyHostToDevice, hp->in) != cudaSuccess ||
-            cudaMemcpyAsync(dv + b * kbb, vh + b * kbb, kbb, cudaMemcpyHostToDevice, hp->in) != cudaSuccess ||
-            cudaEventRecord(hp->in_done[e2], hp->in) != cudaSuccess ||
-            cudaStreamWaitEvent(s, hp->in_done[e2], 0) != cudaSuccess)
-            return POLAR_ERR_CUDA;
-        st = polar_attn_fwd_ws(dq + b * qbb, dk + b * kbb, dv + b * kbb, reinterpret_cast<float *>(du),
-                               &p1, dout + b * qbb,
-                               neff_h ? reinterpret_cast<float *>(dne + b * nbb) : nullptr,
-                               wsb ? dws : nullptr, wsb, stream);
-        if (st != POLAR_OK) return st;
-        if (cudaEventRecord(hp->comp_done[e2], s) != cudaSuccess ||
-            cudaStreamWaitEvent(hp->out, hp->comp_done[e2], 0) != cudaSuccess ||
-            cudaMemcpyAsync(oh + b * qbb, dout + b * qbb, qbb, cudaMemcpyDeviceToHost, hp->out) != cudaSuccess)
-            return POLAR_ERR_CUDA;
-        if (neff_h && cudaMemcpyAsync(nh + b * nbb, dne + b * nbb, nbb, cudaMemcpyDeviceToHost,
-                                      hp->out) != cudaSuccess)
-            return POLAR_ERR_CUDA;
+        for (int r0 = 0; r0 < p->T; r0 += seg_rows, ++ev) {
+            const int r1 = std::min(p->T, r0 + seg_rows);
+            const size_t rows_s = static_cast<size_t>(r1 - r0);
+            const size_t qo = b * qbb + r0 * qrow, ko = b * kbb + r0 * krow;
+            const int e2 = ev & 1;
+            if (cudaMemcpyAsync(dq + qo, qh + qo, rows_s * qrow, cudaMemcpyHostToDevice, hp->in) != cudaSuccess ||
+                cudaMemcpyAsync(dk + ko, kh + ko, rows_s * krow, cudaMemcpyHostToDevice, hp->in) != cudaSuccess ||
+                cudaMemcpyAsync(dv + ko, vh + ko, rows_s * krow, cudaMemcpyHostToDevice, hp->in) != cudaSuccess ||
+                cudaEventRecord(hp->in_done[e2], hp->in) != cudaSuccess ||
+                cudaStreamWaitEvent(s, hp->in_done[e2], 0) != cudaSuccess)
+                return POLAR_ERR_CUDA;
+            float *ne = neff_h ? reinterpret_cast<float *>(dne + b * nbb) : nullptr;
+            if (tc) {
+                FwdLaunch a = make_fwd(dq + b * qbb, dk + b * kbb, dv + b * kbb,
+                                       reinterpret_cast<float *>(du), &p1, dout + b * qbb, ne, status, s);
+                a.moments = fwd_moment_records(p->T) > 0 && p->window == 0 && wsb
+                                ? reinterpret_cast<float *>(dws)
+                                : nullptr;
+                a.qt_lo = r0 / 128;
+                a.qt_cnt = (r1 + 127) / 128 - a.qt_lo;
+                st = from_cuda(launch_fwd_tc(a));
+            } else {
+                st = polar_attn_fwd_ws(dq + b * qbb, dk + b * kbb, dv + b * kbb,
+                                       reinterpret_cast<float *>(du), &p1, dout + b * qbb, ne,
+                                       wsb ? dws : nullptr, wsb, stream);
+            }
+            if (st != POLAR_OK) return st;
+            if (cudaEventRecord(hp->comp_done[e2], s) != cudaSuccess ||
+                cudaStreamWaitEvent(hp->out, hp->comp_done[e2], 0) != cudaSuccess ||
+                cudaMemcpyAsync(oh + qo, dout + qo, rows_s * qrow, cudaMemcpyDeviceToHost, hp->out) != cudaSuccess)
+                return POLAR_ERR_CUDA;
+            // n_eff [B, Hq, T]: this segment's rows of every head of batch b.
+            if (neff_h && cudaMemcpy2DAsync(nh + b * nbb + r0 * 4, static_cast<size_t>(p->T) * 4,
+                                            dne + b * nbb + r0 * 4, static_cast<size_t>(p->T) * 4,
+                                            rows_s * 4, p->Hq, cudaMemcpyDeviceToHost, hp->out) != cudaSuccess)
+                return POLAR_ERR_CUDA;
+        }
     }
     if (cudaEventRecord(hp->out_done, hp->out) != cudaSuccess ||
         cudaStreamWaitEvent(s, hp->out_done, 0) != cudaSuccess)

@@ -61,11 +61,11 @@ __device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4],
 
 __global__ void __launch_bounds__(256)
 fwd_moments_kernel(const __nv_bfloat16 *__restrict__ k, float *__restrict__ rec, int T, int Hkv,
-                   int nrec) {
+                   int nrec, int chunk0) {
     __shared__ __align__(128) uint8_t buf[2][kBufBytes];
     __shared__ float ks_part[4][kHeadDim];
 
-    const int chunk = blockIdx.x, bg = blockIdx.y;  // bg = b * Hkv + g
+    const int chunk = chunk0 + static_cast<int>(blockIdx.x), bg = blockIdx.y;  // bg = b * Hkv + g
     const int b = bg / Hkv, g = bg % Hkv;
     const int t_begin = chunk * kMomChunk;
     const int t_end = min(t_begin + kMomChunk, nrec);
@@ -159,15 +159,18 @@ size_t fwd_moments_bytes(int B, int T, int Hkv) {
     return static_cast<size_t>(B) * Hkv * fwd_moment_records(T) * kMomFloats * sizeof(float);
 }
 
-cudaError_t launch_fwd_moments(const void *k, int B, int T, int Hkv, float *rec,
-                               cudaStream_t stream) {
+cudaError_t launch_fwd_moments(const void *k, int B, int T, int Hkv, float *rec, int rec_lo,
+                               int rec_hi, cudaStream_t stream) {
     const int nrec = fwd_moment_records(T);
     if (nrec == 0 || B == 0) return cudaSuccess;
-    const int nchunks = (nrec + kMomChunk - 1) / kMomChunk;
+    // Whole chunks: every record of a chunk is a running sum from the chunk's start.
+    const int c_lo = max(rec_lo, 0) / kMomChunk;
+    const int c_hi = (min(rec_hi, nrec) + kMomChunk - 1) / kMomChunk;
+    if (c_hi <= c_lo) return cudaSuccess;
     const long long bg = static_cast<long long>(B) * Hkv;
     if (bg > 65535) return cudaErrorInvalidValue;
-    fwd_moments_kernel<<<dim3(nchunks, static_cast<unsigned>(bg)), 256, 0, stream>>>(
-        static_cast<const __nv_bfloat16 *>(k), rec, T, Hkv, nrec);
+    fwd_moments_kernel<<<dim3(c_hi - c_lo, static_cast<unsigned>(bg)), 256, 0, stream>>>(
+        static_cast<const __nv_bfloat16 *>(k), rec, T, Hkv, nrec, c_lo);
     count_launches(1);
     return cudaGetLastError();
 }

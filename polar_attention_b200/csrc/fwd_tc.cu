@@ -318,6 +318,7 @@ struct TcArgs {
     int *status;
     const float *mom;  // key-moment records (kMoments only)
     int B, T, Hq, Hkv, nqt, npairs;
+    int qt_lo, qt_cnt;  // the query tiles this launch takes: qt_lo .. qt_lo + qt_cnt - 1
     int window;  // 0: all causal keys; W > 0: the last W of each row's
     float s, alpha, L, beta, inv_ln_L;
     // Backward rows pass (kRows) only: the upstream gradient dL/dout
@@ -497,7 +498,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CU
 
     // Work tile: heaviest query tiles first (longest causal rows).
     const int per_qt = a.npairs * a.B;
-    const int qt = a.nqt - 1 - static_cast<int>(blockIdx.x) / per_qt;
+    const int qt = a.qt_lo + a.qt_cnt - 1 - static_cast<int>(blockIdx.x) / per_qt;
     const int rem = static_cast<int>(blockIdx.x) % per_qt;
     const int pair = rem % a.npairs, b = rem / a.npairs;
     const int h0 = 2 * pair;
@@ -1065,13 +1066,16 @@ cudaError_t launch_fwd_tc(const FwdLaunch &a) {
     ta.mom = a.moments;
     ta.B = a.B; ta.T = a.T; ta.Hq = a.Hq; ta.Hkv = a.Hkv;
     ta.nqt = (a.T + kBM - 1) / kBM;
+    if (a.qt_lo < 0 || a.qt_cnt < 0 || a.qt_lo + a.qt_cnt > ta.nqt) return cudaErrorInvalidValue;
+    ta.qt_lo = a.qt_lo;
+    ta.qt_cnt = a.qt_cnt > 0 ? a.qt_cnt : ta.nqt - a.qt_lo;
     // A window no shorter than the sequence changes nothing.
     const bool windowed = a.window > 0 && a.window < a.T;
     ta.window = windowed ? a.window : 0;
     ta.npairs = a.Hq / 2;
     ta.s = a.s; ta.alpha = a.alpha; ta.L = static_cast<float>(a.L); ta.beta = a.beta;
     ta.inv_ln_L = 1.0f / logf(static_cast<float>(a.L));
-    const long long ctas = static_cast<long long>(ta.nqt) * ta.npairs * a.B;
+    const long long ctas = static_cast<long long>(ta.qt_cnt) * ta.npairs * a.B;
     if (ctas <= 0) return cudaSuccess;
     if (ctas > 0x7fffffffll) return cudaErrorInvalidValue;
     // Fixed exponential reference while the smallest weight squared, 2^(-4 c_max log2e)
@@ -1085,7 +1089,11 @@ cudaError_t launch_fwd_tc(const FwdLaunch &a) {
         if (windowed) {
             fwd_tc_kernel<true, 2, false, true><<<grid, 640, kSmemBytes, a.stream>>>(tq, tk, tv, ta);
         } else if (a.moments && ta.nqt >= kMomMinTiles) {
-            e = launch_fwd_moments(a.k, a.B, a.T, a.Hkv, a.moments, a.stream);
+            // The records the launch's query tiles read: those of key tiles below
+            // its last query tile, from the chunk holding its first query tile's.
+            const int rec_hi = ta.qt_lo + ta.qt_cnt - 1;
+            e = launch_fwd_moments(a.k, a.B, a.T, a.Hkv, a.moments, ta.qt_lo > 0 ? ta.qt_lo - 1 : 0,
+                                   rec_hi, a.stream);
             if (e != cudaSuccess) return e;
             fwd_tc_kernel<true, 2, true, false><<<grid, 640, kSmemBytes, a.stream>>>(tq, tk, tv, ta);
         } else {
@@ -1142,6 +1150,8 @@ cudaError_t launch_bwd_rows_tc(const BwdLaunch &l, float *coef, void *dab, int T
     ta.status = l.status;
     ta.B = l.B; ta.T = l.T; ta.Hq = l.Hq; ta.Hkv = l.Hkv;
     ta.nqt = Tpad / kBM;
+    ta.qt_lo = 0;
+    ta.qt_cnt = ta.nqt;
     ta.npairs = l.Hq / 2;
     ta.window = windowed ? l.window : 0;
     ta.s = l.s; ta.alpha = l.alpha; ta.L = static_cast<float>(l.L); ta.beta = l.beta;
@@ -1220,6 +1230,8 @@ cudaError_t launch_fwd_train_tc(const FwdLaunch &a) {
     ta.state = a.state;
     ta.B = a.B; ta.T = a.T; ta.Hq = a.Hq; ta.Hkv = a.Hkv;
     ta.nqt = (a.T + kBM - 1) / kBM;
+    ta.qt_lo = 0;
+    ta.qt_cnt = ta.nqt;
     const bool windowed = a.window > 0 && a.window < a.T;
     ta.window = windowed ? a.window : 0;
     ta.npairs = a.Hq / 2;

@@ -22,6 +22,7 @@ struct FwdLaunch {
     int *status;  // device status word
     float *moments;  // key-moment records (fwd_moments_bytes), or null
     float *state;    // training forward: saved row state (FwdState layout), or null
+    int qt_lo, qt_cnt;  // query tiles qt_lo .. qt_lo + qt_cnt - 1 (qt_cnt 0: to the end)
     cudaStream_t stream;
 };
 
@@ -141,8 +142,9 @@ constexpr int kMomChunk = 8;
 constexpr int kMomFloats = 64 * 64 + 64;
 int fwd_moment_records(int T);
 size_t fwd_moments_bytes(int B, int T, int Hkv);
-cudaError_t launch_fwd_moments(const void *k, int B, int T, int Hkv, float *rec,
-                               cudaStream_t stream);
+// Computes the records rec_lo .. rec_hi - 1 (rounded out to whole chunks).
+cudaError_t launch_fwd_moments(const void *k, int B, int T, int Hkv, float *rec, int rec_lo,
+                               int rec_hi, cudaStream_t stream);
 
 // Loads the decode kernels' code onto the current device now rather than at
 // their first launch (lazy module loading).

@@ -216,17 +216,20 @@ def test_unnormalised_inputs_are_reported(cuda_ok):
     assert pa.get_status() == 0
 
 
-@pytest.mark.parametrize("T", [300, 4500])
-def test_host_buffers_match_device_buffers(cuda_ok, T):
-    """polar_attn_fwd_host runs the prefill batch by batch, overlapping each
-    batch's copies with its neighbours' compute: with three batches, on the key
-    moments path (T=4500) and below it, its rows equal the device-buffer call's
-    bit for bit (a row does not depend on the other batches)."""
+@pytest.mark.parametrize("T,Wn", [(300, 0), (4500, 0), (4500, 700)])
+def test_host_buffers_match_device_buffers(cuda_ok, T, Wn):
+    """polar_attn_fwd_host runs the prefill batch by batch and, from T = 2048
+    on, in row segments of whole 1024-row key chunks (here 2048, 2048 and 404
+    rows), each segment's copies overlapping its neighbours' compute; the key
+    moments of a segment's keys are formed with it.  With three batches, on the
+    key-moment path (T=4500), below it and with a window, its rows equal the
+    device-buffer call's bit for bit: a row depends on neither the other
+    batches nor the split."""
     w = W.small_prefill(B=3, T=T, Hq=8, Hkv=2, dtype="bf16", seed=T, plant="frac",
-                        plant_frac=0.01, L=512)
+                        plant_frac=0.01, L=512, window=Wn)
     x = W.prefill_inputs(w, "cpu")
     xd = PT.to_device(x)
-    p = dict(s=w.s, alpha=w.alpha, L=w.L, beta=w.beta)
+    p = dict(s=w.s, alpha=w.alpha, L=w.L, beta=w.beta, window=w.window)
     ref, nref = pa.fwd(xd["q"], xd["k"], xd["v"], xd["u"], **p)
     pin = lambda t: t.contiguous().pin_memory()  # noqa: E731
     ho = torch.empty_like(x["q"]).pin_memory()
