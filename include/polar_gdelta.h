@@ -67,8 +67,12 @@ typedef struct {
  *
  * Computed chunk-parallel: tokens in chunks of 64; within a chunk the writes
  * are solved at once (a unit lower-triangular system over the chunk's keys),
- * and the state passes from chunk to chunk, all in fp32.  The result equals
- * the token-by-token recurrence up to fp32 rounding.  alpha below 1.6e-38 acts
+ * and the state passes from chunk to chunk, all in fp32.  With few (sequence,
+ * head) pairs and many chunks (bf16), the chunks also go in groups: each
+ * group's effect on the state is the affine map S -> S M + E, the groups'
+ * initial states follow from those maps in sequence, and the groups then run
+ * side by side.  The result equals the token-by-token recurrence up to fp32
+ * rounding.  alpha below 1.6e-38 acts
  * as 1.6e-38.  B = 0 or T = 0 leaves everything unchanged.
  */
 size_t polar_gdelta_prefill_workspace_size(const polar_gdelta_params_t *params);

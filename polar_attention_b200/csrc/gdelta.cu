@@ -181,6 +181,11 @@ struct GdArgs {
     void *out;
     float *ws;
     int B, T, H, nchunks, zero_init, accumulate;
+    // Two-level scan (groups > 1): chunk groups of cpg chunks; maps[bh][group][2][64][64]
+    // (the group's homogeneous map M, then its state from zero E) and
+    // starts[bh][group][64][64] (each group's initial state).
+    int groups, cpg;
+    float *maps, *starts;
 };
 
 // Kernel 1 for fp32 inputs: one CTA per (chunk, sequence x head), fp32 FMA.
@@ -632,12 +637,28 @@ constexpr int kOffS = 5 * kTB, kOffU = kOffS + 2 * kSB, kOffUK = kOffU + 2 * kUB
 constexpr int kOffScal = kOffUK + 2 * kUB;            // qs[64], ks[64], b_last, 3 pad
 constexpr size_t kScanMmaSmem = kOffScal + 132 * sizeof(float);
 
+// kMode 0: the whole sequence of one (sequence x head) slice: initial state
+// from the caller (or zero), outputs, final state back to the caller.
+// kMode 1 (two-level scan, first pass): chunk group blockIdx.z only, no
+// outputs; blockIdx.x = slice + 2 kind: kind 0 runs the homogeneous recurrence
+// (Ut taken as zero) from the identity, which gives the group's map M, kind 1
+// the full recurrence from zero, which gives its offset E (S_end = S_0 M + E);
+// both go to a.maps.
+// kMode 2 (two-level scan, last pass): chunk group blockIdx.z from its initial
+// state (a.starts; the caller's state for group 0), with outputs; the last
+// group writes the final state back to the caller.
+template <int kMode>
 __global__ void __launch_bounds__(256, 2) gd_scan_mma_kernel(GdArgs a) {
     extern __shared__ __align__(128) uint8_t smb[];
     const uint32_t sb = smem_u32(smb);
     const float *scal = reinterpret_cast<const float *>(smb + kOffScal);
 
-    const int slice = blockIdx.x, bh = blockIdx.y;
+    const int slice = blockIdx.x & 1, kind = kMode == 1 ? static_cast<int>(blockIdx.x >> 1) : 1;
+    const int bh = blockIdx.y, grp = kMode == 0 ? 0 : static_cast<int>(blockIdx.z);
+    const int c_begin = kMode == 0 ? 0 : grp * a.cpg;
+    const int c_end = kMode == 0 ? a.nchunks : min(a.nchunks, c_begin + a.cpg);
+    constexpr bool kOut = kMode != 1;
+    const bool with_ut = kind == 1;  // kind 0 of the first pass: the homogeneous map
     const int b = bh / a.H, h = bh % a.H;
     const int r0 = slice * kMmaRows;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -649,6 +670,12 @@ __global__ void __launch_bounds__(256, 2) gd_scan_mma_kernel(GdArgs a) {
     const __nv_bfloat16 *ksrc = static_cast<const __nv_bfloat16 *>(a.k) + h * kHeadDim;
     __nv_bfloat16 *out = static_cast<__nv_bfloat16 *>(a.out);
 
+    // Initial state of this slice: the caller's (or zero), a group's start, or
+    // for the first pass the identity (kind 0) or zero (kind 1).
+    const float *init = kMode == 2 && grp > 0
+                            ? a.starts + ((static_cast<size_t>(bh) * a.groups + grp) * 64 + r0) * 64
+                            : state;
+    const bool from_mem = kMode == 2 && grp > 0 ? true : kMode == 1 ? false : !a.zero_init;
     float sacc[2][4];
 #pragma unroll
     for (int n = 0; n < 2; ++n)
@@ -656,7 +683,8 @@ __global__ void __launch_bounds__(256, 2) gd_scan_mma_kernel(GdArgs a) {
         for (int hf = 0; hf < 2; ++hf) {
             const int r = 16 * rm + g + 8 * hf, c = 16 * cn + 8 * n + q2;
             float2 v = make_float2(0.0f, 0.0f);
-            if (!a.zero_init) v = *reinterpret_cast<const float2 *>(state + r * 64 + c);
+            if (from_mem) v = *reinterpret_cast<const float2 *>(init + r * 64 + c);
+            if (kMode == 1 && kind == 0) v = make_float2(r0 + r == c ? 1.0f : 0.0f, r0 + r == c + 1 ? 1.0f : 0.0f);
             sacc[n][2 * hf] = v.x;
             sacc[n][2 * hf + 1] = v.y;
         }
@@ -687,24 +715,25 @@ __global__ void __launch_bounds__(256, 2) gd_scan_mma_kernel(GdArgs a) {
         }
     };
     auto issue_wq = [&](int c) {
-        if (c < a.nchunks) {
+        if (c < c_end) {
             const float *wsc = chunk_ws(c);
             const __nv_bfloat16 *wshc = reinterpret_cast<const __nv_bfloat16 *>(wsc);
 #pragma unroll
             for (int i = 0; i < 4; ++i)  // -W hi (rows, rows + 32), then -W lo
                 cp_async_16(sb + kOffW + (i >> 1) * kTB + cp_dst + 32 * (i & 1) * kTP,
                             wshc + (i >> 1) * 4096 + cp_ws + 32 * 64 * (i & 1), 16);
-            issue_rows(kOffQ, qsrc + (static_cast<size_t>(b) * a.T + c * kC) * row_stride,
-                       min(kC, a.T - c * kC));
+            if (kOut)
+                issue_rows(kOffQ, qsrc + (static_cast<size_t>(b) * a.T + c * kC) * row_stride,
+                           min(kC, a.T - c * kC));
             if (tid < 33) cp_async_16(sb + kOffScal + 16 * tid, wsc + kWsQs + 4 * tid, 16);
         }
         asm volatile("cp.async.commit_group;" ::: "memory");
     };
     auto issue_pk = [&](int c) {
-        if (c < a.nchunks) {
+        if (c < c_end) {
             const __nv_bfloat16 *wshc = reinterpret_cast<const __nv_bfloat16 *>(chunk_ws(c));
 #pragma unroll
-            for (int i = 0; i < 2; ++i)
+            for (int i = 0; i < 2 && kOut; ++i)
                 cp_async_16(sb + kOffP + cp_dst + 32 * i * kTP,
                             wshc + 2 * kWsP + cp_ws + 32 * 64 * i, 16);
             issue_rows(kOffK, ksrc + (static_cast<size_t>(b) * a.T + c * kC) * row_stride,
@@ -715,7 +744,14 @@ __global__ void __launch_bounds__(256, 2) gd_scan_mma_kernel(GdArgs a) {
     // This thread's Ut entries of chunk c (the initial value of U).
     const int ut_off = (16 * mt + g) * 64 + r0 + 16 * nh + q2;
     auto load_ut = [&](int c, float (&u)[2][4]) {
-        if (c >= a.nchunks) return;
+        if (c >= c_end) return;
+        if (!with_ut) {
+#pragma unroll
+            for (int n2 = 0; n2 < 2; ++n2)
+#pragma unroll
+                for (int i = 0; i < 4; ++i) u[n2][i] = 0.0f;
+            return;
+        }
         const float *src = chunk_ws(c) + kWsUt + ut_off;
 #pragma unroll
         for (int n2 = 0; n2 < 2; ++n2)
@@ -728,11 +764,11 @@ __global__ void __launch_bounds__(256, 2) gd_scan_mma_kernel(GdArgs a) {
     };
 
     float unext[2][4];
-    issue_wq(0);
-    issue_pk(0);
-    load_ut(0, unext);
+    issue_wq(c_begin);
+    issue_pk(c_begin);
+    load_ut(c_begin, unext);
 
-    for (int ch = 0; ch < a.nchunks; ++ch) {
+    for (int ch = c_begin; ch < c_end; ++ch) {
         const int t0 = ch * kC, n = min(kC, a.T - t0);
         const size_t row0 = static_cast<size_t>(b) * a.T + t0;
 
@@ -766,19 +802,23 @@ __global__ void __launch_bounds__(256, 2) gd_scan_mma_kernel(GdArgs a) {
             uint32_t wh[4], wl[4], aq[4], bh4[4], bl4[4];
             ldsm_x4(sb + kOffW + ao, wh);
             ldsm_x4(sb + kOffW + kTB + ao, wl);
-            ldsm_x4(sb + kOffQ + ao, aq);
+            if (kOut) ldsm_x4(sb + kOffQ + ao, aq);
             const uint32_t bo = (16 * nh + bn_row) * kTP + 2 * (16 * ks + bn_col);
             ldsm_x4(sb + kOffS + bo, bh4);
             ldsm_x4(sb + kOffS + kSB + bo, bl4);
             // consecutive MMAs go to different accumulators
 #pragma unroll
             for (int n2 = 0; n2 < 2; ++n2) mma_bf16(uacc[n2], wh, bh4[2 * n2], bh4[2 * n2 + 1]);
+            if (kOut) {
 #pragma unroll
-            for (int n2 = 0; n2 < 2; ++n2) mma_bf16(oacc[n2], aq, bh4[2 * n2], bh4[2 * n2 + 1]);
+                for (int n2 = 0; n2 < 2; ++n2) mma_bf16(oacc[n2], aq, bh4[2 * n2], bh4[2 * n2 + 1]);
+            }
 #pragma unroll
             for (int n2 = 0; n2 < 2; ++n2) mma_bf16(uacc[n2], wh, bl4[2 * n2], bl4[2 * n2 + 1]);
+            if (kOut) {
 #pragma unroll
-            for (int n2 = 0; n2 < 2; ++n2) mma_bf16(oacc[n2], aq, bl4[2 * n2], bl4[2 * n2 + 1]);
+                for (int n2 = 0; n2 < 2; ++n2) mma_bf16(oacc[n2], aq, bl4[2 * n2], bl4[2 * n2 + 1]);
+            }
 #pragma unroll
             for (int n2 = 0; n2 < 2; ++n2) mma_bf16(uacc[n2], wl, bh4[2 * n2], bh4[2 * n2 + 1]);
         }
@@ -808,7 +848,7 @@ __global__ void __launch_bounds__(256, 2) gd_scan_mma_kernel(GdArgs a) {
         __syncthreads();
 
         // O += P U  (P is zero above the diagonal: k-steps up to the row tile)
-        for (int ks = 0; ks <= mt; ++ks) {
+        for (int ks = 0; ks <= mt && kOut; ++ks) {
             uint32_t ap[4], bh4[4], bl4[4];
             ldsm_x4(sb + kOffP + (16 * mt + a_row) * kTP + 2 * (16 * ks + a_col), ap);
             const uint32_t bo = (16 * ks + bt_row) * kUP + 2 * (16 * nh + bt_col);
@@ -824,7 +864,7 @@ __global__ void __launch_bounds__(256, 2) gd_scan_mma_kernel(GdArgs a) {
 #pragma unroll
             for (int hf = 0; hf < 2; ++hf) {
                 const int t = 16 * mt + g + 8 * hf, r = 16 * nh + 8 * n2 + q2;
-                if (t < n) {
+                if (kOut && t < n) {
                     uint32_t *dst = reinterpret_cast<uint32_t *>(
                         out + ((row0 + t) * a.H + h) * static_cast<size_t>(kHeadDim) + r0 + r);
                     float v0 = oacc[n2][2 * hf], v1 = oacc[n2][2 * hf + 1];
@@ -858,14 +898,63 @@ __global__ void __launch_bounds__(256, 2) gd_scan_mma_kernel(GdArgs a) {
         issue_pk(ch + 1);
     }
     asm volatile("cp.async.wait_group 0;" ::: "memory");
+    // Final state: the caller's, or this group's map / offset (first pass).
+    float *fin = state;
+    if (kMode == 1)
+        fin = a.maps + (((static_cast<size_t>(bh) * a.groups + grp) * 2 + kind) * 64 + r0) * 64;
+    if (kMode == 2 && grp != a.groups - 1) return;
 #pragma unroll
     for (int n2 = 0; n2 < 2; ++n2)
 #pragma unroll
         for (int hf = 0; hf < 2; ++hf) {
             const int r = 16 * rm + g + 8 * hf, c = 16 * cn + 8 * n2 + q2;
-            *reinterpret_cast<float2 *>(state + r * 64 + c) =
+            *reinterpret_cast<float2 *>(fin + r * 64 + c) =
                 make_float2(sacc[n2][2 * hf], sacc[n2][2 * hf + 1]);
         }
+}
+
+// Two-level scan, middle pass: per (sequence x head), the initial state of
+// every chunk group from the groups' maps, S_start(g + 1) = S_start(g) M_g + E_g
+// (fp32 on the CUDA cores; 64 x 64 x 64 per group), S_start(0) the caller's
+// state or zero.  256 threads; thread t owns rows t / 16 + 16 i of columns
+// 4 (t % 16) .. + 3.
+__global__ void __launch_bounds__(256) gd_compose_kernel(GdArgs a) {
+    __shared__ __align__(16) float Ss[64][64];
+    __shared__ __align__(16) float Ms[64][64];
+    const int bh = blockIdx.x, tid = threadIdx.x;
+    const float *st0 = a.state + static_cast<size_t>(bh) * 64 * 64;
+    for (int i = tid; i < 64 * 64; i += 256)
+        Ss[i >> 6][i & 63] = a.zero_init ? 0.0f : st0[i];
+    const int c4 = 4 * (tid & 15), rr = tid >> 4;
+    for (int gi = 0; gi + 1 < a.groups; ++gi) {
+        const float *Mg = a.maps + (static_cast<size_t>(bh) * a.groups + gi) * 2 * 4096;
+        const float *Eg = Mg + 4096;
+        __syncthreads();  // Ss is complete; Ms is free
+        for (int i = tid; i < 64 * 64; i += 256) Ms[i >> 6][i & 63] = Mg[i];
+        __syncthreads();
+        float4 acc[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) acc[i] = *reinterpret_cast<const float4 *>(Eg + (rr + 16 * i) * 64 + c4);
+#pragma unroll 8
+        for (int k = 0; k < 64; ++k) {
+            const float4 m = *reinterpret_cast<const float4 *>(&Ms[k][c4]);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const float sv = Ss[rr + 16 * i][k];
+                acc[i].x = fmaf(sv, m.x, acc[i].x);
+                acc[i].y = fmaf(sv, m.y, acc[i].y);
+                acc[i].z = fmaf(sv, m.z, acc[i].z);
+                acc[i].w = fmaf(sv, m.w, acc[i].w);
+            }
+        }
+        __syncthreads();  // every read of Ss is done
+        float *dst = a.starts + (static_cast<size_t>(bh) * a.groups + gi + 1) * 4096;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            *reinterpret_cast<float4 *>(&Ss[rr + 16 * i][c4]) = acc[i];
+            *reinterpret_cast<float4 *>(dst + (rr + 16 * i) * 64 + c4) = acc[i];
+        }
+    }
 }
 
 // 16 consecutive elements of a row as fp32 (two or four 16-byte loads).
@@ -1057,10 +1146,13 @@ cudaError_t launch_prefill_t(const GdArgs &g, cudaStream_t stream) {
         if constexpr (kMma) {
             e = cudaFuncSetAttribute(gd_chunk_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      static_cast<int>(kChunkMmaSmem));
-            if (e == cudaSuccess)
-                e = cudaFuncSetAttribute(gd_scan_mma_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(kScanMmaSmem));
+            const void *scans[] = {reinterpret_cast<const void *>(gd_scan_mma_kernel<0>),
+                                   reinterpret_cast<const void *>(gd_scan_mma_kernel<1>),
+                                   reinterpret_cast<const void *>(gd_scan_mma_kernel<2>)};
+            for (const void *f : scans)
+                if (e == cudaSuccess)
+                    e = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             static_cast<int>(kScanMmaSmem));
         } else {
             e = cudaFuncSetAttribute(gd_chunk_kernel<Tin>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      static_cast<int>(kChunkSmem));
@@ -1079,19 +1171,49 @@ cudaError_t launch_prefill_t(const GdArgs &g, cudaStream_t stream) {
         gd_chunk_kernel<Tin><<<dim3(g.nchunks, bh), 256, kChunkSmem, stream>>>(g);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    if constexpr (kMma)
-        gd_scan_mma_kernel<<<dim3(64 / kMmaRows, bh), 256, kScanMmaSmem, stream>>>(g);
-    else
+    if constexpr (kMma) {
+        if (g.groups > 1) {
+            // Two-level scan: each chunk group's map and offset, the groups'
+            // initial states in sequence, then every group with its outputs.
+            gd_scan_mma_kernel<1><<<dim3(2 * (64 / kMmaRows), bh, g.groups), 256, kScanMmaSmem, stream>>>(g);
+            gd_compose_kernel<<<bh, 256, 0, stream>>>(g);
+            gd_scan_mma_kernel<2><<<dim3(64 / kMmaRows, bh, g.groups), 256, kScanMmaSmem, stream>>>(g);
+            count_launches(4);
+            return cudaGetLastError();
+        }
+        gd_scan_mma_kernel<0><<<dim3(64 / kMmaRows, bh), 256, kScanMmaSmem, stream>>>(g);
+    } else {
         gd_scan_kernel<Tin><<<dim3(64 / kSlice, bh), 256, kScanSmem, stream>>>(g);
+    }
     count_launches(2);
     return cudaGetLastError();
 }
 
+// Chunk groups of the two-level scan for a bf16 prefill: one (the plain scan)
+// while the (sequence x head) slices alone give the scan at least one CTA per
+// SM; else enough groups of at least 8 chunks to fill about two CTAs per SM,
+// at most kMaxGroups.
+constexpr int kMaxGroups = 32;
+constexpr int kMinGroupChunks = 8;
+// Chunk groups the workspace has room for: none below two groups' worth.
+size_t max_groups(size_t nchunks) {
+    return nchunks < 2 * kMinGroupChunks ? 0 : std::min<size_t>(kMaxGroups, nchunks / kMinGroupChunks);
+}
+int scan_groups(int B, int H, int nchunks, int sms) {
+    const long long slices = 2ll * B * H;
+    if (slices >= sms || nchunks < 2 * kMinGroupChunks) return 1;
+    const long long want = (2ll * sms + slices - 1) / slices;
+    const int most = std::min(kMaxGroups, nchunks / kMinGroupChunks);
+    return static_cast<int>(std::max<long long>(1, std::min<long long>(want, most)));
+}
+
 }  // namespace
 
+// Per-chunk records, then (for the two-level scan) room for the most chunk
+// groups the shape can have: their maps and offsets, and initial states.
 size_t gdelta_workspace_bytes(int B, int T, int H) {
     const size_t nch = (static_cast<size_t>(T) + kC - 1) / kC;
-    return static_cast<size_t>(B) * H * nch * kWsFloats * sizeof(float);
+    return static_cast<size_t>(B) * H * (nch * kWsFloats + max_groups(nch) * 3 * 4096) * sizeof(float);
 }
 
 cudaError_t launch_gdelta_prefill(const GdeltaLaunch &l) {
@@ -1101,6 +1223,26 @@ cudaError_t launch_gdelta_prefill(const GdeltaLaunch &l) {
     g.state = l.state; g.out = l.out; g.ws = static_cast<float *>(l.workspace);
     g.B = l.B; g.T = l.T; g.H = l.H; g.nchunks = (l.T + kC - 1) / kC;
     g.zero_init = l.zero_init; g.accumulate = l.accumulate;
+    g.groups = 1;
+    g.cpg = g.nchunks;
+    g.maps = g.starts = nullptr;
+    if (l.dtype != POLAR_FP32) {
+        int dev = 0, sms = 148;
+        if (cudaGetDevice(&dev) == cudaSuccess)
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        g.groups = scan_groups(l.B, l.H, g.nchunks, sms);
+        if (g.groups > 1) {
+            g.cpg = (g.nchunks + g.groups - 1) / g.groups;
+            g.groups = (g.nchunks + g.cpg - 1) / g.cpg;  // no empty group
+            const size_t nch = static_cast<size_t>(g.nchunks);
+            const size_t gmax = max_groups(nch);
+            float *extra = g.ws + static_cast<size_t>(l.B) * l.H * nch * kWsFloats;
+            g.maps = extra;
+            g.starts = extra + static_cast<size_t>(l.B) * l.H * gmax * 2 * 4096;
+            // The buffers hold gmax groups per (sequence x head); index them by g.groups.
+            if (static_cast<size_t>(g.groups) > gmax) return cudaErrorInvalidValue;
+        }
+    }
     return l.dtype == POLAR_FP32 ? launch_prefill_t<float>(g, l.stream)
                                  : launch_prefill_t<__nv_bfloat16>(g, l.stream);
 }

@@ -145,6 +145,28 @@ def test_prefill_long_sequence_error_stays_bounded(cuda_ok):
     _check(out, state, o_ref, S_ref, "bf16", what="T=16384")
 
 
+@pytest.mark.parametrize("T,given_state", [(3000, True), (2100, False)])
+def test_prefill_two_level_scan(cuda_ok, T, given_state):
+    """Few (sequence x head) slices and many chunks take the two-level scan:
+    each group of chunks gets its map S -> S M + E, the groups' initial states
+    follow in sequence, then every group runs with its outputs.  Here 47 and 33
+    chunks of one sequence and two heads (5 and 4 groups), a given initial state,
+    a ragged last chunk, and the decay gate closed (alpha = 0) at the first
+    token of a group and in its middle."""
+    w = W.small_gdelta(B=1, T=T, H=2, seed=T)
+    x = W.gdelta_inputs(w)
+    x["alpha"][0, [640, 650, 1280], 0] = 0.0
+    x["beta"][0, 641, 1] = 0.0
+    S0 = None
+    if given_state:
+        g = torch.Generator().manual_seed(5)
+        S0 = 0.2 * torch.randn((1, 2, 64, 64), generator=g)
+    o_ref, S_ref = _oracle(x, None if S0 is None else S0.numpy().astype(np.float64))
+    out, state = _run_prefill(_dev(x), state=None if S0 is None else S0.cuda().clone())
+    e = _check(out, state, o_ref, S_ref, "bf16", what=f"two-level T={T}")
+    print(f"two-level T={T}: output {e[0]:.2e}, state {e[1]:.2e}")
+
+
 def _step(x, out=None, accumulate=False):
     o = pa.gdelta_step(x["q"], x["k"], x["v"], x["alpha"], x["beta"], x["state_pool"], x["slots"],
                        out=out, accumulate=accumulate)
