@@ -131,7 +131,9 @@ polar_status_t polar_attn_fwd(const void *q, const void *k, const void *v, const
  *            over the key tiles left of a query tile come from key moments
  *            (sum k, sum k k^T) that a pre-pass writes here, instead of from
  *            every score: the same quantities, computed with less work per
- *            score (used from 32 query tiles on, without a sliding window).
+ *            score (used from 32 query tiles on; with a sliding window, for
+ *            windows of at least 4096 keys, from differences of key-moment
+ *            prefixes over the key tiles every row of a tile sees in full).
  *            Contents on entry are ignored; calls that share a workspace must
  *            not overlap.  A non-NULL workspace smaller than required returns
  *            POLAR_ERR_WORKSPACE.

@@ -239,11 +239,9 @@ polar_status_t polar_attn_fwd_ws(const void *q, const void *k, const void *v, co
     if (!status) return POLAR_ERR_CUDA;
     FwdLaunch a = make_fwd(q, k, v, u, params, out, neff_out, status,
                            static_cast<cudaStream_t>(stream));
-    // Key moments only where they are used: the tensor-core kernel, beyond one
-    // tile, without a window (a window bounds every row's work anyway).
-    a.moments = fwd_moment_records(params->T) > 0 && params->window == 0
-                    ? static_cast<float *>(workspace)
-                    : nullptr;
+    // Key moments beyond one tile; the tensor-core launcher decides where they
+    // pay off (enough query tiles, or a long enough window).
+    a.moments = fwd_moment_records(params->T) > 0 ? static_cast<float *>(workspace) : nullptr;
     // The tensor-core kernel pairs two query heads of one key/value group per
     // CTA, so it needs an even group size; fp32 inputs use the CUDA-core kernel.
     const bool tc_ok = params->dtype == POLAR_BF16 && (params->Hq / params->Hkv) % 2 == 0;
@@ -431,9 +429,7 @@ polar_status_t polar_attn_fwd_host(const void *q_h, const void *k_h, const void 
             if (tc) {
                 FwdLaunch a = make_fwd(dq + b * qbb, dk + b * kbb, dv + b * kbb,
                                        reinterpret_cast<float *>(du), &p1, dout + b * qbb, ne, status, s);
-                a.moments = fwd_moment_records(p->T) > 0 && p->window == 0 && wsb
-                                ? reinterpret_cast<float *>(dws)
-                                : nullptr;
+                a.moments = fwd_moment_records(p->T) > 0 && wsb ? reinterpret_cast<float *>(dws) : nullptr;
                 a.qt_lo = r0 / 128;
                 a.qt_cnt = (r1 + 127) / 128 - a.qt_lo;
                 st = from_cuda(launch_fwd_tc(a));

@@ -318,7 +318,6 @@ struct TcArgs {
     int *status;
     const float *mom;  // key-moment records (kMoments only)
     int B, T, Hq, Hkv, nqt, npairs;
-    int qt_lo, qt_cnt;  // the query tiles this launch takes: qt_lo .. qt_lo + qt_cnt - 1
     int window;  // 0: all causal keys; W > 0: the last W of each row's
     float s, alpha, L, beta, inv_ln_L;
     // Backward rows pass (kRows) only: the upstream gradient dL/dout
@@ -329,6 +328,10 @@ struct TcArgs {
     float *coef;
     __nv_bfloat16 *dab;
     int Tpad;
+    // The prefill's first query tile (a launch takes gridDim.x / (npairs B)
+    // tiles from there).  Kept in the slot beside Tpad, so that the argument
+    // block keeps its size (a larger one cost the training variant spills).
+    int qt_lo;
     // Training forward (kSave) only: the saved row state [B][Hq][T][kFwdStateWords].
     float *state;
 };
@@ -498,7 +501,9 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CU
 
     // Work tile: heaviest query tiles first (longest causal rows).
     const int per_qt = a.npairs * a.B;
-    const int qt = a.qt_lo + a.qt_cnt - 1 - static_cast<int>(blockIdx.x) / per_qt;
+    // (The backward's rows pass and the training forward always take every tile.)
+    const int qt_top = kRows || kSave ? a.nqt : a.qt_lo + static_cast<int>(gridDim.x) / per_qt;
+    const int qt = qt_top - 1 - static_cast<int>(blockIdx.x) / per_qt;
     const int rem = static_cast<int>(blockIdx.x) % per_qt;
     const int pair = rem % a.npairs, b = rem / a.npairs;
     const int h0 = 2 * pair;
@@ -513,6 +518,11 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CU
     // or starts before the window of the tile's last row (min(q0 + 127, T - 1)).
     auto masked_tile = [&](int j) {
         return j == nkv - 1 || (window > 0 && (jt0 + j) * kBN < min(q0 + kBM, a.T) - window);
+    };
+    // Key tiles every row of the tile sees in full: first_full() .. qt - 1 (the
+    // unmasked loop tiles).  Their raw sums come from the key moments.
+    auto first_full = [&]() {
+        return window > 0 ? max(jt0, (min(q0 + kBM, a.T) - window + kBN - 1) / kBN) : 0;
     };
     // Visible key range of row t in loop tile j, in the tile's coordinates.
     auto vis_hi = [&](int j, int t) { return q0 + t - (jt0 + j) * kBN; };
@@ -627,7 +637,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CU
                 if constexpr (kMoments) {
                     // Y_i = Q_i (G_hi + G_lo) into S_i's first 64 columns, once
                     // softmax i has copied out its last score tile.
-                    if (ok && qt >= 1) {
+                    if (ok && first_full() <= qt - 1) {
                         constexpr uint32_t idesc_y = idesc_bf16(kBM, kHeadDim, false);
                         const uint32_t gh = ((smem_u32(sG) & 0x3FFFFu) >> 4) | (1u << 16);
                         const uint32_t gl = gh + (kGramBytes >> 4);
@@ -672,18 +682,45 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CU
         // bf16 per d) split into a bf16 high part and the bf16 of the remainder,
         // so that Q G_hi + Q G_lo carries the Gram to ~2^-16 relative; the key
         // sums stay fp32.
-        if (qt >= 1) {
+        const int jfull = first_full();
+        if (jfull <= qt - 1) {
             constexpr int kRec4 = kMomFloats / 4;
-            const int last = qt - 1, nclose = last / kMomChunk;
             const float4 *rec = reinterpret_cast<const float4 *>(a.mom) +
                                 (static_cast<size_t>(b) * a.Hkv + g) * (a.nqt - 1) * kRec4;
-            for (int i = lane; i < kRec4; i += 32) {
-                float4 v = rec[static_cast<size_t>(last) * kRec4 + i];
+            // Moments of key tiles 0 .. t: the records closing the chunks before
+            // t's, plus t's own running record.
+            auto prefix = [&](int t, int i) {
+                float4 v = rec[static_cast<size_t>(t) * kRec4 + i];
 #pragma unroll 4
-                for (int c = 0; c < nclose; ++c) {
+                for (int c = 0; c < t / kMomChunk; ++c) {
                     const float4 w = rec[static_cast<size_t>((c + 1) * kMomChunk - 1) * kRec4 + i];
                     v.x += w.x; v.y += w.y; v.z += w.z; v.w += w.w;
                 }
+                return v;
+            };
+            // Moments of key tiles lo .. hi (lo > 0): the records closing the
+            // whole chunks between, hi's running record, and lo's chunk from lo
+            // on (its closing record minus the running record before lo).
+            auto range = [&](int lo, int hi, int i) {
+                const int clo = lo / kMomChunk, chi = hi / kMomChunk;
+                float4 v = rec[static_cast<size_t>(hi) * kRec4 + i];
+                if (clo < chi) {
+                    const float4 w = rec[static_cast<size_t>(clo * kMomChunk + kMomChunk - 1) * kRec4 + i];
+                    v.x += w.x; v.y += w.y; v.z += w.z; v.w += w.w;
+                    for (int c = clo + 1; c < chi; ++c) {
+                        const float4 u = rec[static_cast<size_t>(c * kMomChunk + kMomChunk - 1) * kRec4 + i];
+                        v.x += u.x; v.y += u.y; v.z += u.z; v.w += u.w;
+                    }
+                }
+                if (lo % kMomChunk != 0) {
+                    const float4 u = rec[static_cast<size_t>(lo - 1) * kRec4 + i];
+                    v.x -= u.x; v.y -= u.y; v.z -= u.z; v.w -= u.w;
+                }
+                return v;
+            };
+            for (int i = lane; i < kRec4; i += 32) {
+                // Tiles jfull .. qt - 1 (under a window, a range of a few chunks).
+                const float4 v = jfull > 0 ? range(jfull, qt - 1, i) : prefix(qt - 1, i);
                 if (i < kHeadDim * kHeadDim / 4) {
                     const int d = i >> 4, e0 = (i & 15) * 4;
                     const uint32_t off = d * 128 + ((((e0 >> 3) ^ (d & 7))) << 4) + (e0 & 7) * 2;
@@ -780,7 +817,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CU
         if constexpr (kMoments) {
             // Null-floor sums over the full tiles, from the key moments: this
             // thread's 32 of the 64 components of S1 = <sum k, q>, S2 = <G q, q>.
-            if (ok && nkv > 1) {
+            if (ok && (kWindow ? first_full() <= qt - 1 : nkv > 1)) {
                 // g_full orders warp 3's key-sum stores before the reads below.
                 ok = mbar_wait(&y_full[slot], 0, a.status) && mbar_wait(&g_full, 0, a.status);
                 if (__all_sync(0xffffffffu, ok)) {
@@ -1035,7 +1072,8 @@ cudaError_t launch_fwd_tc(const FwdLaunch &a) {
                              reinterpret_cast<const void *>(fwd_tc_kernel<true, 2, false, false>),
                              reinterpret_cast<const void *>(fwd_tc_kernel<false, 1, false, false>),
                              reinterpret_cast<const void *>(fwd_tc_kernel<true, 2, false, true>),
-                             reinterpret_cast<const void *>(fwd_tc_kernel<false, 1, false, true>)};
+                             reinterpret_cast<const void *>(fwd_tc_kernel<false, 1, false, true>),
+                             reinterpret_cast<const void *>(fwd_tc_kernel<true, 2, true, true>)};
         for (const void *f : all) {
             e = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
             if (e != cudaSuccess) return e;
@@ -1045,7 +1083,7 @@ cudaError_t launch_fwd_tc(const FwdLaunch &a) {
         // warpgroups must fit in (registers per thread at launch) x 640.
         const long long need = 64ll * 128 + 104ll * 512;
         bool fits = true;
-        for (int i = 0; i < 5; ++i) {
+        for (int i = 0; i < 6; ++i) {
             if (i == 2 || i == 4) continue;  // the one-warpgroup-per-head kernels
             cudaFuncAttributes fa;
             e = cudaFuncGetAttributes(&fa, all[i]);
@@ -1068,14 +1106,14 @@ cudaError_t launch_fwd_tc(const FwdLaunch &a) {
     ta.nqt = (a.T + kBM - 1) / kBM;
     if (a.qt_lo < 0 || a.qt_cnt < 0 || a.qt_lo + a.qt_cnt > ta.nqt) return cudaErrorInvalidValue;
     ta.qt_lo = a.qt_lo;
-    ta.qt_cnt = a.qt_cnt > 0 ? a.qt_cnt : ta.nqt - a.qt_lo;
+    const int qt_cnt = a.qt_cnt > 0 ? a.qt_cnt : ta.nqt - a.qt_lo;
     // A window no shorter than the sequence changes nothing.
     const bool windowed = a.window > 0 && a.window < a.T;
     ta.window = windowed ? a.window : 0;
     ta.npairs = a.Hq / 2;
     ta.s = a.s; ta.alpha = a.alpha; ta.L = static_cast<float>(a.L); ta.beta = a.beta;
     ta.inv_ln_L = 1.0f / logf(static_cast<float>(a.L));
-    const long long ctas = static_cast<long long>(ta.qt_cnt) * ta.npairs * a.B;
+    const long long ctas = static_cast<long long>(qt_cnt) * ta.npairs * a.B;
     if (ctas <= 0) return cudaSuccess;
     if (ctas > 0x7fffffffll) return cudaErrorInvalidValue;
     // Fixed exponential reference while the smallest weight squared, 2^(-4 c_max log2e)
@@ -1085,15 +1123,20 @@ cudaError_t launch_fwd_tc(const FwdLaunch &a) {
                           (n_max > a.L ? 1.0f + a.alpha * logf(static_cast<float>(n_max) / a.L) : 1.0f) *
                           1.4426950408889634f;
     const unsigned grid = static_cast<unsigned>(ctas);
+    // The records the launch's query tiles read: those of key tiles below its
+    // last query tile, from the chunk holding its first query tile's.
+    const int rec_lo = ta.qt_lo > 0 ? ta.qt_lo - 1 : 0, rec_hi = ta.qt_lo + qt_cnt - 1;
     if (cl2_max <= 28.0f && (split_ok.load() & bit)) {
-        if (windowed) {
+        if (windowed && a.moments && a.window >= kMomMinTiles * kBN) {
+            // A window of at least kMomMinTiles tiles: the full tiles' raw sums
+            // from differences of key-moment prefixes (every record below rec_hi).
+            e = launch_fwd_moments(a.k, a.B, a.T, a.Hkv, a.moments, 0, rec_hi, a.stream);
+            if (e != cudaSuccess) return e;
+            fwd_tc_kernel<true, 2, true, true><<<grid, 640, kSmemBytes, a.stream>>>(tq, tk, tv, ta);
+        } else if (windowed) {
             fwd_tc_kernel<true, 2, false, true><<<grid, 640, kSmemBytes, a.stream>>>(tq, tk, tv, ta);
         } else if (a.moments && ta.nqt >= kMomMinTiles) {
-            // The records the launch's query tiles read: those of key tiles below
-            // its last query tile, from the chunk holding its first query tile's.
-            const int rec_hi = ta.qt_lo + ta.qt_cnt - 1;
-            e = launch_fwd_moments(a.k, a.B, a.T, a.Hkv, a.moments, ta.qt_lo > 0 ? ta.qt_lo - 1 : 0,
-                                   rec_hi, a.stream);
+            e = launch_fwd_moments(a.k, a.B, a.T, a.Hkv, a.moments, rec_lo, rec_hi, a.stream);
             if (e != cudaSuccess) return e;
             fwd_tc_kernel<true, 2, true, false><<<grid, 640, kSmemBytes, a.stream>>>(tq, tk, tv, ta);
         } else {
@@ -1151,7 +1194,6 @@ cudaError_t launch_bwd_rows_tc(const BwdLaunch &l, float *coef, void *dab, int T
     ta.B = l.B; ta.T = l.T; ta.Hq = l.Hq; ta.Hkv = l.Hkv;
     ta.nqt = Tpad / kBM;
     ta.qt_lo = 0;
-    ta.qt_cnt = ta.nqt;
     ta.npairs = l.Hq / 2;
     ta.window = windowed ? l.window : 0;
     ta.s = l.s; ta.alpha = l.alpha; ta.L = static_cast<float>(l.L); ta.beta = l.beta;
@@ -1231,7 +1273,6 @@ cudaError_t launch_fwd_train_tc(const FwdLaunch &a) {
     ta.B = a.B; ta.T = a.T; ta.Hq = a.Hq; ta.Hkv = a.Hkv;
     ta.nqt = (a.T + kBM - 1) / kBM;
     ta.qt_lo = 0;
-    ta.qt_cnt = ta.nqt;
     const bool windowed = a.window > 0 && a.window < a.T;
     ta.window = windowed ? a.window : 0;
     ta.npairs = a.Hq / 2;

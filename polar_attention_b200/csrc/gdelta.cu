@@ -1227,9 +1227,17 @@ cudaError_t launch_gdelta_prefill(const GdeltaLaunch &l) {
     g.cpg = g.nchunks;
     g.maps = g.starts = nullptr;
     if (l.dtype != POLAR_FP32) {
-        int dev = 0, sms = 148;
-        if (cudaGetDevice(&dev) == cudaSuccess)
-            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        static std::atomic<int> sm_cache[64];  // SMs per device, 0 until read
+        int dev = 0;
+        cudaError_t e = cudaGetDevice(&dev);
+        if (e != cudaSuccess) return e;
+        if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+        int sms = sm_cache[dev].load();
+        if (sms == 0) {
+            e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+            if (e != cudaSuccess) return e;
+            sm_cache[dev].store(sms);
+        }
         g.groups = scan_groups(l.B, l.H, g.nchunks, sms);
         if (g.groups > 1) {
             g.cpg = (g.nchunks + g.groups - 1) / g.groups;

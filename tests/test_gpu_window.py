@@ -44,6 +44,23 @@ def test_tc_prefill_window_all_rows(cuda_ok, T, G, Wn):
     _check_prefill(w, x, out, neff)
 
 
+@pytest.mark.parametrize("T,Wn", [(6000, 4200), (4700, 4096)])
+def test_tc_window_key_moments_all_rows(cuda_ok, T, Wn):
+    """A window of at least 4096 keys with a workspace: the raw sums of the key
+    tiles every row of a query tile sees in full come from differences of
+    key-moment prefixes (the tiles before the window and the diagonal tile
+    score by score).  Every row against the oracle; the no-workspace call
+    forms the same sums score by score and agrees to rounding."""
+    w = W.small_prefill(B=1, T=T, Hq=4, Hkv=2, dtype="bf16", seed=T, plant="frac",
+                        plant_frac=0.01, L=1024, window=Wn)
+    x = W.prefill_inputs(w, "cpu")
+    out, neff = _prefill(w, x)
+    _check_prefill(w, x, out, neff)
+    out0, neff0 = _prefill(w, x, moments=False)
+    assert ((neff - neff0).abs() / neff0).max().item() < 1e-4
+    assert (out.float() - out0.float()).abs().max().item() <= 2.0 ** -6
+
+
 def test_tc_window_running_max_path(cuda_ok):
     """A logit scale too large for the fixed reference takes the running-max
     kernel; its masked tiles honour the window too."""
