@@ -154,7 +154,15 @@ class ClockSampler:
               "clocks_event_reasons.sw_power_cap")
 
     def __init__(self, gpu_indices):
-        self.idx = [str(i) for i in gpu_indices]
+        # nvidia-smi numbers the GPUs of the host; name the process's own by UUID
+        # where torch knows it, so that CUDA_VISIBLE_DEVICES does not matter.
+        self.idx = []
+        for i in gpu_indices:
+            try:
+                u = str(torch.cuda.get_device_properties(i).uuid)
+                self.idx.append(u if u.startswith("GPU-") else "GPU-" + u)
+            except Exception:  # noqa: BLE001
+                self.idx.append(str(i))
         self.proc = None
 
     def __enter__(self):
@@ -199,6 +207,72 @@ class ClockSampler:
         return {"sm_mhz": statistics.median(use) if use else None,
                 "sm_max_mhz": max(mx) if mx else None, "reasons": sorted(reasons),
                 "samples": len(rows), "samples_under_load": len(load)}
+
+
+class NvmlSampler:
+    """The SM clock and the active clock-event reasons read through NVML about
+    every millisecond, on a thread, while the timed step loop runs: at small
+    step counts the whole loop is shorter than nvidia-smi's sampling interval.
+    Read-only queries; the device is found by its UUID, so a remapped
+    CUDA_VISIBLE_DEVICES still names the right GPU."""
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
+
+    def __init__(self, dev):
+        self.samples, self.max_mhz, self.err = [], None, None
+        self._stop = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            uuid = str(torch.cuda.get_device_properties(dev).uuid)
+            self.nvml = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByUUID(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception as e:  # noqa: BLE001 -- NVML is optional; the record says why it is absent
+            self.h, self.err = None, f"nvml unavailable: {type(e).__name__}"
+
+    def _run(self):
+        n = self.nvml
+        while not self._stop.is_set():
+            try:
+                self.samples.append((n.nvmlDeviceGetClockInfo(self.h, n.NVML_CLOCK_SM),
+                                     n.nvmlDeviceGetCurrentClocksEventReasons(self.h)))
+            except Exception as e:  # noqa: BLE001
+                self.err = f"nvml read failed: {type(e).__name__}"
+                return
+            self._stop.wait(0.001)
+
+    def start(self):
+        if self.h is None:
+            return
+        import threading
+        self._stop = threading.Event()
+        self._t = threading.Thread(target=self._run, daemon=True)
+        self._t.start()
+
+    def stop(self):
+        if self._stop is not None:
+            self._stop.set()
+            self._t.join(timeout=5)
+
+    def summary(self):
+        if not self.samples:
+            return None
+        mhz = [m for m, _ in self.samples]
+        reasons = sorted({name for _, r in self.samples for bit, name in self.REASONS.items() if r & bit})
+        return {"sm_mhz": statistics.median(mhz), "sm_min_mhz": min(mhz), "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(mhz)}
+
+
+def clock_record(fast: NvmlSampler, smi: ClockSampler) -> dict:
+    """The clock record of the line: NVML samples taken during the timed step
+    loop where there are any, else nvidia-smi's; nvidia-smi's samples over all
+    timed legs are kept beside them."""
+    s = smi.summary()
+    f = fast.summary()
+    if f is None:
+        return dict(s, source="nvidia-smi over the timed legs", nvml=fast.err)
+    return dict(f, source="nvml during the timed step loop, about 1 ms apart", nvidia_smi=s)
 
 
 # -------------------------------------------------------------- CPU oracle --
@@ -356,19 +430,10 @@ def run_ours(args):
     import atexit
     atexit.register(clk.__exit__, None, None, None)  # stop the sampler on any exit path
     time.sleep(0.3)  # let the sampler start before the timed region
-    # A step takes a few ms, so the timed loop alone can end between two
-    # samples.  Untimed steps run first, under the same sampler, until the GPU
-    # has been busy for about 0.6 s: the samples then see this workload's
-    # clocks and throttle reasons, and the timed loop follows without a gap.
-    load_steps, t_load = 0, time.perf_counter()
-    while time.perf_counter() - t_load < 0.6 and load_steps < 2000:
-        prefill()
-        decode()
-        load_steps += 1
-        if load_steps % 8 == 0:
-            torch.cuda.synchronize(dev)
+    fast_clk = NvmlSampler(dev)
     barrier(world, dev)
     torch.cuda.synchronize(dev)
+    fast_clk.start()
     n0 = pa.launch_count()
     outer[0].record(stream)
     for i in range(K):
@@ -379,6 +444,7 @@ def run_ours(args):
         ev[i][2].record(stream)
     outer[1].record(stream)
     torch.cuda.synchronize(dev)
+    fast_clk.stop()
     launches = pa.launch_count() - n0
     barrier(world, dev)
     st = pa.get_status()
@@ -708,7 +774,7 @@ def run_ours(args):
                                 "traffic": profiled_traffic("decode", sha_d),
                                 "peak_source": f"{peak_src} (copy bandwidth)"},
             "gpu_launches": int(launches),
-            "clocks": dict(clk.summary(), load_steps=load_steps),
+            "clocks": clock_record(fast_clk, clk),
             "e2e": e2e,
         }
         if bwd_res is not None:

@@ -227,14 +227,18 @@ size_t polar_attn_fwd_staging_size(const polar_params_t *params);
  * caller, at least polar_attn_fwd_staging_size bytes), runs the prefill
  * (polar_attn_fwd_ws with its workspace in the staging buffer), copies
  * out and n_eff back to host memory, and synchronises `stream`.  The work
- * goes batch by batch and, for the tensor-core prefill from T = 2048 on, in
- * row segments of whole 1024-row key chunks (about T/4 rows): the query tiles
- * of rows r0 .. r1 - 1 run on `stream` as soon as the rows 0 .. r1 - 1 of q,
- * k and v are in, while the next segment's inputs are copied in and the
- * previous segment's outputs copied out, on two copy streams the library
- * creates once per device and joins to `stream` through events.  The results
- * are those of polar_attn_fwd_ws, bit for bit.  Host-buffer calls on one
- * device are serialised.
+ * goes batch by batch.  For the tensor-core prefill a batch's k and v go in
+ * first and its key moments are formed; its queries then go in row segment
+ * by row segment (about T/4 rows from the top, then halves down to 1024 rows;
+ * one segment below T = 2048), from the LAST rows to the first, so that the
+ * longest causal rows start first and the call ends on the lightest segment.
+ * Each segment's prefill starts as soon as its queries are in, alternating
+ * between `stream` and a second compute stream, and its outputs are copied
+ * back as soon as it is done.  The copies run on two copy streams; the library
+ * creates these three streams once per device and joins them to `stream`
+ * through events.  The CUDA-core prefill goes whole batch by whole batch.  The
+ * results are those of polar_attn_fwd_ws, bit for bit.  Host-buffer calls on
+ * one device are serialised.
  */
 polar_status_t polar_attn_fwd_host(const void *q_h, const void *k_h, const void *v_h,
                                    const float *u_h, const polar_params_t *params, void *out_h,

@@ -38,14 +38,16 @@ int *status_ptr() {
 }
 
 // Copy streams and events of the host-buffer prefill, created once per device:
-// inputs go in on `in`, outputs come back on `out` (two copy engines), joined to
-// the caller's stream through events.  `mu` serialises host-buffer calls on a
-// device, which share these.
+// inputs go in on `in`, outputs come back on `out` (two copy engines), and a
+// second compute stream `comp2` lets consecutive row segments' prefills
+// overlap; all are joined to the caller's stream through events.  `mu`
+// serialises host-buffer calls on a device, which share these.
 struct HostPipe {
     std::mutex mu;
     bool ready = false;
-    cudaStream_t in = nullptr, out = nullptr;
-    cudaEvent_t start = nullptr, out_done = nullptr, in_done[2] = {}, comp_done[2] = {};
+    cudaStream_t in = nullptr, out = nullptr, comp2 = nullptr;
+    cudaEvent_t start = nullptr, out_done = nullptr, kv_in = nullptr, mom_done = nullptr,
+                comp2_done = nullptr, in_done[2] = {}, comp_done[2] = {};
 };
 HostPipe g_pipe[kMaxDevices];
 
@@ -58,8 +60,12 @@ HostPipe *host_pipe() {
         const unsigned ef = cudaEventDisableTiming;
         if (cudaStreamCreateWithFlags(&hp.in, cudaStreamNonBlocking) != cudaSuccess ||
             cudaStreamCreateWithFlags(&hp.out, cudaStreamNonBlocking) != cudaSuccess ||
+            cudaStreamCreateWithFlags(&hp.comp2, cudaStreamNonBlocking) != cudaSuccess ||
             cudaEventCreateWithFlags(&hp.start, ef) != cudaSuccess ||
-            cudaEventCreateWithFlags(&hp.out_done, ef) != cudaSuccess)
+            cudaEventCreateWithFlags(&hp.out_done, ef) != cudaSuccess ||
+            cudaEventCreateWithFlags(&hp.kv_in, ef) != cudaSuccess ||
+            cudaEventCreateWithFlags(&hp.mom_done, ef) != cudaSuccess ||
+            cudaEventCreateWithFlags(&hp.comp2_done, ef) != cudaSuccess)
             return nullptr;
         for (int i = 0; i < 2; ++i)
             if (cudaEventCreateWithFlags(&hp.in_done[i], ef) != cudaSuccess ||
@@ -155,7 +161,7 @@ FwdLaunch make_fwd(const void *q, const void *k, const void *v, const float *u,
     a.s = p->logit_scale; a.alpha = p->alpha; a.beta = p->beta; a.L = p->L_train;
     a.window = p->window;
     a.status = status; a.moments = nullptr; a.state = nullptr; a.stream = stream;
-    a.qt_lo = 0; a.qt_cnt = 0;
+    a.qt_lo = 0; a.qt_cnt = 0; a.moments_ready = false;
     return a;
 }
 
@@ -384,8 +390,6 @@ polar_status_t polar_attn_fwd_host(const void *q_h, const void *k_h, const void 
     char *dout = du + round_up(ub, 256);
     char *dne = dout + round_up(qb, 256);
     char *dws = dne + round_up(nb, 256);
-    // Batch by batch: the inputs of batch b+1 go in and the outputs of batch b-1
-    // come back while batch b runs on `stream`.
     HostPipe *hp = host_pipe();
     if (!hp) return POLAR_ERR_CUDA;
     std::lock_guard<std::mutex> lk(hp->mu);
@@ -396,59 +400,106 @@ polar_status_t polar_attn_fwd_host(const void *q_h, const void *k_h, const void 
     const char *qh = static_cast<const char *>(q_h), *kh = static_cast<const char *>(k_h),
                *vh = static_cast<const char *>(v_h);
     char *oh = static_cast<char *>(out_h), *nh = reinterpret_cast<char *>(neff_h);
-    // The copies start after earlier work on `stream` (which may still use the staging).
+    // The copies and the second compute stream start after earlier work on
+    // `stream` (which may still use the staging).
     if (cudaEventRecord(hp->start, s) != cudaSuccess ||
         cudaStreamWaitEvent(hp->in, hp->start, 0) != cudaSuccess ||
         cudaStreamWaitEvent(hp->out, hp->start, 0) != cudaSuccess ||
+        cudaStreamWaitEvent(hp->comp2, hp->start, 0) != cudaSuccess ||
         cudaMemcpyAsync(du, u_h, ub, cudaMemcpyHostToDevice, hp->in) != cudaSuccess)
         return POLAR_ERR_CUDA;
-    // Each batch goes in row segments of whole 1024-row key chunks, so that a
-    // segment's copies in and out overlap the prefill of its neighbours: the
-    // query tiles of rows r0 .. r1 - 1 need the keys of rows 0 .. r1 - 1 only,
-    // and the key-moment records of those keys.  The tensor-core prefill takes
-    // a query-tile range; the CUDA-core one runs whole batches.
     const bool tc = p->dtype == POLAR_BF16 && (p->Hq / p->Hkv) % 2 == 0 && p->impl != POLAR_IMPL_SIMT;
     const size_t qrow = static_cast<size_t>(p->Hq) * kHeadDim * e, krow = static_cast<size_t>(p->Hkv) * kHeadDim * e;
-    const int seg_rows = tc && p->T >= 2048 ? static_cast<int>(round_up((p->T + 3) / 4, 1024)) : p->T;
     int *status = status_ptr();
     if (!status) return POLAR_ERR_CUDA;
-    int ev = 0;
-    for (int b = 0; b < p->B; ++b) {
-        for (int r0 = 0; r0 < p->T; r0 += seg_rows, ++ev) {
-            const int r1 = std::min(p->T, r0 + seg_rows);
-            const size_t rows_s = static_cast<size_t>(r1 - r0);
-            const size_t qo = b * qbb + r0 * qrow, ko = b * kbb + r0 * krow;
-            const int e2 = ev & 1;
-            if (cudaMemcpyAsync(dq + qo, qh + qo, rows_s * qrow, cudaMemcpyHostToDevice, hp->in) != cudaSuccess ||
-                cudaMemcpyAsync(dk + ko, kh + ko, rows_s * krow, cudaMemcpyHostToDevice, hp->in) != cudaSuccess ||
-                cudaMemcpyAsync(dv + ko, vh + ko, rows_s * krow, cudaMemcpyHostToDevice, hp->in) != cudaSuccess ||
+    // Copies rows lo .. hi - 1 of batch b's output (and their n_eff, [B, Hq, T])
+    // back once `done` (recorded on the stream that computed them) has passed.
+    auto send_back = [&](int b, int lo, int hi, cudaEvent_t done) {
+        const size_t rows_s = static_cast<size_t>(hi - lo);
+        const size_t qo = b * qbb + lo * qrow;
+        if (cudaStreamWaitEvent(hp->out, done, 0) != cudaSuccess ||
+            cudaMemcpyAsync(oh + qo, dout + qo, rows_s * qrow, cudaMemcpyDeviceToHost, hp->out) != cudaSuccess)
+            return false;
+        return !neff_h || cudaMemcpy2DAsync(nh + b * nbb + lo * 4, static_cast<size_t>(p->T) * 4,
+                                            dne + b * nbb + lo * 4, static_cast<size_t>(p->T) * 4,
+                                            rows_s * 4, p->Hq, cudaMemcpyDeviceToHost, hp->out) == cudaSuccess;
+    };
+    if (!tc) {
+        // CUDA-core prefill: whole batches; the inputs of batch b+1 go in and
+        // the outputs of batch b-1 come back while batch b runs.
+        for (int b = 0; b < p->B; ++b) {
+            const int e2 = b & 1;
+            if (cudaMemcpyAsync(dq + b * qbb, qh + b * qbb, qbb, cudaMemcpyHostToDevice, hp->in) != cudaSuccess ||
+                cudaMemcpyAsync(dk + b * kbb, kh + b * kbb, kbb, cudaMemcpyHostToDevice, hp->in) != cudaSuccess ||
+                cudaMemcpyAsync(dv + b * kbb, vh + b * kbb, kbb, cudaMemcpyHostToDevice, hp->in) != cudaSuccess ||
                 cudaEventRecord(hp->in_done[e2], hp->in) != cudaSuccess ||
                 cudaStreamWaitEvent(s, hp->in_done[e2], 0) != cudaSuccess)
                 return POLAR_ERR_CUDA;
             float *ne = neff_h ? reinterpret_cast<float *>(dne + b * nbb) : nullptr;
-            if (tc) {
-                FwdLaunch a = make_fwd(dq + b * qbb, dk + b * kbb, dv + b * kbb,
-                                       reinterpret_cast<float *>(du), &p1, dout + b * qbb, ne, status, s);
-                a.moments = fwd_moment_records(p->T) > 0 && wsb ? reinterpret_cast<float *>(dws) : nullptr;
-                a.qt_lo = r0 / 128;
-                a.qt_cnt = (r1 + 127) / 128 - a.qt_lo;
-                st = from_cuda(launch_fwd_tc(a));
-            } else {
-                st = polar_attn_fwd_ws(dq + b * qbb, dk + b * kbb, dv + b * kbb,
-                                       reinterpret_cast<float *>(du), &p1, dout + b * qbb, ne,
-                                       wsb ? dws : nullptr, wsb, stream);
-            }
+            st = polar_attn_fwd_ws(dq + b * qbb, dk + b * kbb, dv + b * kbb, reinterpret_cast<float *>(du),
+                                   &p1, dout + b * qbb, ne, wsb ? dws : nullptr, wsb, stream);
             if (st != POLAR_OK) return st;
-            if (cudaEventRecord(hp->comp_done[e2], s) != cudaSuccess ||
-                cudaStreamWaitEvent(hp->out, hp->comp_done[e2], 0) != cudaSuccess ||
-                cudaMemcpyAsync(oh + qo, dout + qo, rows_s * qrow, cudaMemcpyDeviceToHost, hp->out) != cudaSuccess)
-                return POLAR_ERR_CUDA;
-            // n_eff [B, Hq, T]: this segment's rows of every head of batch b.
-            if (neff_h && cudaMemcpy2DAsync(nh + b * nbb + r0 * 4, static_cast<size_t>(p->T) * 4,
-                                            dne + b * nbb + r0 * 4, static_cast<size_t>(p->T) * 4,
-                                            rows_s * 4, p->Hq, cudaMemcpyDeviceToHost, hp->out) != cudaSuccess)
+            if (cudaEventRecord(hp->comp_done[e2], s) != cudaSuccess || !send_back(b, 0, p->T, hp->comp_done[e2]))
                 return POLAR_ERR_CUDA;
         }
+    } else {
+        // Tensor-core prefill, batch by batch.  A batch's keys and values go in
+        // first and its key moments are formed; then its queries go in row
+        // segment by row segment from the LAST rows to the first.  A segment's
+        // prefill then needs nothing that is still in flight but its own
+        // queries, so the heaviest segments (the longest causal rows) start
+        // first and the call ends on the lightest one, whose output copy is
+        // short.  Segments alternate between `stream` and a second compute
+        // stream, so that a segment's prefill fills the SMs that the previous
+        // one's last wave leaves idle; every segment's outputs go back as soon
+        // as it is done.  Boundaries fall on 128-row query tiles: segments of
+        // about T/4 rows from the top, then halves down to 1024 rows.
+        const int nqt = (p->T + 127) / 128;
+        const int seg = p->T >= 2048 ? static_cast<int>(round_up((p->T + 3) / 4, 128)) : p->T;
+        int ev = 0;
+        for (int b = 0; b < p->B; ++b) {
+            if (cudaMemcpyAsync(dk + b * kbb, kh + b * kbb, kbb, cudaMemcpyHostToDevice, hp->in) != cudaSuccess ||
+                cudaMemcpyAsync(dv + b * kbb, vh + b * kbb, kbb, cudaMemcpyHostToDevice, hp->in) != cudaSuccess ||
+                cudaEventRecord(hp->kv_in, hp->in) != cudaSuccess ||
+                cudaStreamWaitEvent(s, hp->kv_in, 0) != cudaSuccess)
+                return POLAR_ERR_CUDA;
+            float *ne = neff_h ? reinterpret_cast<float *>(dne + b * nbb) : nullptr;
+            FwdLaunch a = make_fwd(dq + b * qbb, dk + b * kbb, dv + b * kbb, reinterpret_cast<float *>(du),
+                                   &p1, dout + b * qbb, ne, status, s);
+            a.moments = wsb ? reinterpret_cast<float *>(dws + b * wsb) : nullptr;
+            if (fwd_tc_reads_moments(a) &&
+                launch_fwd_moments(a.k, 1, p->T, p->Hkv, a.moments, 0, nqt - 1, s) != cudaSuccess)
+                return POLAR_ERR_CUDA;
+            a.moments_ready = true;
+            if (cudaEventRecord(hp->mom_done, s) != cudaSuccess ||
+                cudaStreamWaitEvent(hp->comp2, hp->mom_done, 0) != cudaSuccess)
+                return POLAR_ERR_CUDA;
+            for (int hi = p->T, lo = 0; hi > 0; hi = lo, ++ev) {
+                lo = seg == p->T ? 0
+                     : hi > seg  ? static_cast<int>(round_up(static_cast<size_t>(hi - seg), 128))
+                     : hi > 1024 ? hi / 2 / 128 * 128
+                                 : 0;
+                const int e2 = ev & 1;
+                cudaStream_t cs = e2 ? hp->comp2 : s;
+                const size_t qo = b * qbb + lo * qrow;
+                if (cudaMemcpyAsync(dq + qo, qh + qo, static_cast<size_t>(hi - lo) * qrow,
+                                    cudaMemcpyHostToDevice, hp->in) != cudaSuccess ||
+                    cudaEventRecord(hp->in_done[e2], hp->in) != cudaSuccess ||
+                    cudaStreamWaitEvent(cs, hp->in_done[e2], 0) != cudaSuccess)
+                    return POLAR_ERR_CUDA;
+                a.stream = cs;
+                a.qt_lo = lo / 128;
+                a.qt_cnt = (hi + 127) / 128 - a.qt_lo;
+                st = from_cuda(launch_fwd_tc(a));
+                if (st != POLAR_OK) return st;
+                if (cudaEventRecord(hp->comp_done[e2], cs) != cudaSuccess ||
+                    !send_back(b, lo, hi, hp->comp_done[e2]))
+                    return POLAR_ERR_CUDA;
+            }
+        }
+        if (cudaEventRecord(hp->comp2_done, hp->comp2) != cudaSuccess ||
+            cudaStreamWaitEvent(s, hp->comp2_done, 0) != cudaSuccess)
+            return POLAR_ERR_CUDA;
     }
     if (cudaEventRecord(hp->out_done, hp->out) != cudaSuccess ||
         cudaStreamWaitEvent(s, hp->out_done, 0) != cudaSuccess)

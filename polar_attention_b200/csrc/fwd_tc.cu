@@ -1058,6 +1058,17 @@ bool make_qkv_maps(const void *q, const void *k, const void *v, int B, int T, in
 
 }  // namespace
 
+bool fwd_tc_reads_moments(const FwdLaunch &a) {
+    if (!a.moments || a.dtype != POLAR_BF16 || (a.Hq / a.Hkv) % 2 != 0) return false;
+    const bool windowed = a.window > 0 && a.window < a.T;
+    const int n_max = windowed ? a.window : a.T;
+    const float cl2_max = a.s *
+                          (n_max > a.L ? 1.0f + a.alpha * logf(static_cast<float>(n_max) / a.L) : 1.0f) *
+                          1.4426950408889634f;
+    if (cl2_max > 28.0f) return false;
+    return windowed ? a.window >= kMomMinTiles * kBN : (a.T + kBM - 1) / kBM >= kMomMinTiles;
+}
+
 cudaError_t launch_fwd_tc(const FwdLaunch &a) {
     const int G = a.Hq / a.Hkv;
     if (a.dtype != POLAR_BF16 || G % 2 != 0) return cudaErrorNotSupported;
@@ -1130,14 +1141,18 @@ cudaError_t launch_fwd_tc(const FwdLaunch &a) {
         if (windowed && a.moments && a.window >= kMomMinTiles * kBN) {
             // A window of at least kMomMinTiles tiles: the full tiles' raw sums
             // from differences of key-moment prefixes (every record below rec_hi).
-            e = launch_fwd_moments(a.k, a.B, a.T, a.Hkv, a.moments, 0, rec_hi, a.stream);
-            if (e != cudaSuccess) return e;
+            if (!a.moments_ready) {
+                e = launch_fwd_moments(a.k, a.B, a.T, a.Hkv, a.moments, 0, rec_hi, a.stream);
+                if (e != cudaSuccess) return e;
+            }
             fwd_tc_kernel<true, 2, true, true><<<grid, 640, kSmemBytes, a.stream>>>(tq, tk, tv, ta);
         } else if (windowed) {
             fwd_tc_kernel<true, 2, false, true><<<grid, 640, kSmemBytes, a.stream>>>(tq, tk, tv, ta);
         } else if (a.moments && ta.nqt >= kMomMinTiles) {
-            e = launch_fwd_moments(a.k, a.B, a.T, a.Hkv, a.moments, rec_lo, rec_hi, a.stream);
-            if (e != cudaSuccess) return e;
+            if (!a.moments_ready) {
+                e = launch_fwd_moments(a.k, a.B, a.T, a.Hkv, a.moments, rec_lo, rec_hi, a.stream);
+                if (e != cudaSuccess) return e;
+            }
             fwd_tc_kernel<true, 2, true, false><<<grid, 640, kSmemBytes, a.stream>>>(tq, tk, tv, ta);
         } else {
             fwd_tc_kernel<true, 2, false, false><<<grid, 640, kSmemBytes, a.stream>>>(tq, tk, tv, ta);

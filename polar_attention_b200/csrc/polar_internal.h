@@ -23,6 +23,7 @@ struct FwdLaunch {
     float *moments;  // key-moment records (fwd_moments_bytes), or null
     float *state;    // training forward: saved row state (FwdState layout), or null
     int qt_lo, qt_cnt;  // query tiles qt_lo .. qt_lo + qt_cnt - 1 (qt_cnt 0: to the end)
+    bool moments_ready;  // `moments` already holds the records of every key tile: no pre-pass
     cudaStream_t stream;
 };
 
@@ -141,6 +142,9 @@ size_t gdelta_workspace_bytes(int B, int T, int H);
 constexpr int kMomChunk = 8;
 constexpr int kMomFloats = 64 * 64 + 64;
 int fwd_moment_records(int T);
+// Whether launch_fwd_tc would read key-moment records for this launch (and so
+// run the pre-pass for its tiles unless they are ready).
+bool fwd_tc_reads_moments(const FwdLaunch &a);
 size_t fwd_moments_bytes(int B, int T, int Hkv);
 // Computes the records rec_lo .. rec_hi - 1 (rounded out to whole chunks).
 cudaError_t launch_fwd_moments(const void *k, int B, int T, int Hkv, float *rec, int rec_lo,
