@@ -128,30 +128,34 @@ def test_host_buffers_match_device_buffers(cuda_ok):
     assert torch.equal(oh, a.cpu()) and torch.equal(nh, na.cpu())
 
 
-def test_full_workload_sampled(cuda_ok):
+def test_full_workload_every_sequence(cuda_ok):
     """The 32-sequence, 128K-256K-context pool (6.6 GB, shuffled pages) in the
-    launch configuration the bench times: every head of four sequences against
-    the oracle, which reads a host copy of just those sequences' pages."""
+    launch configuration the bench times: every head of every sequence against
+    the oracle, eight sequences at a time, each group's oracle reading a host
+    copy of just that group's pages."""
     w = W.DECODE
     x = W.decode_inputs(w, "cuda")
     out, neff = _decode(w, x)
     assert pa.get_status() == 0
     assert torch.isfinite(out.float()).all() and (neff >= 1).all()
-    seqs = [0, 7, 19, 31]
-    pt = x["page_table"][seqs].cpu()
-    sl = x["seqlens"][seqs].cpu()
-    used = [int(pt[i, p]) for i in range(len(seqs)) for p in range((int(sl[i]) + 63) // 64)]
-    remap = {pg: k for k, pg in enumerate(used)}
-    sub = x["kv_pages"][torch.tensor(used, device="cuda")]
-    pt2 = torch.full_like(pt, -1)
-    for i in range(len(seqs)):
-        for p in range((int(sl[i]) + 63) // 64):
-            pt2[i, p] = remap[int(pt[i, p])]
-    xs = {"q": x["q"][seqs], "kv_pages": sub, "page_table": pt2, "seqlens": sl, "u": x["u"]}
-    ref = PT.oracle_decode(w, xs)
-    o = out[seqs].float().cpu().numpy().reshape(len(seqs) * w.Hq, -1).astype(np.float64)
-    n = neff[seqs].cpu().numpy().reshape(-1).astype(np.float64)
-    PT.compare(o, n, ref, np.arange(len(seqs) * w.Hq), PT.OUT_TOL_BF16, what="decode full")
+    for g0 in range(0, w.num_seqs, 8):
+        seqs = list(range(g0, min(g0 + 8, w.num_seqs)))
+        pt = x["page_table"][seqs].cpu()
+        sl = x["seqlens"][seqs].cpu()
+        used = [int(pt[i, p]) for i in range(len(seqs)) for p in range((int(sl[i]) + 63) // 64)]
+        remap = {pg: k for k, pg in enumerate(used)}
+        sub = x["kv_pages"][torch.tensor(used, device="cuda")]
+        pt2 = torch.full_like(pt, -1)
+        for i in range(len(seqs)):
+            for p in range((int(sl[i]) + 63) // 64):
+                pt2[i, p] = remap[int(pt[i, p])]
+        xs = {"q": x["q"][seqs], "kv_pages": sub, "page_table": pt2, "seqlens": sl, "u": x["u"]}
+        ref = PT.oracle_decode(w, xs)
+        o = out[seqs].float().cpu().numpy().reshape(len(seqs) * w.Hq, -1).astype(np.float64)
+        n = neff[seqs].cpu().numpy().reshape(-1).astype(np.float64)
+        PT.compare(o, n, ref, np.arange(len(seqs) * w.Hq), PT.OUT_TOL_BF16,
+                   what=f"decode full, sequences {seqs[0]}-{seqs[-1]}")
+        del sub, xs, ref
 
 
 def test_per_head_variant_reads_the_same_pages(cuda_ok):
