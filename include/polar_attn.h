@@ -238,7 +238,10 @@ size_t polar_attn_fwd_staging_size(const polar_params_t *params);
  * creates these three streams once per device and joins them to `stream`
  * through events.  The CUDA-core prefill goes whole batch by whole batch.  The
  * results are those of polar_attn_fwd_ws, bit for bit.  Host-buffer calls on
- * one device are serialised.
+ * one device are serialised.  Argument errors return before anything is
+ * queued; after a POLAR_ERR_CUDA return, copies or prefills already queued on
+ * the library's streams may still run, so synchronise the device before the
+ * staging buffer or the host buffers are reused.
  */
 polar_status_t polar_attn_fwd_host(const void *q_h, const void *k_h, const void *v_h,
                                    const float *u_h, const polar_params_t *params, void *out_h,

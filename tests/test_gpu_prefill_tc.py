@@ -218,16 +218,18 @@ def test_unnormalised_inputs_are_reported(cuda_ok):
     assert pa.get_status() == 0
 
 
-@pytest.mark.parametrize("T,Wn", [(300, 0), (4500, 0), (4500, 700), (8192, 0), (8192, 1500)])
+@pytest.mark.parametrize("T,Wn", [(300, 0), (4500, 0), (4500, 700), (8192, 0), (8192, 1500),
+                                   (8192, 4200)])
 def test_host_buffers_match_device_buffers(cuda_ok, T, Wn):
     """polar_attn_fwd_host runs the prefill batch by batch: a batch's keys and
     values first (and its key moments), then its queries in row segments from
     the last rows to the first, on two compute streams (T=4500: rows 3456-4499,
     2304-3455, 1152-2303, 512-1151, 0-511; T=8192: 6144-8191, 4096-6143,
     2048-4095, 1024-2047, 0-1023; T=300: one segment).  With three batches, on
-    the key-moment path (T=4500, 8192), below it and with a window, its rows
-    equal the device-buffer call's bit for bit: a row depends on neither the
-    other batches nor the split."""
+    the key-moment path (T=4500, 8192), below it, with a window and with a
+    window long enough for key moments (W=4200), its rows equal the
+    device-buffer call's bit for bit: a row depends on neither the other
+    batches nor the split."""
     w = W.small_prefill(B=3, T=T, Hq=8, Hkv=2, dtype="bf16", seed=T, plant="frac",
                         plant_frac=0.01, L=512, window=Wn)
     x = W.prefill_inputs(w, "cpu")
