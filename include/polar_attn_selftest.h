@@ -49,6 +49,17 @@ polar_status_t polar_attn_selftest_decode_per_head(const void *q, const void *kv
                                                    float *neff_out, void *workspace,
                                                    size_t ws_bytes, void *stream);
 
+/*
+ * Host logic only (no device work): the row segments polar_attn_fwd_host uses
+ * for the tensor-core prefill of T rows, in the order it sends them, from the
+ * last rows to the first.  Segment i covers rows seg_lo[i] .. seg_hi[i] - 1;
+ * about T/4 rows from the top, then halves down to 1024 rows, boundaries on
+ * 128-row query tiles, one segment below T = 2048.  Writes at most `cap`
+ * segments (the last always reaches row 0) and returns their number, or -1
+ * for T < 0, cap < 1 or a NULL pointer.  Host pointers, owned by the caller.
+ */
+int polar_attn_selftest_fwd_host_segments(int T, int *seg_lo, int *seg_hi, int cap);
+
 #ifdef __cplusplus
 }
 #endif

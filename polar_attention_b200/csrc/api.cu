@@ -353,6 +353,35 @@ polar_status_t polar_attn_bwd_from_state(const void *q, const void *k, const voi
     return from_cuda(launch_bwd_from_state(a, out, state));
 }
 
+namespace {
+
+// Row segments of a host-buffer tensor-core prefill of T rows, from the last
+// rows to the first: about T/4 rows from the top, then halves down to 1024
+// rows (one segment below T = 2048).  Boundaries fall on 128-row query tiles.
+// Writes at most `cap` segments (the last one always ends at row 0) and
+// returns how many.
+int fwd_host_segments(int T, int *seg_lo, int *seg_hi, int cap) {
+    const int seg = T >= 2048 ? static_cast<int>(round_up((T + 3) / 4, 128)) : T;
+    int n = 0;
+    for (int hi = T, lo = 0; hi > 0 && n < cap; hi = lo, ++n) {
+        lo = seg == T ? 0
+             : hi > seg  ? static_cast<int>(round_up(static_cast<size_t>(hi - seg), 128))
+             : hi > 1024 ? hi / 2 / 128 * 128
+                         : 0;
+        if (n == cap - 1) lo = 0;
+        seg_lo[n] = lo;
+        seg_hi[n] = hi;
+    }
+    return n;
+}
+
+}  // namespace
+
+int polar_attn_selftest_fwd_host_segments(int T, int *seg_lo, int *seg_hi, int cap) {
+    if (T < 0 || cap < 1 || !seg_lo || !seg_hi) return -1;
+    return fwd_host_segments(T, seg_lo, seg_hi, cap);
+}
+
 size_t polar_attn_fwd_staging_size(const polar_params_t *p) {
     if (check_fwd(p) != POLAR_OK) return 0;
     const size_t e = dtype_bytes(p->dtype);
@@ -452,10 +481,11 @@ polar_status_t polar_attn_fwd_host(const void *q_h, const void *k_h, const void 
         // short.  Segments alternate between `stream` and a second compute
         // stream, so that a segment's prefill fills the SMs that the previous
         // one's last wave leaves idle; every segment's outputs go back as soon
-        // as it is done.  Boundaries fall on 128-row query tiles: segments of
-        // about T/4 rows from the top, then halves down to 1024 rows.
+        // as it is done (segments: fwd_host_segments).
         const int nqt = (p->T + 127) / 128;
-        const int seg = p->T >= 2048 ? static_cast<int>(round_up((p->T + 3) / 4, 128)) : p->T;
+        constexpr int kMaxSeg = 64;
+        int seg_lo[kMaxSeg], seg_hi[kMaxSeg];
+        const int nseg = fwd_host_segments(p->T, seg_lo, seg_hi, kMaxSeg);
         int ev = 0;
         for (int b = 0; b < p->B; ++b) {
             if (cudaMemcpyAsync(dk + b * kbb, kh + b * kbb, kbb, cudaMemcpyHostToDevice, hp->in) != cudaSuccess ||
@@ -474,11 +504,8 @@ polar_status_t polar_attn_fwd_host(const void *q_h, const void *k_h, const void 
             if (cudaEventRecord(hp->mom_done, s) != cudaSuccess ||
                 cudaStreamWaitEvent(hp->comp2, hp->mom_done, 0) != cudaSuccess)
                 return POLAR_ERR_CUDA;
-            for (int hi = p->T, lo = 0; hi > 0; hi = lo, ++ev) {
-                lo = seg == p->T ? 0
-                     : hi > seg  ? static_cast<int>(round_up(static_cast<size_t>(hi - seg), 128))
-                     : hi > 1024 ? hi / 2 / 128 * 128
-                                 : 0;
+            for (int k = 0; k < nseg; ++k, ++ev) {
+                const int lo = seg_lo[k], hi = seg_hi[k];
                 const int e2 = ev & 1;
                 cudaStream_t cs = e2 ? hp->comp2 : s;
                 const size_t qo = b * qbb + lo * qrow;
