@@ -34,7 +34,8 @@ EXPORTS = ["polar_attn_default_params", "polar_attn_fwd_workspace_size", "polar_
            "polar_attn_bwd_workspace_size", "polar_attn_bwd",
            "polar_gdelta_prefill_workspace_size", "polar_gdelta_prefill", "polar_gdelta_step",
            "polar_attn_selftest_timeout", "polar_attn_selftest_decode_per_head",
-           "polar_attn_fwd_state_size", "polar_attn_fwd_train", "polar_attn_bwd_from_state"]
+           "polar_attn_fwd_state_size", "polar_attn_fwd_train", "polar_attn_bwd_from_state",
+           "polar_attn_selftest_fwd_host_segments"]
 
 
 class PolarError(RuntimeError):
@@ -106,6 +107,9 @@ def lib() -> ctypes.CDLL:
             L.polar_attn_selftest_timeout.argtypes = [P]
             L.polar_attn_selftest_decode_per_head.argtypes = [P, P, I, P, I, P, I, P, PP, P, P, P,
                                                               Z, P]
+            IP = ctypes.POINTER(ctypes.c_int)
+            L.polar_attn_selftest_fwd_host_segments.argtypes = [I, IP, IP, I]
+            L.polar_attn_selftest_fwd_host_segments.restype = I
             GP = ctypes.POINTER(GdeltaParams)
             L.polar_gdelta_prefill_workspace_size.argtypes = [GP]
             L.polar_gdelta_prefill_workspace_size.restype = Z
@@ -125,6 +129,17 @@ def lib() -> ctypes.CDLL:
                 getattr(L, name).restype = I
             _lib = L
     return _lib
+
+
+def fwd_host_segments(T: int, cap: int = 64):
+    """The row segments polar_attn_fwd_host sends for a tensor-core prefill of
+    T rows, in order: a list of (lo, hi) (host logic; no device work)."""
+    lo = (ctypes.c_int * max(cap, 1))()
+    hi = (ctypes.c_int * max(cap, 1))()
+    n = lib().polar_attn_selftest_fwd_host_segments(int(T), lo, hi, int(cap))
+    if n < 0:
+        raise ValueError(f"polar_attn_selftest_fwd_host_segments: bad arguments (T={T}, cap={cap})")
+    return [(lo[i], hi[i]) for i in range(n)]
 
 
 def status_string(code: int) -> str:
