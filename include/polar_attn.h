@@ -233,8 +233,9 @@ size_t polar_attn_fwd_staging_size(const polar_params_t *params);
  * one segment below T = 2048), from the LAST rows to the first, so that the
  * longest causal rows start first and the call ends on the lightest segment.
  * Each segment's prefill starts as soon as its queries are in, alternating
- * between `stream` and a second compute stream, and its outputs are copied
- * back as soon as it is done.  The copies run on two copy streams; the library
+ * between `stream` and a second compute stream, and its output rows are
+ * copied back as soon as it is done (a batch's n_eff in one copy after its
+ * last segment).  The copies run on two copy streams; the library
  * creates these three streams once per device and joins them to `stream`
  * through events.  The CUDA-core prefill goes whole batch by whole batch.  The
  * results are those of polar_attn_fwd_ws, bit for bit.  Host-buffer calls on

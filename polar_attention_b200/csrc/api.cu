@@ -441,17 +441,22 @@ polar_status_t polar_attn_fwd_host(const void *q_h, const void *k_h, const void 
     const size_t qrow = static_cast<size_t>(p->Hq) * kHeadDim * e, krow = static_cast<size_t>(p->Hkv) * kHeadDim * e;
     int *status = status_ptr();
     if (!status) return POLAR_ERR_CUDA;
-    // Copies rows lo .. hi - 1 of batch b's output (and their n_eff, [B, Hq, T])
-    // back once `done` (recorded on the stream that computed them) has passed.
+    // Copies rows lo .. hi - 1 of batch b's output back once `done` (recorded on
+    // the stream that computed them) has passed.
     auto send_back = [&](int b, int lo, int hi, cudaEvent_t done) {
         const size_t rows_s = static_cast<size_t>(hi - lo);
         const size_t qo = b * qbb + lo * qrow;
-        if (cudaStreamWaitEvent(hp->out, done, 0) != cudaSuccess ||
-            cudaMemcpyAsync(oh + qo, dout + qo, rows_s * qrow, cudaMemcpyDeviceToHost, hp->out) != cudaSuccess)
-            return false;
-        return !neff_h || cudaMemcpy2DAsync(nh + b * nbb + lo * 4, static_cast<size_t>(p->T) * 4,
-                                            dne + b * nbb + lo * 4, static_cast<size_t>(p->T) * 4,
-                                            rows_s * 4, p->Hq, cudaMemcpyDeviceToHost, hp->out) == cudaSuccess;
+        return cudaStreamWaitEvent(hp->out, done, 0) == cudaSuccess &&
+               cudaMemcpyAsync(oh + qo, dout + qo, rows_s * qrow, cudaMemcpyDeviceToHost, hp->out) ==
+                   cudaSuccess;
+    };
+    // Batch b's n_eff ([Hq, T], contiguous) in one copy, queued on the output
+    // stream after the copies of all its segments, which waited for each of
+    // their prefills: one 2-D copy per segment (Hq strided runs) costs the
+    // output stream far more than the bytes.
+    auto send_neff = [&](int b) {
+        return !neff_h || cudaMemcpyAsync(nh + b * nbb, dne + b * nbb, nbb, cudaMemcpyDeviceToHost,
+                                          hp->out) == cudaSuccess;
     };
     if (!tc) {
         // CUDA-core prefill: whole batches; the inputs of batch b+1 go in and
@@ -468,7 +473,8 @@ polar_status_t polar_attn_fwd_host(const void *q_h, const void *k_h, const void 
             st = polar_attn_fwd_ws(dq + b * qbb, dk + b * kbb, dv + b * kbb, reinterpret_cast<float *>(du),
                                    &p1, dout + b * qbb, ne, wsb ? dws : nullptr, wsb, stream);
             if (st != POLAR_OK) return st;
-            if (cudaEventRecord(hp->comp_done[e2], s) != cudaSuccess || !send_back(b, 0, p->T, hp->comp_done[e2]))
+            if (cudaEventRecord(hp->comp_done[e2], s) != cudaSuccess ||
+                !send_back(b, 0, p->T, hp->comp_done[e2]) || !send_neff(b))
                 return POLAR_ERR_CUDA;
         }
     } else {
@@ -523,6 +529,7 @@ polar_status_t polar_attn_fwd_host(const void *q_h, const void *k_h, const void 
                     !send_back(b, lo, hi, hp->comp_done[e2]))
                     return POLAR_ERR_CUDA;
             }
+            if (!send_neff(b)) return POLAR_ERR_CUDA;
         }
         if (cudaEventRecord(hp->comp2_done, hp->comp2) != cudaSuccess ||
             cudaStreamWaitEvent(s, hp->comp2_done, 0) != cudaSuccess)
